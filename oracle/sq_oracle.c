@@ -1,0 +1,267 @@
+/*
+ * sq_oracle.c -- plain, slow, obviously-correct CPU oracle for the SmoothQuant
+ * W8A8 linear layer (per-token activation scales x per-output-channel weight
+ * scales, int8 x int8 -> int32, dequantised epilogue).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the package smoke check and
+ * the CPU-baseline leg of the benchmark may load this library.  The product
+ * path (the CUDA library) never calls it and shares no code with it.
+ *
+ * Arithmetic contract (kept deliberately plain so it can be checked by eye):
+ *   - every floating-point step is one IEEE-754 binary32 operation with
+ *     round-to-nearest-even; the file is compiled with -ffp-contract=off so no
+ *     multiply-add is fused, and without -ffast-math;
+ *   - bf16 inputs are widened to fp32 exactly (the 16 bf16 bits become the
+ *     high half of the fp32 word);
+ *   - "round" is round-half-to-even (nearbyint under the default
+ *     FE_TONEAREST mode), then clamp to the symmetric range [-127, 127];
+ *   - a zero absolute maximum gives scale 0 and all-zero codes (no division);
+ *   - inputs must be finite; non-finite inputs are outside the contract.
+ *
+ * Sources, by page and section:
+ *   [W]  "Understanding W8A8 INT8 LLM Quantization", section "Why Naive
+ *        Weight Quantization Doesn't Work, and How GPTQ Fixes It": the
+ *        per-channel weight scale max|w|/127 and code round(w/scale).
+ *   [A]  same page, section "Why Activation Quantization Is Hard, and How
+ *        SmoothQuant Fixes It": one dynamic scale per token over all channels.
+ *   [S]  same page, sections "Where the outlier actually comes from" and
+ *        "How the smoothing factor is computed": per-input-channel absmax over
+ *        calibration samples, smoothing factor s_j, activations divided by s,
+ *        the matching weight input channel multiplied by s.
+ *   [V]  "quant_llm_int8" (LLM.int8() architecture page), sections "The
+ *        architecture: every piece explained" and "End-to-end flow": int8
+ *        matmul accumulating in int32, dequantised by the outer product of the
+ *        per-row activation scales and the per-column weight scales.
+ *   [C]  "How does SmoothQuant int8 LLM calibration work...", section "The
+ *        Technical Workflow for Int8 Quantization Deployment": calibration
+ *        records the maximum absolute value of every channel.
+ *
+ * The smoothing-factor equation itself did not survive the page's text
+ * extraction; this oracle uses s_j = A_j^alpha / B_j^(1-alpha), with A_j the
+ * calibration absmax of input channel j and B_j the absmax of input channel j
+ * of the weight, evaluated in fp64 with libm pow and rounded once to fp32.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#include <stddef.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* dtype codes shared with the Python wrapper: 0 = fp32, 1 = bf16 */
+#define SQO_F32 0
+#define SQO_BF16 1
+
+static float widen_bf16(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* element i of a row-major fp32 or bf16 buffer, widened to fp32 exactly */
+static float elem(const void *p, int dt, size_t i)
+{
+    if (dt == SQO_BF16)
+        return widen_bf16(((const uint16_t *)p)[i]);
+    return ((const float *)p)[i];
+}
+
+/* round-half-to-even of an fp32 value to the nearest bf16 (16-bit pattern) */
+uint16_t sqo_f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu))
+        return (uint16_t)((u >> 16) | 0x0040u); /* keep NaN a NaN */
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* [C], [S]: A_j = max over calibration tokens t of |X[t, j]|.
+ * x: [T, K] with row stride ldx elements.  ax: [K], overwritten. */
+void sqo_calib_absmax(const void *x, int dt, int64_t T, int64_t K, int64_t ldx, float *ax)
+{
+    for (int64_t j = 0; j < K; ++j)
+        ax[j] = 0.0f;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t j = 0; j < K; ++j) {
+            float v = fabsf(elem(x, dt, (size_t)(t * ldx + j)));
+            if (v > ax[j])
+                ax[j] = v;
+        }
+}
+
+/* [S]: B_j = max over output channels n of |W[n, j]|, W stored [N, K]
+ * (out x in), so input channel j is column j. */
+void sqo_weight_in_absmax(const void *w, int dt, int64_t N, int64_t K, float *aw)
+{
+    for (int64_t j = 0; j < K; ++j)
+        aw[j] = 0.0f;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < K; ++j) {
+            float v = fabsf(elem(w, dt, (size_t)(n * K + j)));
+            if (v > aw[j])
+                aw[j] = v;
+        }
+}
+
+/* [S]: s_j = A_j^alpha / B_j^(1 - alpha) in fp64, rounded once to fp32.
+ * alpha is the fp32 argument widened to fp64.  A channel with A_j == 0 or
+ * B_j == 0 is left unmigrated (s_j = 1). */
+void sqo_smooth_factors(const float *ax, const float *aw, int64_t K, float alpha, float *s)
+{
+    double a = (double)alpha;
+    for (int64_t j = 0; j < K; ++j) {
+        if (ax[j] == 0.0f || aw[j] == 0.0f) {
+            s[j] = 1.0f;
+            continue;
+        }
+        double num = pow((double)ax[j], a);
+        double den = pow((double)aw[j], 1.0 - a);
+        s[j] = (float)(num / den);
+    }
+}
+
+/* [S] then [W]: W'[n, k] = W[n, k] * s[k] (the weight's input channel k is
+ * scaled up by s_k); sw[n] = max_k |W'[n, k]| / 127;
+ * wq[n, k] = clamp(round(W'[n, k] / sw[n]), -127, 127). */
+void sqo_smooth_quant_weight(const void *w, int dt, int64_t N, int64_t K, const float *s,
+                             int8_t *wq, float *sw)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = fabsf(elem(w, dt, (size_t)(n * K + k)) * s[k]);
+            if (v > amax)
+                amax = v;
+        }
+        float scale = amax / 127.0f;
+        sw[n] = scale;
+        for (int64_t k = 0; k < K; ++k) {
+            int8_t q = 0;
+            if (amax != 0.0f) {
+                float wp = elem(w, dt, (size_t)(n * K + k)) * s[k];
+                float r = nearbyintf(wp / scale);
+                if (r > 127.0f)
+                    r = 127.0f;
+                if (r < -127.0f)
+                    r = -127.0f;
+                q = (int8_t)r;
+            }
+            wq[n * K + k] = q;
+        }
+    }
+}
+
+/* [S] then [A]: x^[m, k] = X[m, k] / s[k]; sx[m] = max_k |x^[m, k]| / 127;
+ * xq[m, k] = clamp(round(x^[m, k] / sx[m]), -127, 127).  Only the rows listed
+ * in `rows` (or all M rows when rows == NULL) are computed; row i of the
+ * outputs corresponds to rows[i].  x has row stride ldx elements. */
+void sqo_quant_act_rows(const void *x, int dt, int64_t ldx, int64_t K, const float *s,
+                        const int64_t *rows, int64_t nrows, int8_t *xq, float *sx)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = fabsf(elem(x, dt, (size_t)(m * ldx + k)) / s[k]);
+            if (v > amax)
+                amax = v;
+        }
+        float scale = amax / 127.0f;
+        sx[i] = scale;
+        for (int64_t k = 0; k < K; ++k) {
+            int8_t q = 0;
+            if (amax != 0.0f) {
+                float xh = elem(x, dt, (size_t)(m * ldx + k)) / s[k];
+                float r = nearbyintf(xh / scale);
+                if (r > 127.0f)
+                    r = 127.0f;
+                if (r < -127.0f)
+                    r = -127.0f;
+                q = (int8_t)r;
+            }
+            xq[i * K + k] = q;
+        }
+    }
+}
+
+void sqo_quant_act(const void *x, int dt, int64_t M, int64_t K, const float *s, int8_t *xq,
+                   float *sx)
+{
+    sqo_quant_act_rows(x, dt, K, K, s, NULL, M, xq, sx);
+}
+
+/* [V]: acc[m, n] = sum_k xq[m, k] * wq[n, k], exact in int32 (|acc| is at
+ * most K * 127^2, below 2^31 for K <= 133144).  Both operands are K-major. */
+void sqo_gemm_i32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K,
+                  int32_t *acc)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int32_t a = 0;
+            for (int64_t k = 0; k < K; ++k)
+                a += (int32_t)xq[m * K + k] * (int32_t)wq[n * K + k];
+            acc[m * N + n] = a;
+        }
+}
+
+/* [V]: one accumulator for each listed (m, n) pair. */
+void sqo_gemm_i32_pairs(const int8_t *xq, int64_t ldxq, const int8_t *wq, int64_t K,
+                        const int64_t *ms, const int64_t *ns, int64_t npairs, int32_t *acc)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < npairs; ++i) {
+        int32_t a = 0;
+        for (int64_t k = 0; k < K; ++k)
+            a += (int32_t)xq[ms[i] * ldxq + k] * (int32_t)wq[ns[i] * K + k];
+        acc[i] = a;
+    }
+}
+
+/* [V]: y = ((float)acc * sx[m]) * sw[n], two fp32 multiplies in this order.
+ * y_f32 and/or y_bf16 may be NULL. */
+void sqo_dequant(const int32_t *acc, const float *sx, const float *sw, int64_t M, int64_t N,
+                 float *y_f32, uint16_t *y_bf16)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            float t = (float)acc[m * N + n] * sx[m];
+            float y = t * sw[n];
+            if (y_f32)
+                y_f32[m * N + n] = y;
+            if (y_bf16)
+                y_bf16[m * N + n] = sqo_f32_to_bf16(y);
+        }
+}
+
+/* [V]: the dequantised value for each listed (m, n) pair, same arithmetic as
+ * sqo_dequant; acc[i], sx[i] and sw[i] belong to pair i. */
+void sqo_dequant_pairs(const int32_t *acc, const float *sx, const float *sw, int64_t npairs,
+                       float *y_f32, uint16_t *y_bf16)
+{
+    for (int64_t i = 0; i < npairs; ++i) {
+        float t = (float)acc[i] * sx[i];
+        float y = t * sw[i];
+        if (y_f32)
+            y_f32[i] = y;
+        if (y_bf16)
+            y_bf16[i] = sqo_f32_to_bf16(y);
+    }
+}
+
+int sqo_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

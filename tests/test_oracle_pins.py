@@ -1,0 +1,391 @@
+"""Pins for the CPU oracle against what the pages and the mathematics fix.
+
+Each test ties the oracle to something other than itself: a worked example
+printed on the pages (tests/golden, cited there), a closed form, an invariant
+of round-to-nearest quantisation, or brute force on tiny inputs.  Together they
+are chosen so that a plausible slip in the oracle (a dropped term, a wrong sign
+or index, a transposed operand, the wrong rounding rule) fails at least one.
+"""
+import math
+
+import numpy as np
+import pytest
+
+F32 = np.float32
+
+
+def f32(x):
+    return np.asarray(x, dtype=np.float32)
+
+
+# ---------------------------------------------------------------------------
+# Worked examples printed on the pages
+# ---------------------------------------------------------------------------
+
+def test_weight_rtn_worked_example(oracle, golden):
+    """Per-output-channel scale max|w|/127 and round(w/scale): "Understanding
+    W8A8 INT8 LLM Quantization", "Why Naive Weight Quantization Doesn't Work"."""
+    g = golden("weight_rtn_example.json")
+    w = f32([g["w_page_columns"]["ch0"], g["w_page_columns"]["ch1"]])  # [N=2, K=3]
+    s = np.ones(3, F32)
+    wq, sw = oracle.smooth_quant_weight(w, s)
+    for i, ch in enumerate(("ch0", "ch1")):
+        # the scales the page prints (4 significant digits)
+        assert float(sw[i]) == pytest.approx(g["scales_page"][ch], rel=5e-4)
+        assert wq[i].tolist() == g["q_expected"][ch]
+    # every printed code except the page's arithmetic slip matches the page
+    diffs = [(ch, k) for ch in ("ch0", "ch1") for k in range(3)
+             if g["q_page"][ch][k] != g["q_expected"][ch][k]]
+    assert diffs == [("ch1", 1)]
+    # reconstruction and the page's output for x = [1, 2, 0.5]
+    x = np.asarray(g["x_page"], np.float64)
+    rec = wq.astype(np.float64) * sw.astype(np.float64)[:, None]
+    for i, ch in enumerate(("ch0", "ch1")):
+        assert rec[i] == pytest.approx(g["reconstructed_expected"][ch], abs=6e-5)
+        assert float(rec[i] @ x) == pytest.approx(g["y_reconstructed_expected"][ch], abs=6e-4)
+        assert float(w[i].astype(np.float64) @ x) == pytest.approx(g["y_original_page"][ch], abs=1e-6)
+    # the page's own (slipped) code reproduces its printed 2.193
+    q_slip = np.asarray(g["q_page"]["ch1"], np.float64) * float(sw[1])
+    assert float(q_slip @ x) == pytest.approx(g["y_reconstructed_page"]["ch1"], abs=6e-4)
+
+
+def test_activation_outlier_worked_example(oracle, golden):
+    """One dynamic scale per token across all channels: "Why Activation
+    Quantization Is Hard, and How SmoothQuant Fixes It"."""
+    g = golden("activation_outlier_example.json")
+    x = f32([g["x"]])
+    xq, sx = oracle.quant_act(x, np.ones(4, F32))
+    assert float(sx[0]) == pytest.approx(g["scale_page"], rel=5e-4)
+    assert xq[0].tolist() == g["q_expected"] == g["q_page"]
+
+
+def test_smoothed_activation_worked_example(oracle, golden):
+    """Dividing the outlier channel by s removes the outlier: "Where the outlier
+    actually comes from" (gamma of channel 3 divided by 100)."""
+    g = golden("smoothed_activation_example.json")
+    x = f32([g["x_before_smoothing"]])
+    s = f32(g["s"])
+    xq, sx = oracle.quant_act(x, s)
+    assert float(sx[0]) == pytest.approx(g["scale_page"], rel=2e-2)  # page prints 0.012
+    assert float(sx[0]) == float(F32(1.53) / F32(127.0))
+    assert xq[0].tolist() == g["q_expected"]
+    # the page's printed 63 is reproduced only by its rounded scale and half-up rounding
+    assert math.floor(0.75 / g["scale_page"] + 0.5) == g["q_page"][1]
+
+
+# ---------------------------------------------------------------------------
+# Rounding rule, clamping, zero scales
+# ---------------------------------------------------------------------------
+
+def test_round_half_to_even_activation(oracle):
+    """amax = 127 gives scale exactly 1, so exact .5 quotients expose the tie rule."""
+    row = f32([[127.0, 2.5, 3.5, -2.5, 0.5, 1.5, -126.5, 126.5]])
+    xq, sx = oracle.quant_act(row, np.ones(8, F32))
+    assert float(sx[0]) == 1.0
+    assert xq[0].tolist() == [127, 2, 4, -2, 0, 2, -126, 126]
+
+
+def test_round_half_to_even_weight(oracle):
+    w = f32([[-127.0, 2.5, 3.5, -0.5, 5.5, -6.5, 0.0, 1.0]])
+    wq, sw = oracle.smooth_quant_weight(w, np.ones(8, F32))
+    assert float(sw[0]) == 1.0
+    assert wq[0].tolist() == [-127, 2, 4, 0, 6, -6, 0, 1]
+
+
+def test_symmetric_range_never_minus_128(oracle):
+    rng = np.random.default_rng(1)
+    x = f32(rng.standard_normal((64, 96)) * 5)
+    xq, _ = oracle.quant_act(x, np.ones(96, F32))
+    assert xq.min() >= -127 and xq.max() <= 127
+    w = f32(rng.standard_normal((64, 96)))
+    wq, _ = oracle.smooth_quant_weight(w, np.ones(96, F32))
+    assert wq.min() >= -127
+
+
+def test_zero_rows_and_channels(oracle):
+    x = np.zeros((3, 16), F32)
+    x[1, 5] = -2.0
+    xq, sx = oracle.quant_act(x, np.ones(16, F32))
+    assert sx.tolist() == [0.0, float(F32(2.0) / F32(127.0)), 0.0]
+    assert not xq[0].any() and not xq[2].any() and xq[1, 5] == -127
+    w = np.zeros((2, 16), F32)
+    w[0, 3] = 0.5
+    wq, sw = oracle.smooth_quant_weight(w, np.ones(16, F32))
+    assert sw[1] == 0.0 and not wq[1].any() and wq[0, 3] == 127
+    # degenerate channels are not migrated
+    s = oracle.smooth_factors(f32([0.0, 3.0, 2.0]), f32([1.0, 0.0, 2.0]), 0.5)
+    assert s.tolist() == [1.0, 1.0, 1.0]
+
+
+# ---------------------------------------------------------------------------
+# Smoothing factor: closed forms and the alpha special cases
+# ---------------------------------------------------------------------------
+
+def test_smooth_factor_closed_forms(oracle):
+    ax = f32([100.0, 4.0, 32.0, 7.25, 1e-3])
+    aw = f32([1.0, 16.0, 0.5, 7.25, 0.04])
+    s = oracle.smooth_factors(ax, aw, 0.5)
+    assert s[0] == 10.0 and s[1] == 0.5 and s[3] == 1.0
+    assert s[4] == pytest.approx(math.sqrt(1e-3 / 0.04), rel=1e-6)
+    # alpha = 0.8: 32^0.8 / 0.5^0.2 = 2^4 * 2^0.2 = 2^4.2
+    s8 = oracle.smooth_factors(ax, aw, 0.8)
+    a = float(F32(0.8))  # the fp32 argument, widened
+    assert s8[2] == F32(32.0 ** a / 0.5 ** (1.0 - a))
+    assert float(s8[2]) == pytest.approx(2 ** 4.2, rel=1e-6)
+
+
+def test_smooth_factor_alpha_one_is_activation_absmax(oracle):
+    rng = np.random.default_rng(2)
+    ax = f32(np.abs(rng.standard_normal(257)) * 30 + 0.01)
+    aw = f32(np.abs(rng.standard_normal(257)) * 0.1 + 1e-4)
+    s = oracle.smooth_factors(ax, aw, 1.0)
+    assert np.array_equal(s, ax)
+
+
+def test_smooth_factor_alpha_zero_depends_only_on_weight(oracle):
+    """alpha = 0: s_j = 1 / B_j, independent of the calibration statistics."""
+    rng = np.random.default_rng(3)
+    aw = f32(np.abs(rng.standard_normal(300)) * 0.1 + 1e-4)
+    s1 = oracle.smooth_factors(f32(np.abs(rng.standard_normal(300)) + 1), aw, 0.0)
+    s2 = oracle.smooth_factors(f32(np.abs(rng.standard_normal(300)) * 50 + 1), aw, 0.0)
+    assert np.array_equal(s1, s2)
+    assert np.array_equal(s1, (1.0 / aw.astype(np.float64)).astype(F32))
+
+
+def test_alpha_zero_unit_weight_leaves_x_unchanged(oracle):
+    """The plain reading of "alpha near zero preserves the original
+    distribution": with every weight input channel's absmax equal to 1 the
+    factors are all 1 and X/s is X bit for bit."""
+    rng = np.random.default_rng(4)
+    K = 64
+    w = f32(rng.uniform(-1, 1, (32, K)))
+    w[0, :] = 1.0
+    xcal = f32(rng.standard_normal((40, K)) * 9)
+    ax, aw, s, _, _ = oracle.prepare(xcal, w, 0.0)
+    assert np.all(aw == 1.0) and np.all(s == 1.0)
+    x = f32(rng.standard_normal((5, K)))
+    a = oracle.quant_act(x, s)
+    b = oracle.quant_act(x, np.ones(K, F32))
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_alpha_one_flattens_calibration_channels(oracle):
+    """alpha = 1 migrates all difficulty: every calibration channel of X/s has
+    absmax exactly 1 (a / a = 1 in IEEE arithmetic)."""
+    rng = np.random.default_rng(5)
+    K = 48
+    xcal = f32(rng.standard_normal((30, K)) * rng.uniform(0.1, 80, K))
+    w = f32(rng.standard_normal((16, K)) * 0.02)
+    ax, aw, s, _, _ = oracle.prepare(xcal, w, 1.0)
+    assert np.array_equal(s, ax)
+    assert np.all(np.max(np.abs(xcal / s), axis=0) == 1.0)
+
+
+def test_smooth_factor_monotone(oracle):
+    """A larger calibration outlier gives a larger s (for alpha > 0); a larger
+    weight range gives a smaller one (for alpha < 1)."""
+    ax = f32([1.0, 2.0, 10.0, 100.0])
+    s = oracle.smooth_factors(ax, f32([0.1] * 4), 0.5)
+    assert np.all(np.diff(s) > 0)
+    s = oracle.smooth_factors(f32([5.0] * 4), ax, 0.5)
+    assert np.all(np.diff(s) < 0)
+
+
+# ---------------------------------------------------------------------------
+# Calibration absmax
+# ---------------------------------------------------------------------------
+
+def test_calib_absmax_bruteforce_and_merge(oracle):
+    rng = np.random.default_rng(6)
+    x = f32(rng.standard_normal((37, 80)) * 3)
+    ax = oracle.calib_absmax(x)
+    assert np.array_equal(ax, np.abs(x).max(axis=0))
+    # statistics of two calibration batches merge by max
+    a1 = oracle.calib_absmax(x[:20])
+    a2 = oracle.calib_absmax(x[20:])
+    assert np.array_equal(ax, np.maximum(a1, a2))
+    # bf16 input: exact widening
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    axb = oracle.calib_absmax(xb)
+    assert np.array_equal(axb, np.abs(oracle.bf16_bits_to_f32(xb)).max(axis=0))
+
+
+def test_small_workload_outliers_dominate_calibration(oracle):
+    from w8a8_int8_gemm_channel_b200 import workloads as wls
+
+    wl = wls.WORKLOADS["small"]
+    lin = wl.linears[0]
+    xcal = wls.calibration(wl, lin).numpy()
+    ax = oracle.calib_absmax(xcal)
+    assert sorted(np.argsort(ax)[-4:].tolist()) == [3, 77, 150, 201]
+
+
+# ---------------------------------------------------------------------------
+# Smoothing: identity and direction
+# ---------------------------------------------------------------------------
+
+def _small_case(oracle):
+    from w8a8_int8_gemm_channel_b200 import workloads as wls
+
+    wl = wls.WORKLOADS["small"]
+    lin = wl.linears[0]
+    xcal = wls.calibration(wl, lin).numpy()
+    w = wls.weight(wl, lin).numpy()
+    x = wls.inputs(wl, lin, 16).numpy()
+    return wl, xcal, w, x
+
+
+def test_smoothing_identity_fp64(oracle):
+    """(X diag(s)^-1)(W diag(s))^T = X W^T to 1e-10 relative in fp64."""
+    wl, xcal, w, x = _small_case(oracle)
+    _, _, s, _, _ = oracle.prepare(xcal, w, wl.alpha)
+    assert s.max() > 5 * np.median(s)  # the outlier channels were migrated
+    smoothed, plain = oracle.smoothing_identity_fp64(x, w, s)
+    rel = np.linalg.norm(smoothed - plain) / np.linalg.norm(plain)
+    assert rel < 1e-10
+
+
+def test_smoothing_direction(oracle):
+    """The weight's INPUT channel k is multiplied by s_k and the activation
+    channel k divided by it; the dequantised operands reproduce W diag(s) and
+    X diag(s)^-1 to within half a quantisation step."""
+    wl, xcal, w, x = _small_case(oracle)
+    _, _, s, wq, sw = oracle.prepare(xcal, w, wl.alpha)
+    ws = w.astype(np.float64) * s.astype(np.float64)[None, :]
+    err_w = np.abs(wq * sw.astype(np.float64)[:, None] - ws)
+    assert np.all(err_w <= sw.astype(np.float64)[:, None] * (0.5 + 1e-5))
+    xq, sx = oracle.quant_act(x, s)
+    xs = x.astype(np.float64) / s.astype(np.float64)[None, :]
+    err_x = np.abs(xq * sx.astype(np.float64)[:, None] - xs)
+    assert np.all(err_x <= sx.astype(np.float64)[:, None] * (0.5 + 1e-5))
+    # the max-magnitude element of every nonzero row lands on +-127
+    assert np.all(np.abs(xq).max(axis=1) == 127)
+    assert np.all(np.abs(wq).max(axis=1) == 127)
+
+
+def test_scales_are_per_token_and_per_output_channel(oracle):
+    """Scaling one token row by 2 doubles only its scale; scaling one output
+    row of W by 2 doubles only its scale; the codes stay put."""
+    rng = np.random.default_rng(7)
+    x = f32(rng.standard_normal((6, 32)))
+    s = f32(rng.uniform(0.5, 4, 32))
+    xq, sx = oracle.quant_act(x, s)
+    x2 = x.copy()
+    x2[2] *= 2
+    xq2, sx2 = oracle.quant_act(x2, s)
+    assert np.array_equal(xq, xq2)
+    assert sx2[2] == 2 * sx[2] and np.array_equal(np.delete(sx, 2), np.delete(sx2, 2))
+    w = f32(rng.standard_normal((5, 32)))
+    wq, sw = oracle.smooth_quant_weight(w, s)
+    w2 = w.copy()
+    w2[3] *= 2
+    wq2, sw2 = oracle.smooth_quant_weight(w2, s)
+    assert np.array_equal(wq, wq2)
+    assert sw2[3] == 2 * sw[3] and np.array_equal(np.delete(sw, 3), np.delete(sw2, 3))
+
+
+def test_quant_act_row_subset(oracle):
+    rng = np.random.default_rng(8)
+    x = f32(rng.standard_normal((9, 48)))
+    s = f32(rng.uniform(0.5, 4, 48))
+    xq, sx = oracle.quant_act(x, s)
+    rows = np.array([7, 0, 3])
+    xq_r, sx_r = oracle.quant_act(x, s, rows=rows)
+    assert np.array_equal(xq_r, xq[rows]) and np.array_equal(sx_r, sx[rows])
+
+
+def test_smoothing_reduces_quantisation_error(oracle):
+    """Sanity signal, not a parity criterion: on the outlier-bearing small
+    workload, W8A8 with smoothing is closer to the unquantised X W^T than
+    per-token W8A8 without it."""
+    wl, xcal, w, x = _small_case(oracle)
+    ref = oracle.fp64_reference_linear(x, w)
+
+    def err(alpha):
+        if alpha is None:
+            s = np.ones(w.shape[1], F32)
+            wq, sw = oracle.smooth_quant_weight(w, s)
+        else:
+            _, _, s, wq, sw = oracle.prepare(xcal, w, alpha)
+        y, _, _, _ = oracle.linear(x, s, wq, sw, "f32")
+        return np.linalg.norm(y - ref) / np.linalg.norm(ref)
+
+    assert err(wl.alpha) < 0.5 * err(None)
+
+
+# ---------------------------------------------------------------------------
+# int32 GEMM and dequantisation
+# ---------------------------------------------------------------------------
+
+def test_gemm_bruteforce_tiny(oracle):
+    rng = np.random.default_rng(9)
+    for M, N, K in [(1, 1, 1), (2, 3, 5), (8, 8, 8), (3, 7, 4), (5, 2, 8)]:
+        xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+        wq = rng.integers(-127, 128, (N, K)).astype(np.int8)
+        acc = oracle.gemm_i32(xq, wq)
+        for m in range(M):
+            for n in range(N):
+                ref = 0
+                for k in range(K):
+                    ref += int(xq[m, k]) * int(wq[n, k])
+                assert int(acc[m, n]) == ref
+    pairs = oracle.gemm_i32_pairs(xq, wq, [4, 0, 2], [1, 0, 1])
+    assert pairs.tolist() == [int(acc[4, 1]), int(acc[0, 0]), int(acc[2, 1])]
+
+
+def test_int32_accumulator_extremes():
+    """|acc| <= K * 127^2 < 2^31 for every K in the workloads (K <= 28672); the bound holds up to K = 133144."""
+    from oracle import oracle as o
+
+    K = 28672
+    assert K * 127 * 127 < 2 ** 31 and 133144 * 127 * 127 < 2 ** 31 <= 133145 * 127 * 127
+    xq = np.full((1, K), 127, np.int8)
+    wq = np.full((2, K), -127, np.int8)
+    wq[1, ::2] = 127
+    acc = o.gemm_i32(xq, wq)
+    assert acc.tolist() == [[-K * 127 * 127, 0]]
+
+
+def test_dequant_against_fp64(oracle):
+    """y = (acc * sx) * sw: two correctly rounded fp32 products, so within
+    2 ulp (plus the int->float rounding) of the exact product."""
+    rng = np.random.default_rng(10)
+    acc = rng.integers(-400_000_000, 400_000_000, (7, 9)).astype(np.int32)
+    sx = f32(rng.uniform(1e-3, 3, 7))
+    sw = f32(rng.uniform(1e-5, 1e-2, 9))
+    y = oracle.dequant(acc, sx, sw, "f32")
+    exact = acc.astype(np.float64) * sx.astype(np.float64)[:, None] * sw.astype(np.float64)[None, :]
+    assert np.all(np.abs(y - exact) <= 3 * 2.0 ** -24 * np.abs(exact))
+    # order: acc times the token scale first
+    assert np.array_equal(y, (acc.astype(F32) * sx[:, None]) * sw[None, :])
+    yb = oracle.dequant(acc, sx, sw, "bf16")
+    assert np.array_equal(yb, oracle.f32_to_bf16_bits(y))
+    yp = oracle.dequant_pairs(acc[[1, 6], [2, 8]], sx[[1, 6]], sw[[2, 8]], "f32")
+    assert np.array_equal(yp, y[[1, 6], [2, 8]])
+
+
+def test_bf16_round_half_to_even(oracle):
+    """bf16 keeps 7 fraction bits: ulp(1) = 2^-7."""
+    cases = {
+        1.0: 0x3F80,
+        1.0 + 2 ** -8: 0x3F80,          # tie -> even (down)
+        1.0 + 3 * 2 ** -8: 0x3F82,      # tie -> even (up)
+        1.0 + 2 ** -8 + 2 ** -20: 0x3F81,
+        -(1.0 + 2 ** -8 + 2 ** -20): 0xBF81,
+        3.0e38: 0x7F62,
+        0.0: 0x0000,
+    }
+    got = oracle.f32_to_bf16_bits(f32(list(cases)))
+    assert got.tolist() == list(cases.values())
+    # a value just below the largest finite fp32 rounds to +inf in bf16
+    assert int(oracle.f32_to_bf16_bits(f32([3.4e38]))[0]) == 0x7F80
+
+
+def test_linear_end_to_end_small(oracle):
+    """The whole path on the small workload stays close to fp64 X W^T."""
+    wl, xcal, w, x = _small_case(oracle)
+    _, _, s, wq, sw = oracle.prepare(xcal, w, wl.alpha)
+    y, xq, sx, acc = oracle.linear(x, s, wq, sw, "f32")
+    ref = oracle.fp64_reference_linear(x, w)
+    assert y.shape == (16, 256) and y.dtype == np.float32
+    assert np.linalg.norm(y - ref) / np.linalg.norm(ref) < 0.05
