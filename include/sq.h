@@ -1,0 +1,198 @@
+/*
+ * sq.h -- C ABI of libsq, the SmoothQuant W8A8 INT8 linear layer for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The layer computes Y[M, N] = X[M, K] W[N, K]^T with both operands in int8:
+ *   offline   A_j   = max over calibration tokens of |X_cal[t, j]|
+ *             B_j   = max over output channels of |W[n, j]|
+ *             s_j   = A_j^alpha / B_j^(1 - alpha)
+ *             W'    = W diag(s), quantised per output channel (row n) to int8
+ *   online    X^    = X diag(s)^-1, quantised per token (row m) to int8
+ *             acc   = Xq Wq^T in int32, Y = (acc * sx[m]) * sw[n]
+ *
+ * Sources (page title, section):
+ *   "Understanding W8A8 INT8 LLM Quantization": "Why Naive Weight Quantization
+ *     Doesn't Work, and How GPTQ Fixes It" (per-channel scale max|w|/127 and
+ *     round(w/scale)); "Why Activation Quantization Is Hard, and How
+ *     SmoothQuant Fixes It" (one dynamic scale per token); "Where the outlier
+ *     actually comes from" and "How the smoothing factor is computed"
+ *     (calibration absmax per channel, the factor s, dividing the activation
+ *     and multiplying the matching weight input channel by s).
+ *   "quant_llm_int8": "The architecture: every piece explained" and "End-to-end
+ *     flow" (int8 matmul accumulating in int32, dequantised by the outer
+ *     product of per-row activation scales and per-column weight scales).
+ *   "How does SmoothQuant int8 LLM calibration work...": "The Technical
+ *     Workflow for Int8 Quantization Deployment" (absmax per channel over
+ *     calibration samples; alpha between 0 and 1).
+ *
+ * Numerics (every entry point): fp32 IEEE arithmetic, round-to-nearest-even,
+ * no fused multiply-add in any step whose result is rounded; codes are
+ * clamp(round_half_even(v / scale), -127, 127) (-128 is never produced); a
+ * zero absolute maximum gives scale 0 and all-zero codes; s_j is evaluated in
+ * fp64 and rounded once to fp32, and is 1 where A_j or B_j is 0.  Inputs must
+ * be finite.  Results are bit-identical to the plain CPU definition, except
+ * that s_j may differ in its last bit where the fp64 quotient lies within a
+ * few fp64 ulps of an fp32 rounding midpoint (libm and CUDA pow differ by up
+ * to 2 fp64 ulps).
+ *
+ * Conventions (every entry point):
+ *   - Every pointer is a DEVICE pointer owned by the caller; the library never
+ *     allocates or frees caller memory.  Buffers must not alias unless stated.
+ *   - Every pointer must be 16-byte aligned.
+ *   - Matrices are row-major; X is [rows, K] (K contiguous), W is [N, K]
+ *     (output channels x input channels, K contiguous), Y is [M, N].
+ *   - K and N must be multiples of 16; M, T >= 1.
+ *   - All work is enqueued on `stream` (0 = legacy default stream) and is
+ *     asynchronous; results are valid once the stream has been synchronised.
+ *   - Argument errors are detected on the host before anything is enqueued
+ *     and return SQ_ERR_INVALID_ARG (or SQ_ERR_UNSUPPORTED for sizes beyond a
+ *     stated limit); a failed launch returns SQ_ERR_CUDA.  No C++ exception
+ *     crosses this interface.
+ *   - Kernels that wait on on-chip barriers give up after about two seconds,
+ *     record an error word on the device and return; sq_device_status()
+ *     reports it as SQ_ERR_TIMEOUT.  No kernel traps.
+ */
+#ifndef SQ_H_
+#define SQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SQ_API __attribute__((visibility("default")))
+#else
+#define SQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *sq_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    SQ_OK = 0,
+    SQ_ERR_INVALID_ARG = 1,
+    SQ_ERR_UNSUPPORTED = 2,
+    SQ_ERR_CUDA = 3,
+    SQ_ERR_TIMEOUT = 4
+} sq_status;
+
+typedef enum {
+    SQ_F32 = 0, /* IEEE binary32 */
+    SQ_BF16 = 1 /* bfloat16, 16-bit pattern */
+} sq_dtype;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+SQ_API const char *sq_status_string(sq_status st);
+
+/* Library version as 10000*major + 100*minor + patch. */
+SQ_API int sq_version(void);
+
+/*
+ * Calibration statistics ("How the smoothing factor is computed": A_j is the
+ * largest activation magnitude seen in channel j over calibration samples).
+ *   x    [T, K] of dtype dt, row stride ldx elements (ldx >= K, and ldx times
+ *        the element size a multiple of 16 bytes).
+ *   ax   [K] fp32, ACCUMULATED: ax[j] = max(ax[j], max_t |x[t, j]|).  The
+ *        caller zero-fills ax before the first batch of a calibration run and
+ *        may then call this once per calibration batch.
+ * Errors: SQ_ERR_INVALID_ARG for NULL/misaligned pointers, T < 1, K < 16,
+ * K % 16 != 0, bad ldx or dt.
+ */
+SQ_API sq_status sq_calib_absmax(const void *x, sq_dtype dt, int64_t T, int64_t K, int64_t ldx,
+                          float *ax, sq_stream_t stream);
+
+/*
+ * Smoothing factors ("How the smoothing factor is computed"):
+ *   B_j = max_n |w[n, j]|,  s_j = A_j^alpha / B_j^(1-alpha) (fp64, rounded
+ *   once to fp32; s_j = 1 where A_j == 0 or B_j == 0).
+ *   ax   [K] fp32 calibration absmax (from sq_calib_absmax).
+ *   w    [N, K] of dtype dt (the unsmoothed weight).
+ *   alpha in [0, 1] (migration strength), finite.
+ *   s    [K] fp32 output.
+ *   aw   [K] fp32 output with B_j, or NULL.  s and aw must not alias ax.
+ * Errors: as above, plus alpha outside [0, 1].
+ */
+SQ_API sq_status sq_smooth_factors(const float *ax, const void *w, sq_dtype dt, int64_t N, int64_t K,
+                            float alpha, float *s, float *aw, sq_stream_t stream);
+
+/*
+ * Smoothed per-output-channel weight quantisation ("Where the outlier actually
+ * comes from": multiply the matching weight input channel by s; "Why Naive
+ * Weight Quantization Doesn't Work": scale = max|w'|/127, q = round(w'/scale)):
+ *   w'[n, k] = w[n, k] * s[k];  sw[n] = max_k |w'[n, k]| / 127;
+ *   wq[n, k] = clamp(round(w'[n, k] / sw[n]), -127, 127).
+ *   w [N, K] dtype dt; s [K] fp32; wq [N, K] int8 out; sw [N] fp32 out.
+ * K is at most 65536 (bf16) or 32768 (fp32); larger K is SQ_ERR_UNSUPPORTED.
+ */
+SQ_API sq_status sq_smooth_quant_weight(const void *w, sq_dtype dt, int64_t N, int64_t K,
+                                 const float *s, int8_t *wq, float *sw, sq_stream_t stream);
+
+/*
+ * Dynamic per-token activation quantisation ("Why Activation Quantization Is
+ * Hard": one scale per token over all channels, computed at run time), of the
+ * smoothed activation:
+ *   x^[m, k] = x[m, k] / s[k];  sx[m] = max_k |x^[m, k]| / 127;
+ *   xq[m, k] = clamp(round(x^[m, k] / sx[m]), -127, 127).
+ *   x [M, K] dtype dt; s [K] fp32; xq [M, K] int8 out; sx [M] fp32 out.
+ * K limits as for sq_smooth_quant_weight.
+ */
+SQ_API sq_status sq_quant_act(const void *x, sq_dtype dt, int64_t M, int64_t K, const float *s,
+                       int8_t *xq, float *sx, sq_stream_t stream);
+
+/*
+ * W8A8 GEMM with the dequantising epilogue ("quant_llm_int8": int32
+ * accumulation, outer product of row and column scales):
+ *   acc[m, n] = sum_k xq[m, k] * wq[n, k]   (exact int32; K * 127^2 < 2^31,
+ *                                            so K <= 133144)
+ *   y[m, n]   = ((float)acc[m, n] * sx[m]) * sw[n], stored as out_dt
+ *               (SQ_BF16: round-half-to-even of the fp32 value).
+ *   xq [M, K] int8, sx [M] fp32, wq [N, K] int8, sw [N] fp32, y [M, N].
+ * Runs on the 5th-generation tensor cores (tcgen05, int8 x int8 -> int32 in
+ * tensor memory); y must not alias any input.
+ */
+SQ_API sq_status sq_w8a8_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
+                       int64_t M, int64_t N, int64_t K, void *y, sq_dtype out_dt,
+                       sq_stream_t stream);
+
+/*
+ * The raw int32 accumulators acc[m, n] = sum_k xq[m, k] * wq[n, k] of the same
+ * tensor-core kernels (no scales), for verification.  acc is [M, N] int32.
+ */
+SQ_API sq_status sq_w8a8_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K,
+                           int32_t *acc, sq_stream_t stream);
+
+/*
+ * The online linear layer: sq_quant_act followed by sq_w8a8_gemm, i.e. the
+ * per-layer work that "Understanding W8A8 INT8 LLM Quantization", section
+ * "Inter-Token Latency (ITL)", charges to every generated token: find each
+ * token's range and scale, cast to int8, multiply in int8, dequantise.
+ *   x [M, K] dtype in_dt; s [K]; wq [N, K]; sw [N]; y [M, N] dtype out_dt.
+ *   workspace: device scratch of at least sq_linear_workspace_size(M, N, K)
+ *   bytes (may be NULL when that size is 0), 16-byte aligned, owned by the
+ *   caller and not read by the caller afterwards; calls that run concurrently
+ *   need separate workspaces.
+ * Small M (decode) quantises the activations inside the GEMM kernel and needs
+ * no workspace.
+ */
+SQ_API sq_status sq_linear(const void *x, sq_dtype in_dt, const float *s, const int8_t *wq,
+                    const float *sw, int64_t M, int64_t N, int64_t K, void *y, sq_dtype out_dt,
+                    void *workspace, size_t ws_bytes, sq_stream_t stream);
+
+/* Bytes of workspace sq_linear needs for these sizes (0 when none). */
+SQ_API size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * Device error word: synchronises `stream`, then reads and clears the error
+ * word the kernels set when a bounded on-chip wait gives up.  Returns SQ_OK,
+ * SQ_ERR_TIMEOUT (with the kernel's location code in *code when code is not
+ * NULL) or SQ_ERR_CUDA if the synchronisation itself failed.
+ */
+SQ_API sq_status sq_device_status(sq_stream_t stream, uint32_t *code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H_ */

@@ -1,0 +1,138 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load, export every function include/sq.h declares, and turn
+every malformed argument into SQ_ERR_INVALID_ARG / SQ_ERR_UNSUPPORTED on the
+host before anything is enqueued: none of these calls reaches the CUDA
+runtime, so they run on a machine without a GPU.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import w8a8_int8_gemm_channel_b200 as sq
+from w8a8_int8_gemm_channel_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sq.h")
+
+A = 0x7F0000001000  # a 16-byte aligned fake device address (never dereferenced)
+B = 0x7F0000002000
+C = 0x7F0000003000
+D = 0x7F0000004000
+E = 0x7F0000005000
+MIS = 0x7F0000001004  # misaligned
+INV, UNS = sq.SQ_ERR_INVALID_ARG, sq.SQ_ERR_UNSUPPORTED
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return sq.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^SQ_API\s+[\w\s\*]*?\b(sq_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert header_functions() == sorted(sq.ABI_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", sq.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = sorted({l.split()[-1] for l in out.splitlines() if l.split()[-1].startswith("sq_")})
+    assert exported == header_functions()
+
+
+def test_status_strings(lib):
+    names = [sq.status_string(i) for i in range(5)]
+    assert names == ["SQ_OK", "SQ_ERR_INVALID_ARG", "SQ_ERR_UNSUPPORTED", "SQ_ERR_CUDA",
+                     "SQ_ERR_TIMEOUT"]
+    assert sq.status_string(99) == "SQ_ERR_UNKNOWN"
+    assert lib.sq_version() >= 100
+
+
+def test_calib_absmax_rejects(lib):
+    f = lib.sq_calib_absmax
+    assert f(None, 1, 8, 64, 64, B, None) == INV           # null x
+    assert f(A, 1, 8, 64, 64, None, None) == INV           # null ax
+    assert f(A, 7, 8, 64, 64, B, None) == INV              # bad dtype
+    assert f(A, 1, 0, 64, 64, B, None) == INV              # T = 0
+    assert f(A, 1, 8, 40, 40, B, None) == INV              # K % 16
+    assert f(A, 1, 8, 64, 60, B, None) == INV              # ldx < K
+    assert f(A, 1, 8, 64, 68, B, None) == INV              # ldx * 2 bytes not a multiple of 16
+    assert f(MIS, 1, 8, 64, 64, B, None) == INV            # misaligned x
+    assert f(A, 0, 8, 64, 64, MIS, None) == INV            # misaligned ax
+
+
+def test_smooth_factors_rejects(lib):
+    f = lib.sq_smooth_factors
+    assert f(A, B, 1, 32, 64, 1.5, C, None, None) == INV   # alpha > 1
+    assert f(A, B, 1, 32, 64, -0.1, C, None, None) == INV  # alpha < 0
+    assert f(A, B, 1, 32, 64, float("nan"), C, None, None) == INV
+    assert f(A, B, 1, 32, 64, 0.5, A, None, None) == INV   # s aliases ax
+    assert f(A, B, 1, 32, 64, 0.5, C, C, None) == INV      # aw aliases s
+    assert f(A, B, 1, 32, 64, 0.5, C, MIS, None) == INV    # misaligned aw
+    assert f(A, B, 1, 0, 64, 0.5, C, None, None) == INV    # N = 0
+    assert f(A, B, 1, 32, 8, 0.5, C, None, None) == INV    # K < 16
+    assert f(None, B, 1, 32, 64, 0.5, C, None, None) == INV
+
+
+def test_quantisers_reject(lib):
+    for f in (lib.sq_smooth_quant_weight, lib.sq_quant_act):
+        assert f(None, 1, 4, 64, B, C, D, None) == INV
+        assert f(A, 1, 0, 64, B, C, D, None) == INV       # zero rows
+        assert f(A, 1, 4, 50, B, C, D, None) == INV       # K % 16
+        assert f(A, 1, 4, 64, B, MIS, D, None) == INV     # misaligned codes
+        assert f(A, 3, 4, 64, B, C, D, None) == INV       # bad dtype
+        assert f(A, 1, 4, 65536 + 16, B, C, D, None) == UNS   # bf16 row longer than supported
+        assert f(A, 0, 4, 32768 + 16, B, C, D, None) == UNS   # fp32 row longer than supported
+
+
+def test_quantisers_do_not_run_without_valid_args(lib):
+    # same calls but with one bad pointer so nothing is launched
+    assert lib.sq_quant_act(A, 1, 4, 64, None, C, D, None) == INV
+    assert lib.sq_smooth_quant_weight(A, 1, 4, 64, B, C, None, None) == INV
+
+
+def test_gemm_rejects(lib):
+    f = lib.sq_w8a8_gemm
+    assert f(A, B, C, D, 0, 64, 64, E, 1, None) == INV     # M = 0
+    assert f(A, B, C, D, 4, 40, 64, E, 1, None) == INV     # N % 16
+    assert f(A, B, C, D, 4, 64, 72, E, 1, None) == INV     # K % 16
+    assert f(A, B, C, D, 4, 64, 133152, E, 1, None) == UNS  # K * 127^2 would overflow int32
+    assert f(A, B, C, D, 4, 64, 64, MIS, 1, None) == INV   # misaligned y
+    assert f(A, None, C, D, 4, 64, 64, E, 1, None) == INV  # null sx
+    assert f(A, B, C, D, 4, 64, 64, E, 2, None) == INV     # bad out dtype
+    g = lib.sq_w8a8_gemm_s32
+    assert g(A, B, 4, 64, 64, None, None) == INV
+    assert g(A, B, -1, 64, 64, C, None) == INV
+    assert g(MIS, B, 4, 64, 64, C, None) == INV
+
+
+def test_linear_rejects_and_workspace_size(lib):
+    M, N, K = 100, 64, 256
+    need = sq.sq_linear_workspace_size(M, N, K)
+    assert need >= M * K + 4 * M and need % 16 == 0
+    f = lib.sq_linear
+    assert need > 0 and f(A, 1, B, C, D, M, N, K, E, 1, None, 0, None) == INV
+    assert f(A, 1, B, C, D, M, N, K, E, 1, A + 0x100000, need - 1, None) == INV
+    assert f(A, 1, B, C, D, M, N, K, E, 1, MIS, need, None) == INV
+    assert f(A, 1, B, C, D, 0, N, K, E, 1, A, need, None) == INV
+    assert f(A, 1, B, C, D, M, 24, K, E, 1, A, need, None) == INV
+    assert f(A, 5, B, C, D, M, N, K, E, 1, A, need, None) == INV
+    assert sq.sq_linear_workspace_size(0, 64, 64) == 0
+
+
+def test_binding_fails_loudly_without_device_tensors():
+    torch = pytest.importorskip("torch")
+    x = torch.zeros(4, 16)
+    with pytest.raises(ValueError):
+        sq.sq_calib_absmax(x, torch.zeros(16))

@@ -1,0 +1,259 @@
+"""GPU parity: every stage of the CUDA path against the CPU oracle on the same
+seeded bytes, through the C ABI (via the thin Python binding).
+
+Sizes span several tiles with ragged tails (M not a multiple of the 128-row
+tile, N not a multiple of the 256-column tile, K not a multiple of the 128-byte
+stage), the degenerate cases (one token, a zero token row, a zero input
+channel, a zero weight row, a large-magnitude row) and the smallest legal K.
+"""
+import numpy as np
+import pytest
+import torch
+
+import w8a8_int8_gemm_channel_b200 as sq
+from w8a8_int8_gemm_channel_b200 import workloads as wls
+from tests.gpu_util import (assert_bits_equal, assert_output_close, assert_smooth_factors,
+                            exact_fraction, to_dev, to_np)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from w8a8_int8_gemm_channel_b200 import _build
+
+    _build.build()
+    sq.lib()
+    yield
+    st, code = sq.sq_device_status()
+    assert st == sq.SQ_OK, f"device error word {code:#x}"
+
+
+def rand(shape, seed, dtype=torch.bfloat16, scale=1.0):
+    return wls.random_tensor(shape, seed, dtype=dtype, scale=scale)
+
+
+# ---------------------------------------------------------------------------
+# the small workload, stage by stage (fp32 in, fp32 out)
+# ---------------------------------------------------------------------------
+
+def test_small_workload_all_stages(oracle):
+    wl = wls.WORKLOADS["small"]
+    lin = wl.linears[0]
+    xcal = wls.calibration(wl, lin)
+    w = wls.weight(wl, lin)
+    x = wls.inputs(wl, lin, wl.Ms[0])
+    ax_o, aw_o, s_o, wq_o, sw_o = oracle.prepare(to_np(xcal), to_np(w), wl.alpha)
+
+    ax = sq.calibrate(xcal.cuda())
+    assert_bits_equal(to_np(ax), ax_o, "ax")
+    s = torch.empty(lin.K, device="cuda")
+    aw = torch.empty(lin.K, device="cuda")
+    sq.sq_smooth_factors(ax, w.cuda(), wl.alpha, s, aw)
+    assert_bits_equal(to_np(aw), aw_o, "aw")
+    assert_smooth_factors(to_np(s), s_o, ax_o, aw_o, wl.alpha)
+    # downstream stages get the oracle's s on both sides
+    s_np = s_o
+    s = to_dev(s_o)
+    wq = torch.empty(lin.N, lin.K, dtype=torch.int8, device="cuda")
+    sw = torch.empty(lin.N, device="cuda")
+    sq.sq_smooth_quant_weight(w.cuda(), s, wq, sw)
+    assert_bits_equal(to_np(wq), wq_o, "wq")
+    assert_bits_equal(to_np(sw), sw_o, "sw")
+
+    M = x.shape[0]
+    xq = torch.empty(M, lin.K, dtype=torch.int8, device="cuda")
+    sx = torch.empty(M, device="cuda")
+    sq.sq_quant_act(x.cuda(), s, xq, sx)
+    xq_o, sx_o = oracle.quant_act(to_np(x), s_np)
+    assert_bits_equal(to_np(xq), xq_o, "xq")
+    assert_bits_equal(to_np(sx), sx_o, "sx")
+
+    acc = torch.empty(M, lin.N, dtype=torch.int32, device="cuda")
+    sq.sq_w8a8_gemm_s32(xq, wq, acc)
+    acc_o = oracle.gemm_i32(xq_o, wq_o)
+    assert_bits_equal(to_np(acc), acc_o, "acc")
+
+    y = torch.empty(M, lin.N, device="cuda")
+    sq.sq_w8a8_gemm(xq, sx, wq, sw, y)
+    y_o = oracle.dequant(acc_o, sx_o, sw_o, "f32")
+    assert_output_close(to_np(y), y_o, "y")
+    assert exact_fraction(to_np(y), y_o) == 1.0
+
+    y2 = sq.linear(x.cuda(), s, wq, sw, out_dtype=torch.float32)
+    assert_bits_equal(to_np(y2), to_np(y), "sq_linear vs stages")
+
+
+# ---------------------------------------------------------------------------
+# calibration absmax
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,K,dtype", [(1, 16, torch.bfloat16), (7, 48, torch.float32),
+                                       (1000, 4112, torch.bfloat16), (333, 272, torch.float32),
+                                       (70000, 64, torch.bfloat16)])
+def test_calib_absmax(oracle, T, K, dtype):
+    x = rand((T, K), seed=T * 7 + K, dtype=dtype, scale=3.0)
+    if K > 20:
+        x[:, 5] = 0  # a zero channel
+    ax = torch.zeros(K, device="cuda")
+    sq.sq_calib_absmax(x.cuda(), ax)
+    torch.cuda.synchronize()
+    assert_bits_equal(to_np(ax), oracle.calib_absmax(to_np(x)), "ax")
+
+
+def test_calib_absmax_accumulates_over_batches(oracle):
+    x = rand((513, 256), seed=11, scale=5.0)
+    ax = sq.calibrate([x[:200].cuda(), x[200:].cuda()])
+    assert_bits_equal(to_np(ax), oracle.calib_absmax(to_np(x)), "ax over batches")
+
+
+def test_calib_absmax_row_stride(oracle):
+    """ldx > K: a column slice of a wider row-major buffer."""
+    T, K, ldx = 300, 128, 192
+    full = rand((T, ldx), seed=12, scale=2.0).cuda()
+    ax = torch.zeros(K, device="cuda")
+    st = sq.lib().sq_calib_absmax(full.data_ptr(), sq.SQ_BF16, T, K, ldx, ax.data_ptr(),
+                                  torch.cuda.current_stream().cuda_stream)
+    assert st == sq.SQ_OK
+    torch.cuda.synchronize()
+    assert_bits_equal(to_np(ax), oracle.calib_absmax(to_np(full[:, :K])), "ax strided")
+
+
+# ---------------------------------------------------------------------------
+# smoothing factors
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("alpha", [0.0, 0.5, 0.8, 0.85, 1.0])
+@pytest.mark.parametrize("N,K,dtype", [(16, 16, torch.float32), (300, 4112, torch.bfloat16)])
+def test_smooth_factors(oracle, alpha, N, K, dtype):
+    rng = np.random.default_rng(N + K)
+    ax_np = np.abs(rng.standard_normal(K)).astype(np.float32) * 10
+    ax_np[rng.integers(0, K, 3)] *= 60
+    ax_np[0] = 0.0  # dead calibration channel
+    w = rand((N, K), seed=N * K, dtype=dtype, scale=0.02)
+    if K > 3:
+        w[:, 2] = 0  # dead weight input channel
+    s = torch.empty(K, device="cuda")
+    aw = torch.empty(K, device="cuda")
+    sq.sq_smooth_factors(to_dev(ax_np), w.cuda(), alpha, s, aw)
+    aw_o = oracle.weight_in_absmax(to_np(w))
+    s_o = oracle.smooth_factors(ax_np, aw_o, alpha)
+    assert_bits_equal(to_np(aw), aw_o, "aw")
+    assert_smooth_factors(to_np(s), s_o, ax_np, aw_o, alpha)
+    assert float(to_np(s)[0]) == 1.0 and (K <= 3 or float(to_np(s)[2]) == 1.0)
+
+
+# ---------------------------------------------------------------------------
+# weight and activation quantisers
+# ---------------------------------------------------------------------------
+
+QUANT_SHAPES = [(1, 16, torch.float32), (3, 48, torch.bfloat16), (37, 4096, torch.bfloat16),
+                (130, 4112, torch.bfloat16), (5, 14336, torch.bfloat16), (2, 28672, torch.bfloat16),
+                (9, 8192, torch.float32), (4, 65536, torch.bfloat16), (2, 32768, torch.float32)]
+
+
+@pytest.mark.parametrize("R,K,dtype", QUANT_SHAPES)
+def test_quant_act(oracle, R, K, dtype):
+    x = rand((R, K), seed=R * 31 + K, dtype=dtype)
+    if R > 2:
+        x[1] = 0          # zero token row
+        x[2] *= 1000      # large-magnitude row
+    s_np = np.random.default_rng(K).uniform(0.25, 8.0, K).astype(np.float32)
+    s = to_dev(s_np)
+    xq = torch.empty(R, K, dtype=torch.int8, device="cuda")
+    sx = torch.empty(R, device="cuda")
+    sq.sq_quant_act(x.cuda(), s, xq, sx)
+    xq_o, sx_o = oracle.quant_act(to_np(x), s_np)
+    assert_bits_equal(to_np(sx), sx_o, "sx")
+    assert_bits_equal(to_np(xq), xq_o, "xq")
+
+
+@pytest.mark.parametrize("R,K,dtype", QUANT_SHAPES)
+def test_smooth_quant_weight(oracle, R, K, dtype):
+    w = rand((R, K), seed=R * 17 + K, dtype=dtype, scale=0.02)
+    if R > 2:
+        w[0] = 0
+    s_np = np.random.default_rng(K + 1).uniform(0.1, 30.0, K).astype(np.float32)
+    s = to_dev(s_np)
+    wq = torch.empty(R, K, dtype=torch.int8, device="cuda")
+    sw = torch.empty(R, device="cuda")
+    sq.sq_smooth_quant_weight(w.cuda(), s, wq, sw)
+    wq_o, sw_o = oracle.smooth_quant_weight(to_np(w), s_np)
+    assert_bits_equal(to_np(sw), sw_o, "sw")
+    assert_bits_equal(to_np(wq), wq_o, "wq")
+
+
+# ---------------------------------------------------------------------------
+# GEMM: int32 accumulators and the dequantised output
+# ---------------------------------------------------------------------------
+
+GEMM_SHAPES = [(1, 16, 16), (5, 32, 48), (16, 256, 256), (31, 272, 4112), (33, 128, 128),
+               (64, 64, 256), (100, 48, 1024), (128, 512, 4096), (129, 272, 4112),
+               (300, 528, 1040), (257, 784, 2064), (512, 1024, 512)]
+
+
+def _int8(shape, seed):
+    return wls.random_int8(shape, seed)
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_s32_exact(oracle, M, N, K):
+    xq = _int8((M, K), seed=M * 1000 + K)
+    wq = _int8((N, K), seed=N * 1000 + K + 1)
+    acc = torch.empty(M, N, dtype=torch.int32, device="cuda")
+    sq.sq_w8a8_gemm_s32(xq.cuda(), wq.cuda(), acc)
+    assert_bits_equal(to_np(acc), oracle.gemm_i32(to_np(xq), to_np(wq)), f"acc {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+@pytest.mark.parametrize("M,N,K", [(1, 16, 16), (31, 272, 4112), (129, 272, 4112), (300, 528, 1040)])
+def test_gemm_dequant(oracle, M, N, K, out):
+    xq = _int8((M, K), seed=M + 5 * K)
+    wq = _int8((N, K), seed=N + 7 * K)
+    rng = np.random.default_rng(M * N)
+    sx_np = rng.uniform(1e-3, 2.0, M).astype(np.float32)
+    sw_np = rng.uniform(1e-5, 1e-3, N).astype(np.float32)
+    if M > 1:
+        sx_np[0] = 0.0  # a zero token row
+    y = torch.empty(M, N, dtype=torch.bfloat16 if out == "bf16" else torch.float32, device="cuda")
+    sq.sq_w8a8_gemm(xq.cuda(), to_dev(sx_np), wq.cuda(), to_dev(sw_np), y)
+    acc_o = oracle.gemm_i32(to_np(xq), to_np(wq))
+    y_o = oracle.dequant(acc_o, sx_np, sw_np, out)
+    assert_output_close(to_np(y), y_o, f"y {out}")
+    assert exact_fraction(to_np(y), y_o) == 1.0
+
+
+def test_gemm_extreme_accumulators(oracle):
+    """All +127 against all -127 at K = 28672: |acc| = K * 127^2, the largest magnitude."""
+    M, N, K = 3, 32, 28672
+    xq = torch.full((M, K), 127, dtype=torch.int8)
+    wq = torch.full((N, K), -127, dtype=torch.int8)
+    wq[1::2] = 127
+    acc = torch.empty(M, N, dtype=torch.int32, device="cuda")
+    sq.sq_w8a8_gemm_s32(xq.cuda(), wq.cuda(), acc)
+    assert_bits_equal(to_np(acc), oracle.gemm_i32(to_np(xq), to_np(wq)), "acc extremes")
+    assert int(to_np(acc)[0, 0]) == -K * 127 * 127
+
+
+# ---------------------------------------------------------------------------
+# the online linear (sq_linear) against the oracle, bf16 in / bf16 out
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (8, 272, 4112), (32, 6144, 1024),
+                                   (77, 512, 2048), (256, 768, 4096)])
+def test_linear_bf16(oracle, M, N, K):
+    x = rand((M, K), seed=M + N + K)
+    x[:, 7] *= 60.0
+    w = rand((N, K), seed=N + K + 3, scale=0.02)
+    xcal = rand((512, K), seed=K + 9)
+    xcal[:, 7] *= 60.0
+    _, _, s_o, wq_o, sw_o = oracle.prepare(to_np(xcal), to_np(w), 0.5)
+    s = to_dev(s_o)
+    wq = to_dev(wq_o)
+    sw = to_dev(sw_o)
+    y = sq.linear(x.cuda(), s, wq, sw, out_dtype=torch.bfloat16)
+    y_o, _, _, _ = oracle.linear(to_np(x), s_o, wq_o, sw_o, "bf16")
+    assert_output_close(to_np(y), y_o, "linear")
+    assert exact_fraction(to_np(y), y_o) == 1.0

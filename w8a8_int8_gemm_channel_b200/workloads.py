@@ -194,10 +194,14 @@ def inputs(wl: Workload, lin: Linear, M: int, device="cpu", base_seed: int = 0):
     return activations(wl, lin, M, "x", device=device, base_seed=base_seed)
 
 
-def weight(wl: Workload, lin: Linear, device="cpu", base_seed: int = 0) -> torch.Tensor:
-    """Weight [N, K] (out x in), N(0, sigma)."""
-    g = _gen(device, seed_for(wl.name, f"w/{lin.name}", base_seed))
-    w = torch.randn(lin.N, lin.K, generator=g, device=device, dtype=torch.float32) * wl.w_sigma
+def weight(wl: Workload, lin: Linear, device="cpu", base_seed: int = 0,
+           rows: Optional[int] = None) -> torch.Tensor:
+    """Weight [N, K] (out x in), N(0, sigma); `rows` draws a smaller [rows, K]
+    sample with the same distribution (its own seed)."""
+    tag = f"w/{lin.name}" if rows is None else f"w/{lin.name}/rows{rows}"
+    g = _gen(device, seed_for(wl.name, tag, base_seed))
+    n = lin.N if rows is None else rows
+    w = torch.randn(n, lin.K, generator=g, device=device, dtype=torch.float32) * wl.w_sigma
     return w.to(_torch_dtype(wl.dtype))
 
 
