@@ -184,6 +184,35 @@ SQ_API sq_status sq_linear(const void *x, sq_dtype in_dt, const float *s, const 
 SQ_API size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
+ * sq_linear without any allocation, for callers that cannot allocate device
+ * memory: for example a plugin inside a host framework that owns every device
+ * allocation and hands the library only its input and output buffers, or a
+ * latency-critical serving loop in which a cudaMalloc (which can synchronise
+ * the whole device) is not allowed.  The pages have no counterpart to this
+ * entry point; it is a packaging of sq_linear.
+ *
+ * Same arguments, arithmetic and results as sq_linear, but the workspace is a
+ * fixed scratch array that lives in the library itself (a file-scope device
+ * array of SQ_LINEAR_NOALLOC_SCRATCH_BYTES bytes, held by every GPU that loads
+ * the library until the process exits).  The call makes no cudaMalloc or
+ * cudaFree and calls no allocating library routine.
+ *   - Sizes whose sq_linear_workspace_size(M, N, K) exceeds
+ *     SQ_LINEAR_NOALLOC_SCRATCH_BYTES are rejected with SQ_ERR_UNSUPPORTED
+ *     before anything is enqueued.
+ *   - The first call on a device (with that device current) looks up the
+ *     device address of the scratch array once; make that first call before
+ *     any stream capture on the device.
+ *   - All calls on a device share the one scratch array, which keeps the
+ *     previous call's contents (nothing in it needs to start at zero).  Calls
+ *     that can overlap on the GPU (different streams without ordering between
+ *     them) race on it: order them, or use sq_linear with separate workspaces.
+ */
+#define SQ_LINEAR_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+SQ_API sq_status sq_linear_noalloc(const void *x, sq_dtype in_dt, const float *s,
+                                   const int8_t *wq, const float *sw, int64_t M, int64_t N,
+                                   int64_t K, void *y, sq_dtype out_dt, sq_stream_t stream);
+
+/*
  * Device error word: synchronises `stream`, then reads and clears the error
  * word the kernels set when a bounded on-chip wait gives up.  Returns SQ_OK,
  * SQ_ERR_TIMEOUT (with the kernel's location code in *code when code is not

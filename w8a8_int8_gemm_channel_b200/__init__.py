@@ -17,6 +17,7 @@ The raw entry points keep the C names and take caller-allocated outputs:
     sq_w8a8_gemm_s32(xq, wq, acc)
     sq_linear(x, s, wq, sw, y, workspace)
     sq_linear_workspace_size(M, N, K)
+    sq_linear_noalloc(x, s, wq, sw, y)          no workspace, no allocation
     sq_device_status()
 
 ``calibrate``, ``prepare_weight`` and ``linear`` are conveniences that allocate
@@ -47,6 +48,7 @@ ABI_SYMBOLS = (
     "sq_w8a8_gemm_s32",
     "sq_linear",
     "sq_linear_workspace_size",
+    "sq_linear_noalloc",
     "sq_device_status",
 )
 
@@ -76,6 +78,7 @@ def _declare(lib):
         "sq_w8a8_gemm_s32": ([P, P, I, I, I, P, P], E),
         "sq_linear": ([P, E, P, P, P, I, I, I, P, E, P, ctypes.c_size_t, P], E),
         "sq_linear_workspace_size": ([I, I, I], ctypes.c_size_t),
+        "sq_linear_noalloc": ([P, E, P, P, P, I, I, I, P, E, P], E),
         "sq_device_status": ([P, ctypes.POINTER(ctypes.c_uint32)], E),
     }
     for name, (args, res) in sig.items():
@@ -199,6 +202,22 @@ def sq_linear(x, s, wq, sw, y, workspace=None, stream=None):
     _check("sq_linear",
            lib().sq_linear(_ptr(x), _dtype_code(x), _ptr(s), _ptr(wq), _ptr(sw), M, N, K, _ptr(y),
                            _dtype_code(y), ws_ptr, ws_bytes, _stream(stream)))
+
+
+# bytes of the library's fixed scratch array used by sq_linear_noalloc
+LINEAR_NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def sq_linear_noalloc(x, s, wq, sw, y, stream=None):
+    """sq_linear with the library's own fixed scratch array instead of a
+    caller workspace; allocates nothing.  Raises SQError(SQ_ERR_UNSUPPORTED)
+    when sq_linear_workspace_size(M, N, K) exceeds
+    LINEAR_NOALLOC_SCRATCH_BYTES."""
+    M, K = x.shape
+    N = wq.shape[0]
+    _check("sq_linear_noalloc",
+           lib().sq_linear_noalloc(_ptr(x), _dtype_code(x), _ptr(s), _ptr(wq), _ptr(sw), M, N, K,
+                                   _ptr(y), _dtype_code(y), _stream(stream)))
 
 
 def sq_device_status(stream=None) -> Tuple[int, int]:

@@ -234,6 +234,33 @@ sq_status check_gemm_dims(int64_t M, int64_t N, int64_t K)
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// ---- fixed scratch for sq_linear_noalloc -----------------------------------
+// The array belongs to this translation unit; in host code its name only
+// stands in for the symbol, so the device address is looked up once per
+// device with cudaGetSymbolAddress and handed to the kernels as a pointer.
+static __device__ __align__(256) uint8_t g_linear_noalloc_scratch[SQ_LINEAR_NOALLOC_SCRATCH_BYTES];
+
+// Device address of the scratch array on the current device (looked up on the
+// first call for that device), or nullptr if the lookup fails.
+void *noalloc_scratch()
+{
+    static void *addr[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_linear_noalloc_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -387,6 +414,29 @@ sq_status sq_linear(const void *x, sq_dtype in_dt, const float *s, const int8_t 
     if (r != SQ_OK)
         return r;
     return sq_w8a8_gemm(xq, sx, wq, sw, M, N, K, y, out_dt, stream);
+}
+
+sq_status sq_linear_noalloc(const void *x, sq_dtype in_dt, const float *s, const int8_t *wq,
+                            const float *sw, int64_t M, int64_t N, int64_t K, void *y,
+                            sq_dtype out_dt, sq_stream_t stream)
+{
+    if (x == nullptr || s == nullptr || wq == nullptr || sw == nullptr || y == nullptr ||
+        !valid_dtype(in_dt) || !valid_dtype(out_dt) || !aligned16(x) || !aligned16(s) ||
+        !aligned16(wq) || !aligned16(sw) || !aligned16(y))
+        return SQ_ERR_INVALID_ARG;
+    sq_status r = check_gemm_dims(M, N, K);
+    if (r != SQ_OK)
+        return r;
+    const size_t need = sq_linear_workspace_size(M, N, K);
+    if (need > SQ_LINEAR_NOALLOC_SCRATCH_BYTES)
+        return SQ_ERR_UNSUPPORTED;
+    void *ws = nullptr;
+    if (need > 0) {
+        ws = noalloc_scratch();
+        if (ws == nullptr)
+            return SQ_ERR_CUDA;
+    }
+    return sq_linear(x, in_dt, s, wq, sw, M, N, K, y, out_dt, ws, need, stream);
 }
 
 sq_status sq_device_status(sq_stream_t stream, uint32_t *code)
