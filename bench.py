@@ -435,6 +435,100 @@ def workload_config(wl):
 
 
 # ---------------------------------------------------------------------------
+# single-call cases (per-kernel timing and profiler captures)
+# ---------------------------------------------------------------------------
+
+def run_case(spec, steps, warmup, flush_l2=True):
+    """Time one C-ABI call on synthetic data.  spec is one of
+    gemm:M,N,K  linear:M,N,K  quant_act:M,K  quant_w:N,K  calib:T,K
+    smooth_factors:N,K.  Prints one JSON line with the median time."""
+    import w8a8_int8_gemm_channel_b200 as sq
+
+    lib = sq.lib()
+    kind, dims = spec.split(":")
+    d = [int(v) for v in dims.split(",")]
+    dev = torch.device("cuda", 0)
+    st = torch.cuda.current_stream().cuda_stream
+    peaks = load_peaks()
+    bf, i8, f32 = torch.bfloat16, torch.int8, torch.float32
+    r = lambda *shape, dt=bf, sc=1.0: (torch.randn(*shape, device=dev) * sc).to(dt)
+    ops, nbytes = 0, 0
+    if kind in ("gemm", "linear"):
+        M, N, K = d
+        wq = torch.randint(-127, 128, (N, K), device=dev, dtype=i8)
+        sw = torch.rand(N, device=dev) * 1e-3
+        y = torch.empty(M, N, device=dev, dtype=bf)
+        ops = 2 * M * N * K
+        if kind == "gemm":
+            xq = torch.randint(-127, 128, (M, K), device=dev, dtype=i8)
+            sx = torch.rand(M, device=dev)
+            fn = lambda: lib.sq_w8a8_gemm(xq.data_ptr(), sx.data_ptr(), wq.data_ptr(), sw.data_ptr(),
+                                          M, N, K, y.data_ptr(), sq.SQ_BF16, st)
+            nbytes = M * K + N * K + 4 * (M + N) + 2 * M * N
+        else:
+            x = r(M, K)
+            s = torch.rand(K, device=dev) + 0.5
+            ws_n = sq.sq_linear_workspace_size(M, N, K)
+            ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
+            fn = lambda: lib.sq_linear(x.data_ptr(), sq.SQ_BF16, s.data_ptr(), wq.data_ptr(),
+                                       sw.data_ptr(), M, N, K, y.data_ptr(), sq.SQ_BF16,
+                                       ws.data_ptr() if ws_n else None, ws_n, st)
+            nbytes = 2 * M * K + 4 * K + N * K + 4 * N + 2 * M * N
+    elif kind == "quant_act":
+        M, K = d
+        x, s = r(M, K), torch.rand(K, device=dev) + 0.5
+        xq, sx = torch.empty(M, K, dtype=i8, device=dev), torch.empty(M, device=dev)
+        fn = lambda: lib.sq_quant_act(x.data_ptr(), sq.SQ_BF16, M, K, s.data_ptr(), xq.data_ptr(),
+                                      sx.data_ptr(), st)
+        nbytes = 3 * M * K + 4 * K + 4 * M
+    elif kind == "quant_w":
+        N, K = d
+        w, s = r(N, K, sc=0.02), torch.rand(K, device=dev) + 0.5
+        wq, sw = torch.empty(N, K, dtype=i8, device=dev), torch.empty(N, device=dev)
+        fn = lambda: lib.sq_smooth_quant_weight(w.data_ptr(), sq.SQ_BF16, N, K, s.data_ptr(),
+                                                wq.data_ptr(), sw.data_ptr(), st)
+        nbytes = 3 * N * K + 4 * K + 4 * N
+    elif kind == "calib":
+        T, K = d
+        x, ax = r(T, K), torch.zeros(K, device=dev)
+        fn = lambda: lib.sq_calib_absmax(x.data_ptr(), sq.SQ_BF16, T, K, K, ax.data_ptr(), st)
+        nbytes = 2 * T * K
+    elif kind == "smooth_factors":
+        N, K = d
+        w, ax, s = r(N, K, sc=0.02), torch.rand(K, device=dev) * 10, torch.empty(K, device=dev)
+        fn = lambda: lib.sq_smooth_factors(ax.data_ptr(), w.data_ptr(), sq.SQ_BF16, N, K, 0.5,
+                                           s.data_ptr(), None, st)
+        nbytes = 2 * N * K + 8 * K
+    else:
+        raise SystemExit(f"unknown case {spec}")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush_l2 else None
+    for _ in range(warmup):
+        assert fn() == 0
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        if flush is not None:
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        rc = fn()
+        e1.record()
+        assert rc == 0, sq.status_string(rc)
+        times.append((e0, e1))
+    torch.cuda.synchronize()
+    us = statistics.median(a.elapsed_time(b) for a, b in times) * 1e3
+    out = {"case": spec, "us": round(us, 2), "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1),
+           "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3), "l2_flushed": flush_l2}
+    if ops:
+        out["TOPS"] = round(ops / (us * 1e-6) / 1e12, 1)
+        out["tensor_frac_burst"] = round(out["TOPS"] / (INT8_PER_BF16 * peaks["bf16_tflops"]), 3)
+    stc, code = sq.sq_device_status()
+    assert stc == 0, f"device error {code:#x}"
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
 # main arm
 # ---------------------------------------------------------------------------
 
@@ -449,7 +543,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--breakdown-steps", type=int, default=20)
+    ap.add_argument("--case", action="append", default=None,
+                    help="time single calls instead of the step, e.g. gemm:4096,6144,4096")
+    ap.add_argument("--no-flush", action="store_true")
     args = ap.parse_args()
+    if args.case:
+        for c in args.case:
+            run_case(c, args.steps, max(args.warmup, 3), flush_l2=not args.no_flush)
+        return 0
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

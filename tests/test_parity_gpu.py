@@ -257,3 +257,80 @@ def test_linear_bf16(oracle, M, N, K):
     y_o, _, _, _ = oracle.linear(to_np(x), s_o, wq_o, sw_o, "bf16")
     assert_output_close(to_np(y), y_o, "linear")
     assert exact_fraction(to_np(y), y_o) == 1.0
+
+
+# ---------------------------------------------------------------------------
+# numerics of the quantisers' fast paths: ties, near-ties, tiny and huge
+# magnitudes, divisors outside the fast range, zero chunks
+# ---------------------------------------------------------------------------
+
+def _edge_rows(K, seed):
+    rng = np.random.default_rng(seed)
+    rows = []
+    # exact ties and 1-ulp neighbours: amax 127 gives scale 1 when s == 1
+    t = np.array([127.0] + [k + 0.5 for k in range(-60, 60)] * 4, np.float32)[:K]
+    rows.append(t)
+    rows.append(np.nextafter(t, np.float32(np.inf)))
+    rows.append(np.nextafter(t, np.float32(-np.inf)))
+    # tiny, subnormal-adjacent and huge rows (scale outside the fast range)
+    rows.append((rng.standard_normal(K) * 1e-33).astype(np.float32))
+    rows.append((rng.standard_normal(K) * 1e-40).astype(np.float32))
+    rows.append((rng.standard_normal(K) * 1e30).astype(np.float32))
+    # a zero row and a row with zero chunks
+    rows.append(np.zeros(K, np.float32))
+    z = rng.standard_normal(K).astype(np.float32)
+    z[: K // 2] = 0.0
+    rows.append(z)
+    # near-ties for a generic scale: values placed at (k + 1/2) * scale * s_k
+    return np.stack(rows).astype(np.float32)
+
+
+@pytest.mark.parametrize("s_kind", ["ones", "random", "extreme"])
+def test_quant_act_fast_path_edges(oracle, s_kind):
+    K = 256
+    x = _edge_rows(K, 5)
+    rng = np.random.default_rng(6)
+    if s_kind == "ones":
+        s_np = np.ones(K, np.float32)
+    elif s_kind == "random":
+        s_np = rng.uniform(0.05, 20.0, K).astype(np.float32)
+    else:  # divisors outside [2^-60, 2^61): exercises the IEEE fallback
+        s_np = rng.uniform(0.5, 2.0, K).astype(np.float32)
+        s_np[3] = 1e-25
+        s_np[9] = 1e25
+        # keep every smoothed value x/s finite (an overflowing quotient is outside the contract)
+        x[np.abs(x[:, 3]) > 1e10, 3] = 1.0
+    # a generic-scale near-tie row: amax fixed by one element, others at half-integers
+    sc = np.float32(0.0123)
+    nt = (np.arange(K) % 200 - 100 + 0.5).astype(np.float32) * sc * s_np
+    nt[0] = np.float32(127.0) * sc * s_np[0]
+    x = np.vstack([x, nt.astype(np.float32)])
+    xq = torch.empty(x.shape, dtype=torch.int8, device="cuda")
+    sx = torch.empty(x.shape[0], device="cuda")
+    sq.sq_quant_act(to_dev(x), to_dev(s_np), xq, sx)
+    xq_o, sx_o = oracle.quant_act(x, s_np)
+    assert_bits_equal(to_np(sx), sx_o, "sx")
+    assert_bits_equal(to_np(xq), xq_o, "xq")
+    # the fused decode path (all rows fit one call) on the same inputs
+    wq = wls.random_int8((64, K), seed=7)
+    sw = np.full(64, 1e-3, np.float32)
+    y = torch.empty(x.shape[0], 64, dtype=torch.float32, device="cuda")
+    sq.sq_linear(to_dev(x), to_dev(s_np), wq.cuda(), to_dev(sw), y)
+    acc_o = oracle.gemm_i32(xq_o, to_np(wq))
+    assert_output_close(to_np(y), oracle.dequant(acc_o, sx_o, sw, "f32"), "fused linear")
+
+
+@pytest.mark.parametrize("s_kind", ["ones", "random", "extreme"])
+def test_smooth_quant_weight_fast_path_edges(oracle, s_kind):
+    K = 256
+    w = _edge_rows(K, 8)
+    rng = np.random.default_rng(9)
+    s_np = {"ones": np.ones(K, np.float32),
+            "random": rng.uniform(0.05, 20.0, K).astype(np.float32),
+            "extreme": np.where(np.arange(K) % 17 == 0, 1e-20, 1.0).astype(np.float32)}[s_kind]
+    wq = torch.empty(w.shape, dtype=torch.int8, device="cuda")
+    sw = torch.empty(w.shape[0], device="cuda")
+    sq.sq_smooth_quant_weight(to_dev(w), to_dev(s_np), wq, sw)
+    wq_o, sw_o = oracle.smooth_quant_weight(w, s_np)
+    assert_bits_equal(to_np(sw), sw_o, "sw")
+    assert_bits_equal(to_np(wq), wq_o, "wq")

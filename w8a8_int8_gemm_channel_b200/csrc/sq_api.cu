@@ -9,12 +9,18 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <cstdio>
+#include <cstdlib>
 #include <mutex>
+#include <tuple>
+#include <vector>
+#include <climits>
 
 #include "sq.h"
 #include "sq_gemm.cuh"
 #include "sq_mem.cuh"
 #include "sq_ptx.cuh"
+#include "sq_splitk.cuh"
 
 namespace {
 
@@ -23,6 +29,7 @@ using sq::OUT_F32;
 using sq::OUT_S32;
 
 constexpr int kMaxDevices = 64;
+constexpr int kMaxDynSmem = 232448;  // 227 KB of dynamic shared memory per CTA on sm_100
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -62,6 +69,13 @@ bool device_info(DeviceInfo &info)
     }
     info = cache[dev];
     return true;
+}
+
+// Launch plans are printed to stderr when SQ_DEBUG_PLAN is set (diagnostics).
+bool debug_plan()
+{
+    static const bool on = std::getenv("SQ_DEBUG_PLAN") != nullptr;
+    return on;
 }
 
 // ---- tensor maps -----------------------------------------------------------
@@ -125,58 +139,69 @@ sq_status launch_col_absmax(const T *x, int64_t R, int64_t K, int64_t ld, float 
     if (!device_info(di))
         return SQ_ERR_CUDA;
     constexpr int V = sq::Vec<T>::N;
+    constexpr int CL = sq::kColClusterRows;
     const int64_t chunks = K / V;
-    const int threads = static_cast<int>(std::min<int64_t>(256, ((chunks + 31) / 32) * 32));
-    const int64_t col_blocks = (chunks + threads - 1) / threads;
-    // about 8 CTAs of 256 threads per SM in total
-    const int64_t want = std::max<int64_t>(1, (int64_t)di.sms * 8 * 256 / threads / col_blocks);
-    int64_t rows_per_block = std::max<int64_t>(4, (R + want - 1) / want);
+    const int64_t col_blocks = (chunks + sq::kColThreads - 1) / sq::kColThreads;
+    // about 8 CTAs of 256 threads per SM in total, in clusters of CL row bands
+    const int64_t want = std::max<int64_t>(CL, (int64_t)di.sms * 8 / col_blocks);
+    int64_t rows_per_block = std::max<int64_t>(32, (R + want - 1) / want);
     int64_t row_blocks = (R + rows_per_block - 1) / rows_per_block;
-    if (row_blocks > 65535) {
-        row_blocks = 65535;
-        rows_per_block = (R + row_blocks - 1) / row_blocks;
+    while (row_blocks > 65528) {
+        rows_per_block *= 2;
         row_blocks = (R + rows_per_block - 1) / rows_per_block;
     }
-    dim3 grid(static_cast<unsigned>(col_blocks), static_cast<unsigned>(row_blocks));
-    sq::col_absmax_kernel<T><<<grid, threads, 0, st>>>(
-        x, R, K, ld, rows_per_block, reinterpret_cast<unsigned int *>(out));
+    row_blocks = (row_blocks + CL - 1) / CL * CL;  // whole clusters; surplus bands are empty
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(col_blocks), static_cast<unsigned>(row_blocks));
+    cfg.blockDim = dim3(sq::kColThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = CL;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, sq::col_absmax_kernel<T>, x, R, K, ld, rows_per_block,
+                           reinterpret_cast<unsigned int *>(out)) != cudaSuccess) {
+        cudaGetLastError();
+        return SQ_ERR_CUDA;
+    }
     return launch_status();
 }
 
 // ---- row quantisers ----------------------------------------------------------
+template <typename T, int MODE, int SEG, bool SMEM_S>
+sq_status launch_quant_rows_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
+                                float *scale, cudaStream_t st, const DeviceInfo &di)
+{
+    auto kernel = sq::quant_rows_kernel<T, MODE, SEG, SMEM_S>;
+    const int smem = SMEM_S ? static_cast<int>(K * sizeof(float)) : 0;
+    static std::atomic<uint64_t> attr_done{0};
+    if (SMEM_S && !ensure_smem_attr(kernel, kMaxDynSmem, attr_done))
+        return SQ_ERR_CUDA;
+    const int warps = sq::kQuantThreads / 32;
+    const int per_sm = smem <= 64 * 1024 ? 3 : 2;
+    const int64_t blocks = std::min<int64_t>((rows + warps - 1) / warps, per_sm * (int64_t)di.sms);
+    kernel<<<static_cast<unsigned>(blocks), sq::kQuantThreads, smem, st>>>(in, rows, K, s, q, scale);
+    return launch_status();
+}
+
+constexpr int64_t kSmemFactorBytes = 112 * 1024;
+
 template <typename T, int MODE>
 sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
                             float *scale, cudaStream_t st)
 {
-    constexpr int V = sq::Vec<T>::N;
-    const int64_t chunks = K / V;
-    int cpt = 1;
-    while (cpt < 8 && (chunks + cpt - 1) / cpt > 1024)
-        cpt *= 2;
-    if ((chunks + cpt - 1) / cpt > 1024)
-        return SQ_ERR_UNSUPPORTED;
-    // prefer >= 128 threads per row block when the row is long enough
-    while (cpt > 1 && (chunks + cpt - 1) / cpt < 128)
-        cpt /= 2;
-    const int threads = static_cast<int>(std::max<int64_t>(32, (((chunks + cpt - 1) / cpt + 31) / 32) * 32));
+    DeviceInfo di;
+    if (!device_info(di))
+        return SQ_ERR_CUDA;
     if (rows > 2147483647LL)
         return SQ_ERR_UNSUPPORTED;
-    dim3 grid(static_cast<unsigned>(rows));
-    switch (cpt) {
-    case 1:
-        sq::quant_rows_kernel<T, 1, MODE><<<grid, threads, 0, st>>>(in, K, s, q, scale);
-        break;
-    case 2:
-        sq::quant_rows_kernel<T, 2, MODE><<<grid, threads, 0, st>>>(in, K, s, q, scale);
-        break;
-    case 4:
-        sq::quant_rows_kernel<T, 4, MODE><<<grid, threads, 0, st>>>(in, K, s, q, scale);
-        break;
-    default:
-        sq::quant_rows_kernel<T, 8, MODE><<<grid, threads, 0, st>>>(in, K, s, q, scale);
-        break;
-    }
-    return launch_status();
+    if (K * (int64_t)sizeof(float) <= kSmemFactorBytes)
+        return launch_quant_rows_cfg<T, MODE, 16, true>(in, rows, K, s, q, scale, st, di);
+    return launch_quant_rows_cfg<T, MODE, 16, false>(in, rows, K, s, q, scale, st, di);
 }
 
 int64_t max_quant_k(sq_dtype dt) { return dt == SQ_BF16 ? 65536 : 32768; }
@@ -208,17 +233,167 @@ sq_status launch_gemm_cfg(const int8_t *xq, const float *sx, const int8_t *wq, c
     return launch_status();
 }
 
+// ---- split-K small-M GEMM (optionally with the activation quant fused in) --
+constexpr int64_t kFusedSliceBytes = 128 * 1024;  // resident token operand per CTA
+
+struct SplitPlan {
+    int splits = 1, kbps = 1, stages = 2, smem = 0;
+    bool ok = false;
+};
+
+// Clusters of `splits` CTAs with `smem` bytes each that the device can hold at
+// once (cudaOccupancyMaxActiveClusters), cached per kernel and shape.
+template <typename KernelT>
+int active_clusters(KernelT kernel, int splits, int smem)
+{
+    static std::mutex mu;
+    static std::vector<std::tuple<int, int, int, int>> cache;  // dev, splits, smem -> clusters
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (auto &e : cache)
+            if (std::get<0>(e) == dev && std::get<1>(e) == splits && std::get<2>(e) == smem)
+                return std::get<3>(e);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(splits * 64));
+    cfg.blockDim = dim3(sq::kSplitThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    std::lock_guard<std::mutex> lk(mu);
+    cache.emplace_back(dev, splits, smem, n);
+    return n;
+}
+
+template <int BNX, bool FUSED, typename KernelT>
+SplitPlan plan_splitk(KernelT kernel, int64_t N, int64_t K)
+{
+    SplitPlan best;
+    const int64_t n_tiles = (N + sq::kBM - 1) / sq::kBM;
+    const int64_t k_blocks = (K + sq::kBK - 1) / sq::kBK;
+    int64_t best_cost = INT64_MAX;
+    // tuning overrides (same work, different decomposition): SQ_SPLITK_SPLITS, SQ_SPLITK_STAGES
+    static const int force_splits = std::getenv("SQ_SPLITK_SPLITS") ? std::atoi(std::getenv("SQ_SPLITK_SPLITS")) : 0;
+    static const int force_stages = std::getenv("SQ_SPLITK_STAGES") ? std::atoi(std::getenv("SQ_SPLITK_STAGES")) : 0;
+    for (int64_t want = 1; want <= std::min<int64_t>(sq::kMaxSplits, k_blocks); ++want) {
+        if (force_splits > 0 && want != force_splits)
+            continue;
+        const int64_t kbps = (k_blocks + want - 1) / want;
+        const int64_t sp = (k_blocks + kbps - 1) / kbps;
+        if (sp != want)
+            continue;
+        if (FUSED && (int64_t)BNX * sq::kBK * kbps > kFusedSliceBytes)
+            continue;
+        int stages = force_stages > 1 ? force_stages : 8;
+        while (stages > 2 &&
+               sq::split_layout<BNX>(stages, FUSED, (int)kbps).total + 1024 > (uint32_t)kMaxDynSmem)
+            --stages;
+        const int smem = (int)sq::split_layout<BNX>(stages, FUSED, (int)kbps).total + 1024;
+        if (smem > kMaxDynSmem)
+            continue;
+        const int active = active_clusters(kernel, (int)sp, smem);
+        if (active <= 0)
+            continue;
+        const int64_t waves = (n_tiles + active - 1) / active;
+        const int64_t cost = waves * (kbps + 4);  // +4: fixed per-CTA cost in k-block units
+        if (cost < best_cost) {
+            best_cost = cost;
+            best.splits = (int)sp;
+            best.kbps = (int)kbps;
+            best.stages = stages;
+            best.smem = smem;
+            best.ok = true;
+        }
+    }
+    return best;
+}
+
+template <int BNX, int OUT, bool FUSED, typename TIN>
+sq_status launch_splitk_cfg(const TIN *x, const float *s, const int8_t *xq, const float *sx,
+                            const int8_t *wq, const float *sw, int64_t M, int64_t N, int64_t K,
+                            void *y, cudaStream_t st)
+{
+    auto kernel = sq::gemm_splitk_kernel<BNX, OUT, FUSED, TIN>;
+    static std::atomic<uint64_t> attr_done{0};
+    if (!ensure_smem_attr(kernel, kMaxDynSmem, attr_done))
+        return SQ_ERR_CUDA;
+    const SplitPlan p = plan_splitk<BNX, FUSED>(kernel, N, K);
+    if (!p.ok)
+        return SQ_ERR_UNSUPPORTED;
+    if (debug_plan())
+        std::fprintf(stderr, "[sq] splitk BNX=%d fused=%d M=%lld N=%lld K=%lld: splits=%d kb/split=%d stages=%d smem=%d clusters=%lld active=%d\n",
+                     BNX, (int)FUSED, (long long)M, (long long)N, (long long)K, p.splits, p.kbps, p.stages, p.smem,
+                     (long long)((N + sq::kBM - 1) / sq::kBM), active_clusters(kernel, p.splits, p.smem));
+    CUtensorMap tw, tx;
+    if (!make_tmap_i8(&tw, wq, N, K, sq::kBM))
+        return SQ_ERR_CUDA;
+    if (FUSED)
+        tx = tw;  // unused by the fused kernel
+    else if (!make_tmap_i8(&tx, xq, M, K, BNX))
+        return SQ_ERR_CUDA;
+    const int64_t n_tiles = (N + sq::kBM - 1) / sq::kBM;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(n_tiles * p.splits));
+    cfg.blockDim = dim3(sq::kSplitThreads);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, tw, tx, x, s, sx, sw, y, static_cast<int>(M),
+                           static_cast<int>(N), static_cast<int>(K), p.splits, p.kbps,
+                           p.stages) != cudaSuccess) {
+        cudaGetLastError();
+        return SQ_ERR_CUDA;
+    }
+    return launch_status();
+}
+
 template <int OUT>
 sq_status launch_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
                       int64_t M, int64_t N, int64_t K, void *y, cudaStream_t st)
 {
+    const float *nf = nullptr;
     if (M <= 32)
-        return launch_gemm_cfg<32, 8, OUT, true>(xq, sx, wq, sw, M, N, K, y, st);
+        return launch_splitk_cfg<32, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
     if (M <= 64)
-        return launch_gemm_cfg<64, 8, OUT, true>(xq, sx, wq, sw, M, N, K, y, st);
+        return launch_splitk_cfg<64, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
     if (M <= 128)
-        return launch_gemm_cfg<128, 6, OUT, true>(xq, sx, wq, sw, M, N, K, y, st);
+        return launch_splitk_cfg<128, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
     return launch_gemm_cfg<256, 4, OUT, false>(xq, sx, wq, sw, M, N, K, y, st);
+}
+
+// The fused decode path (activation quant inside the GEMM, no workspace)
+// applies to at most 32 tokens when K fits the per-CTA token operand.
+bool fused_decode_applies(int64_t M, int64_t K)
+{
+    return M <= 32 && K <= sq::kMaxSplits * (kFusedSliceBytes / (32 * sq::kBK)) * sq::kBK;
+}
+
+template <typename TIN>
+sq_status launch_fused_linear(const TIN *x, const float *s, const int8_t *wq, const float *sw,
+                              int64_t M, int64_t N, int64_t K, void *y, sq_dtype out_dt,
+                              cudaStream_t st)
+{
+    if (out_dt == SQ_BF16)
+        return launch_splitk_cfg<32, OUT_BF16, true, TIN>(x, s, nullptr, nullptr, wq, sw, M, N, K, y, st);
+    return launch_splitk_cfg<32, OUT_F32, true, TIN>(x, s, nullptr, nullptr, wq, sw, M, N, K, y, st);
 }
 
 constexpr int64_t kMaxDim = 2147483647LL;
@@ -385,7 +560,7 @@ sq_status sq_w8a8_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_
 size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K)
 {
     (void)N;
-    if (M < 1 || K < 1)
+    if (M < 1 || K < 1 || fused_decode_applies(M, K))
         return 0;
     return align_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256) +
            align_up(static_cast<size_t>(M) * sizeof(float), 256);
@@ -404,6 +579,13 @@ sq_status sq_linear(const void *x, sq_dtype in_dt, const float *s, const int8_t 
         return r;
     if (K > max_quant_k(in_dt))
         return SQ_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (fused_decode_applies(M, K)) {
+        if (in_dt == SQ_BF16)
+            return launch_fused_linear(static_cast<const __nv_bfloat16 *>(x), s, wq, sw, M, N, K, y,
+                                       out_dt, st);
+        return launch_fused_linear(static_cast<const float *>(x), s, wq, sw, M, N, K, y, out_dt, st);
+    }
     const size_t need = sq_linear_workspace_size(M, N, K);
     if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned16(workspace)))
         return SQ_ERR_INVALID_ARG;

@@ -20,6 +20,7 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include "sq_div.cuh"
 #include "sq_ptx.cuh"
 
 namespace sq {
@@ -98,60 +99,159 @@ __device__ __forceinline__ void load_vec_stream<float>(const float *p, float (&v
     v[3] = u.w;
 }
 
-// clamp(round_half_even(v / scale), -127, 127) as a byte; scale > 0.
-__device__ __forceinline__ uint32_t quant_code(float v, float scale)
+template <typename T>
+__device__ __forceinline__ uint4 ld_chunk(const T *p)
 {
-    int q = __float2int_rn(__fdiv_rn(v, scale));
-    q = max(-127, min(127, q));
-    return static_cast<uint32_t>(q) & 0xFFu;
+    return __ldcs(reinterpret_cast<const uint4 *>(p));
+}
+
+template <typename T>
+__device__ __forceinline__ void widen(const uint4 &u, float (&v)[Vec<T>::N]);
+
+template <>
+__device__ __forceinline__ void widen<__nv_bfloat16>(const uint4 &u, float (&v)[8])
+{
+    v[0] = __uint_as_float(u.x << 16);
+    v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(u.y << 16);
+    v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    v[4] = __uint_as_float(u.z << 16);
+    v[5] = __uint_as_float(u.z & 0xFFFF0000u);
+    v[6] = __uint_as_float(u.w << 16);
+    v[7] = __uint_as_float(u.w & 0xFFFF0000u);
+}
+
+template <>
+__device__ __forceinline__ void widen<float>(const uint4 &u, float (&v)[4])
+{
+    v[0] = __uint_as_float(u.x);
+    v[1] = __uint_as_float(u.y);
+    v[2] = __uint_as_float(u.z);
+    v[3] = __uint_as_float(u.w);
 }
 
 // ----------------------------------------------------------------------------
 // Column absmax: out[j] = max(out[j], max_r |x[r, j]|), out as fp32 bit
 // patterns (non-negative floats order like their unsigned bit patterns).
 // Block: 256 threads = 256 consecutive 16-byte column chunks; blockIdx.y
-// selects a band of `rows_per_block` rows.  Coalesced 16-byte loads, one
-// atomicMax per channel per CTA.
+// selects a band of `rows_per_block` rows.  The CTAs of a cluster (consecutive
+// bands, kColClusterRows of them) combine their partial maxima through
+// distributed shared memory, and the cluster's first CTA issues one atomicMax
+// per channel, so the global atomics are 1/kColClusterRows of one per CTA.
 // ----------------------------------------------------------------------------
+constexpr int kColThreads = 256;
+constexpr int kColClusterRows = 8;
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+// address of the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_shared_rank(uint32_t local, uint32_t rank)
+{
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+    return remote;
+}
+
+__device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
 template <typename T>
-__global__ void __launch_bounds__(256) col_absmax_kernel(const T *__restrict__ x, int64_t R,
-                                                          int64_t K, int64_t ld,
-                                                          int64_t rows_per_block,
-                                                          unsigned int *__restrict__ out_bits)
+__global__ void __launch_bounds__(kColThreads) col_absmax_kernel(const T *__restrict__ x, int64_t R,
+                                                                  int64_t K, int64_t ld,
+                                                                  int64_t rows_per_block,
+                                                                  unsigned int *__restrict__ out_bits)
 {
     constexpr int V = Vec<T>::N;
+    constexpr int SLOTS = kColThreads / kColClusterRows;  // chunk columns each CTA combines
+    __shared__ __align__(16) float part[kColThreads * V];
     const int64_t chunks = K / V;
     const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (c >= chunks)
-        return;
-    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_block;
-    const int64_t r1 = min(R, r0 + rows_per_block);
     float m[V];
 #pragma unroll
     for (int i = 0; i < V; ++i)
         m[i] = 0.0f;
-    const T *p = x + r0 * ld + c * V;
-    int64_t r = r0;
-    for (; r + 4 <= r1; r += 4, p += 4 * ld) {
-        float a[V], b[V], d[V], e[V];
-        load_vec_stream<T>(p, a);
-        load_vec_stream<T>(p + ld, b);
-        load_vec_stream<T>(p + 2 * ld, d);
-        load_vec_stream<T>(p + 3 * ld, e);
+    if (c < chunks) {
+        const int64_t r0 = min(R, static_cast<int64_t>(blockIdx.y) * rows_per_block);
+        const int64_t r1 = min(R, r0 + rows_per_block);
+        const T *p = x + r0 * ld + c * V;
+        int64_t r = r0;
+        for (; r + 8 <= r1; r += 8, p += 8 * ld) {
+            uint4 raw[8];  // eight rows in flight per thread
 #pragma unroll
-        for (int i = 0; i < V; ++i)
-            m[i] = fmaxf(m[i], fmaxf(fmaxf(fabsf(a[i]), fabsf(b[i])), fmaxf(fabsf(d[i]), fabsf(e[i]))));
+            for (int u = 0; u < 8; ++u)
+                raw[u] = __ldcs(reinterpret_cast<const uint4 *>(p + u * ld));
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                float a[V];
+                widen<T>(raw[u], a);
+#pragma unroll
+                for (int i = 0; i < V; ++i)
+                    m[i] = fmaxf(m[i], fabsf(a[i]));
+            }
+        }
+        for (; r < r1; ++r, p += ld) {
+            float a[V];
+            load_vec_stream<T>(p, a);
+#pragma unroll
+            for (int i = 0; i < V; ++i)
+                m[i] = fmaxf(m[i], fabsf(a[i]));
+        }
     }
-    for (; r < r1; ++r, p += ld) {
-        float a[V];
-        load_vec_stream<T>(p, a);
 #pragma unroll
-        for (int i = 0; i < V; ++i)
-            m[i] = fmaxf(m[i], fabsf(a[i]));
+    for (int i = 0; i < V; i += 4)
+        *reinterpret_cast<float4 *>(part + threadIdx.x * V + i) = make_float4(m[i], m[i + 1], m[i + 2], m[i + 3]);
+    __syncwarp();
+    cluster_sync_all();  // every CTA's partial maxima are visible cluster-wide
+    // CTA `rank` combines chunk slots [rank*SLOTS, rank*SLOTS + SLOTS) across the cluster
+    if (threadIdx.x < SLOTS) {
+        const int slot = static_cast<int>(cluster_ctarank()) * SLOTS + threadIdx.x;
+        const int64_t cc = static_cast<int64_t>(blockIdx.x) * blockDim.x + slot;
+        if (cc < chunks) {
+            const uint32_t local = smem_u32(part + slot * V);
+            float t[kColClusterRows][V];
+#pragma unroll
+            for (int rk = 0; rk < kColClusterRows; ++rk) {
+                const uint32_t remote = map_shared_rank(local, rk);
+#pragma unroll
+                for (int i = 0; i < V; i += 4) {
+                    const float4 q = ld_shared_cluster_f4(remote + 4u * i);
+                    t[rk][i] = q.x;
+                    t[rk][i + 1] = q.y;
+                    t[rk][i + 2] = q.z;
+                    t[rk][i + 3] = q.w;
+                }
+            }
+            float mm[V];
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                mm[i] = t[0][i];
+#pragma unroll
+                for (int rk = 1; rk < kColClusterRows; ++rk)
+                    mm[i] = fmaxf(mm[i], t[rk][i]);
+                atomicMax(out_bits + cc * V + i, __float_as_uint(mm[i]));
+            }
+        }
     }
-#pragma unroll
-    for (int i = 0; i < V; ++i)
-        atomicMax(out_bits + c * V + i, __float_as_uint(m[i]));
+    __syncwarp();
+    cluster_sync_all();  // no CTA leaves while its shared memory may still be read
 }
 
 // ----------------------------------------------------------------------------
@@ -221,65 +321,94 @@ __device__ __forceinline__ void store_codes<4>(int8_t *dst, const uint32_t (&q)[
 }
 
 // ----------------------------------------------------------------------------
-// Row quantiser shared by the weight and the activation paths.  One CTA per
-// row; each thread keeps CPT 16-byte chunks of the row in registers so the
-// row is read from memory once.
-//   MODE_W:  v = w * s   (smoothed weight, "multiply the weight input channel")
-//   MODE_X:  v = x / s   (smoothed activation, "divide the activation by s")
-//   scale = max|v| / 127;  code = clamp(rint(v / scale)).
+// Row quantiser shared by the weight and the activation paths: one warp per
+// row, persistent over rows.
+//   MODE_W:  v = w * s   (smoothed weight: the weight input channel times s)
+//   MODE_X:  v = x / s   (smoothed activation: the activation divided by s)
+//   scale = max_k |v| / 127;  code = clamp(round_half_even(v / scale), -127, 127)
+// Each lane reads 16-byte chunks c = lane + 32 i of the row, SEG chunks at a
+// time (a short, fixed instruction footprint).  The row is read twice: the
+// second (code) pass hits L1/L2, so HBM sees it once.  With SMEM_S the factors
+// s (and for MODE_X their reciprocals) are staged in shared memory once per CTA.
 // ----------------------------------------------------------------------------
 enum RowMode { MODE_W = 0, MODE_X = 1 };
 
-template <typename T, int CPT, int MODE>
-__global__ void __launch_bounds__(1024) quant_rows_kernel(const T *__restrict__ in, int64_t K,
-                                                           const float *__restrict__ s,
-                                                           int8_t *__restrict__ q,
-                                                           float *__restrict__ scale_out)
+__device__ __forceinline__ float warp_max(float v)
 {
-    constexpr int V = Vec<T>::N;
-    __shared__ float red[32];
-    const int64_t row = blockIdx.x;
-    const int64_t chunks = K / V;
-    const T *src = in + row * K;
-    float v[CPT][V];
-    float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < CPT; ++i) {
-        const int64_t c = threadIdx.x + static_cast<int64_t>(i) * blockDim.x;
-        if (c < chunks) {
-            float x[V];
-            load_vec_stream<T>(src + c * V, x);
-            const float4 *sp = reinterpret_cast<const float4 *>(s + c * V);
-#pragma unroll
-            for (int h = 0; h < V / 4; ++h) {
-                const float4 s4 = __ldg(sp + h);
-                const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float t = (MODE == MODE_W) ? __fmul_rn(x[h * 4 + e], sv[e])
-                                                     : __fdiv_rn(x[h * 4 + e], sv[e]);
-                    v[i][h * 4 + e] = t;
-                    amax = fmaxf(amax, fabsf(t));
-                }
-            }
-        }
+    for (int o = 16; o > 0; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+constexpr int kQuantThreads = 256;
+
+// Chunks of up to 8 values passed by value to the out-of-line slow paths.
+struct Chunk8 {
+    float v[8];
+};
+
+// Exact maximum of |x / s| over the elements of one chunk whose approximate
+// magnitude a = RN(|x| * RN(1/s)) reaches `thr` (rare: the row's top element).
+__device__ __noinline__ float chunk_max_exact(Chunk8 x, Chunk8 a, const float *__restrict__ s_chunk,
+                                              int n, float thr)
+{
+    float em = 0.0f;
+    for (int e = 0; e < n; ++e)
+        if (a.v[e] >= thr)
+            em = fmaxf(em, fabsf(__fdiv_rn(x.v[e], __ldg(s_chunk + e))));
+    return em;
+}
+
+// Exact codes of one chunk (rare: near ties, scales outside the fast range).
+// MODE_W: v = x * s; MODE_X: v = x / s.
+__device__ __noinline__ Chunk8 chunk_codes_exact(Chunk8 x, const float *__restrict__ s_chunk, int n,
+                                                 int mode_x, float scale)
+{
+    Chunk8 y;
+    for (int e = 0; e < n; ++e) {
+        const float sv = __ldg(s_chunk + e);
+        const float v = mode_x ? __fdiv_rn(x.v[e], sv) : __fmul_rn(x.v[e], sv);
+        y.v[e] = __uint_as_float(scale != 0.0f ? exact_code_bits(v, scale) : code_bits(0.0f));
     }
-    amax = block_max(amax, red);
-    const float scale = __fdiv_rn(amax, 127.0f);
-    if (threadIdx.x == 0)
-        scale_out[row] = scale;
-    int8_t *dst = q + row * K;
+    return y;
+}
+
+// Exact max of |x / s| over one chunk (rows whose divisors leave the fast range).
+__device__ __noinline__ float chunk_absmax_div(Chunk8 x, const float *__restrict__ s_chunk, int n)
+{
+    float m = 0.0f;
+    for (int e = 0; e < n; ++e)
+        m = fmaxf(m, fabsf(__fdiv_rn(x.v[e], __ldg(s_chunk + e))));
+    return m;
+}
+
+// Approximate magnitudes a = RN(|x| * r) of one chunk and their maximum.
+template <int V>
+__device__ __forceinline__ float chunk_approx(const float (&x)[V], const float (&r)[V], Chunk8 &a)
+{
+    float hi = 0.0f;
 #pragma unroll
-    for (int i = 0; i < CPT; ++i) {
-        const int64_t c = threadIdx.x + static_cast<int64_t>(i) * blockDim.x;
-        if (c < chunks) {
-            uint32_t code[V];
-#pragma unroll
-            for (int e = 0; e < V; ++e)
-                code[e] = (amax != 0.0f) ? quant_code(v[i][e], scale) : 0u;
-            store_codes<V>(dst + c * V, code);
-        }
+    for (int e = 0; e < V; ++e) {
+        a.v[e] = fabsf(__fmul_rn(x[e], r[e]));
+        hi = fmaxf(hi, a.v[e]);
     }
+    return hi;
+}
+
+// Exact-maximum contribution of one chunk given the row's candidate threshold.
+template <int V>
+__device__ __forceinline__ float chunk_candidates(const float (&x)[V], const float (&r)[V],
+                                                  const float *__restrict__ s_chunk, float thr)
+{
+    Chunk8 a, xv;
+    const float hi = chunk_approx<V>(x, r, a);
+    if (hi < thr)
+        return 0.0f;
+#pragma unroll
+    for (int e = 0; e < V; ++e)
+        xv.v[e] = x[e];
+    return chunk_max_exact(xv, a, s_chunk, V, thr);
 }
 
 }  // namespace sq
