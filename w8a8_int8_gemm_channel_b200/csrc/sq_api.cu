@@ -172,23 +172,24 @@ sq_status launch_col_absmax(const T *x, int64_t R, int64_t K, int64_t ld, float 
 }
 
 // ---- row quantisers ----------------------------------------------------------
-template <typename T, int MODE, int SEG, bool SMEM_S>
-sq_status launch_quant_rows_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
-                                float *scale, cudaStream_t st, const DeviceInfo &di)
+constexpr int64_t kSmemFactorBytes = 112 * 1024;  // per-column factors staged in shared memory
+
+// Two launches: row scales (one warp per row), then the codes (elementwise).
+template <typename T, int MODE, bool SMEM_S>
+sq_status launch_row_scale(const T *in, int64_t rows, int64_t K, const float *s, float *scale,
+                           cudaStream_t st, const DeviceInfo &di)
 {
-    auto kernel = sq::quant_rows_kernel<T, MODE, SEG, SMEM_S>;
+    auto kernel = sq::row_scale_kernel<T, MODE, 16, SMEM_S>;
     const int smem = SMEM_S ? static_cast<int>(K * sizeof(float)) : 0;
     static std::atomic<uint64_t> attr_done{0};
     if (SMEM_S && !ensure_smem_attr(kernel, kMaxDynSmem, attr_done))
         return SQ_ERR_CUDA;
+    const int per_sm = smem <= 96 * 1024 ? 2 : 1;
     const int warps = sq::kQuantThreads / 32;
-    const int per_sm = smem <= 64 * 1024 ? 3 : 2;
-    const int64_t blocks = std::min<int64_t>((rows + warps - 1) / warps, per_sm * (int64_t)di.sms);
-    kernel<<<static_cast<unsigned>(blocks), sq::kQuantThreads, smem, st>>>(in, rows, K, s, q, scale);
+    const int64_t blocks = std::min<int64_t>((rows + warps - 1) / warps, (int64_t)per_sm * di.sms);
+    kernel<<<static_cast<unsigned>(blocks), sq::kQuantThreads, smem, st>>>(in, rows, K, s, scale);
     return launch_status();
 }
-
-constexpr int64_t kSmemFactorBytes = 112 * 1024;
 
 template <typename T, int MODE>
 sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
@@ -199,9 +200,25 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
         return SQ_ERR_CUDA;
     if (rows > 2147483647LL)
         return SQ_ERR_UNSUPPORTED;
-    if (K * (int64_t)sizeof(float) <= kSmemFactorBytes)
-        return launch_quant_rows_cfg<T, MODE, 16, true>(in, rows, K, s, q, scale, st, di);
-    return launch_quant_rows_cfg<T, MODE, 16, false>(in, rows, K, s, q, scale, st, di);
+    sq_status r = (K * (int64_t)sizeof(float) <= kSmemFactorBytes)
+                      ? launch_row_scale<T, MODE, true>(in, rows, K, s, scale, st, di)
+                      : launch_row_scale<T, MODE, false>(in, rows, K, s, scale, st, di);
+    if (r != SQ_OK)
+        return r;
+    constexpr int V = sq::Vec<T>::N;
+    const int64_t chunks = K / V;
+    const int threads = static_cast<int>(std::min<int64_t>(256, (chunks + 31) / 32 * 32));
+    const int64_t col_blocks = (chunks + threads - 1) / threads;
+    const int64_t want = std::max<int64_t>(1, (int64_t)di.sms * 8 * 256 / threads / col_blocks);
+    int64_t rpb = std::max<int64_t>(4, (rows + want - 1) / want);
+    int64_t row_blocks = (rows + rpb - 1) / rpb;
+    while (row_blocks > 65535) {
+        rpb *= 2;
+        row_blocks = (rows + rpb - 1) / rpb;
+    }
+    dim3 grid(static_cast<unsigned>(col_blocks), static_cast<unsigned>(row_blocks));
+    sq::row_codes_kernel<T, MODE><<<grid, threads, 0, st>>>(in, rows, K, s, scale, rpb, q);
+    return launch_status();
 }
 
 int64_t max_quant_k(sq_dtype dt) { return dt == SQ_BF16 ? 65536 : 32768; }

@@ -45,45 +45,48 @@ __device__ __forceinline__ float warp_slice_absmax(const T *__restrict__ src, in
 {
     constexpr int V = Vec<T>::N;
     const bool single = nch <= 32 * SEG;
-    if (MODE == MODE_X && single && !bad_divisor) {
-        // one load; per-chunk approximate maxima stay in registers, so the
-        // exact pass only revisits the chunk(s) near the row maximum
-        warp_load_slice<T, SEG>(src, nch, 0, lane, raw);
-        float hi[SEG];
+    constexpr int HI = 16;  // chunks per lane covered by the kept maxima (slices up to 32*HI chunks)
+    if (MODE == MODE_X && nch <= 32 * HI && !bad_divisor) {
+        // the slice is read once; approximate maxima of chunk pairs stay in
+        // registers and the exact pass only revisits the pairs near the row maximum
+        float hi[HI / 2];
         float amax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < SEG; ++i) {
-            const int c = min(lane + 32 * i, nch - 1);
-            float x[V], f[V];
-            Chunk8 a;
-            widen<T>(raw[i], x);
-            factor(c, f);
-            hi[i] = chunk_approx<V>(x, f, a);
-            amax = fmaxf(amax, hi[i]);
+        for (int g = 0; g < HI / SEG; ++g) {
+            warp_load_slice<T, SEG>(src, nch, g * 32 * SEG, lane, raw);
+#pragma unroll
+            for (int i = 0; i < SEG; ++i) {
+                const int j = g * SEG + i;
+                const int c = min(g * 32 * SEG + lane + 32 * i, nch - 1);
+                float x[V], f[V];
+                Chunk8 a;
+                widen<T>(raw[i], x);
+                factor(c, f);
+                const float h = chunk_approx<V>(x, f, a);
+                hi[j / 2] = (j & 1) ? fmaxf(hi[j / 2], h) : h;
+                amax = fmaxf(amax, h);
+            }
         }
         const float A = warp_max(amax);
         const float thr = __fmul_rn(A, kCandidateScale);
         const bool exact_all = A < kTinyQuotient;
         float emax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < SEG; ++i) {
-            if (exact_all || hi[i] >= thr) {
-                const int c = min(lane + 32 * i, nch - 1);
+        for (int j = 0; j < HI; ++j) {
+            const int cj = (j / SEG) * 32 * SEG + lane + 32 * (j % SEG);
+            if ((exact_all || hi[j / 2] >= thr) && cj < nch) {
                 float x[V], f[V];
                 // re-read the chunk (L1) so the row need not stay in registers
-                const uint4 u = (lane + 32 * i < nch)
-                                    ? __ldg(reinterpret_cast<const uint4 *>(src + static_cast<int64_t>(c) * V))
-                                    : make_uint4(0u, 0u, 0u, 0u);
-                widen<T>(u, x);
+                widen<T>(__ldg(reinterpret_cast<const uint4 *>(src + static_cast<int64_t>(cj) * V)), x);
                 if (!exact_all) {
-                    factor(c, f);
-                    emax = fmaxf(emax, chunk_candidates<V>(x, f, sptr(c), thr));
+                    factor(cj, f);
+                    emax = fmaxf(emax, chunk_candidates<V>(x, f, sptr(cj), thr));
                 } else {
                     Chunk8 xv;
 #pragma unroll
                     for (int e = 0; e < V; ++e)
                         xv.v[e] = x[e];
-                    emax = fmaxf(emax, chunk_absmax_div(xv, sptr(c), V));
+                    emax = fmaxf(emax, chunk_absmax_div(xv, sptr(cj), V));
                 }
             }
         }
@@ -150,7 +153,7 @@ __device__ __forceinline__ void warp_slice_codes(const T *__restrict__ src, int 
 {
     uint4 raw[SEG];
     constexpr int V = Vec<T>::N;
-    const float rsc = __frcp_rn(scale);
+    const float rsc = rcp_approx(scale);
     const bool fast = scale_in_fast_range(scale) && !bad_divisor;
 #pragma unroll 1
     for (int base = 0; base < nch; base += 32 * SEG) {
@@ -165,12 +168,16 @@ __device__ __forceinline__ void warp_slice_codes(const T *__restrict__ src, int 
             bool tie = !fast;
             if (fast) {
                 factor(cc, f);
+                // y = RN(a * rsc + 1.5*2^23) rounds the product a*rsc half-even to an
+                // integer in one step (the code is y's low byte); d = a*rsc - that
+                // integer decides whether the fast result is safe (|d| < 0.5 - 2^-13)
                 float dmax = 0.0f;
 #pragma unroll
                 for (int e = 0; e < V; ++e) {
-                    const float t = __fmul_rn(__fmul_rn(x[e], f[e]), rsc);
-                    const float yy = __fadd_rn(t, kRoundMagic);
-                    dmax = fmaxf(dmax, fabsf(__fsub_rn(t, __fsub_rn(yy, kRoundMagic))));
+                    const float a = __fmul_rn(x[e], f[e]);
+                    const float yy = __fmaf_rn(a, rsc, kRoundMagic);
+                    const float r = __fsub_rn(yy, kRoundMagic);
+                    dmax = fmaxf(dmax, fabsf(__fmaf_rn(a, rsc, -r)));
                     y[e] = __float_as_uint(yy);
                 }
                 tie = !(dmax < kTieLimit);  // NaN (scale too small) also takes the exact path
@@ -196,42 +203,67 @@ __device__ __forceinline__ void warp_slice_codes(const T *__restrict__ src, int 
     }
 }
 
+// Stage n factors from s into dst (RN(1/s) when RECIP, else s itself; nothing
+// stored unless STORE), threads t, t+nt, ... of a group, four float4 loads in
+// flight per thread per round.  Returns non-zero when some reciprocal is
+// unusable by the fast division (its divisor lies outside [2^-60, 2^61)).
+template <bool RECIP, bool STORE>
+__device__ __forceinline__ int stage_factors(const float *__restrict__ s, int n, float *dst, int t, int nt)
+{
+    int bad = 0;
+    const int nv = n >> 2;  // n is a multiple of 16
+    const float4 *s4 = reinterpret_cast<const float4 *>(s);
+    for (int j0 = t; j0 < nv; j0 += 4 * nt) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + u * nt;
+            v[u] = j < nv ? __ldg(s4 + j) : make_float4(1.f, 1.f, 1.f, 1.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + u * nt;
+            if (j < nv) {
+                float4 r = v[u];
+                if (RECIP) {
+                    r = make_float4(fast_recip(v[u].x), fast_recip(v[u].y), fast_recip(v[u].z), fast_recip(v[u].w));
+                    bad |= (r.x == 0.0f) | (r.y == 0.0f) | (r.z == 0.0f) | (r.w == 0.0f);
+                }
+                if (STORE)
+                    reinterpret_cast<float4 *>(dst)[j] = r;
+            }
+        }
+    }
+    return bad;
+}
+
 // ----------------------------------------------------------------------------
-// Standalone quantiser: one warp per row, persistent over rows.  With SMEM_S
-// the per-column factors (MODE_X: RN(1/s); MODE_W: s) are staged in shared
-// memory once per CTA.
+// Standalone quantiser, two kernels:
+//   row_scale_kernel  one warp per row (persistent): the exact row maximum and
+//                     scale = RN(max/127), read-only, no CTA barriers;
+//   row_codes_kernel  elementwise given the row scales: each thread owns one
+//                     16-byte column chunk (its factors live in registers) and
+//                     walks a band of rows with several rows in flight.
+// The codes kernel re-reads the rows; for activations (and weights) that fit
+// the 126 MB L2 that second read is served from L2.
 // ----------------------------------------------------------------------------
 template <typename T, int MODE, int SEG, bool SMEM_S>
 __global__ void __launch_bounds__(kQuantThreads, 2)
-    quant_rows_kernel(const T *__restrict__ in, int64_t rows, int64_t K,
-                      const float *__restrict__ s, int8_t *__restrict__ q,
-                      float *__restrict__ scale_out)
+    row_scale_kernel(const T *__restrict__ in, int64_t rows, int64_t K, const float *__restrict__ s,
+                     float *__restrict__ scale_out)
 {
     constexpr int V = Vec<T>::N;
     extern __shared__ float4 smem_f4[];
     float *f_sm = reinterpret_cast<float *>(smem_f4);
     int bad_divisor = 0;
-    if constexpr (SMEM_S) {
-        for (int64_t j = threadIdx.x; j < K; j += blockDim.x) {
-            const float sv = __ldg(s + j);
-            if constexpr (MODE == MODE_X) {
-                const float rv = div_recip(sv);
-                bad_divisor |= (rv == 0.0f);
-                f_sm[j] = rv;
-            } else {
-                f_sm[j] = sv;
-            }
-        }
-        bad_divisor = __syncthreads_or(bad_divisor);
-    } else if constexpr (MODE == MODE_X) {
-        for (int64_t j = threadIdx.x; j < K; j += blockDim.x)
-            bad_divisor |= (div_recip(__ldg(s + j)) == 0.0f);
+    if constexpr (SMEM_S || MODE == MODE_X) {
+        bad_divisor = stage_factors<MODE == MODE_X, SMEM_S>(s, static_cast<int>(K), f_sm, threadIdx.x,
+                                                            blockDim.x);
         bad_divisor = __syncthreads_or(bad_divisor);
     }
     const int lane = threadIdx.x & 31;
     const int warps = blockDim.x >> 5;
     const int nch = static_cast<int>(K / V);
-
     auto factor = [&](int c, float (&f)[V]) {
 #pragma unroll
         for (int h = 0; h < V / 4; ++h) {
@@ -241,7 +273,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
             } else {
                 v4 = __ldg(reinterpret_cast<const float4 *>(s + static_cast<int64_t>(c) * V) + h);
                 if constexpr (MODE == MODE_X)
-                    v4 = make_float4(div_recip(v4.x), div_recip(v4.y), div_recip(v4.z), div_recip(v4.w));
+                    v4 = make_float4(fast_recip(v4.x), fast_recip(v4.y), fast_recip(v4.z), fast_recip(v4.w));
             }
             f[4 * h] = v4.x;
             f[4 * h + 1] = v4.y;
@@ -250,23 +282,89 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
         }
     };
     auto sptr = [&](int c) { return s + static_cast<int64_t>(c) * V; };
-
     for (int64_t row = static_cast<int64_t>(blockIdx.x) * warps + (threadIdx.x >> 5); row < rows;
          row += static_cast<int64_t>(gridDim.x) * warps) {
-        const T *src = in + row * K;
         uint4 raw[SEG];
-        const float E = warp_slice_absmax<T, MODE, SEG>(src, nch, lane, bad_divisor != 0, factor, sptr, raw);
-        const float scale = __fdiv_rn(E, 127.0f);
+        const float E = warp_slice_absmax<T, MODE, SEG>(in + row * K, nch, lane, bad_divisor != 0, factor,
+                                                        sptr, raw);
         if (lane == 0)
-            scale_out[row] = scale;
-        int8_t *dst = q + row * K;
-        auto store = [&](int c, uint2 u) {
-            if constexpr (V == 8)
-                *reinterpret_cast<uint2 *>(dst + static_cast<int64_t>(c) * 8) = u;
-            else
-                *reinterpret_cast<uint32_t *>(dst + static_cast<int64_t>(c) * 4) = u.x;
-        };
-        warp_slice_codes<T, MODE, 4>(src, nch, lane, bad_divisor != 0, scale, factor, sptr, store);
+            scale_out[row] = scale_from_max(E);
+    }
+}
+
+template <typename T, int MODE>
+__global__ void __launch_bounds__(256) row_codes_kernel(const T *__restrict__ in, int64_t rows, int64_t K,
+                                                        const float *__restrict__ s,
+                                                        const float *__restrict__ scale,
+                                                        int64_t rows_per_block, int8_t *__restrict__ q)
+{
+    constexpr int V = Vec<T>::N;
+    constexpr int U = 4;  // rows in flight per thread
+    const int64_t nch = K / V;
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (c >= nch)
+        return;
+    // this thread's factors: MODE_X -> 1/s (1 ulp), MODE_W -> s
+    float f[V];
+    bool bad = false;
+#pragma unroll
+    for (int h = 0; h < V; h += 4) {
+        const float4 v4 = __ldg(reinterpret_cast<const float4 *>(s + c * V + h));
+        const float sv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            f[h + e] = (MODE == MODE_X) ? fast_recip(sv[e]) : sv[e];
+            bad |= (MODE == MODE_X) && f[h + e] == 0.0f;
+        }
+    }
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_block;
+    const int64_t r1 = min(rows, r0 + rows_per_block);
+    for (int64_t r = r0; r < r1; r += U) {
+        uint4 raw[U];
+        float sc[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const bool ok = r + u < r1;
+            raw[u] = ok ? __ldg(reinterpret_cast<const uint4 *>(in + (r + u) * K + c * V)) : make_uint4(0u, 0u, 0u, 0u);
+            sc[u] = ok ? __ldg(scale + r + u) : 1.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const bool live = r + u < r1;
+            float x[V];
+            widen<T>(raw[u], x);
+            const float rsc = rcp_approx(sc[u]);
+            bool tie = bad || !scale_in_fast_range(sc[u]);
+            uint32_t y[V];
+            float dmax = 0.0f;
+#pragma unroll
+            for (int e = 0; e < V; ++e) {
+                const float a = __fmul_rn(x[e], f[e]);
+                const float yy = __fmaf_rn(a, rsc, kRoundMagic);
+                const float rr = __fsub_rn(yy, kRoundMagic);
+                dmax = fmaxf(dmax, fabsf(__fmaf_rn(a, rsc, -rr)));
+                y[e] = __float_as_uint(yy);
+            }
+            tie |= !(dmax < kTieLimit);
+            if (tie && live) {
+                Chunk8 xv;
+#pragma unroll
+                for (int e = 0; e < V; ++e)
+                    xv.v[e] = x[e];
+                const Chunk8 yy = chunk_codes_exact(xv, s + c * V, V, MODE == MODE_X, sc[u]);
+#pragma unroll
+                for (int e = 0; e < V; ++e)
+                    y[e] = __float_as_uint(yy.v[e]);
+            }
+            if (live) {
+                int8_t *dst = q + (r + u) * K + c * V;
+                if constexpr (V == 8)
+                    *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_code_bytes(y[0], y[1], y[2], y[3]),
+                                                                 pack_code_bytes(y[4], y[5], y[6], y[7]));
+                else
+                    *reinterpret_cast<uint32_t *>(dst) = pack_code_bytes(y[0], y[1], y[2], y[3]);
+            }
+        }
     }
 }
 

@@ -294,12 +294,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             const int nch = static_cast<int>((k1 - k0) / V);
             float *rsl = reinterpret_cast<float *>(g + L.rsl);
             volatile int *bad_flag = reinterpret_cast<volatile int *>(g + L.misc + 8);
-            int bad = 0;
-            for (int j = wi; j < static_cast<int>(k1 - k0); j += kSplitWorkers) {
-                const float rv = div_recip(__ldg(s + k0 + j));
-                rsl[j] = rv;
-                bad |= (rv == 0.0f);
-            }
+            const int bad = stage_factors<true, true>(s + k0, static_cast<int>(k1 - k0), rsl, wi, kSplitWorkers);
             if (bad)
                 *bad_flag = 1;
             named_bar_sync(1, kSplitWorkers);
@@ -318,8 +313,8 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             // (a) exact partial absmax of x/s per token over the slice
 #pragma unroll 1
             for (int m = ww; m < M; m += kSplitWorkers / 32) {
-                uint4 raw[16];
-                const float E = warp_slice_absmax<TIN, MODE_X, 16>(x + static_cast<int64_t>(m) * K + k0, nch,
+                uint4 raw[8];
+                const float E = warp_slice_absmax<TIN, MODE_X, 8>(x + static_cast<int64_t>(m) * K + k0, nch,
                                                                    lane, bad_divisor, factor, sptr, raw);
                 if (lane == 0)
                     wpmax[m] = E;
@@ -342,7 +337,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                 float a = 0.0f;
                 for (int r = 0; r < splits; ++r)
                     a = fmaxf(a, pmax[r * BNX + wi]);
-                sxs[wi] = __fdiv_rn(a, 127.0f);
+                sxs[wi] = scale_from_max(a);
             }
             named_bar_sync(1, kSplitWorkers);
             // (d) codes of the slice into the swizzled K-major B operand
