@@ -207,10 +207,15 @@ class Step:
         return sum(y.numel() * y.element_size() for d in self.lins for y in d["y"].values())
 
     def launches_per_step(self):
-        n = 1  # calibration absmax
-        n += 3 * len(self.lins)  # weight in-channel absmax + factors, weight quantiser
+        """Kernels of this library one step launches: the calibration absmax
+        (1); per linear the weight's input-channel absmax and the factors (2)
+        and the weight quantiser's scale and code kernels (2); per token count
+        and linear either the fused linear (1) or the activation quantiser's
+        two kernels and the GEMM (3)."""
+        n = 1
+        n += 4 * len(self.lins)
         for M in self.wl.Ms:
-            n += len(self.lins) * (1 if self.fused(M) else 2)
+            n += len(self.lins) * (1 if self.fused(M) else 3)
         return n
 
     def fused(self, M):
@@ -374,7 +379,7 @@ def cpu_baseline(wl, target_s=12.0):
     samp.step()  # warm (builds/loads the oracle)
     spent_total, est_total, ops = 0.0, 0.0, 0
     n = 0
-    while spent_total < target_s and n < 200:
+    while spent_total < target_s and n < 5000:
         spent, est, ops = samp.step()
         spent_total += spent
         est_total += est
@@ -529,6 +534,26 @@ def run_case(spec, steps, warmup, flush_l2=True):
 
 
 # ---------------------------------------------------------------------------
+# replicas: one process per GPU, each running the whole step on its own data
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(ms, world, device):
+    """The slowest rank's device time; every rank calls this at the same point."""
+    if world == 1:
+        return ms
+    import torch.distributed as dist
+
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tops(world, ops_per_step, steps, ms):
+    """Whole-job throughput: every replica's ops over the slowest rank's time."""
+    return world * ops_per_step * steps / (ms * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------
 # main arm
 # ---------------------------------------------------------------------------
 
@@ -565,7 +590,7 @@ def main():
 
     if world > 1:
         torch.cuda.set_device(local_rank)
-        dist.init_process_group(backend="nccl", timeout=datetime.timedelta(seconds=300))
+        dist.init_process_group(backend="nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", local_rank if world > 1 else 0)
     torch.cuda.set_device(device)
     wl = wls.WORKLOADS[args.workload]
@@ -605,18 +630,14 @@ def main():
     torch.cuda.synchronize()
     clocks = sampler.stop(visible_gpu_index(local_rank)) if sampler else None
     barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world, device)
     st, code = step.sq.sq_device_status(stream)
     if st != 0:
         raise RuntimeError(f"device error word {code:#x} after the timed region")
 
     ms_per_step = elapsed_ms / args.steps
     ops_step = step.gemm_ops()
-    value = world * ops_step * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = aggregate_tops(world, ops_step, args.steps, elapsed_ms)
 
     # roofline of the dominant kernel: the prefill tcgen05 GEMM (M >= 1024)
     g_ops = 0
@@ -702,12 +723,8 @@ def main():
                 e2e_step()
             e1.record(stream)
         stream.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * ops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+        e2e = {"value": aggregate_tops(world, ops_step, e2e_steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps}
 
