@@ -222,15 +222,17 @@ class Step:
         return self.sq.sq_linear_workspace_size(M, self.lins[0]["lin"].N, self.K) == 0
 
     # -- the call sequence -------------------------------------------------------
-    def run(self, stream, gemm_events=None, stage_events=None):
+    def run(self, stream, gemm_events=None, stage_events=None, capturing=False):
         """Enqueue one step on `stream`.  gemm_events: list receiving
         (M, N, start, end) around each prefill GEMM; stage_events: list
-        receiving (name, start, end) around every call."""
+        receiving (name, start, end) around every call.  capturing: the
+        stream is being captured into a CUDA graph (events become graph
+        nodes that record on every replay)."""
         lib, K = self.lib, self.K
         st = stream.cuda_stream
 
         def ev():
-            e = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True, external=capturing)
             e.record(stream)
             return e
 
@@ -443,7 +445,7 @@ def workload_config(wl):
 # single-call cases (per-kernel timing and profiler captures)
 # ---------------------------------------------------------------------------
 
-def run_case(spec, steps, warmup, flush_l2=True):
+def run_case(spec, steps, warmup, flush_l2=True, settle_us=0.0):
     """Time one C-ABI call on synthetic data.  spec is one of
     gemm:M,N,K  linear:M,N,K  quant_act:M,K  quant_w:N,K  calib:T,K
     smooth_factors:N,K.  Prints one JSON line with the median time."""
@@ -514,6 +516,9 @@ def run_case(spec, steps, warmup, flush_l2=True):
     for _ in range(steps):
         if flush is not None:
             flush.zero_()
+        if settle_us > 0:
+            # idle the GPU after the flush so its write-back does not overlap the call
+            torch.cuda._sleep(int(settle_us * 1965))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         rc = fn()
@@ -522,7 +527,7 @@ def run_case(spec, steps, warmup, flush_l2=True):
         times.append((e0, e1))
     torch.cuda.synchronize()
     us = statistics.median(a.elapsed_time(b) for a, b in times) * 1e3
-    out = {"case": spec, "us": round(us, 2), "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1),
+    out = {"case": spec, "us": round(us, 2), "settle_us": settle_us, "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1),
            "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3), "l2_flushed": flush_l2}
     if ops:
         out["TOPS"] = round(ops / (us * 1e-6) / 1e12, 1)
@@ -571,10 +576,14 @@ def main():
     ap.add_argument("--case", action="append", default=None,
                     help="time single calls instead of the step, e.g. gemm:4096,6144,4096")
     ap.add_argument("--no-flush", action="store_true")
+    ap.add_argument("--settle-us", type=float, default=0.0,
+                    help="--case: GPU idle time between the L2 flush and the timed call")
+    ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=False,
+                    help="replay the step as a CUDA graph in the timed region")
     args = ap.parse_args()
     if args.case:
         for c in args.case:
-            run_case(c, args.steps, max(args.warmup, 3), flush_l2=not args.no_flush)
+            run_case(c, args.steps, max(args.warmup, 3), flush_l2=not args.no_flush, settle_us=args.settle_us)
         return 0
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -611,8 +620,25 @@ def main():
     if st != 0:
         raise RuntimeError(f"device error word {code:#x} after warm-up")
 
-    # timed region
+    # The step as a CUDA graph: S steps per graph (S divides the step count),
+    # replayed steps / S times.  The GEMM events inside the graph record on
+    # every replay, so after the timed region they hold the last replay's S
+    # steps.  Without --graph the steps are enqueued eagerly and every GEMM
+    # launch of the timed region is bracketed by its own events.
+    graph = None
     gemm_events = []
+    per_graph = 1
+    if args.graph:
+        per_graph = max(d for d in range(1, min(args.steps, 10) + 1) if args.steps % d == 0)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for _ in range(per_graph):
+                step.run(stream, gemm_events=gemm_events, capturing=True)
+        for _ in range(2):
+            graph.replay()
+        stream.synchronize()
+
+    # timed region
     sampler = ClockSampler() if rank == 0 else None
     barrier()
     torch.cuda.synchronize()
@@ -623,8 +649,12 @@ def main():
     t_end = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         t_start.record(stream)
-        for _ in range(args.steps):
-            step.run(stream, gemm_events=gemm_events)
+        if graph is not None:
+            for _ in range(args.steps // per_graph):
+                graph.replay()
+        else:
+            for _ in range(args.steps):
+                step.run(stream, gemm_events=gemm_events)
         t_end.record(stream)
     stream.synchronize()
     torch.cuda.synchronize()
@@ -663,6 +693,8 @@ def main():
         "peak_note": f"int8 dense = 2 x {peaks['source']} sustained bf16 cuBLAS "
                      f"({peaks['bf16_tflops_sustained']:.0f} TFLOP/s); 'TFLOP/s' here counts int8 ops",
         "launches": g_n, "avg_launch_us": g_ms / max(g_n, 1) * 1e3,
+        "events": (f"the timed region's last graph replay ({per_graph} steps)" if graph is not None
+                   else "every launch of the timed region"),
         "ops_per_launch": g_ops / max(g_n, 1),
     }
 
@@ -737,7 +769,8 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": workload_config(wl),
+            "config": dict(workload_config(wl),
+                           launch="cuda_graph" if graph is not None else "eager"),
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -747,6 +780,7 @@ def main():
             "stages": stages,
         }
         print(json.dumps(line), flush=True)
+    graph = None
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

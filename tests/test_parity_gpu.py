@@ -225,6 +225,35 @@ def test_gemm_dequant(oracle, M, N, K, out):
     assert exact_fraction(to_np(y), y_o) == 1.0
 
 
+# Shapes whose tile counts select each tile width of the CTA-pair prefill
+# kernel on 74 pairs (256, 256, 192 and 128 output columns per 256-row tile),
+# with ragged M and K; checked exactly on every row and column at the tile edges
+# plus a random sample of (token, channel) pairs.
+@pytest.mark.parametrize("M,N,K", [(2000, 4096, 272), (4000, 6144, 528), (1000, 6144, 1040), (300, 1040, 2064)])
+def test_gemm_pair_widths_sampled(oracle, M, N, K):
+    xq = _int8((M, K), seed=M * 7 + K)
+    wq = _int8((N, K), seed=N * 11 + K)
+    acc = torch.empty(M, N, dtype=torch.int32, device="cuda")
+    sq.sq_w8a8_gemm_s32(xq.cuda(), wq.cuda(), acc)
+    rng = np.random.default_rng(M + N + K)
+    ms = np.unique(np.concatenate([[0, 127, 128, 255, 256, M - 1], rng.integers(0, M, 24)]))
+    ns = np.unique(np.concatenate([[0, 63, 64, 95, 96, 127, 128, 191, 192, 255, 256, N - 1],
+                                   rng.integers(0, N, 40)]))
+    mm, nn = np.meshgrid(ms, ns, indexing="ij")
+    xq_h, wq_h = to_np(xq), to_np(wq)
+    im, jn = np.meshgrid(np.arange(ms.size), np.arange(ns.size), indexing="ij")
+    acc_o = oracle.gemm_i32_pairs(xq_h[ms], wq_h[ns], im.ravel(), jn.ravel())
+    assert_bits_equal(to_np(acc)[mm.ravel(), nn.ravel()], acc_o, f"acc {M}x{N}x{K} sampled")
+    # y through the dequantising epilogue on the same sample
+    rng2 = np.random.default_rng(K)
+    sx_np = rng2.uniform(1e-3, 2.0, M).astype(np.float32)
+    sw_np = rng2.uniform(1e-5, 1e-3, N).astype(np.float32)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    sq.sq_w8a8_gemm(xq.cuda(), to_dev(sx_np), wq.cuda(), to_dev(sw_np), y)
+    y_o = oracle.dequant_pairs(acc_o, sx_np[mm.ravel()], sw_np[nn.ravel()], "bf16")
+    assert_output_close(to_np(y)[mm.ravel(), nn.ravel()], y_o, "y sampled")
+
+
 def test_gemm_extreme_accumulators(oracle):
     """All +127 against all -127 at K = 28672: |acc| = K * 127^2, the largest magnitude."""
     M, N, K = 3, 32, 28672

@@ -18,6 +18,7 @@
 
 #include "sq.h"
 #include "sq_gemm.cuh"
+#include "sq_gemm_pair.cuh"
 #include "sq_mem.cuh"
 #include "sq_ptx.cuh"
 #include "sq_splitk.cuh"
@@ -191,6 +192,46 @@ sq_status launch_row_scale(const T *in, int64_t rows, int64_t K, const float *s,
     return launch_status();
 }
 
+// Single-pass quantiser (row in registers): 2^log2g warps per row, CH chunks
+// per lane.  Returns false when the row is too long for it.
+template <typename T, int MODE, int CH>
+sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
+                               float *scale, int log2g, cudaStream_t st, const DeviceInfo &di)
+{
+    auto kernel = sq::row_quant_kernel<T, MODE, CH>;
+    const int smem = static_cast<int>(K * sizeof(float));
+    static std::atomic<uint64_t> attr_done{0};
+    // the kernel also has a little static shared memory (the group maxima)
+    if (!ensure_smem_attr(kernel, kMaxDynSmem - 1024, attr_done))
+        return SQ_ERR_CUDA;
+    // resident CTAs per SM for this shared-memory size, cached per size
+    static std::mutex mu;
+    static std::vector<std::pair<int, int>> occ;  // smem -> CTAs per SM (one device type)
+    int per_sm = 0;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (auto &e : occ)
+            if (e.first == smem)
+                per_sm = e.second;
+    }
+    if (per_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, sq::kQuantThreads, smem) !=
+                cudaSuccess ||
+            per_sm < 1) {
+            cudaGetLastError();
+            return SQ_ERR_CUDA;
+        }
+        std::lock_guard<std::mutex> lk(mu);
+        occ.emplace_back(smem, per_sm);
+    }
+    const int slots = (sq::kQuantThreads / 32) >> log2g;
+    const int64_t blocks = std::min<int64_t>((rows + slots - 1) / slots, (int64_t)per_sm * di.sms);
+    kernel<<<static_cast<unsigned>(blocks), sq::kQuantThreads, smem, st>>>(in, rows, K, s, log2g, q, scale);
+    return launch_status();
+}
+
+constexpr int kRowQuantCh = 8;  // chunks per lane of the single-pass quantiser (3 CTAs per SM)
+
 template <typename T, int MODE>
 sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
                             float *scale, cudaStream_t st)
@@ -200,6 +241,23 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
         return SQ_ERR_CUDA;
     if (rows > 2147483647LL)
         return SQ_ERR_UNSUPPORTED;
+    {
+        constexpr int V = sq::Vec<T>::N;
+        const int64_t nch = K / V;
+        // tuning override (same arithmetic, different decomposition): SQ_QUANT_CH=16
+        static const int force_ch = std::getenv("SQ_QUANT_CH") ? std::atoi(std::getenv("SQ_QUANT_CH")) : 0;
+        const int ch = force_ch == 16 ? 16 : kRowQuantCh;
+        int log2g = 0;
+        while (log2g < 3 && (int64_t)32 * ch << log2g < nch)
+            ++log2g;
+        if ((int64_t)32 * ch << log2g >= nch) {
+            if (debug_plan())
+                std::fprintf(stderr, "sq quant rows=%lld K=%lld: single pass CH=%d G=%d\n", (long long)rows,
+                             (long long)K, ch, 1 << log2g);
+            return ch == 16 ? launch_row_quant_cfg<T, MODE, 16>(in, rows, K, s, q, scale, log2g, st, di)
+                            : launch_row_quant_cfg<T, MODE, kRowQuantCh>(in, rows, K, s, q, scale, log2g, st, di);
+        }
+    }
     sq_status r = (K * (int64_t)sizeof(float) <= kSmemFactorBytes)
                       ? launch_row_scale<T, MODE, true>(in, rows, K, s, scale, st, di)
                       : launch_row_scale<T, MODE, false>(in, rows, K, s, scale, st, di);
@@ -254,32 +312,38 @@ sq_status launch_gemm_cfg(const int8_t *xq, const float *sx, const int8_t *wq, c
 constexpr int64_t kFusedSliceBytes = 128 * 1024;  // resident token operand per CTA
 
 struct SplitPlan {
-    int splits = 1, kbps = 1, stages = 2, smem = 0;
+    int splits = 1, kbps = 1, stages = 2, smem = 0, kbs = 1;
     bool ok = false;
 };
 
-// Clusters of `splits` CTAs with `smem` bytes each that the device can hold at
-// once (cudaOccupancyMaxActiveClusters), cached per kernel and shape.
+// Clusters of `csize` CTAs of `threads` threads and `smem` bytes each that the
+// device can hold at once (cudaOccupancyMaxActiveClusters), cached per kernel
+// and shape.
 template <typename KernelT>
-int active_clusters(KernelT kernel, int splits, int smem)
+int active_clusters(KernelT kernel, int csize, int smem, int threads)
 {
     static std::mutex mu;
-    static std::vector<std::tuple<int, int, int, int>> cache;  // dev, splits, smem -> clusters
+    struct Entry {
+        const void *fn;
+        int dev, csize, smem, threads, n;
+    };
+    static std::vector<Entry> cache;
     int dev = 0;
     cudaGetDevice(&dev);
+    const void *fn = reinterpret_cast<const void *>(kernel);
     {
         std::lock_guard<std::mutex> lk(mu);
         for (auto &e : cache)
-            if (std::get<0>(e) == dev && std::get<1>(e) == splits && std::get<2>(e) == smem)
-                return std::get<3>(e);
+            if (e.fn == fn && e.dev == dev && e.csize == csize && e.smem == smem && e.threads == threads)
+                return e.n;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(splits * 64));
-    cfg.blockDim = dim3(sq::kSplitThreads);
+    cfg.gridDim = dim3(static_cast<unsigned>(csize * 64));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = splits;
+    attr[0].val.clusterDim.x = csize;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
@@ -290,7 +354,7 @@ int active_clusters(KernelT kernel, int splits, int smem)
         n = 0;
     }
     std::lock_guard<std::mutex> lk(mu);
-    cache.emplace_back(dev, splits, smem, n);
+    cache.push_back(Entry{fn, dev, csize, smem, threads, n});
     return n;
 }
 
@@ -304,6 +368,8 @@ SplitPlan plan_splitk(KernelT kernel, int64_t N, int64_t K)
     // tuning overrides (same work, different decomposition): SQ_SPLITK_SPLITS, SQ_SPLITK_STAGES
     static const int force_splits = std::getenv("SQ_SPLITK_SPLITS") ? std::atoi(std::getenv("SQ_SPLITK_SPLITS")) : 0;
     static const int force_stages = std::getenv("SQ_SPLITK_STAGES") ? std::atoi(std::getenv("SQ_SPLITK_STAGES")) : 0;
+    static const int force_kbs = std::getenv("SQ_SPLITK_KBS") ? std::atoi(std::getenv("SQ_SPLITK_KBS")) : 0;
+    const int kbs = force_kbs > 0 ? force_kbs : 1;
     for (int64_t want = 1; want <= std::min<int64_t>(sq::kMaxSplits, k_blocks); ++want) {
         if (force_splits > 0 && want != force_splits)
             continue;
@@ -315,12 +381,12 @@ SplitPlan plan_splitk(KernelT kernel, int64_t N, int64_t K)
             continue;
         int stages = force_stages > 1 ? force_stages : 8;
         while (stages > 2 &&
-               sq::split_layout<BNX>(stages, FUSED, (int)kbps).total + 1024 > (uint32_t)kMaxDynSmem)
+               sq::split_layout<BNX>(stages, FUSED, (int)kbps, kbs).total + 1024 > (uint32_t)kMaxDynSmem)
             --stages;
-        const int smem = (int)sq::split_layout<BNX>(stages, FUSED, (int)kbps).total + 1024;
+        const int smem = (int)sq::split_layout<BNX>(stages, FUSED, (int)kbps, kbs).total + 1024;
         if (smem > kMaxDynSmem)
             continue;
-        const int active = active_clusters(kernel, (int)sp, smem);
+        const int active = active_clusters(kernel, (int)sp, smem, sq::kSplitThreads);
         if (active <= 0)
             continue;
         const int64_t waves = (n_tiles + active - 1) / active;
@@ -331,6 +397,7 @@ SplitPlan plan_splitk(KernelT kernel, int64_t N, int64_t K)
             best.kbps = (int)kbps;
             best.stages = stages;
             best.smem = smem;
+            best.kbs = kbs;
             best.ok = true;
         }
     }
@@ -350,9 +417,9 @@ sq_status launch_splitk_cfg(const TIN *x, const float *s, const int8_t *xq, cons
     if (!p.ok)
         return SQ_ERR_UNSUPPORTED;
     if (debug_plan())
-        std::fprintf(stderr, "[sq] splitk BNX=%d fused=%d M=%lld N=%lld K=%lld: splits=%d kb/split=%d stages=%d smem=%d clusters=%lld active=%d\n",
-                     BNX, (int)FUSED, (long long)M, (long long)N, (long long)K, p.splits, p.kbps, p.stages, p.smem,
-                     (long long)((N + sq::kBM - 1) / sq::kBM), active_clusters(kernel, p.splits, p.smem));
+        std::fprintf(stderr, "[sq] splitk BNX=%d fused=%d M=%lld N=%lld K=%lld: splits=%d kb/split=%d stages=%d kbs=%d smem=%d clusters=%lld active=%d\n",
+                     BNX, (int)FUSED, (long long)M, (long long)N, (long long)K, p.splits, p.kbps, p.stages, p.kbs, p.smem,
+                     (long long)((N + sq::kBM - 1) / sq::kBM), active_clusters(kernel, p.splits, p.smem, sq::kSplitThreads));
     CUtensorMap tw, tx;
     if (!make_tmap_i8(&tw, wq, N, K, sq::kBM))
         return SQ_ERR_CUDA;
@@ -375,11 +442,79 @@ sq_status launch_splitk_cfg(const TIN *x, const float *s, const int8_t *xq, cons
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kernel, tw, tx, x, s, sx, sw, y, static_cast<int>(M),
                            static_cast<int>(N), static_cast<int>(K), p.splits, p.kbps,
-                           p.stages) != cudaSuccess) {
+                           p.stages, p.kbs) != cudaSuccess) {
         cudaGetLastError();
         return SQ_ERR_CUDA;
     }
     return launch_status();
+}
+
+// Prefill GEMM on CTA pairs: 256 x BN output tiles, persistent over tiles.
+template <int BN, int STAGES, int OUT>
+sq_status launch_gemm_pair_cfg(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
+                               int64_t M, int64_t N, int64_t K, void *y, cudaStream_t st)
+{
+    using Cfg = sq::PairCfg<BN, STAGES>;
+    CUtensorMap ta, tb;
+    if (!make_tmap_i8(&ta, xq, M, K, 128) || !make_tmap_i8(&tb, wq, N, K, BN / 2))
+        return SQ_ERR_CUDA;
+    auto kernel = sq::gemm_i8_pair_kernel<BN, STAGES, OUT>;
+    static std::atomic<uint64_t> attr_done{0};
+    if (!ensure_smem_attr(kernel, Cfg::SMEM_BYTES, attr_done))
+        return SQ_ERR_CUDA;
+    const int active = active_clusters(kernel, 2, Cfg::SMEM_BYTES, sq::kPairThreads);
+    if (active <= 0)
+        return SQ_ERR_CUDA;
+    const int64_t tiles = ((M + sq::kPairBM - 1) / sq::kPairBM) * ((N + BN - 1) / BN);
+    const int64_t pairs = std::min<int64_t>(tiles, active);
+    if (debug_plan())
+        std::fprintf(stderr, "sq gemm pair M=%lld N=%lld K=%lld: BN=%d stages=%d tiles=%lld pairs=%lld\n",
+                     (long long)M, (long long)N, (long long)K, BN, STAGES, (long long)tiles, (long long)pairs);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cfg.blockDim = dim3(sq::kPairThreads);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, sx, sw, y, static_cast<int>(M), static_cast<int>(N),
+                           static_cast<int>(K)) != cudaSuccess) {
+        cudaGetLastError();
+        return SQ_ERR_CUDA;
+    }
+    return launch_status();
+}
+
+// Tile width of the pair GEMM: the fewest rounds of tiles over the
+// co-resident pairs, each round costing one tile's time.  Narrower tiles
+// re-read more operand bytes per operation from L2, so a tile's time is not
+// proportional to its width: measured on B200 (8192 x 28672 x 4096, many
+// rounds), 256 / 192 / 128-wide tiles reach 0.94 / 0.81 / 0.62 of the int8
+// peak, i.e. relative tile times 271 : 237 : 206.
+inline int pick_pair_bn(int64_t M, int64_t N, int pairs)
+{
+    static const int force = std::getenv("SQ_GEMM_PAIR_BN") ? std::atoi(std::getenv("SQ_GEMM_PAIR_BN")) : -1;
+    if (force >= 0)
+        return force;
+    constexpr int cand[3] = {256, 192, 128};
+    constexpr int64_t tile_time[3] = {271, 237, 206};
+    int best = 256;
+    int64_t best_cost = INT64_MAX;
+    for (int i = 0; i < 3; ++i) {
+        const int64_t tiles = ((M + sq::kPairBM - 1) / sq::kPairBM) * ((N + cand[i] - 1) / cand[i]);
+        const int64_t rounds = (tiles + pairs - 1) / std::max(pairs, 1);
+        const int64_t cost = rounds * tile_time[i];
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = cand[i];
+        }
+    }
+    return best;
 }
 
 template <int OUT>
@@ -393,7 +528,20 @@ sq_status launch_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const
         return launch_splitk_cfg<64, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
     if (M <= 128)
         return launch_splitk_cfg<128, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
-    return launch_gemm_cfg<256, 4, OUT, false>(xq, sx, wq, sw, M, N, K, y, st);
+    DeviceInfo di;
+    if (!device_info(di))
+        return SQ_ERR_CUDA;
+    const int bn = pick_pair_bn(M, N, di.sms / 2);
+    switch (bn) {
+    case 256:
+        return launch_gemm_pair_cfg<256, 6, OUT>(xq, sx, wq, sw, M, N, K, y, st);
+    case 192:
+        return launch_gemm_pair_cfg<192, 7, OUT>(xq, sx, wq, sw, M, N, K, y, st);
+    case 128:
+        return launch_gemm_pair_cfg<128, 8, OUT>(xq, sx, wq, sw, M, N, K, y, st);
+    default:  // single-SM 128 x 256 tiles
+        return launch_gemm_cfg<256, 4, OUT, false>(xq, sx, wq, sw, M, N, K, y, st);
+    }
 }
 
 // The fused decode path (activation quant inside the GEMM, no workspace)

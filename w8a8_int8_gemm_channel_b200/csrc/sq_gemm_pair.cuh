@@ -1,0 +1,254 @@
+// sq_gemm_pair.cuh -- the prefill W8A8 GEMM on CTA pairs (tcgen05 cta_group::2).
+//
+//   acc[m, n] = sum_k xq[m, k] * wq[n, k]      (int8 x int8 -> int32, exact)
+//   y[m, n]   = ((float)acc[m, n] * sx[m]) * sw[n]
+//
+// Source: "quant_llm_int8", sections "The architecture: every piece explained"
+// and "End-to-end flow" (integer matmul accumulating in int32, dequantisation
+// by the outer product of the per-row and per-column scales).
+//
+// An output tile is 256 rows (tokens) x BN columns (output channels) and is
+// computed by the two CTAs of a cluster pair, one per SM:
+//   * CTA r of the pair loads A rows [m0 + 128 r, +128) and B rows
+//     [n0 + r BN/2, +BN/2) into its own shared memory (plain TMA, no
+//     multicast); the completion bytes of both CTAs' loads land on the stage's
+//     barrier in the first CTA;
+//   * the first CTA issues tcgen05.mma.cta_group::2 (M = 256, N = BN, K = 32),
+//     which reads both CTAs' halves and accumulates 128 rows in each CTA's
+//     TMEM; its commits free the stage in both CTAs and publish the
+//     accumulator to both epilogues;
+//   * both CTAs' epilogues read their own 128 accumulator rows and store them;
+//     all eight epilogue warps release the accumulator on the first CTA's
+//     barrier.
+// Per SM and 128-byte k block this moves 16 KB of A and BN/2 x 128 bytes of B
+// for 128 x BN outputs: with BN = 256 a third less operand traffic from L2
+// per operation than a 128 x 256 tile on one SM.  Two accumulators in TMEM
+// let the epilogue of one tile overlap the main loop of the next.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sq_gemm.cuh"
+#include "sq_ptx.cuh"
+
+namespace sq {
+
+constexpr int kPairThreads = 192;
+constexpr int kPairBM = 256;  // rows of an output tile (128 per CTA)
+
+template <int BN, int STAGES>
+struct PairCfg {
+    static constexpr int A_BYTES = 128 * kBK;       // this CTA's 128 rows of A
+    static constexpr int B_BYTES = (BN / 2) * kBK;  // this CTA's BN/2 rows of B
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int TMEM_COLS = pow2_at_least(2 * BN, 32);
+    static constexpr int NUM_BARS = 2 * STAGES + 5;  // full, empty, tfull[2], tempty[2], drain
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + NUM_BARS * 8 + 16;
+    static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "MMA N (multiple of 32 for the epilogue)");
+    static_assert(B_BYTES % 1024 == 0, "stage alignment (8-row swizzle atoms)");
+    static_assert(TMEM_COLS <= 512, "TMEM");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+template <int BN, int STAGES, int OUT>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const float *__restrict__ sx, const float *__restrict__ sw, void *__restrict__ y,
+                        int M, int N, int K)
+{
+    using Cfg = PairCfg<BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+    const uint32_t sA = base;
+    const uint32_t sB = base + STAGES * Cfg::A_BYTES;
+    const uint32_t sBar = sB + STAGES * Cfg::B_BYTES;
+    auto full_bar = [&](int s) { return sBar + 8u * s; };
+    auto empty_bar = [&](int s) { return sBar + 8u * (STAGES + s); };
+    auto tfull_bar = [&](int b) { return sBar + 8u * (2 * STAGES + b); };
+    auto tempty_bar = [&](int b) { return sBar + 8u * (2 * STAGES + 2 + b); };
+    const uint32_t drain_bar = sBar + 8u * (2 * STAGES + 4);
+    const uint32_t slot_off = (sBar - base) + 8u * Cfg::NUM_BARS;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(gbase + slot_off);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + slot_off + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0: the pair's first CTA (issues the MMAs)
+    const int pair = static_cast<int>(blockIdx.x >> 1);
+    const int pairs = static_cast<int>(gridDim.x >> 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 8);  // 4 epilogue warps in each CTA
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(const_cast<uint32_t *>(tmem_slot)), Cfg::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    cluster_arrive();  // both CTAs' barriers and TMEM exist before any cross-CTA use
+    cluster_wait();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int m_tiles = (M + kPairBM - 1) / kPairBM;
+    const int n_tiles = (N + BN - 1) / BN;
+    const int total = m_tiles * n_tiles;
+    const int k_blocks = (K + kBK - 1) / kBK;
+
+    uint32_t issued_mask = 0, issued_parity = 0;  // producer: last phase issued per stage
+    bool mma_issued_any = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int t = pair; t < total; t += pairs) {
+                const int m_blk = t % m_tiles, n_blk = t / m_tiles;
+                const int a_row = m_blk * kPairBM + static_cast<int>(rank) * 128;
+                const int b_row = n_blk * BN + static_cast<int>(rank) * (BN / 2);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!bounded_wait(empty_bar(stage), phase ^ 1u, kErrWaitProducer, abort_flag))
+                        goto producer_done;
+                    if (rank == 0)
+                        mbar_arrive_expect_tx(full_bar(stage), 2u * Cfg::STAGE_BYTES);
+                    const uint32_t fb = map_shared_rank(full_bar(stage), 0);
+                    tma_load_2d_pair(sA + stage * Cfg::A_BYTES, &tmA, fb, kb * kBK, a_row);
+                    tma_load_2d_pair(sB + stage * Cfg::B_BYTES, &tmB, fb, kb * kBK, b_row);
+                    issued_mask |= 1u << stage;
+                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // every commit that frees a stage of this CTA has arrived before
+            // the CTA may leave (they are multicast from the first CTA)
+            for (int s = 0; s < STAGES; ++s)
+                if (issued_mask & (1u << s))
+                    if (!bounded_wait(empty_bar(s), (issued_parity >> s) & 1u, kErrWaitDrain, abort_flag))
+                        break;
+        producer_done:;
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = idesc_i8(kPairBM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int t = pair; t < total; t += pairs) {
+                if (!bounded_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, kErrWaitAccEmpty, abort_flag))
+                    break;
+                tc_fence_after_sync();
+                const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
+                bool ok = true;
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!bounded_wait(full_bar(stage), phase, kErrWaitMma, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a0 = sA + stage * Cfg::A_BYTES;
+                    const uint32_t b0 = sB + stage * Cfg::B_BYTES;
+#pragma unroll
+                    for (int k = 0; k < kBK / 32; ++k)
+                        mma_i8_pair(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k), idesc,
+                                    (kb | k) != 0 ? 1u : 0u);
+                    mma_issued_any = true;
+                    mma_commit_pair(empty_bar(stage), 0x3);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                mma_commit_pair(tfull_bar(acc), 0x3);
+                acc ^= 1;
+                if (acc == 0)
+                    acc_phase ^= 1u;
+            }
+        }
+    } else {
+        // epilogue warps 2..5: warp w reads TMEM lanes 32 (w % 4) .. +31
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t tempty_first = map_shared_rank(tempty_bar(0), 0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = pair; t < total; t += pairs) {
+            const int m_blk = t % m_tiles, n_blk = t / m_tiles;
+            const bool ok = bounded_wait(tfull_bar(acc), acc_phase, kErrWaitAccFull, abort_flag);
+            if (!__all_sync(0xFFFFFFFFu, ok))
+                break;
+            tc_fence_after_sync();
+            const int64_t m = static_cast<int64_t>(m_blk) * kPairBM + rank * 128 + row;
+            const uint32_t tbase =
+                tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+            const float sxm = (m < M && OUT != OUT_S32) ? __ldg(sx + m) : 0.0f;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                const int n0 = n_blk * BN + c * 32;
+                if (n0 >= N)
+                    break;
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tbase + c * 32, r);
+                tmem_ld_wait();
+                if (m < M)
+                    store_row_chunk<OUT>(r, sxm, sw, n0, N, y, m);
+                __syncwarp();
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_remote_release(tempty_first + 8u * acc);
+            acc ^= 1;
+            if (acc == 0)
+                acc_phase ^= 1u;
+        }
+    }
+
+    // ---- teardown ----------------------------------------------------------
+    if (warp == 1 && lane == 0 && rank == 0 && *abort_flag && mma_issued_any) {
+        // every MMA of the pair finishes before either CTA releases TMEM
+        mma_commit_pair_local(drain_bar);
+        bounded_wait(drain_bar, 0, kErrWaitDrain, nullptr, kWaitTimeoutNs / 4);
+    }
+    if (warp == 0 && lane == 0 && rank == 0 && *abort_flag) {
+        // copies still in flight complete on the first CTA's full barriers
+        for (int s = 0; s < STAGES; ++s)
+            if (issued_mask & (1u << s))
+                bounded_wait(full_bar(s), (issued_parity >> s) & 1u, kErrWaitDrain, nullptr, kWaitTimeoutNs / 4);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    cluster_arrive();  // neither CTA leaves while the other may still touch its memory
+    cluster_wait();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after_sync();
+        tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+}  // namespace sq

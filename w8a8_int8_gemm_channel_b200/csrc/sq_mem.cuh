@@ -142,25 +142,10 @@ __device__ __forceinline__ void widen<float>(const uint4 &u, float (&v)[4])
 constexpr int kColThreads = 256;
 constexpr int kColClusterRows = 8;
 
-__device__ __forceinline__ uint32_t cluster_ctarank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
 __device__ __forceinline__ void cluster_sync_all()
 {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
-}
-
-// address of the same shared-memory location in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t map_shared_rank(uint32_t local, uint32_t rank)
-{
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
-    return remote;
 }
 
 __device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr)

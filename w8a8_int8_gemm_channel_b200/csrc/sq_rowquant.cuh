@@ -368,4 +368,198 @@ __global__ void __launch_bounds__(256) row_codes_kernel(const T *__restrict__ in
     }
 }
 
+// ----------------------------------------------------------------------------
+// Single-pass quantiser: each row is read from HBM once and stays in
+// registers from the maximum to the codes.  G = 2^log2g warps share one row
+// (a CTA of 8 warps holds 8/G rows at a time); lane L of warp g holds the
+// 16-byte chunks c = 32 g + L + 32 G i, i < CH, so each step i of the G warps
+// covers 32 G consecutive chunks.  Rows of up to 32 * CH * 8 chunks.  The
+// factors (RN(1/s) for activations, s for weights) are staged in shared
+// memory while the first row's loads are in flight.  Persistent over rows.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void named_barrier_sync(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+template <typename T, int MODE, int CH>
+__global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
+    row_quant_kernel(const T *__restrict__ in, int64_t rows, int64_t K, const float *__restrict__ s,
+                     int log2g, int8_t *__restrict__ q, float *__restrict__ scale_out)
+{
+    constexpr int V = Vec<T>::N;
+    constexpr int WARPS = kQuantThreads / 32;
+    extern __shared__ float4 smem_f4[];
+    float *f_sm = reinterpret_cast<float *>(smem_f4);
+    __shared__ float red[2][WARPS];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = 1 << log2g;
+    const int slot = warp >> log2g;
+    const int g = warp & (G - 1);
+    const int slots = WARPS >> log2g;
+    const int nch = static_cast<int>(K / V);
+    const int c0 = 32 * g + lane;
+    const int cstep = 32 * G;
+    int64_t row = static_cast<int64_t>(blockIdx.x) * slots + slot;
+    const int64_t rstride = static_cast<int64_t>(gridDim.x) * slots;
+
+    uint4 raw[CH];
+    auto load_row = [&](int64_t r) {
+        const T *src = in + r * K;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int c = c0 + cstep * i;
+            raw[i] = c < nch ? ld_chunk<T>(src + static_cast<int64_t>(c) * V) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    if (row < rows)
+        load_row(row);
+    const bool bad_divisor =
+        __syncthreads_or(stage_factors<MODE == MODE_X, true>(s, static_cast<int>(K), f_sm, threadIdx.x,
+                                                             blockDim.x)) != 0;
+    auto factor = [&](int c, float (&f)[V]) {
+#pragma unroll
+        for (int h = 0; h < V / 4; ++h) {
+            const float4 v4 = reinterpret_cast<const float4 *>(f_sm + static_cast<int64_t>(c) * V)[h];
+            f[4 * h] = v4.x;
+            f[4 * h + 1] = v4.y;
+            f[4 * h + 2] = v4.z;
+            f[4 * h + 3] = v4.w;
+        }
+    };
+    // maximum over the G warps of this row; alternating buffers, so a buffer
+    // is rewritten only after every warp of the group has passed the barrier
+    // that follows its last read
+    int nred = 0;
+    auto group_max = [&](float v) -> float {
+        v = warp_max(v);
+        if (G == 1)
+            return v;
+        float *r = red[nred & 1];
+        ++nred;
+        if (lane == 0)
+            r[warp] = v;
+        named_barrier_sync(1 + slot, 32 * G);
+        float m = r[slot << log2g];
+        for (int j = 1; j < G; ++j)
+            m = fmaxf(m, r[(slot << log2g) + j]);
+        return m;
+    };
+
+    while (row < rows) {
+        // 1. exact row maximum E = max |v|
+        float E;
+        if constexpr (MODE == MODE_W) {
+            float m = 0.0f;
+#pragma unroll
+            for (int i = 0; i < CH; ++i) {
+                const int c = c0 + cstep * i;
+                if (c < nch) {
+                    float x[V], f[V];
+                    widen<T>(raw[i], x);
+                    factor(c, f);
+#pragma unroll
+                    for (int e = 0; e < V; ++e)
+                        m = fmaxf(m, fabsf(__fmul_rn(x[e], f[e])));
+                }
+            }
+            E = group_max(m);
+        } else {
+            float hmax[CH];
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < CH; ++i) {
+                const int c = c0 + cstep * i;
+                hmax[i] = 0.0f;
+                if (c < nch && !bad_divisor) {
+                    float x[V], f[V];
+                    Chunk8 a;
+                    widen<T>(raw[i], x);
+                    factor(c, f);
+                    hmax[i] = chunk_approx<V>(x, f, a);
+                    amax = fmaxf(amax, hmax[i]);
+                }
+            }
+            const float A = group_max(amax);
+            // exact everywhere when a divisor or the row's magnitude leaves the
+            // range the approximate maximum is proven for
+            const bool exact_all = bad_divisor || A < kTinyQuotient || !(A <= 0x1.fffffep127f);
+            const float thr = __fmul_rn(A, kCandidateScale);
+            float emax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < CH; ++i) {
+                const int c = c0 + cstep * i;
+                if (c < nch && (exact_all || hmax[i] >= thr)) {
+                    float x[V];
+                    widen<T>(raw[i], x);
+                    if (exact_all) {
+                        Chunk8 xv;
+#pragma unroll
+                        for (int e = 0; e < V; ++e)
+                            xv.v[e] = x[e];
+                        emax = fmaxf(emax, chunk_absmax_div(xv, s + static_cast<int64_t>(c) * V, V));
+                    } else {
+                        float f[V];
+                        factor(c, f);
+                        emax = fmaxf(emax, chunk_candidates<V>(x, f, s + static_cast<int64_t>(c) * V, thr));
+                    }
+                }
+            }
+            E = group_max(emax);
+        }
+
+        // 2. scale and codes, from the registers
+        const float scale = scale_from_max(E);
+        if (g == 0 && lane == 0)
+            scale_out[row] = scale;
+        const float rsc = rcp_approx(scale);
+        const bool fast = scale_in_fast_range(scale) && !bad_divisor;
+        int8_t *dst = q + row * K;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int c = c0 + cstep * i;
+            if (c < nch) {
+                float x[V];
+                uint32_t y[V];
+                widen<T>(raw[i], x);
+                bool tie = !fast;
+                if (fast) {
+                    float f[V];
+                    factor(c, f);
+                    float dmax = 0.0f;
+#pragma unroll
+                    for (int e = 0; e < V; ++e) {
+                        const float a = __fmul_rn(x[e], f[e]);
+                        const float yy = __fmaf_rn(a, rsc, kRoundMagic);
+                        const float rr = __fsub_rn(yy, kRoundMagic);
+                        dmax = fmaxf(dmax, fabsf(__fmaf_rn(a, rsc, -rr)));
+                        y[e] = __float_as_uint(yy);
+                    }
+                    tie = !(dmax < kTieLimit);
+                }
+                if (tie) {
+                    Chunk8 xv;
+#pragma unroll
+                    for (int e = 0; e < V; ++e)
+                        xv.v[e] = x[e];
+                    const Chunk8 yy = chunk_codes_exact(xv, s + static_cast<int64_t>(c) * V, V, MODE == MODE_X, scale);
+#pragma unroll
+                    for (int e = 0; e < V; ++e)
+                        y[e] = __float_as_uint(yy.v[e]);
+                }
+                int8_t *d = dst + static_cast<int64_t>(c) * V;
+                if constexpr (V == 8)
+                    *reinterpret_cast<uint2 *>(d) = make_uint2(pack_code_bytes(y[0], y[1], y[2], y[3]),
+                                                               pack_code_bytes(y[4], y[5], y[6], y[7]));
+                else
+                    *reinterpret_cast<uint32_t *>(d) = pack_code_bytes(y[0], y[1], y[2], y[3]);
+            }
+        }
+        row += rstride;
+        if (row < rows)
+            load_row(row);
+    }
+}
+
 }  // namespace sq

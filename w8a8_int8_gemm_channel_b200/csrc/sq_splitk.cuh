@@ -51,57 +51,6 @@ __device__ __forceinline__ void st_shared_cluster_f32(uint32_t addr, float v)
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_remote_release(uint32_t cluster_addr)
-{
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ bool bounded_wait_cluster(uint32_t bar, uint32_t parity, unsigned int code,
-                                                     volatile int *abort_flag)
-{
-    if (mbar_try_wait_acq_cluster(bar, parity))
-        return true;
-    const unsigned long long t0 = globaltimer_ns();
-    for (;;) {
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait_acq_cluster(bar, parity))
-                return true;
-        if (*abort_flag)
-            return false;
-        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-            record_error(code);
-            *abort_flag = 1;
-            return false;
-        }
-    }
-}
-
-// Split cluster barrier (not .aligned: the lanes of a warp may reach it apart).
-__device__ __forceinline__ void cluster_arrive()
-{
-    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
-}
-
-__device__ __forceinline__ void cluster_wait()
-{
-    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
-}
-
 __device__ __forceinline__ void named_bar_sync(int id, int threads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
@@ -122,15 +71,17 @@ struct SplitLayout {
     uint32_t a, b, part, pmax, wpmax, sxs, rsl, bars, misc, total;
 };
 
+// A stage holds `kbs` consecutive 128-byte k blocks (one barrier handshake per stage).
 template <int BNX>
-__host__ __device__ inline SplitLayout split_layout(int stages, bool fused, int kb_per_split)
+__host__ __device__ inline SplitLayout split_layout(int stages, bool fused, int kb_per_split, int kbs)
 {
     SplitLayout L;
     uint32_t o = 0;
     L.a = o;
-    o += stages * kBM * kBK;
+    o += stages * kbs * kBM * kBK;
     L.b = o;
-    o += fused ? static_cast<uint32_t>(BNX) * kBK * kb_per_split : static_cast<uint32_t>(stages) * BNX * kBK;
+    o += fused ? static_cast<uint32_t>(BNX) * kBK * kb_per_split
+               : static_cast<uint32_t>(stages) * kbs * BNX * kBK;
     L.part = o;
     o += kBM * (BNX + 4) * 4;
     L.pmax = o;
@@ -156,13 +107,18 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                        const TIN *__restrict__ x, const float *__restrict__ s,
                        const float *__restrict__ sx, const float *__restrict__ sw,
                        void *__restrict__ y, int M, int N, int K, int splits, int kb_per_split,
-                       int stages)
+                       int stages, int kbs)
 {
     static_assert(BNX % 32 == 0 && BNX <= 128, "token tile");
     static_assert(!FUSED || BNX == 32, "the fused prologue handles up to 32 tokens");
-    constexpr uint32_t TMEM_COLS = BNX < 32 ? 32 : BNX;
+    // NACC independent accumulators: consecutive MMAs rotate over them so no
+    // MMA waits on the previous one's accumulation (with N = BNX this small
+    // the accumulate dependency, not the tensor pipe, would set the pace);
+    // the epilogue adds them (exact int32).
+    constexpr int NACC = BNX <= 128 ? 4 : 2;
+    constexpr uint32_t TMEM_COLS = BNX * NACC;
     constexpr int PSTRIDE = BNX + 4;  // padded int32 row stride of the partial buffer
-    const SplitLayout L = split_layout<BNX>(stages, FUSED, kb_per_split);
+    const SplitLayout L = split_layout<BNX>(stages, FUSED, kb_per_split, kbs);
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -210,6 +166,21 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         if (!FUSED)
             tma_prefetch_desc(&tmX);
     }
+    if (warp == 2 && lane == 0) {
+        // request this CTA's whole weight slice into L2 at once: the ring's
+        // loads then wait on L2 rather than on HBM latency
+        for (int kb = kb0; kb < kb1; ++kb)
+            tma_prefetch_l2_2d(&tmW, kb * kBK, n_blk * kBM);
+    }
+    // the epilogue's scales, fetched while the main loop runs
+    float swn_pre = 0.0f;
+    if (warp >= 4) {
+        const int64_t n = static_cast<int64_t>(n_blk) * kBM + (warp & 3) * 32 + lane;
+        if (OUT != OUT_S32 && n < N)
+            swn_pre = __ldg(sw + n);
+        if (!FUSED && OUT != OUT_S32 && threadIdx.x - 128 < M)
+            sxs[threadIdx.x - 128] = __ldg(sx + (threadIdx.x - 128));
+    }
     if (warp == 1) {
         tmem_alloc(smem_u32(const_cast<uint32_t *>(tmem_slot)), TMEM_COLS);
         tmem_relinquish();
@@ -224,19 +195,26 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     uint32_t issued_mask = 0, issued_parity = 0;
     bool mma_issued_any = false;
 
+    const int nst = (nkb + kbs - 1) / kbs;  // stages this CTA streams
+    const uint32_t a_stage = static_cast<uint32_t>(kbs) * kBM * kBK;
+    const uint32_t b_stage = static_cast<uint32_t>(kbs) * BNX * kBK;
     if (warp == 0) {
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            const uint32_t bytes = kBM * kBK + (FUSED ? 0 : BNX * kBK);
-            for (int j = 0; j < nkb; ++j) {
-                const int kb = kb0 + j;
+            for (int g = 0; g < nst; ++g) {
+                const int cnt = min(kbs, nkb - g * kbs);
                 if (!bounded_wait(empty_bar(stage), phase ^ 1u, kErrWaitProducer, abort_flag))
                     break;
-                mbar_arrive_expect_tx(full_bar(stage), bytes);
-                tma_load_2d(sA + stage * (kBM * kBK), &tmW, full_bar(stage), kb * kBK, n_blk * kBM);
-                if (!FUSED)
-                    tma_load_2d(sB + stage * (BNX * kBK), &tmX, full_bar(stage), kb * kBK, 0);
+                mbar_arrive_expect_tx(full_bar(stage),
+                                      static_cast<uint32_t>(cnt) * (kBM * kBK + (FUSED ? 0 : BNX * kBK)));
+                for (int i = 0; i < cnt; ++i) {
+                    const int kb = kb0 + g * kbs + i;
+                    tma_load_2d(sA + stage * a_stage + i * (kBM * kBK), &tmW, full_bar(stage), kb * kBK,
+                                n_blk * kBM);
+                    if (!FUSED)
+                        tma_load_2d(sB + stage * b_stage + i * (BNX * kBK), &tmX, full_bar(stage), kb * kBK, 0);
+                }
                 issued_mask |= 1u << stage;
                 issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                 if (++stage == stages) {
@@ -255,18 +233,25 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                 tc_fence_after_sync();
                 int stage = 0;
                 uint32_t phase = 0;
-                for (int j = 0; j < nkb; ++j) {
+                for (int g = 0; g < nst; ++g) {
                     if (!bounded_wait(full_bar(stage), phase, kErrWaitMma, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t a0 = sA + stage * (kBM * kBK);
-                    const uint32_t b0 = FUSED ? sB + j * (BNX * kBK) : sB + stage * (BNX * kBK);
+                    const int cnt = min(kbs, nkb - g * kbs);
+                    for (int i = 0; i < cnt; ++i) {
+                        const int j = g * kbs + i;  // k block within this CTA's slice
+                        const uint32_t a0 = sA + stage * a_stage + i * (kBM * kBK);
+                        const uint32_t b0 = FUSED ? sB + j * (BNX * kBK) : sB + stage * b_stage + i * (BNX * kBK);
 #pragma unroll
-                    for (int k = 0; k < kBK / 32; ++k)
-                        mma_i8(tmem_base, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k),
-                               idesc, (j | k) != 0 ? 1u : 0u);
+                        for (int k = 0; k < kBK / 32; ++k) {
+                            const int step = j * (kBK / 32) + k;  // MMA index within the slice
+                            mma_i8(tmem_base + static_cast<uint32_t>((step % NACC) * BNX),
+                                   smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k), idesc,
+                                   step >= NACC ? 1u : 0u);
+                        }
+                    }
                     mma_issued_any = true;
                     mma_commit(empty_bar(stage));
                     if (++stage == stages) {
@@ -372,9 +357,18 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             tc_fence_after_sync();
 #pragma unroll 1
             for (int c = 0; c < BNX / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + c * 32, r);
+                uint32_t r[32], t[32];
+                const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + c * 32;
+                tmem_ld_32x32b_x32(lane_addr, r);
                 tmem_ld_wait();
+#pragma unroll 1
+                for (int a = 1; a < NACC; ++a) {
+                    tmem_ld_32x32b_x32(lane_addr + static_cast<uint32_t>(a * BNX), t);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 32; ++q)
+                        r[q] += t[q];  // exact int32 sums
+                }
                 int4 *dst = reinterpret_cast<int4 *>(part + row * PSTRIDE + c * 32);
 #pragma unroll
                 for (int v = 0; v < 8; ++v)
@@ -406,7 +400,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const int64_t n = static_cast<int64_t>(n_blk) * kBM + row;
-        const float swn = (n < N && OUT != OUT_S32) ? __ldg(sw + n) : 0.0f;
+        const float swn = swn_pre;
         const uint32_t my = smem_u32(part + row * PSTRIDE);
 #pragma unroll 1
         for (int c = 0; c < BNX / 32; ++c) {
@@ -442,7 +436,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                         if constexpr (OUT == OUT_S32) {
                             reinterpret_cast<int32_t *>(y)[idx] = acc[jj];
                         } else {
-                            const float sxm = FUSED ? sxs[m] : __ldg(sx + m);
+                            const float sxm = sxs[m];
                             const float o = __fmul_rn(__fmul_rn(__int2float_rn(acc[jj]), sxm), swn);
                             if constexpr (OUT == OUT_F32)
                                 reinterpret_cast<float *>(y)[idx] = o;
