@@ -206,16 +206,27 @@ class Step:
     def output_bytes(self):
         return sum(y.numel() * y.element_size() for d in self.lins for y in d["y"].values())
 
+    def quant_kernels(self):
+        """Kernels one quantiser call launches: one single-pass kernel while
+        the factor tables fit shared memory and a row fits 16 chunks per lane
+        of 8 warps, else a scale kernel and a code kernel."""
+        esize = 2 if self.in_code == self.sq.SQ_BF16 else 4
+        nch = self.K * esize // 16
+        smem = self.K * 4 + (self.K * 2 if esize == 2 else 0)
+        if os.environ.get("SQ_QUANT_KIND") == "2":
+            return 2
+        return 1 if smem <= 232448 - 1024 and nch <= 32 * 16 * 8 else 2
+
     def launches_per_step(self):
         """Kernels of this library one step launches: the calibration absmax
         (1); per linear the weight's input-channel absmax and the factors (2)
-        and the weight quantiser's scale and code kernels (2); per token count
-        and linear either the fused linear (1) or the activation quantiser's
-        two kernels and the GEMM (3)."""
+        and the weight quantiser; per token count and linear either the fused
+        linear (1) or the activation quantiser and the GEMM (1)."""
+        q = self.quant_kernels()
         n = 1
-        n += 4 * len(self.lins)
+        n += (2 + q) * len(self.lins)
         for M in self.wl.Ms:
-            n += len(self.lins) * (1 if self.fused(M) else 3)
+            n += len(self.lins) * (1 if self.fused(M) else q + 1)
         return n
 
     def fused(self, M):

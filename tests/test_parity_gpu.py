@@ -363,3 +363,49 @@ def test_smooth_quant_weight_fast_path_edges(oracle, s_kind):
     wq_o, sw_o = oracle.smooth_quant_weight(w, s_np)
     assert_bits_equal(to_np(sw), sw_o, "sw")
     assert_bits_equal(to_np(wq), wq_o, "wq")
+
+
+# ---------------------------------------------------------------------------
+# bf16 rows: the quantisers bound |v| in bf16 arithmetic (within about 0.8%)
+# and recompute exactly every chunk within 2^-5 of the largest bound; these
+# rows crowd the top of the range so that the bound alone could not order them
+# ---------------------------------------------------------------------------
+
+def _bf16_crowded_rows(K, s_np, mode, seed):
+    """bf16 rows (as fp32 values) whose smoothed magnitudes crowd the maximum."""
+    rng = np.random.default_rng(seed)
+    f = (1.0 / s_np) if mode == "x" else s_np  # v = x * f in exact arithmetic
+    rows = []
+    # 300 elements within 0.5% of 3.0, the rest far below
+    r = rng.standard_normal(K) * 0.3
+    idx = rng.choice(K, 300, replace=False)
+    r[idx] = 3.0 * (1.0 + rng.uniform(-0.005, 0.005, 300)) * np.sign(rng.standard_normal(300))
+    rows.append(r / f)
+    # every smoothed magnitude equal up to bf16 rounding of x: all chunks are candidates
+    rows.append(np.where(rng.random(K) < 0.5, -1.0, 1.0) / f)
+    # Gaussian with a few outlier channels, a tiny row and a zero row
+    r = rng.standard_normal(K)
+    r[rng.choice(K, 5, replace=False)] *= 60.0
+    rows.append(r / f)
+    rows.append(rng.standard_normal(K) * 1e-33 / f)
+    rows.append(np.zeros(K))
+    x = torch.from_numpy(np.stack(rows).astype(np.float32)).to(torch.bfloat16)
+    return x
+
+
+@pytest.mark.parametrize("K", [4096, 14336])
+@pytest.mark.parametrize("mode", ["x", "w"])
+def test_quant_bf16_crowded_maxima(oracle, K, mode):
+    rng = np.random.default_rng(K + (1 if mode == "x" else 2))
+    s_np = rng.uniform(0.3, 3.0, K).astype(np.float32)
+    x = _bf16_crowded_rows(K, s_np, mode, seed=K)
+    q = torch.empty(x.shape, dtype=torch.int8, device="cuda")
+    sc = torch.empty(x.shape[0], device="cuda")
+    if mode == "x":
+        sq.sq_quant_act(x.cuda(), to_dev(s_np), q, sc)
+        q_o, sc_o = oracle.quant_act(to_np(x), s_np)
+    else:
+        sq.sq_smooth_quant_weight(x.cuda(), to_dev(s_np), q, sc)
+        q_o, sc_o = oracle.smooth_quant_weight(to_np(x), s_np)
+    assert_bits_equal(to_np(sc), sc_o, f"scales ({mode})")
+    assert_bits_equal(to_np(q), q_o, f"codes ({mode})")

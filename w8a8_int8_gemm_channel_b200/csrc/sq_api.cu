@@ -14,6 +14,7 @@
 #include <mutex>
 #include <tuple>
 #include <vector>
+#include <utility>
 #include <climits>
 
 #include "sq.h"
@@ -77,6 +78,51 @@ bool debug_plan()
 {
     static const bool on = std::getenv("SQ_DEBUG_PLAN") != nullptr;
     return on;
+}
+
+// Programmatic dependent launch for every kernel of the library (each one
+// begins with griddepcontrol.wait, so it sees all work before it on the
+// stream); SQ_PDL=0 turns the attribute off.
+bool pdl_enabled()
+{
+    static const bool on = !(std::getenv("SQ_PDL") && std::atoi(std::getenv("SQ_PDL")) == 0);
+    return on;
+}
+
+// Launch `kernel` on `st`.  Kernels that use cluster features (distributed
+// shared memory, cluster barriers, remote mbarrier arrivals) pass their
+// cluster shape cx x cy, which is set even when it is 1 x 1; other kernels
+// pass cx = 0.
+template <typename... KArgs, typename... Args>
+sq_status launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t st, int cx,
+                        int cy, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    if (cx > 0) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = static_cast<unsigned>(cx);
+        attr[n].val.clusterDim.y = static_cast<unsigned>(cy);
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+        cudaGetLastError();
+        return SQ_ERR_CUDA;
+    }
+    return launch_status();
 }
 
 // ---- tensor maps -----------------------------------------------------------
@@ -143,33 +189,19 @@ sq_status launch_col_absmax(const T *x, int64_t R, int64_t K, int64_t ld, float 
     constexpr int CL = sq::kColClusterRows;
     const int64_t chunks = K / V;
     const int64_t col_blocks = (chunks + sq::kColThreads - 1) / sq::kColThreads;
-    // about 8 CTAs of 256 threads per SM in total, in clusters of CL row bands
-    const int64_t want = std::max<int64_t>(CL, (int64_t)di.sms * 8 / col_blocks);
-    int64_t rows_per_block = std::max<int64_t>(32, (R + want - 1) / want);
+    // one wave of about 4 CTAs of 256 threads per SM, in clusters of CL row
+    // bands; bands are whole multiples of the 8 rows a thread keeps in flight
+    const int64_t want = std::max<int64_t>(CL, (int64_t)di.sms * 4 / col_blocks);
+    int64_t rows_per_block = std::max<int64_t>(8, ((R + want - 1) / want + 7) / 8 * 8);
     int64_t row_blocks = (R + rows_per_block - 1) / rows_per_block;
     while (row_blocks > 65528) {
         rows_per_block *= 2;
         row_blocks = (R + rows_per_block - 1) / rows_per_block;
     }
     row_blocks = (row_blocks + CL - 1) / CL * CL;  // whole clusters; surplus bands are empty
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(col_blocks), static_cast<unsigned>(row_blocks));
-    cfg.blockDim = dim3(sq::kColThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = CL;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, sq::col_absmax_kernel<T>, x, R, K, ld, rows_per_block,
-                           reinterpret_cast<unsigned int *>(out)) != cudaSuccess) {
-        cudaGetLastError();
-        return SQ_ERR_CUDA;
-    }
-    return launch_status();
+    return launch_kernel(sq::col_absmax_kernel<T>, dim3(static_cast<unsigned>(col_blocks), static_cast<unsigned>(row_blocks)),
+                         dim3(sq::kColThreads), 0, st, 1, CL, x, R, K, ld, rows_per_block,
+                         reinterpret_cast<unsigned int *>(out));
 }
 
 // ---- row quantisers ----------------------------------------------------------
@@ -188,18 +220,18 @@ sq_status launch_row_scale(const T *in, int64_t rows, int64_t K, const float *s,
     const int per_sm = smem <= 96 * 1024 ? 2 : 1;
     const int warps = sq::kQuantThreads / 32;
     const int64_t blocks = std::min<int64_t>((rows + warps - 1) / warps, (int64_t)per_sm * di.sms);
-    kernel<<<static_cast<unsigned>(blocks), sq::kQuantThreads, smem, st>>>(in, rows, K, s, scale);
-    return launch_status();
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(sq::kQuantThreads), smem, st, 0, 0, in, rows,
+                         K, s, scale);
 }
 
 // Single-pass quantiser (row in registers): 2^log2g warps per row, CH chunks
-// per lane.  Returns false when the row is too long for it.
+// per lane.
 template <typename T, int MODE, int CH>
 sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
                                float *scale, int log2g, cudaStream_t st, const DeviceInfo &di)
 {
     auto kernel = sq::row_quant_kernel<T, MODE, CH>;
-    const int smem = static_cast<int>(K * sizeof(float));
+    const int smem = static_cast<int>(sq::row_quant_smem(K, sq::Vec<T>::N == 8));
     static std::atomic<uint64_t> attr_done{0};
     // the kernel also has a little static shared memory (the group maxima)
     if (!ensure_smem_attr(kernel, kMaxDynSmem - 1024, attr_done))
@@ -224,13 +256,17 @@ sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float
         std::lock_guard<std::mutex> lk(mu);
         occ.emplace_back(smem, per_sm);
     }
+    // few rows: spread each row over more warps so that every SM has work
+    while (log2g < 3 && rows * (1 << log2g) < (int64_t)di.sms * per_sm * (sq::kQuantThreads / 32))
+        ++log2g;
     const int slots = (sq::kQuantThreads / 32) >> log2g;
     const int64_t blocks = std::min<int64_t>((rows + slots - 1) / slots, (int64_t)per_sm * di.sms);
-    kernel<<<static_cast<unsigned>(blocks), sq::kQuantThreads, smem, st>>>(in, rows, K, s, log2g, q, scale);
-    return launch_status();
+    if (debug_plan())
+        std::fprintf(stderr, "sq quant rows=%lld K=%lld: single pass CH=%d G=%d per_sm=%d blocks=%lld\n",
+                     (long long)rows, (long long)K, CH, 1 << log2g, per_sm, (long long)blocks);
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(sq::kQuantThreads), smem, st, 0, 0, in, rows,
+                         K, s, log2g, q, scale);
 }
-
-constexpr int kRowQuantCh = 8;  // chunks per lane of the single-pass quantiser (3 CTAs per SM)
 
 template <typename T, int MODE>
 sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
@@ -241,21 +277,21 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
         return SQ_ERR_CUDA;
     if (rows > 2147483647LL)
         return SQ_ERR_UNSUPPORTED;
-    {
-        constexpr int V = sq::Vec<T>::N;
-        const int64_t nch = K / V;
-        // tuning override (same arithmetic, different decomposition): SQ_QUANT_CH=16
-        static const int force_ch = std::getenv("SQ_QUANT_CH") ? std::atoi(std::getenv("SQ_QUANT_CH")) : 0;
-        const int ch = force_ch == 16 ? 16 : kRowQuantCh;
-        int log2g = 0;
-        while (log2g < 3 && (int64_t)32 * ch << log2g < nch)
-            ++log2g;
-        if ((int64_t)32 * ch << log2g >= nch) {
-            if (debug_plan())
-                std::fprintf(stderr, "sq quant rows=%lld K=%lld: single pass CH=%d G=%d\n", (long long)rows,
-                             (long long)K, ch, 1 << log2g);
-            return ch == 16 ? launch_row_quant_cfg<T, MODE, 16>(in, rows, K, s, q, scale, log2g, st, di)
-                            : launch_row_quant_cfg<T, MODE, kRowQuantCh>(in, rows, K, s, q, scale, log2g, st, di);
+    // tuning override (same arithmetic, other kernels): SQ_QUANT_KIND=2 takes
+    // the two-kernel path for every K
+    static const int force_kind = std::getenv("SQ_QUANT_KIND") ? std::atoi(std::getenv("SQ_QUANT_KIND")) : 0;
+    constexpr int V = sq::Vec<T>::N;
+    const int64_t nch = K / V;
+    if (force_kind != 2 && sq::row_quant_smem(K, V == 8) <= kMaxDynSmem - 1024) {
+        // 8 chunks per lane (three CTAs per SM), 16 for rows too long for that
+        for (int ch : {8, 16}) {
+            int log2g = 0;
+            while (log2g < 3 && ((int64_t)32 * ch << log2g) < nch)
+                ++log2g;
+            if (((int64_t)32 * ch << log2g) < nch)
+                continue;
+            return ch == 8 ? launch_row_quant_cfg<T, MODE, 8>(in, rows, K, s, q, scale, log2g, st, di)
+                           : launch_row_quant_cfg<T, MODE, 16>(in, rows, K, s, q, scale, log2g, st, di);
         }
     }
     sq_status r = (K * (int64_t)sizeof(float) <= kSmemFactorBytes)
@@ -263,7 +299,6 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
                       : launch_row_scale<T, MODE, false>(in, rows, K, s, scale, st, di);
     if (r != SQ_OK)
         return r;
-    constexpr int V = sq::Vec<T>::N;
     const int64_t chunks = K / V;
     const int threads = static_cast<int>(std::min<int64_t>(256, (chunks + 31) / 32 * 32));
     const int64_t col_blocks = (chunks + threads - 1) / threads;
@@ -275,8 +310,8 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
         row_blocks = (rows + rpb - 1) / rpb;
     }
     dim3 grid(static_cast<unsigned>(col_blocks), static_cast<unsigned>(row_blocks));
-    sq::row_codes_kernel<T, MODE><<<grid, threads, 0, st>>>(in, rows, K, s, scale, rpb, q);
-    return launch_status();
+    return launch_kernel(sq::row_codes_kernel<T, MODE>, grid, dim3(threads), 0, st, 0, 0, in, rows, K, s,
+                         static_cast<const float *>(scale), rpb, q);
 }
 
 int64_t max_quant_k(sq_dtype dt) { return dt == SQ_BF16 ? 65536 : 32768; }
@@ -303,9 +338,8 @@ sq_status launch_gemm_cfg(const int8_t *xq, const float *sx, const int8_t *wq, c
         return SQ_ERR_CUDA;
     const int64_t tiles = ((ra + sq::kBM - 1) / sq::kBM) * ((rb + BN - 1) / BN);
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, di.sms));
-    kernel<<<grid, sq::kGemmThreads, Cfg::SMEM_BYTES, st>>>(ta, tb, sx, sw, y, static_cast<int>(M),
-                                                           static_cast<int>(N), static_cast<int>(K));
-    return launch_status();
+    return launch_kernel(kernel, dim3(grid), dim3(sq::kGemmThreads), Cfg::SMEM_BYTES, st, 0, 0, ta, tb, sx, sw, y,
+                         static_cast<int>(M), static_cast<int>(N), static_cast<int>(K));
 }
 
 // ---- split-K small-M GEMM (optionally with the activation quant fused in) --
@@ -428,25 +462,9 @@ sq_status launch_splitk_cfg(const TIN *x, const float *s, const int8_t *xq, cons
     else if (!make_tmap_i8(&tx, xq, M, K, BNX))
         return SQ_ERR_CUDA;
     const int64_t n_tiles = (N + sq::kBM - 1) / sq::kBM;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(n_tiles * p.splits));
-    cfg.blockDim = dim3(sq::kSplitThreads);
-    cfg.dynamicSmemBytes = p.smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p.splits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kernel, tw, tx, x, s, sx, sw, y, static_cast<int>(M),
-                           static_cast<int>(N), static_cast<int>(K), p.splits, p.kbps,
-                           p.stages, p.kbs) != cudaSuccess) {
-        cudaGetLastError();
-        return SQ_ERR_CUDA;
-    }
-    return launch_status();
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(n_tiles * p.splits)), dim3(sq::kSplitThreads), p.smem, st,
+                         p.splits, 1, tw, tx, x, s, sx, sw, y, static_cast<int>(M), static_cast<int>(N),
+                         static_cast<int>(K), p.splits, p.kbps, p.stages, p.kbs);
 }
 
 // Prefill GEMM on CTA pairs: 256 x BN output tiles, persistent over tiles.
@@ -470,24 +488,8 @@ sq_status launch_gemm_pair_cfg(const int8_t *xq, const float *sx, const int8_t *
     if (debug_plan())
         std::fprintf(stderr, "sq gemm pair M=%lld N=%lld K=%lld: BN=%d stages=%d tiles=%lld pairs=%lld\n",
                      (long long)M, (long long)N, (long long)K, BN, STAGES, (long long)tiles, (long long)pairs);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-    cfg.blockDim = dim3(sq::kPairThreads);
-    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, sx, sw, y, static_cast<int>(M), static_cast<int>(N),
-                           static_cast<int>(K)) != cudaSuccess) {
-        cudaGetLastError();
-        return SQ_ERR_CUDA;
-    }
-    return launch_status();
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(2 * pairs)), dim3(sq::kPairThreads), Cfg::SMEM_BYTES, st, 2,
+                         1, ta, tb, sx, sw, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K));
 }
 
 // Tile width of the pair GEMM: the fewest rounds of tiles over the
@@ -656,8 +658,7 @@ sq_status sq_smooth_factors(const float *ax, const void *w, sq_dtype dt, int64_t
         return r;
     const int threads = 256;
     const unsigned blocks = static_cast<unsigned>((K + threads - 1) / threads);
-    sq::smooth_factors_kernel<<<blocks, threads, 0, st>>>(ax, s, aw, K, alpha);
-    return launch_status();
+    return launch_kernel(sq::smooth_factors_kernel, dim3(blocks), dim3(threads), 0, st, 0, 0, ax, s, aw, K, alpha);
 }
 
 sq_status sq_smooth_quant_weight(const void *w, sq_dtype dt, int64_t N, int64_t K, const float *s,

@@ -149,6 +149,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                    const float *__restrict__ sx, const float *__restrict__ sw,
                    void *__restrict__ y, int M, int N, int K)
 {
+    pdl_prologue();
     using Cfg = GemmCfg<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);

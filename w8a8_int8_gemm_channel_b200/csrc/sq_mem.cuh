@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(kColThreads) col_absmax_kernel(const T *__rest
                                                                   int64_t rows_per_block,
                                                                   unsigned int *__restrict__ out_bits)
 {
+    pdl_prologue();
     constexpr int V = Vec<T>::N;
     constexpr int SLOTS = kColThreads / kColClusterRows;  // chunk columns each CTA combines
     __shared__ __align__(16) float part[kColThreads * V];
@@ -247,6 +248,7 @@ __global__ void __launch_bounds__(kColThreads) col_absmax_kernel(const T *__rest
 __global__ void smooth_factors_kernel(const float *__restrict__ ax, float *s, float *aw, int64_t K,
                                       float alpha)
 {
+    pdl_prologue();
     const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (j >= K)
         return;
@@ -365,6 +367,15 @@ __device__ __noinline__ float chunk_absmax_div(Chunk8 x, const float *__restrict
     float m = 0.0f;
     for (int e = 0; e < n; ++e)
         m = fmaxf(m, fabsf(__fdiv_rn(x.v[e], __ldg(s_chunk + e))));
+    return m;
+}
+
+// Exact max of |x * s| over one chunk (weights: the smoothed values).
+__device__ __noinline__ float chunk_absmax_mul(Chunk8 x, const float *__restrict__ s_chunk, int n)
+{
+    float m = 0.0f;
+    for (int e = 0; e < n; ++e)
+        m = fmaxf(m, fabsf(__fmul_rn(x.v[e], __ldg(s_chunk + e))));
     return m;
 }
 

@@ -26,6 +26,7 @@ enum : unsigned int {
     kErrWaitPrologue = 0x500,   // MMA issuer waiting for the in-kernel quantised operand
     kErrWaitCluster = 0x600,    // cross-CTA exchange inside a cluster
     kErrWaitDrain = 0x700,      // teardown drain of in-flight copies
+    kErrWaitRow = 0x800,        // quantiser waiting for a staged row
 };
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
@@ -40,6 +41,17 @@ __device__ __forceinline__ unsigned long long globaltimer_ns()
 __device__ __forceinline__ void record_error(unsigned int code)
 {
     atomicCAS(&g_sq_device_error, 0u, code);
+}
+
+// Programmatic dependent launch.  Every kernel of the library starts with
+// pdl_prologue(): it waits until the grid before it on the stream has
+// completed and its memory is visible (a no-op when the launch did not allow
+// an early start), then lets the next grid begin launching, so that grid's
+// launch overlaps this one's execution.
+__device__ __forceinline__ void pdl_prologue()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
@@ -203,6 +215,83 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
         : "memory");
+}
+
+// Contiguous copy global -> shared of `bytes` (multiple of 16, both addresses
+// 16-byte aligned); completion is signalled on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// ----------------------------------------------------------------------------
+// packed fp32 pairs (sm_100): two independent IEEE round-to-nearest
+// operations per instruction, exactly the scalar _rn results.  The pairs are
+// formed inside the asm (mov.b64 {lo, hi}), which only names a register pair.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float2 f2_mul(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// packed bfloat16 pairs: products rounded to bf16 (only used for bounds
+// that are re-checked exactly)
+__device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t bf2_max(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// the larger half of a pair of non-negative bf16 values, as fp32 (exact)
+__device__ __forceinline__ float bf2_hmax_f32(uint32_t v)
+{
+    return fmaxf(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
 
 // Prefetch one 2-D tile into L2 (no shared-memory destination, no completion).

@@ -252,6 +252,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     row_scale_kernel(const T *__restrict__ in, int64_t rows, int64_t K, const float *__restrict__ s,
                      float *__restrict__ scale_out)
 {
+    pdl_prologue();
     constexpr int V = Vec<T>::N;
     extern __shared__ float4 smem_f4[];
     float *f_sm = reinterpret_cast<float *>(smem_f4);
@@ -298,6 +299,7 @@ __global__ void __launch_bounds__(256) row_codes_kernel(const T *__restrict__ in
                                                         const float *__restrict__ scale,
                                                         int64_t rows_per_block, int8_t *__restrict__ q)
 {
+    pdl_prologue();
     constexpr int V = Vec<T>::N;
     constexpr int U = 4;  // rows in flight per thread
     const int64_t nch = K / V;
@@ -373,24 +375,79 @@ __global__ void __launch_bounds__(256) row_codes_kernel(const T *__restrict__ in
 // registers from the maximum to the codes.  G = 2^log2g warps share one row
 // (a CTA of 8 warps holds 8/G rows at a time); lane L of warp g holds the
 // 16-byte chunks c = 32 g + L + 32 G i, i < CH, so each step i of the G warps
-// covers 32 G consecutive chunks.  Rows of up to 32 * CH * 8 chunks.  The
-// factors (RN(1/s) for activations, s for weights) are staged in shared
-// memory while the first row's loads are in flight.  Persistent over rows.
+// covers 32 G consecutive chunks.  Persistent over rows.
+//
+// Maximum.  bf16 rows: a bound p_k = RN_bf16(|x_k| * RN_bf16(|f_k|)) in
+// packed bf16 arithmetic, with f_k = RN(1/s_k) to 1 ulp (activations) or s_k
+// (weights), lies within a factor 1 +- 0.0079 of |v_k| (two bf16 roundings of
+// relative size 2^-8 each, plus the reciprocal's and v's fp32 roundings).  So
+// the element attaining the exact maximum E has p_k >= A (1 - 2^-5), A the
+// largest bound, and only the chunks reaching that threshold are recomputed
+// exactly (IEEE x/s or x*s).  fp32 rows: fp32 bounds a_k = RN(|x_k| f_k)
+// within 2^-21 and the threshold A (1 - 2^-20); weights need none (a_k is
+// v_k).  Rows whose bound leaves [2^-100, FLT_MAX], or whose divisors leave
+// the fast range, are recomputed exactly throughout.
+// Codes.  The rounding fast path of sq_div.cuh, in packed fp32 pairs.
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void named_barrier_sync(int id, int threads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Factor tables in shared memory: f[K] fp32 (RN(1/s) when RECIP, else s)
+// and, with BF, fb[K] = RN_bf16(|f|) as bf16 pairs.  Returns non-zero when
+// some reciprocal is unusable by the fast paths.
+template <bool RECIP, bool BF>
+__device__ __forceinline__ int stage_factor_tables(const float *__restrict__ s, int n, float *f, uint32_t *fb,
+                                                   int t, int nt)
+{
+    int bad = 0;
+    const int nv = n >> 2;  // n is a multiple of 16
+    const float4 *s4 = reinterpret_cast<const float4 *>(s);
+    for (int j0 = t; j0 < nv; j0 += 4 * nt) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + u * nt;
+            v[u] = j < nv ? __ldg(s4 + j) : make_float4(1.f, 1.f, 1.f, 1.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + u * nt;
+            if (j < nv) {
+                float4 r = v[u];
+                if (RECIP) {
+                    r = make_float4(fast_recip(v[u].x), fast_recip(v[u].y), fast_recip(v[u].z), fast_recip(v[u].w));
+                    bad |= (r.x == 0.0f) | (r.y == 0.0f) | (r.z == 0.0f) | (r.w == 0.0f);
+                }
+                reinterpret_cast<float4 *>(f)[j] = r;
+                if (BF) {
+                    const __nv_bfloat162 lo = __floats2bfloat162_rn(fabsf(r.x), fabsf(r.y));
+                    const __nv_bfloat162 hi = __floats2bfloat162_rn(fabsf(r.z), fabsf(r.w));
+                    reinterpret_cast<uint2 *>(fb)[j] =
+                        make_uint2(*reinterpret_cast<const uint32_t *>(&lo), *reinterpret_cast<const uint32_t *>(&hi));
+                }
+            }
+        }
+    }
+    return bad;
+}
+
+// bytes of shared memory the factor tables of a K-column row take
+__host__ __device__ constexpr int64_t row_quant_smem(int64_t K, bool bf) { return K * 4 + (bf ? K * 2 : 0); }
+
 template <typename T, int MODE, int CH>
 __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
     row_quant_kernel(const T *__restrict__ in, int64_t rows, int64_t K, const float *__restrict__ s,
                      int log2g, int8_t *__restrict__ q, float *__restrict__ scale_out)
 {
+    pdl_prologue();
     constexpr int V = Vec<T>::N;
+    constexpr bool BF = (V == 8);  // bf16 rows
     constexpr int WARPS = kQuantThreads / 32;
     extern __shared__ float4 smem_f4[];
     float *f_sm = reinterpret_cast<float *>(smem_f4);
+    uint32_t *fb_sm = reinterpret_cast<uint32_t *>(f_sm + K);
     __shared__ float red[2][WARPS];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -415,17 +472,15 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
     };
     if (row < rows)
         load_row(row);
-    const bool bad_divisor =
-        __syncthreads_or(stage_factors<MODE == MODE_X, true>(s, static_cast<int>(K), f_sm, threadIdx.x,
-                                                             blockDim.x)) != 0;
-    auto factor = [&](int c, float (&f)[V]) {
+    // factor tables staged while the first row's loads are in flight
+    const bool bad_divisor = __syncthreads_or(stage_factor_tables<MODE == MODE_X, BF>(
+                                 s, static_cast<int>(K), f_sm, fb_sm, threadIdx.x, blockDim.x)) != 0;
+    auto factor_pairs = [&](int c, float2 (&f2)[V / 2]) {
 #pragma unroll
         for (int h = 0; h < V / 4; ++h) {
             const float4 v4 = reinterpret_cast<const float4 *>(f_sm + static_cast<int64_t>(c) * V)[h];
-            f[4 * h] = v4.x;
-            f[4 * h + 1] = v4.y;
-            f[4 * h + 2] = v4.z;
-            f[4 * h + 3] = v4.w;
+            f2[2 * h] = make_float2(v4.x, v4.y);
+            f2[2 * h + 1] = make_float2(v4.z, v4.w);
         }
     };
     // maximum over the G warps of this row; alternating buffers, so a buffer
@@ -448,65 +503,58 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
     };
 
     while (row < rows) {
-        // 1. exact row maximum E = max |v|
-        float E;
-        if constexpr (MODE == MODE_W) {
-            float m = 0.0f;
+        // 1. bounds of |v| per chunk, the row's largest bound A, the exact maximum E
+        float hm[CH];
+        float am = 0.0f;
 #pragma unroll
-            for (int i = 0; i < CH; ++i) {
-                const int c = c0 + cstep * i;
-                if (c < nch) {
-                    float x[V], f[V];
+        for (int i = 0; i < CH; ++i) {
+            const int c = c0 + cstep * i;
+            hm[i] = 0.0f;
+            if (c < nch) {
+                if constexpr (BF) {
+                    const uint4 fb = *reinterpret_cast<const uint4 *>(fb_sm + static_cast<int64_t>(c) * 4);
+                    uint32_t p = bf2_mul(raw[i].x & 0x7FFF7FFFu, fb.x);
+                    p = bf2_max(p, bf2_mul(raw[i].y & 0x7FFF7FFFu, fb.y));
+                    p = bf2_max(p, bf2_mul(raw[i].z & 0x7FFF7FFFu, fb.z));
+                    p = bf2_max(p, bf2_mul(raw[i].w & 0x7FFF7FFFu, fb.w));
+                    hm[i] = bf2_hmax_f32(p);
+                } else {
+                    float x[V];
+                    float2 f2[V / 2];
                     widen<T>(raw[i], x);
-                    factor(c, f);
+                    factor_pairs(c, f2);
+                    float h = 0.0f;
 #pragma unroll
-                    for (int e = 0; e < V; ++e)
-                        m = fmaxf(m, fabsf(__fmul_rn(x[e], f[e])));
+                    for (int e = 0; e < V; e += 2) {
+                        const float2 a = f2_mul(make_float2(x[e], x[e + 1]), f2[e / 2]);
+                        h = fmaxf(h, fmaxf(fabsf(a.x), fabsf(a.y)));
+                    }
+                    hm[i] = h;
                 }
+                am = fmaxf(am, hm[i]);
             }
-            E = group_max(m);
-        } else {
-            float hmax[CH];
-            float amax = 0.0f;
+        }
+        const float A = group_max(am);
+        float E = A;  // fp32 weights: the bounds are the values themselves
+        if (BF || MODE == MODE_X) {
+            const bool exact_all = bad_divisor || !(A >= kTinyQuotient) || !(A <= 0x1.fffffep127f);
+            const float thr = __fmul_rn(A, BF ? 0.96875f : kCandidateScale);
+            float em = 0.0f;
 #pragma unroll
             for (int i = 0; i < CH; ++i) {
                 const int c = c0 + cstep * i;
-                hmax[i] = 0.0f;
-                if (c < nch && !bad_divisor) {
-                    float x[V], f[V];
-                    Chunk8 a;
-                    widen<T>(raw[i], x);
-                    factor(c, f);
-                    hmax[i] = chunk_approx<V>(x, f, a);
-                    amax = fmaxf(amax, hmax[i]);
-                }
-            }
-            const float A = group_max(amax);
-            // exact everywhere when a divisor or the row's magnitude leaves the
-            // range the approximate maximum is proven for
-            const bool exact_all = bad_divisor || A < kTinyQuotient || !(A <= 0x1.fffffep127f);
-            const float thr = __fmul_rn(A, kCandidateScale);
-            float emax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < CH; ++i) {
-                const int c = c0 + cstep * i;
-                if (c < nch && (exact_all || hmax[i] >= thr)) {
+                if (c < nch && (exact_all || hm[i] >= thr)) {
+                    Chunk8 xv;
                     float x[V];
                     widen<T>(raw[i], x);
-                    if (exact_all) {
-                        Chunk8 xv;
 #pragma unroll
-                        for (int e = 0; e < V; ++e)
-                            xv.v[e] = x[e];
-                        emax = fmaxf(emax, chunk_absmax_div(xv, s + static_cast<int64_t>(c) * V, V));
-                    } else {
-                        float f[V];
-                        factor(c, f);
-                        emax = fmaxf(emax, chunk_candidates<V>(x, f, s + static_cast<int64_t>(c) * V, thr));
-                    }
+                    for (int e = 0; e < V; ++e)
+                        xv.v[e] = x[e];
+                    const float *sc = s + static_cast<int64_t>(c) * V;
+                    em = fmaxf(em, MODE == MODE_X ? chunk_absmax_div(xv, sc, V) : chunk_absmax_mul(xv, sc, V));
                 }
             }
-            E = group_max(emax);
+            E = group_max(em);
         }
 
         // 2. scale and codes, from the registers
@@ -515,6 +563,10 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
             scale_out[row] = scale;
         const float rsc = rcp_approx(scale);
         const bool fast = scale_in_fast_range(scale) && !bad_divisor;
+        const float2 rsc2 = make_float2(rsc, rsc);
+        const float2 nrsc2 = make_float2(-rsc, -rsc);
+        const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
+        const float2 nmagic2 = make_float2(-kRoundMagic, -kRoundMagic);
         int8_t *dst = q + row * K;
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
@@ -525,18 +577,22 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
                 widen<T>(raw[i], x);
                 bool tie = !fast;
                 if (fast) {
-                    float f[V];
-                    factor(c, f);
+                    float2 f2[V / 2];
+                    factor_pairs(c, f2);
                     float dmax = 0.0f;
 #pragma unroll
-                    for (int e = 0; e < V; ++e) {
-                        const float a = __fmul_rn(x[e], f[e]);
-                        const float yy = __fmaf_rn(a, rsc, kRoundMagic);
-                        const float rr = __fsub_rn(yy, kRoundMagic);
-                        dmax = fmaxf(dmax, fabsf(__fmaf_rn(a, rsc, -rr)));
-                        y[e] = __float_as_uint(yy);
+                    for (int e = 0; e < V; e += 2) {
+                        // yy = RN(a * rsc + 1.5*2^23): a*rsc rounded half-even to an
+                        // integer r (the code is yy's low byte); dd = r - a*rsc
+                        const float2 a = f2_mul(make_float2(x[e], x[e + 1]), f2[e / 2]);
+                        const float2 yy = f2_fma(a, rsc2, magic2);
+                        const float2 rr = f2_add(yy, nmagic2);
+                        const float2 dd = f2_fma(a, nrsc2, rr);
+                        dmax = fmaxf(dmax, fmaxf(fabsf(dd.x), fabsf(dd.y)));
+                        y[e] = __float_as_uint(yy.x);
+                        y[e + 1] = __float_as_uint(yy.y);
                     }
-                    tie = !(dmax < kTieLimit);
+                    tie = !(dmax < kTieLimit);  // NaN (scale too small) also takes the exact path
                 }
                 if (tie) {
                     Chunk8 xv;

@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                        void *__restrict__ y, int M, int N, int K, int splits, int kb_per_split,
                        int stages, int kbs)
 {
+    pdl_prologue();
     static_assert(BNX % 32 == 0 && BNX <= 128, "token tile");
     static_assert(!FUSED || BNX == 32, "the fused prologue handles up to 32 tokens");
     // NACC independent accumulators: consecutive MMAs rotate over them so no
