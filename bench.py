@@ -10,10 +10,10 @@ bf16 out):
   1. calibration absmax over the 65536-token batch      (sq_calib_absmax)
   2. smoothing factors for each linear                    (sq_smooth_factors)
   3. smoothed per-output-channel int8 weights             (sq_smooth_quant_weight)
-  4. for every token count M and linear: the online linear
-       M <= 32: sq_linear (activation quant fused into the GEMM kernel)
-       M >  32: sq_quant_act then sq_w8a8_gemm (what sq_linear runs, split so
-                the GEMM kernel can be timed on its own)
+  4. for every token count M and linear: the online linear, sq_quant_act
+     then sq_w8a8_gemm (the two kernels sq_linear runs, called separately so
+     the GEMM kernel can be timed on its own; with SQ_LINEAR_FUSED=1 up to 32
+     tokens run sq_linear's fused kernel instead)
 
 value = int8 operations of all GEMMs in the step (2 M N K each) / step time,
 in TOPS, inputs resident in HBM.  e2e = the same through the same C-ABI calls

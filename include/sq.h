@@ -173,8 +173,10 @@ SQ_API sq_status sq_w8a8_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M,
  *   bytes (may be NULL when that size is 0), 16-byte aligned, owned by the
  *   caller and not read by the caller afterwards; calls that run concurrently
  *   need separate workspaces.
- * Small M (decode) quantises the activations inside the GEMM kernel and needs
- * no workspace.
+ * Two kernels run back to back (the second launch overlaps the first);
+ * the workspace holds the int8 activations and their scales in between.
+ * With the environment variable SQ_LINEAR_FUSED=1, up to 32 tokens are
+ * instead quantised inside the GEMM kernel (no workspace; slower on B200).
  */
 SQ_API sq_status sq_linear(const void *x, sq_dtype in_dt, const float *s, const int8_t *wq,
                     const float *sw, int64_t M, int64_t N, int64_t K, void *y, sq_dtype out_dt,

@@ -340,13 +340,15 @@ def test_quant_act_fast_path_edges(oracle, s_kind):
     xq_o, sx_o = oracle.quant_act(x, s_np)
     assert_bits_equal(to_np(sx), sx_o, "sx")
     assert_bits_equal(to_np(xq), xq_o, "xq")
-    # the fused decode path (all rows fit one call) on the same inputs
+    # the online linear on the same inputs (quantiser, then GEMM)
     wq = wls.random_int8((64, K), seed=7)
     sw = np.full(64, 1e-3, np.float32)
     y = torch.empty(x.shape[0], 64, dtype=torch.float32, device="cuda")
-    sq.sq_linear(to_dev(x), to_dev(s_np), wq.cuda(), to_dev(sw), y)
+    need = sq.sq_linear_workspace_size(x.shape[0], 64, K)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
+    sq.sq_linear(to_dev(x), to_dev(s_np), wq.cuda(), to_dev(sw), y, ws if need else None)
     acc_o = oracle.gemm_i32(xq_o, to_np(wq))
-    assert_output_close(to_np(y), oracle.dequant(acc_o, sx_o, sw, "f32"), "fused linear")
+    assert_output_close(to_np(y), oracle.dequant(acc_o, sx_o, sw, "f32"), "linear")
 
 
 @pytest.mark.parametrize("s_kind", ["ones", "random", "extreme"])

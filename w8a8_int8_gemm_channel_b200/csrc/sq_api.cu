@@ -438,17 +438,17 @@ SplitPlan plan_splitk(KernelT kernel, int64_t N, int64_t K)
     return best;
 }
 
-template <int BNX, int OUT, bool FUSED, typename TIN>
+template <int BNX, int OUT, bool FUSED, typename TIN, bool LSU = false>
 sq_status launch_splitk_cfg(const TIN *x, const float *s, const int8_t *xq, const float *sx,
                             const int8_t *wq, const float *sw, int64_t M, int64_t N, int64_t K,
                             void *y, cudaStream_t st)
 {
-    auto kernel = sq::gemm_splitk_kernel<BNX, OUT, FUSED, TIN>;
+    auto kernel = sq::gemm_splitk_kernel<BNX, OUT, FUSED, TIN, LSU>;
     static std::atomic<uint64_t> attr_done{0};
     if (!ensure_smem_attr(kernel, kMaxDynSmem, attr_done))
         return SQ_ERR_CUDA;
     const SplitPlan p = plan_splitk<BNX, FUSED>(kernel, N, K);
-    if (!p.ok)
+    if (!p.ok || (LSU && p.kbs != 1))
         return SQ_ERR_UNSUPPORTED;
     if (debug_plan())
         std::fprintf(stderr, "[sq] splitk BNX=%d fused=%d M=%lld N=%lld K=%lld: splits=%d kb/split=%d stages=%d kbs=%d smem=%d clusters=%lld active=%d\n",
@@ -463,7 +463,7 @@ sq_status launch_splitk_cfg(const TIN *x, const float *s, const int8_t *xq, cons
         return SQ_ERR_CUDA;
     const int64_t n_tiles = (N + sq::kBM - 1) / sq::kBM;
     return launch_kernel(kernel, dim3(static_cast<unsigned>(n_tiles * p.splits)), dim3(sq::kSplitThreads), p.smem, st,
-                         p.splits, 1, tw, tx, x, s, sx, sw, y, static_cast<int>(M), static_cast<int>(N),
+                         p.splits, 1, tw, tx, wq, xq, x, s, sx, sw, y, static_cast<int>(M), static_cast<int>(N),
                          static_cast<int>(K), p.splits, p.kbps, p.stages, p.kbs);
 }
 
@@ -524,12 +524,17 @@ sq_status launch_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const
                       int64_t M, int64_t N, int64_t K, void *y, cudaStream_t st)
 {
     const float *nf = nullptr;
+    // weight tiles through the load/store unit (cp.async) or TMA
+    static const bool lsu = std::getenv("SQ_SPLITK_LSU") && std::atoi(std::getenv("SQ_SPLITK_LSU")) == 1;
     if (M <= 32)
-        return launch_splitk_cfg<32, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
+        return lsu ? launch_splitk_cfg<32, OUT, false, float, true>(nf, nf, xq, sx, wq, sw, M, N, K, y, st)
+                   : launch_splitk_cfg<32, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
     if (M <= 64)
-        return launch_splitk_cfg<64, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
+        return lsu ? launch_splitk_cfg<64, OUT, false, float, true>(nf, nf, xq, sx, wq, sw, M, N, K, y, st)
+                   : launch_splitk_cfg<64, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
     if (M <= 128)
-        return launch_splitk_cfg<128, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
+        return lsu ? launch_splitk_cfg<128, OUT, false, float, true>(nf, nf, xq, sx, wq, sw, M, N, K, y, st)
+                   : launch_splitk_cfg<128, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
     DeviceInfo di;
     if (!device_info(di))
         return SQ_ERR_CUDA;
@@ -547,10 +552,15 @@ sq_status launch_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const
 }
 
 // The fused decode path (activation quant inside the GEMM, no workspace)
-// applies to at most 32 tokens when K fits the per-CTA token operand.
+// applies to at most 32 tokens when K fits the per-CTA token operand, and
+// only when selected.
 bool fused_decode_applies(int64_t M, int64_t K)
 {
-    return M <= 32 && K <= sq::kMaxSplits * (kFusedSliceBytes / (32 * sq::kBK)) * sq::kBK;
+    // off unless SQ_LINEAR_FUSED=1: on B200 the quantiser kernel followed by
+    // the split-K GEMM (launch overlapped) is faster than quantising inside
+    // the GEMM kernel's prologue
+    static const bool on = std::getenv("SQ_LINEAR_FUSED") && std::atoi(std::getenv("SQ_LINEAR_FUSED")) == 1;
+    return on && M <= 32 && K <= sq::kMaxSplits * (kFusedSliceBytes / (32 * sq::kBK)) * sq::kBK;
 }
 
 template <typename TIN>

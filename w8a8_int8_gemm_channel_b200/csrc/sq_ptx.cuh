@@ -294,6 +294,24 @@ __device__ __forceinline__ float bf2_hmax_f32(uint32_t v)
     return fmaxf(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
 
+// 16-byte asynchronous copy global -> shared through the load/store unit
+// (L2 only), zero-filling the destination when `valid` is false.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the barrier's expected count includes this arrival).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Prefetch one 2-D tile into L2 (no shared-memory destination, no completion).
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int32_t x, int32_t y)
 {

@@ -101,9 +101,15 @@ __host__ __device__ inline SplitLayout split_layout(int stages, bool fused, int 
     return L;
 }
 
-template <int BNX, int OUT, bool FUSED, typename TIN>
+// LSU: the weight and token tiles are copied by warps 4..7 with 16-byte
+// cp.async (load/store unit) straight into the swizzled operand layout
+// instead of by TMA; the epilogue runs on the same warps afterwards.
+constexpr int kLsuLoaders = 128;
+
+template <int BNX, int OUT, bool FUSED, typename TIN, bool LSU = false>
 __global__ void __launch_bounds__(kSplitThreads, 1)
     gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                       const int8_t *__restrict__ wq, const int8_t *__restrict__ xq,
                        const TIN *__restrict__ x, const float *__restrict__ s,
                        const float *__restrict__ sx, const float *__restrict__ sw,
                        void *__restrict__ y, int M, int N, int K, int splits, int kb_per_split,
@@ -151,7 +157,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < stages; ++i) {
-            mbar_init(full_bar(i), 1);
+            mbar_init(full_bar(i), LSU ? kLsuLoaders : 1);
             mbar_init(empty_bar(i), 1);
         }
         mbar_init(xready_bar, kSplitWorkers);
@@ -199,7 +205,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     const int nst = (nkb + kbs - 1) / kbs;  // stages this CTA streams
     const uint32_t a_stage = static_cast<uint32_t>(kbs) * kBM * kBK;
     const uint32_t b_stage = static_cast<uint32_t>(kbs) * BNX * kBK;
-    if (warp == 0) {
+    if (warp == 0 && !LSU) {
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
@@ -239,6 +245,8 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (LSU)
+                        fence_proxy_async_smem();  // the tiles were written through the generic proxy
                     tc_fence_after_sync();
                     const int cnt = min(kbs, nkb - g * kbs);
                     for (int i = 0; i < cnt; ++i) {
@@ -346,6 +354,49 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             }
             fence_proxy_async_smem();
             mbar_arrive(xready_bar);
+        }
+    }
+
+    if constexpr (LSU) {
+        // ---- weight and token tiles through the load/store unit ------------
+        // thread t copies 16-byte chunk (t & 7) of rows (t >> 3) + 16 i of the
+        // 128-byte k block, to the position the 128-byte swizzle gives it
+        if (warp >= 4) {
+            const int t = static_cast<int>(threadIdx.x) - 128;
+            const int j = t & 7;
+            const int rbase = t >> 3;
+            const int64_t n0 = static_cast<int64_t>(n_blk) * kBM;
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int g = 0; g < nkb; ++g) {
+                if (!bounded_wait(empty_bar(stage), phase ^ 1u, kErrWaitProducer, abort_flag))
+                    break;
+                const int64_t kk = static_cast<int64_t>(kb0 + g) * kBK + j * 16;
+                const bool kv = kk < K;
+                const uint32_t sa = sA + stage * (kBM * kBK);
+#pragma unroll
+                for (int i = 0; i < kBM / 16; ++i) {
+                    const int r = rbase + 16 * i;
+                    const int64_t n = n0 + r;
+                    const bool v = kv && n < N;
+                    cp_async_16(sa + (r >> 3) * 1024u + (r & 7) * 128u + (((j ^ r) & 7) << 4), wq + (v ? n * K + kk : 0),
+                                v);
+                }
+                const uint32_t sb = sB + stage * (BNX * kBK);
+#pragma unroll
+                for (int i = 0; i < BNX / 16; ++i) {
+                    const int r = rbase + 16 * i;
+                    const bool v = kv && r < M;
+                    cp_async_16(sb + (r >> 3) * 1024u + (r & 7) * 128u + (((j ^ r) & 7) << 4),
+                                xq + (v ? static_cast<int64_t>(r) * K + kk : 0), v);
+                }
+                cp_async_arrive(full_bar(stage));
+                if (++stage == stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            cp_async_wait_all();  // nothing of this thread's is in flight past here
         }
     }
 
