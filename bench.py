@@ -57,11 +57,16 @@ DEFAULT_WORKLOAD = "llama3_8b_attn"
 INT8_PER_BF16 = 2.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic per launch of the prefill GEMM kernel, from the committed ncu
-# summary named below (dram__bytes_read.sum + dram__bytes_write.sum), keyed by
-# (M, N, K).  Empty until a capture of the current kernel exists.
-GEMM_TRAFFIC_BYTES = {}
-GEMM_TRAFFIC_SOURCE = None
+# DRAM traffic per launch of the prefill GEMM kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum), keyed by (M, N, K), from the ncu capture summarised
+# in the profile named below.
+GEMM_TRAFFIC_BYTES = {
+    (1024, 6144, 4096): 29417216 + 256,
+    (1024, 4096, 4096): 21018880 + 0,
+    (4096, 6144, 4096): 42038528 + 3244032,
+    (4096, 4096, 4096): 33625600 + 16128,
+}
+GEMM_TRAFFIC_SOURCE = "profiles/gemm_i8_pair_4096x6144x4096.md"
 
 
 # ---------------------------------------------------------------------------
@@ -697,10 +702,11 @@ def main():
     int8_peak = INT8_PER_BF16 * peaks["bf16_tflops_sustained"]
     achieved = g_ops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
     roofline = {
-        "kernel": "gemm_i8_kernel (tcgen05.mma kind::i8, prefill tiles 128x256)",
+        "kernel": "gemm_i8_pair_kernel (tcgen05.mma.cta_group::2 kind::i8, 256-row tiles on CTA pairs)",
         "bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s",
         "frac": (achieved / int8_peak) if achieved else None,
         "traffic": (sum(g_traffic) / len(g_traffic)) if len(g_traffic) == g_n and g_n else None,
+        "traffic_source": GEMM_TRAFFIC_SOURCE,
         "peak_note": f"int8 dense = 2 x {peaks['source']} sustained bf16 cuBLAS "
                      f"({peaks['bf16_tflops_sustained']:.0f} TFLOP/s); 'TFLOP/s' here counts int8 ops",
         "launches": g_n, "avg_launch_us": g_ms / max(g_n, 1) * 1e3,

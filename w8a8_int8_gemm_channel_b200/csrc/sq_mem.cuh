@@ -108,16 +108,20 @@ __device__ __forceinline__ uint4 ld_chunk(const T *p)
 template <typename T>
 __device__ __forceinline__ void widen(const uint4 &u, float (&v)[Vec<T>::N]);
 
+// bf16 bits -> fp32: the low half moved up by a byte permute (no shift), the
+// high half masked
+__device__ __forceinline__ uint32_t bf16_lo_bits(uint32_t u) { return __byte_perm(u, 0u, 0x1044u); }
+
 template <>
 __device__ __forceinline__ void widen<__nv_bfloat16>(const uint4 &u, float (&v)[8])
 {
-    v[0] = __uint_as_float(u.x << 16);
+    v[0] = __uint_as_float(bf16_lo_bits(u.x));
     v[1] = __uint_as_float(u.x & 0xFFFF0000u);
-    v[2] = __uint_as_float(u.y << 16);
+    v[2] = __uint_as_float(bf16_lo_bits(u.y));
     v[3] = __uint_as_float(u.y & 0xFFFF0000u);
-    v[4] = __uint_as_float(u.z << 16);
+    v[4] = __uint_as_float(bf16_lo_bits(u.z));
     v[5] = __uint_as_float(u.z & 0xFFFF0000u);
-    v[6] = __uint_as_float(u.w << 16);
+    v[6] = __uint_as_float(bf16_lo_bits(u.w));
     v[7] = __uint_as_float(u.w & 0xFFFF0000u);
 }
 

@@ -291,7 +291,7 @@ __device__ __forceinline__ uint32_t bf2_max(uint32_t a, uint32_t b)
 // the larger half of a pair of non-negative bf16 values, as fp32 (exact)
 __device__ __forceinline__ float bf2_hmax_f32(uint32_t v)
 {
-    return fmaxf(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+    return fmaxf(__uint_as_float(__byte_perm(v, 0u, 0x1044u)), __uint_as_float(v & 0xFFFF0000u));
 }
 
 // 16-byte asynchronous copy global -> shared through the load/store unit
