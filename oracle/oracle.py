@@ -67,6 +67,8 @@ def _load():
             lib.sqo_gemm_i32_pairs.argtypes = [P, I, P, I, P, P, I, P]
             lib.sqo_dequant.argtypes = [P, P, P, I, I, P, P]
             lib.sqo_dequant_pairs.argtypes = [P, P, P, I, P, P]
+            lib.sqo_fold_gamma.argtypes = [P, P, I, P]
+            lib.sqo_rmsnorm_quant.argtypes = [P, ctypes.c_int, I, I, P, ctypes.c_float, P, P, P]
             lib.sqo_f32_to_bf16.argtypes = [ctypes.c_float]
             lib.sqo_f32_to_bf16.restype = ctypes.c_uint16
             lib.sqo_num_threads.restype = ctypes.c_int
@@ -164,6 +166,30 @@ def quant_act(x: np.ndarray, s: np.ndarray, rows=None):
     sx = np.empty(R, np.float32)
     _load().sqo_quant_act_rows(_ptr(x), _dt(x), K, K, _ptr(s), _ptr(r), R, _ptr(xq), _ptr(sx))
     return xq, sx
+
+
+def fold_gamma(gamma: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """g = gamma / s per channel (fp32): RMSNorm's gamma with the smoothing folded in."""
+    gamma = _c(gamma, np.float32)
+    s = _c(s, np.float32)
+    assert gamma.shape == s.shape and gamma.ndim == 1
+    g = np.empty_like(gamma)
+    _load().sqo_fold_gamma(_ptr(gamma), _ptr(s), gamma.size, _ptr(g))
+    return g
+
+
+def rmsnorm_quant(h: np.ndarray, g: np.ndarray, eps: float):
+    """RMSNorm of each token row with the folded gamma g, then per-token int8
+    quantisation.  Returns (xq int8 [M, K], sx fp32 [M], rinv fp32 [M])."""
+    h = _c(h)
+    g = _c(g, np.float32)
+    M, K = h.shape
+    assert g.shape == (K,)
+    xq = np.empty((M, K), np.int8)
+    sx = np.empty(M, np.float32)
+    rinv = np.empty(M, np.float32)
+    _load().sqo_rmsnorm_quant(_ptr(h), _dt(h), M, K, _ptr(g), float(eps), _ptr(xq), _ptr(sx), _ptr(rinv))
+    return xq, sx, rinv
 
 
 def gemm_i32(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:

@@ -35,6 +35,10 @@
  *   [C]  "How does SmoothQuant int8 LLM calibration work...", section "The
  *        Technical Workflow for Int8 Quantization Deployment": calibration
  *        records the maximum absolute value of every channel.
+ *   [R]  "Understanding W8A8 INT8 LLM Quantization", section "Where the
+ *        outlier actually comes from": RMSNorm (divide by the vector's
+ *        root-mean-square, multiply by gamma) and SmoothQuant's division of
+ *        gamma by s.
  *
  * The smoothing-factor equation itself did not survive the page's text
  * extraction; this oracle uses s_j = A_j^alpha / B_j^(1-alpha), with A_j the
@@ -254,6 +258,64 @@ void sqo_dequant_pairs(const int32_t *acc, const float *sx, const float *sw, int
             y_f32[i] = y;
         if (y_bf16)
             y_bf16[i] = sqo_f32_to_bf16(y);
+    }
+}
+
+/* [R] "Understanding W8A8 INT8 LLM Quantization", section "Where the
+ * outlier actually comes from": RMSNorm divides every value of a token's
+ * vector by the vector's root-mean-square, then multiplies channel j by the
+ * trained gamma_j; SmoothQuant divides gamma by the smoothing factors s, so
+ * the norm's output is already the smoothed activation.
+ *   g[j] = gamma[j] / s[j]   (one IEEE fp32 division per channel, offline) */
+void sqo_fold_gamma(const float *gamma, const float *s, int64_t K, float *g)
+{
+    for (int64_t j = 0; j < K; ++j)
+        g[j] = gamma[j] / s[j];
+}
+
+/* [R] then [A], per token m:
+ *   ms   = (sum_k h[m, k]^2) / K in fp64 (every square is exact in fp64; the
+ *          sum runs in index order);
+ *   rinv = 1 / sqrt(ms + eps) with IEEE fp64 sqrt and division, rounded once
+ *          to fp32 (0 when ms + eps is 0: a zero row stays zero);
+ *   a    = (h[m, k] * rinv) * g[k], two fp32 multiplies;
+ *   sx   = max_k |a| / 127;  xq = clamp(round(a / sx), -127, 127).
+ * rinv_out (may be NULL) receives rinv per token. */
+void sqo_rmsnorm_quant(const void *h, int dt, int64_t M, int64_t K, const float *g, float eps,
+                       int8_t *xq, float *sx, float *rinv_out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double v = (double)elem(h, dt, (size_t)(m * K + k));
+            ss += v * v;
+        }
+        double ms = ss / (double)K + (double)eps;
+        float rinv = ms > 0.0 ? (float)(1.0 / sqrt(ms)) : 0.0f;
+        if (rinv_out)
+            rinv_out[m] = rinv;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf((elem(h, dt, (size_t)(m * K + k)) * rinv) * g[k]);
+            if (a > amax)
+                amax = a;
+        }
+        float scale = amax / 127.0f;
+        sx[m] = scale;
+        for (int64_t k = 0; k < K; ++k) {
+            int8_t q = 0;
+            if (amax != 0.0f) {
+                float a = (elem(h, dt, (size_t)(m * K + k)) * rinv) * g[k];
+                float r = nearbyintf(a / scale);
+                if (r > 127.0f)
+                    r = 127.0f;
+                if (r < -127.0f)
+                    r = -127.0f;
+                q = (int8_t)r;
+            }
+            xq[m * K + k] = q;
+        }
     }
 }
 

@@ -389,3 +389,97 @@ def test_linear_end_to_end_small(oracle):
     ref = oracle.fp64_reference_linear(x, w)
     assert y.shape == (16, 256) and y.dtype == np.float32
     assert np.linalg.norm(y - ref) / np.linalg.norm(ref) < 0.05
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm with gamma / s folded in, then per-token quantisation ("Understanding
+# W8A8 INT8 LLM Quantization", section "Where the outlier actually comes from")
+# ---------------------------------------------------------------------------
+
+def test_rmsnorm_gamma_worked_example(oracle, golden):
+    """The page's example: gamma = [1, 1, 1, 100] turns a balanced normalised
+    vector into an outlier row that destroys three channels; dividing gamma by
+    s = [1, 1, 1, 100] restores them."""
+    g = golden("rmsnorm_gamma_example.json")
+    h = np.array([g["normalized"]], np.float32)
+    gamma = np.array(g["gamma"], np.float32)
+    s = np.array(g["s"], np.float32)
+    folded = oracle.fold_gamma(gamma, s)
+    assert folded.tolist() == g["gamma_smoothed_page"]
+    q0, _, _ = oracle.rmsnorm_quant(h, gamma, 0.0)
+    q1, _, _ = oracle.rmsnorm_quant(h, folded, 0.0)
+    assert q0[0].tolist() == g["q_unsmoothed_expected"]
+    assert q1[0].tolist() == g["q_smoothed_expected"]
+
+
+def test_rmsnorm_power_of_two_scale_invariance(oracle):
+    """With eps = 0, RMSNorm is invariant to scaling a token by any positive
+    number; scaling by 2^k is exact in floating point, so codes, scales and the
+    normalised values agree bit for bit (a missing division by the RMS fails)."""
+    rng = np.random.default_rng(41)
+    h = (rng.standard_normal((6, 640)) * 3).astype(np.float32)
+    g = rng.uniform(0.1, 4.0, 640).astype(np.float32)
+    q, sx, r = oracle.rmsnorm_quant(h, g, 0.0)
+    for k in (-20, 7, 30):
+        q2, sx2, r2 = oracle.rmsnorm_quant((h * np.float32(2.0 ** k)).astype(np.float32), g, 0.0)
+        assert np.array_equal(q, q2) and np.array_equal(sx, sx2)
+        assert np.array_equal(r2 * np.float32(2.0 ** k), r)
+
+
+def test_rmsnorm_constant_rows_and_zero_rows(oracle):
+    """A constant row +-c normalises to +-1 exactly (c a power of two), so the
+    smoothed activation is +-g; a zero row stays zero with or without eps."""
+    K = 48
+    rng = np.random.default_rng(42)
+    g = rng.uniform(0.5, 2.0, K).astype(np.float32)
+    signs = np.where(np.arange(K) % 3 == 0, -1.0, 1.0).astype(np.float32)
+    h = np.stack([signs * 8.0, signs * 0.125, np.zeros(K), np.zeros(K)]).astype(np.float32)
+    q, sx, r = oracle.rmsnorm_quant(h[:3], g, 0.0)
+    assert r[0] == np.float32(0.125) and r[1] == np.float32(8.0) and r[2] == 0.0
+    qa, sxa = oracle.quant_act((signs * g)[None, :].astype(np.float32), np.ones(K, np.float32))
+    assert np.array_equal(q[0], qa[0]) and sx[0] == sxa[0]
+    assert np.array_equal(q[1], qa[0]) and sx[1] == sxa[0]
+    assert not q[2].any() and sx[2] == 0.0
+    q, sx, r = oracle.rmsnorm_quant(h[2:], g, 1e-5)
+    assert not q.any() and not sx.any()
+    assert r[0] == np.float32(1.0 / np.sqrt(np.float64(np.float32(1e-5))))
+
+
+def test_rmsnorm_against_fp64_closed_form(oracle):
+    """max |a| = 127 sx against the exact max_k |h_k| g_k / sqrt(mean(h^2) + eps)
+    in fp64 (three roundings), and every code against round(exact / sx) away
+    from ties: a sum instead of a mean, a missing square root or eps outside
+    the root all fail."""
+    rng = np.random.default_rng(43)
+    M, K, eps = 12, 1024, 1e-5
+    h = (rng.standard_normal((M, K)) * rng.uniform(0.01, 50.0, (M, 1))).astype(np.float32)
+    h[:, 17] *= 60.0
+    g = rng.uniform(0.05, 3.0, K).astype(np.float32)
+    q, sx, r = oracle.rmsnorm_quant(h, g, eps)
+    h64 = h.astype(np.float64)
+    exact = h64 / np.sqrt((h64 * h64).mean(axis=1, keepdims=True) + np.float64(np.float32(eps))) * g
+    amax = np.abs(exact).max(axis=1)
+    assert np.allclose(sx.astype(np.float64) * 127.0, amax, rtol=4 * 2.0 ** -24, atol=0)
+    t = exact / sx[:, None].astype(np.float64)
+    frac = np.abs(t - np.floor(t) - 0.5)
+    safe = frac > 1e-4
+    assert safe.mean() > 0.99
+    assert np.array_equal(q[safe], np.clip(np.rint(t[safe]), -127, 127).astype(np.int8))
+
+
+def test_rmsnorm_fold_matches_unfused_composition(oracle):
+    """Folding gamma / s into the norm gives the codes of quantising
+    X / s with X = RMSNorm(h) * gamma, except where the two fp32 rounding
+    orders straddle a tie (a fold in the wrong direction, gamma * s, fails)."""
+    rng = np.random.default_rng(44)
+    M, K = 16, 512
+    h = rng.standard_normal((M, K)).astype(np.float32)
+    gamma = rng.uniform(0.5, 1.5, K).astype(np.float32)
+    gamma[[3, 77]] *= 60.0
+    s = rng.uniform(0.5, 2.0, K).astype(np.float32)
+    s[[3, 77]] *= 40.0
+    q_fold, _, r = oracle.rmsnorm_quant(h, oracle.fold_gamma(gamma, s), 0.0)
+    x = ((h * r[:, None]) * gamma).astype(np.float32)
+    q_ref, _ = oracle.quant_act(x, s)
+    d = np.abs(q_fold.astype(np.int32) - q_ref.astype(np.int32))
+    assert d.max() <= 1 and (d == 0).mean() > 0.995
