@@ -142,6 +142,34 @@ SQ_API sq_status sq_quant_act(const void *x, sq_dtype dt, int64_t M, int64_t K, 
                        int8_t *xq, float *sx, sq_stream_t stream);
 
 /*
+ * RMSNorm's gamma with the smoothing factors folded in ("Understanding W8A8
+ * INT8 LLM Quantization", section "Where the outlier actually comes from":
+ * SmoothQuant divides the norm's gamma by s, so the norm already produces the
+ * smoothed activation):  g[j] = gamma[j] / s[j] (one IEEE fp32 division).
+ *   gamma [K], s [K], g [K] fp32 device arrays, 16-byte aligned; K a multiple
+ *   of 16.  Offline, once per linear.
+ */
+SQ_API sq_status sq_fold_gamma(const float *gamma, const float *s, int64_t K, float *g,
+                               sq_stream_t stream);
+
+/*
+ * RMSNorm with the folded gamma, then per-token int8 quantisation, in one
+ * pass over the hidden states (same page and section; the per-token scale as
+ * in sq_quant_act):
+ *   ms[m]   = sum_k h[m, k]^2 / K + eps       (squares exact in fp64, fp64 sum)
+ *   rinv[m] = RN_fp32(1 / sqrt(ms[m]))        (IEEE fp64; 0 when ms[m] is 0)
+ *   a[m, k] = (h[m, k] * rinv[m]) * g[k]      (two fp32 multiplies)
+ *   sx[m]   = max_k |a[m, k]| / 127;  xq[m, k] = clamp(round(a[m, k] / sx[m]), -127, 127)
+ *   h [M, K] dtype dt; g [K] fp32 (from sq_fold_gamma); eps >= 0 finite;
+ *   xq [M, K] int8 out; sx [M] fp32 out; rinv [M] fp32 out (may be NULL).
+ * The order of the fp64 sum is unspecified: when the fp64 value of
+ * 1/sqrt(ms) lies at an fp32 rounding midpoint, rinv may round either way.
+ * K limits as for sq_smooth_quant_weight.
+ */
+SQ_API sq_status sq_rmsnorm_quant(const void *h, sq_dtype dt, int64_t M, int64_t K, const float *g,
+                                  float eps, int8_t *xq, float *sx, float *rinv, sq_stream_t stream);
+
+/*
  * W8A8 GEMM with the dequantising epilogue ("quant_llm_int8": int32
  * accumulation, outer product of row and column scales):
  *   acc[m, n] = sum_k xq[m, k] * wq[n, k]   (exact int32; K * 127^2 < 2^31,

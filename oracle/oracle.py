@@ -68,7 +68,7 @@ def _load():
             lib.sqo_dequant.argtypes = [P, P, P, I, I, P, P]
             lib.sqo_dequant_pairs.argtypes = [P, P, P, I, P, P]
             lib.sqo_fold_gamma.argtypes = [P, P, I, P]
-            lib.sqo_rmsnorm_quant.argtypes = [P, ctypes.c_int, I, I, P, ctypes.c_float, P, P, P]
+            lib.sqo_rmsnorm_quant.argtypes = [P, ctypes.c_int, I, I, P, ctypes.c_float, P, P, P, P]
             lib.sqo_f32_to_bf16.argtypes = [ctypes.c_float]
             lib.sqo_f32_to_bf16.restype = ctypes.c_uint16
             lib.sqo_num_threads.restype = ctypes.c_int
@@ -178,18 +178,31 @@ def fold_gamma(gamma: np.ndarray, s: np.ndarray) -> np.ndarray:
     return g
 
 
-def rmsnorm_quant(h: np.ndarray, g: np.ndarray, eps: float):
+def rmsnorm_quant(h: np.ndarray, g: np.ndarray, eps: float, rinv_in=None):
     """RMSNorm of each token row with the folded gamma g, then per-token int8
-    quantisation.  Returns (xq int8 [M, K], sx fp32 [M], rinv fp32 [M])."""
+    quantisation.  Returns (xq int8 [M, K], sx fp32 [M], rinv fp32 [M]).
+    rinv_in (fp32 [M]) replaces the computed 1/RMS when given."""
     h = _c(h)
     g = _c(g, np.float32)
     M, K = h.shape
     assert g.shape == (K,)
+    ri = None if rinv_in is None else _c(rinv_in, np.float32)
+    assert ri is None or ri.shape == (M,)
     xq = np.empty((M, K), np.int8)
     sx = np.empty(M, np.float32)
     rinv = np.empty(M, np.float32)
-    _load().sqo_rmsnorm_quant(_ptr(h), _dt(h), M, K, _ptr(g), float(eps), _ptr(xq), _ptr(sx), _ptr(rinv))
+    _load().sqo_rmsnorm_quant(_ptr(h), _dt(h), M, K, _ptr(g), float(eps), _ptr(ri), _ptr(xq), _ptr(sx), _ptr(rinv))
     return xq, sx, rinv
+
+
+def rmsnorm_rinv_fp64(h: np.ndarray, eps: float) -> np.ndarray:
+    """1 / sqrt(mean(h^2) + eps) per row in fp64 (numpy's summation order), before
+    the rounding to fp32: used to check that two rinv values one fp32 ulp apart
+    both come from an fp64 value at the rounding midpoint."""
+    h64 = _c(h).astype(np.float64) if _c(h).dtype != np.uint16 else bf16_bits_to_f32(h).astype(np.float64)
+    ms = (h64 * h64).sum(axis=1) / h64.shape[1] + np.float64(np.float32(eps))
+    with np.errstate(divide="ignore"):
+        return np.where(ms > 0, 1.0 / np.sqrt(ms), 0.0)
 
 
 def gemm_i32(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:

@@ -280,9 +280,13 @@ void sqo_fold_gamma(const float *gamma, const float *s, int64_t K, float *g)
  *          to fp32 (0 when ms + eps is 0: a zero row stays zero);
  *   a    = (h[m, k] * rinv) * g[k], two fp32 multiplies;
  *   sx   = max_k |a| / 127;  xq = clamp(round(a / sx), -127, 127).
- * rinv_out (may be NULL) receives rinv per token. */
+ * rinv_out (may be NULL) receives rinv per token.  rinv_in (may be NULL)
+ * replaces the computed rinv: the pages fix no summation order for the
+ * squares, so another order may round rinv the other way when the fp64
+ * value lies at an fp32 rounding midpoint; given the same rinv, everything
+ * after it is fixed. */
 void sqo_rmsnorm_quant(const void *h, int dt, int64_t M, int64_t K, const float *g, float eps,
-                       int8_t *xq, float *sx, float *rinv_out)
+                       const float *rinv_in, int8_t *xq, float *sx, float *rinv_out)
 {
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m) {
@@ -293,6 +297,8 @@ void sqo_rmsnorm_quant(const void *h, int dt, int64_t M, int64_t K, const float 
         }
         double ms = ss / (double)K + (double)eps;
         float rinv = ms > 0.0 ? (float)(1.0 / sqrt(ms)) : 0.0f;
+        if (rinv_in)
+            rinv = rinv_in[m];
         if (rinv_out)
             rinv_out[m] = rinv;
         float amax = 0.0f;

@@ -136,3 +136,19 @@ def test_binding_fails_loudly_without_device_tensors():
     x = torch.zeros(4, 16)
     with pytest.raises(ValueError):
         sq.sq_calib_absmax(x, torch.zeros(16))
+
+
+def test_rmsnorm_entry_points_reject_bad_arguments(lib):
+    f = lib.sq_fold_gamma
+    assert f(None, B, 64, C, None) == INV
+    assert f(A, B, 24, C, None) == INV        # K not a multiple of 16
+    assert f(A, MIS, 64, C, None) == INV      # misaligned s
+    g = lib.sq_rmsnorm_quant
+    assert g(None, 1, 4, 64, B, 1e-5, C, D, None, None) == INV
+    assert g(A, 1, 0, 64, B, 1e-5, C, D, None, None) == INV      # M < 1
+    assert g(A, 1, 4, 40, B, 1e-5, C, D, None, None) == INV      # K not a multiple of 16
+    assert g(A, 1, 4, 64, B, -1.0, C, D, None, None) == INV      # eps < 0
+    assert g(A, 1, 4, 64, B, float("nan"), C, D, None, None) == INV
+    assert g(A, 1, 4, 64, B, 1e-5, C, D, MIS, None) == INV       # misaligned rinv
+    assert g(A, 7, 4, 64, B, 1e-5, C, D, None, None) == INV      # bad dtype
+    assert g(A, 1, 4, 65536, B, 1e-5, C, D, None, None) == UNS   # row too long for one pass

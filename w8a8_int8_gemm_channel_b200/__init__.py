@@ -44,6 +44,8 @@ ABI_SYMBOLS = (
     "sq_smooth_factors",
     "sq_smooth_quant_weight",
     "sq_quant_act",
+    "sq_fold_gamma",
+    "sq_rmsnorm_quant",
     "sq_w8a8_gemm",
     "sq_w8a8_gemm_s32",
     "sq_linear",
@@ -74,6 +76,8 @@ def _declare(lib):
         "sq_smooth_factors": ([P, P, E, I, I, F, P, P, P], E),
         "sq_smooth_quant_weight": ([P, E, I, I, P, P, P, P], E),
         "sq_quant_act": ([P, E, I, I, P, P, P, P], E),
+        "sq_fold_gamma": ([P, P, I, P, P], E),
+        "sq_rmsnorm_quant": ([P, E, I, I, P, F, P, P, P, P], E),
         "sq_w8a8_gemm": ([P, P, P, P, I, I, I, P, E, P], E),
         "sq_w8a8_gemm_s32": ([P, P, I, I, I, P, P], E),
         "sq_linear": ([P, E, P, P, P, I, I, I, P, E, P, ctypes.c_size_t, P], E),
@@ -173,6 +177,18 @@ def sq_quant_act(x, s, xq, sx, stream=None):
     _check("sq_quant_act",
            lib().sq_quant_act(_ptr(x), _dtype_code(x), M, K, _ptr(s), _ptr(xq), _ptr(sx),
                               _stream(stream)))
+
+
+def sq_fold_gamma(gamma, s, g, stream=None):
+    K = gamma.shape[0]
+    _check("sq_fold_gamma", lib().sq_fold_gamma(_ptr(gamma), _ptr(s), K, _ptr(g), _stream(stream)))
+
+
+def sq_rmsnorm_quant(h, g, eps, xq, sx, rinv=None, stream=None):
+    M, K = h.shape
+    _check("sq_rmsnorm_quant",
+           lib().sq_rmsnorm_quant(_ptr(h), _dtype_code(h), M, K, _ptr(g), float(eps), _ptr(xq), _ptr(sx),
+                                  None if rinv is None else _ptr(rinv), _stream(stream)))
 
 
 def sq_w8a8_gemm(xq, sx, wq, sw, y, stream=None):

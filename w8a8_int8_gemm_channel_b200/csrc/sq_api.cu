@@ -613,6 +613,51 @@ void *noalloc_scratch()
     return addr[dev];
 }
 
+// Fused RMSNorm + quantiser: 2^log2g warps per row, CH chunks per lane.
+template <typename T, int CH>
+sq_status launch_rmsnorm_quant_cfg(const T *h, int64_t rows, int64_t K, const float *g, float eps, int8_t *q,
+                                   float *sx, float *rinv, int log2g, cudaStream_t st, const DeviceInfo &di)
+{
+    auto kernel = sq::rmsnorm_quant_kernel<T, CH>;
+    const int smem = static_cast<int>(K * 4);
+    static std::atomic<uint64_t> attr_done{0};
+    if (!ensure_smem_attr(kernel, kMaxDynSmem - 1024, attr_done))
+        return SQ_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, sq::kQuantThreads, smem) != cudaSuccess ||
+        per_sm < 1) {
+        cudaGetLastError();
+        return SQ_ERR_CUDA;
+    }
+    while (log2g < 3 && rows * (1 << log2g) < (int64_t)di.sms * per_sm * (sq::kQuantThreads / 32))
+        ++log2g;
+    const int slots = (sq::kQuantThreads / 32) >> log2g;
+    const int64_t blocks = std::min<int64_t>((rows + slots - 1) / slots, (int64_t)per_sm * di.sms);
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(sq::kQuantThreads), smem, st, 0, 0, h, rows,
+                         K, g, eps, log2g, q, sx, rinv);
+}
+
+template <typename T>
+sq_status launch_rmsnorm_quant(const T *h, int64_t rows, int64_t K, const float *g, float eps, int8_t *q, float *sx,
+                               float *rinv, cudaStream_t st)
+{
+    DeviceInfo di;
+    if (!device_info(di))
+        return SQ_ERR_CUDA;
+    constexpr int V = sq::Vec<T>::N;
+    const int64_t nch = K / V;
+    for (int ch : {8, 16}) {
+        int log2g = 0;
+        while (log2g < 3 && ((int64_t)32 * ch << log2g) < nch)
+            ++log2g;
+        if (((int64_t)32 * ch << log2g) < nch)
+            continue;
+        return ch == 8 ? launch_rmsnorm_quant_cfg<T, 8>(h, rows, K, g, eps, q, sx, rinv, log2g, st, di)
+                       : launch_rmsnorm_quant_cfg<T, 16>(h, rows, K, g, eps, q, sx, rinv, log2g, st, di);
+    }
+    return SQ_ERR_UNSUPPORTED;
+}
+
 }  // namespace
 
 extern "C" {
@@ -701,6 +746,36 @@ sq_status sq_quant_act(const void *x, sq_dtype dt, int64_t M, int64_t K, const f
         return launch_quant_rows<__nv_bfloat16, sq::MODE_X>(static_cast<const __nv_bfloat16 *>(x),
                                                              M, K, s, xq, sx, st);
     return launch_quant_rows<float, sq::MODE_X>(static_cast<const float *>(x), M, K, s, xq, sx, st);
+}
+
+sq_status sq_fold_gamma(const float *gamma, const float *s, int64_t K, float *g, sq_stream_t stream)
+{
+    if (gamma == nullptr || s == nullptr || g == nullptr || K < 16 || K % 16 != 0 || !aligned16(gamma) ||
+        !aligned16(s) || !aligned16(g))
+        return SQ_ERR_INVALID_ARG;
+    if (K > kMaxDim)
+        return SQ_ERR_UNSUPPORTED;
+    const unsigned threads = 256;
+    const unsigned blocks = static_cast<unsigned>((K + threads - 1) / threads);
+    return launch_kernel(sq::fold_gamma_kernel, dim3(blocks), dim3(threads), 0, reinterpret_cast<cudaStream_t>(stream),
+                         0, 0, gamma, s, g, K);
+}
+
+sq_status sq_rmsnorm_quant(const void *h, sq_dtype dt, int64_t M, int64_t K, const float *g, float eps,
+                           int8_t *xq, float *sx, float *rinv, sq_stream_t stream)
+{
+    if (h == nullptr || g == nullptr || xq == nullptr || sx == nullptr || !valid_dtype(dt) || M < 1 || K < 16 ||
+        K % 16 != 0 || !aligned16(h) || !aligned16(g) || !aligned16(xq) || !aligned16(sx) ||
+        (rinv != nullptr && !aligned16(rinv)) || !(eps >= 0.0f) || !(eps <= 3.0e38f))
+        return SQ_ERR_INVALID_ARG;
+    // one row of 16 chunks per lane over 8 warps; g staged in shared memory
+    const int64_t kmax = dt == SQ_BF16 ? 32768 : 16384;
+    if (K > kmax || M > kMaxDim)
+        return SQ_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dt == SQ_BF16)
+        return launch_rmsnorm_quant(static_cast<const __nv_bfloat16 *>(h), M, K, g, eps, xq, sx, rinv, st);
+    return launch_rmsnorm_quant(static_cast<const float *>(h), M, K, g, eps, xq, sx, rinv, st);
 }
 
 sq_status sq_w8a8_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,

@@ -245,6 +245,19 @@ __global__ void __launch_bounds__(kColThreads) col_absmax_kernel(const T *__rest
 }
 
 // ----------------------------------------------------------------------------
+// RMSNorm gamma with the smoothing folded in: g_j = gamma_j / s_j (one IEEE
+// fp32 division per channel).
+// ----------------------------------------------------------------------------
+__global__ void fold_gamma_kernel(const float *__restrict__ gamma, const float *__restrict__ s,
+                                  float *__restrict__ g, int64_t K)
+{
+    pdl_prologue();
+    const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (j < K)
+        g[j] = __fdiv_rn(gamma[j], s[j]);
+}
+
+// ----------------------------------------------------------------------------
 // Smoothing factors, in place: on entry s holds B_j (as written by the
 // column-absmax kernel); on exit s_j = A_j^alpha / B_j^(1-alpha) evaluated in
 // fp64 and rounded once, or 1 where A_j or B_j is 0.  aw (optional) receives B_j.
@@ -381,6 +394,16 @@ __device__ __noinline__ float chunk_absmax_mul(Chunk8 x, const float *__restrict
     for (int e = 0; e < n; ++e)
         m = fmaxf(m, fabsf(__fmul_rn(x.v[e], __ldg(s_chunk + e))));
     return m;
+}
+
+// Exact codes of one chunk of known values (rare: near ties, scales outside
+// the fast range).
+__device__ __noinline__ Chunk8 chunk_codes_of_values(Chunk8 a, int n, float scale)
+{
+    Chunk8 y;
+    for (int e = 0; e < n; ++e)
+        y.v[e] = __uint_as_float(scale != 0.0f ? exact_code_bits(a.v[e], scale) : code_bits(0.0f));
+    return y;
 }
 
 // Approximate magnitudes a = RN(|x| * r) of one chunk and their maximum.

@@ -618,4 +618,187 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
     }
 }
 
+// ----------------------------------------------------------------------------
+// RMSNorm with gamma / s folded in, then per-token int8 quantisation: one
+// read of each token's hidden vector h, written as codes and a scale.
+//   ms   = sum_k h_k^2 / K + eps   (squares exact in fp64, fp64 sums)
+//   rinv = RN_f32(1 / sqrt(ms))    (IEEE fp64 sqrt and division; 0 if ms = 0)
+//   a_k  = RN(RN(h_k * rinv) * g_k)
+//   scale = RN(max |a| / 127),  code = clamp(rne(RN(a / scale)), -127, 127)
+// a is computed exactly, so its maximum needs no candidate pass; the codes use
+// the rounding fast path of sq_div.cuh with the exact fallback near ties.
+// Same row layout as row_quant_kernel: G = 2^log2g warps per row, the row in
+// registers, g staged in shared memory.
+// ----------------------------------------------------------------------------
+template <typename T, int CH>
+__global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
+    rmsnorm_quant_kernel(const T *__restrict__ in, int64_t rows, int64_t K, const float *__restrict__ gam,
+                         float eps, int log2g, int8_t *__restrict__ q, float *__restrict__ scale_out,
+                         float *__restrict__ rinv_out)
+{
+    pdl_prologue();
+    constexpr int V = Vec<T>::N;
+    constexpr int WARPS = kQuantThreads / 32;
+    extern __shared__ float4 smem_f4[];
+    float *g_sm = reinterpret_cast<float *>(smem_f4);
+    __shared__ float red[2][WARPS];
+    __shared__ double redd[2][WARPS];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = 1 << log2g;
+    const int slot = warp >> log2g;
+    const int g = warp & (G - 1);
+    const int slots = WARPS >> log2g;
+    const int nch = static_cast<int>(K / V);
+    const int c0 = 32 * g + lane;
+    const int cstep = 32 * G;
+    int64_t row = static_cast<int64_t>(blockIdx.x) * slots + slot;
+    const int64_t rstride = static_cast<int64_t>(gridDim.x) * slots;
+
+    uint4 raw[CH];
+    auto load_row = [&](int64_t r) {
+        const T *src = in + r * K;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int c = c0 + cstep * i;
+            raw[i] = c < nch ? ld_chunk<T>(src + static_cast<int64_t>(c) * V) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    if (row < rows)
+        load_row(row);
+    {
+        const float4 *g4 = reinterpret_cast<const float4 *>(gam);
+        for (int j = threadIdx.x; j < static_cast<int>(K / 4); j += blockDim.x)
+            reinterpret_cast<float4 *>(g_sm)[j] = __ldg(g4 + j);
+    }
+    __syncthreads();
+    auto gvals = [&](int c, float (&f)[V]) {
+#pragma unroll
+        for (int h = 0; h < V / 4; ++h) {
+            const float4 v4 = reinterpret_cast<const float4 *>(g_sm + static_cast<int64_t>(c) * V)[h];
+            f[4 * h] = v4.x;
+            f[4 * h + 1] = v4.y;
+            f[4 * h + 2] = v4.z;
+            f[4 * h + 3] = v4.w;
+        }
+    };
+    // reductions over the G warps of this row (alternating buffers, as in row_quant_kernel)
+    int nred = 0;
+    auto group_max = [&](float v) -> float {
+        v = warp_max(v);
+        if (G == 1)
+            return v;
+        float *r = red[nred & 1];
+        ++nred;
+        if (lane == 0)
+            r[warp] = v;
+        named_barrier_sync(1 + slot, 32 * G);
+        float m = r[slot << log2g];
+        for (int j = 1; j < G; ++j)
+            m = fmaxf(m, r[(slot << log2g) + j]);
+        return m;
+    };
+    int nredd = 0;
+    auto group_sum = [&](double v) -> double {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            v = __dadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+        if (G == 1)
+            return v;
+        double *r = redd[nredd & 1];
+        ++nredd;
+        if (lane == 0)
+            r[warp] = v;
+        named_barrier_sync(1 + slot, 32 * G);
+        double t = r[slot << log2g];
+        for (int j = 1; j < G; ++j)
+            t = __dadd_rn(t, r[(slot << log2g) + j]);
+        return t;
+    };
+
+    while (row < rows) {
+        // 1. 1/RMS of the token
+        double ss = 0.0;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            if (c0 + cstep * i < nch) {
+                float x[V];
+                widen<T>(raw[i], x);
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    const double v = static_cast<double>(x[e]);
+                    ss = __fma_rn(v, v, ss);  // v*v is exact in fp64
+                }
+            }
+        }
+        ss = group_sum(ss);
+        const double ms = __dadd_rn(__ddiv_rn(ss, static_cast<double>(K)), static_cast<double>(eps));
+        const float rinv = ms > 0.0 ? __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(ms))) : 0.0f;
+        if (g == 0 && lane == 0 && rinv_out != nullptr)
+            rinv_out[row] = rinv;
+
+        // 2. the smoothed activations a and their exact maximum
+        float am = 0.0f;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int c = c0 + cstep * i;
+            if (c < nch) {
+                float x[V], f[V];
+                widen<T>(raw[i], x);
+                gvals(c, f);
+#pragma unroll
+                for (int e = 0; e < V; ++e)
+                    am = fmaxf(am, fabsf(__fmul_rn(__fmul_rn(x[e], rinv), f[e])));
+            }
+        }
+        const float E = group_max(am);
+
+        // 3. scale and codes
+        const float scale = scale_from_max(E);
+        if (g == 0 && lane == 0)
+            scale_out[row] = scale;
+        const float rsc = rcp_approx(scale);
+        const bool fast = scale_in_fast_range(scale);
+        int8_t *dst = q + row * K;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int c = c0 + cstep * i;
+            if (c < nch) {
+                float x[V], f[V], a[V];
+                uint32_t y[V];
+                widen<T>(raw[i], x);
+                gvals(c, f);
+                float dmax = 0.0f;
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    a[e] = __fmul_rn(__fmul_rn(x[e], rinv), f[e]);
+                    const float yy = __fmaf_rn(a[e], rsc, kRoundMagic);
+                    const float rr = __fsub_rn(yy, kRoundMagic);
+                    dmax = fmaxf(dmax, fabsf(__fmaf_rn(a[e], -rsc, rr)));
+                    y[e] = __float_as_uint(yy);
+                }
+                if (!fast || !(dmax < kTieLimit)) {
+                    Chunk8 av;
+#pragma unroll
+                    for (int e = 0; e < V; ++e)
+                        av.v[e] = a[e];
+                    const Chunk8 yy = chunk_codes_of_values(av, V, scale);
+#pragma unroll
+                    for (int e = 0; e < V; ++e)
+                        y[e] = __float_as_uint(yy.v[e]);
+                }
+                int8_t *dd = dst + static_cast<int64_t>(c) * V;
+                if constexpr (V == 8)
+                    *reinterpret_cast<uint2 *>(dd) = make_uint2(pack_code_bytes(y[0], y[1], y[2], y[3]),
+                                                                pack_code_bytes(y[4], y[5], y[6], y[7]));
+                else
+                    *reinterpret_cast<uint32_t *>(dd) = pack_code_bytes(y[0], y[1], y[2], y[3]);
+            }
+        }
+        row += rstride;
+        if (row < rows)
+            load_row(row);
+    }
+}
+
 }  // namespace sq
