@@ -190,9 +190,9 @@ sq_status launch_col_absmax(const T *x, int64_t R, int64_t K, int64_t ld, float 
     const int64_t chunks = K / V;
     const int64_t col_blocks = (chunks + sq::kColThreads - 1) / sq::kColThreads;
     // one wave of about 4 CTAs of 256 threads per SM, in clusters of CL row
-    // bands; bands are whole multiples of the 8 rows a thread keeps in flight
+    // bands; bands are whole multiples of the 16 rows a thread keeps in flight
     const int64_t want = std::max<int64_t>(CL, (int64_t)di.sms * 4 / col_blocks);
-    int64_t rows_per_block = std::max<int64_t>(8, ((R + want - 1) / want + 7) / 8 * 8);
+    int64_t rows_per_block = std::max<int64_t>(16, ((R + want - 1) / want + 15) / 16 * 16);
     int64_t row_blocks = (R + rows_per_block - 1) / rows_per_block;
     while (row_blocks > 65528) {
         rows_per_block *= 2;
@@ -226,11 +226,11 @@ sq_status launch_row_scale(const T *in, int64_t rows, int64_t K, const float *s,
 
 // Single-pass quantiser (row in registers): 2^log2g warps per row, CH chunks
 // per lane.
-template <typename T, int MODE, int CH>
+template <typename T, int MODE, int CH, bool FIT>
 sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
                                float *scale, int log2g, cudaStream_t st, const DeviceInfo &di)
 {
-    auto kernel = sq::row_quant_kernel<T, MODE, CH>;
+    auto kernel = sq::row_quant_kernel<T, MODE, CH, FIT>;
     const int smem = static_cast<int>(sq::row_quant_smem(K, sq::Vec<T>::N == 8));
     static std::atomic<uint64_t> attr_done{0};
     // the kernel also has a little static shared memory (the group maxima)
@@ -257,7 +257,8 @@ sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float
         occ.emplace_back(smem, per_sm);
     }
     // few rows: spread each row over more warps so that every SM has work
-    while (log2g < 3 && rows * (1 << log2g) < (int64_t)di.sms * per_sm * (sq::kQuantThreads / 32))
+    // (not for FIT, whose G is fixed by the row length)
+    while (!FIT && log2g < 3 && rows * (1 << log2g) < (int64_t)di.sms * per_sm * (sq::kQuantThreads / 32))
         ++log2g;
     const int slots = (sq::kQuantThreads / 32) >> log2g;
     const int64_t blocks = std::min<int64_t>((rows + slots - 1) / slots, (int64_t)per_sm * di.sms);
@@ -290,8 +291,14 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
                 ++log2g;
             if (((int64_t)32 * ch << log2g) < nch)
                 continue;
-            return ch == 8 ? launch_row_quant_cfg<T, MODE, 8>(in, rows, K, s, q, scale, log2g, st, di)
-                           : launch_row_quant_cfg<T, MODE, 16>(in, rows, K, s, q, scale, log2g, st, di);
+            // an exact fit drops the bounds checks; few rows rather spread over more warps
+            const bool fit = ((int64_t)32 * ch << log2g) == nch &&
+                             rows * (1 << log2g) >= (int64_t)di.sms * 2 * (sq::kQuantThreads / 32);
+            if (ch == 8)
+                return fit ? launch_row_quant_cfg<T, MODE, 8, true>(in, rows, K, s, q, scale, log2g, st, di)
+                           : launch_row_quant_cfg<T, MODE, 8, false>(in, rows, K, s, q, scale, log2g, st, di);
+            return fit ? launch_row_quant_cfg<T, MODE, 16, true>(in, rows, K, s, q, scale, log2g, st, di)
+                       : launch_row_quant_cfg<T, MODE, 16, false>(in, rows, K, s, q, scale, log2g, st, di);
         }
     }
     sq_status r = (K * (int64_t)sizeof(float) <= kSmemFactorBytes)

@@ -183,6 +183,20 @@ __global__ void __launch_bounds__(kColThreads) col_absmax_kernel(const T *__rest
         const int64_t r1 = min(R, r0 + rows_per_block);
         const T *p = x + r0 * ld + c * V;
         int64_t r = r0;
+        for (; r + 16 <= r1; r += 16, p += 16 * ld) {
+            uint4 raw[16];  // sixteen rows in flight per thread
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                raw[u] = __ldcs(reinterpret_cast<const uint4 *>(p + u * ld));
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                float a[V];
+                widen<T>(raw[u], a);
+#pragma unroll
+                for (int i = 0; i < V; ++i)
+                    m[i] = fmaxf(m[i], fabsf(a[i]));
+            }
+        }
         for (; r + 8 <= r1; r += 8, p += 8 * ld) {
             uint4 raw[8];  // eight rows in flight per thread
 #pragma unroll

@@ -436,7 +436,9 @@ __device__ __forceinline__ int stage_factor_tables(const float *__restrict__ s, 
 // bytes of shared memory the factor tables of a K-column row take
 __host__ __device__ constexpr int64_t row_quant_smem(int64_t K, bool bf) { return K * 4 + (bf ? K * 2 : 0); }
 
-template <typename T, int MODE, int CH>
+// FIT: the G warps of a row cover its chunks exactly (32 CH G = K / V), so
+// no chunk needs a bounds check.
+template <typename T, int MODE, int CH, bool FIT>
 __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
     row_quant_kernel(const T *__restrict__ in, int64_t rows, int64_t K, const float *__restrict__ s,
                      int log2g, int8_t *__restrict__ q, float *__restrict__ scale_out)
@@ -467,7 +469,7 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
             const int c = c0 + cstep * i;
-            raw[i] = c < nch ? ld_chunk<T>(src + static_cast<int64_t>(c) * V) : make_uint4(0u, 0u, 0u, 0u);
+            raw[i] = (FIT || c < nch) ? ld_chunk<T>(src + static_cast<int64_t>(c) * V) : make_uint4(0u, 0u, 0u, 0u);
         }
     };
     if (row < rows)
@@ -510,7 +512,7 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
         for (int i = 0; i < CH; ++i) {
             const int c = c0 + cstep * i;
             hm[i] = 0.0f;
-            if (c < nch) {
+            if (FIT || c < nch) {
                 if constexpr (BF) {
                     const uint4 fb = *reinterpret_cast<const uint4 *>(fb_sm + static_cast<int64_t>(c) * 4);
                     uint32_t p = bf2_mul(raw[i].x & 0x7FFF7FFFu, fb.x);
@@ -543,7 +545,7 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
 #pragma unroll
             for (int i = 0; i < CH; ++i) {
                 const int c = c0 + cstep * i;
-                if (c < nch && (exact_all || hm[i] >= thr)) {
+                if ((FIT || c < nch) && (exact_all || hm[i] >= thr)) {
                     Chunk8 xv;
                     float x[V];
                     widen<T>(raw[i], x);
@@ -571,7 +573,7 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
             const int c = c0 + cstep * i;
-            if (c < nch) {
+            if (FIT || c < nch) {
                 float x[V];
                 uint32_t y[V];
                 widen<T>(raw[i], x);
