@@ -744,45 +744,73 @@ def main():
                                            (INT8_PER_BF16 * peaks["bf16_tflops"]), 3)
             stages[name] = ent
 
-    # end to end: inputs from pinned host memory, outputs read back, every step
+    # end to end: every step's inputs copied from pinned host memory and its
+    # outputs read back.  Two device buffer sets alternate, so the upload of
+    # step i+1 (one copy stream) and the download of step i (another) overlap
+    # the computation of step i; each buffer set is reused only after the
+    # computation and the download that used it have finished.
     e2e = None
     if not args.no_e2e:
-        e2e_steps = args.e2e_steps or max(3, min(args.steps, 20))
+        e2e_steps = args.e2e_steps or max(4, min(args.steps, 20))
+        sets = [step, Step(wl, device)]
         h_xcal = step.xcal.cpu().pin_memory()
         h_w = [d["w"].cpu().pin_memory() for d in step.lins]
         h_x = [{M: x.cpu().pin_memory() for M, x in d["x"].items()} for d in step.lins]
-        h_y = [{M: torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for M, y in d["y"].items()}
-               for d in step.lins]
+        h_y = [[{M: torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for M, y in d["y"].items()}
+                for d in step.lins] for _ in range(2)]
         h2d = step.input_bytes()
         d2h = step.output_bytes()
+        s_in = torch.cuda.Stream(device)
+        s_out = torch.cuda.Stream(device)
+        ev = lambda: torch.cuda.Event(enable_timing=False)
+        done = [ev(), ev()]      # computation on set b finished
+        drained = [ev(), ev()]   # download of set b's outputs finished
 
-        def e2e_step():
-            step.xcal.copy_(h_xcal, non_blocking=True)
-            for i, d in enumerate(step.lins):
-                d["w"].copy_(h_w[i], non_blocking=True)
-                for M in wl.Ms:
-                    d["x"][M].copy_(h_x[i][M], non_blocking=True)
-            step.run(stream)
-            for i, d in enumerate(step.lins):
-                for M in wl.Ms:
-                    h_y[i][M].copy_(d["y"][M], non_blocking=True)
+        def e2e_step(i):
+            b = i % 2
+            st = sets[b]
+            loaded = ev()
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(done[b])
+                st.xcal.copy_(h_xcal, non_blocking=True)
+                for j, d in enumerate(st.lins):
+                    d["w"].copy_(h_w[j], non_blocking=True)
+                    for M in wl.Ms:
+                        d["x"][M].copy_(h_x[j][M], non_blocking=True)
+                loaded.record(s_in)
+            with torch.cuda.stream(stream):
+                stream.wait_event(loaded)
+                if i >= 2:
+                    stream.wait_event(drained[b])
+                st.run(stream)
+                done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[b])
+                for j, d in enumerate(st.lins):
+                    for M in wl.Ms:
+                        h_y[b][j][M].copy_(d["y"][M], non_blocking=True)
+                drained[b].record(s_out)
 
-        with torch.cuda.stream(stream):
-            e2e_step()
-        stream.synchronize()
+        for i in range(2):
+            e2e_step(i)
+        torch.cuda.synchronize()
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(e2e_steps):
-                e2e_step()
-            e1.record(stream)
-        stream.synchronize()
+        e0.record(s_in)
+        stream.wait_event(e0)
+        s_out.wait_event(e0)
+        for i in range(e2e_steps):
+            e2e_step(i + 2)
+        e1.record(s_out)
+        torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
         e2e = {"value": aggregate_tops(world, ops_step, e2e_steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps}
+               "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps,
+               "pipelining": "two device buffer sets; uploads, computation and downloads on three streams"}
+        del sets
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
