@@ -250,6 +250,17 @@ SQ_API sq_status sq_linear_noalloc(const void *x, sq_dtype in_dt, const float *s
  */
 SQ_API sq_status sq_device_status(sq_stream_t stream, uint32_t *code);
 
+/*
+ * Self-test of the failure detection: enqueues one tiny kernel whose single
+ * waiting thread waits on an on-chip barrier that nothing ever arrives on,
+ * with a limit of limit_us microseconds (1 .. 2000000).  The wait gives up,
+ * records the location code 0x900 in the device error word and the kernel
+ * returns, so the context stays usable; sq_device_status then reports
+ * SQ_ERR_TIMEOUT with that code.  The pages have no counterpart: this checks
+ * the library's own bounded waits.
+ */
+SQ_API sq_status sq_selftest_wait_timeout(uint32_t limit_us, sq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -152,3 +152,9 @@ def test_rmsnorm_entry_points_reject_bad_arguments(lib):
     assert g(A, 1, 4, 64, B, 1e-5, C, D, MIS, None) == INV       # misaligned rinv
     assert g(A, 7, 4, 64, B, 1e-5, C, D, None, None) == INV      # bad dtype
     assert g(A, 1, 4, 65536, B, 1e-5, C, D, None, None) == UNS   # row too long for one pass
+
+
+def test_selftest_rejects_limits_out_of_range(lib):
+    f = lib.sq_selftest_wait_timeout
+    assert f(0, None) == INV
+    assert f(2000001, None) == INV

@@ -52,6 +52,7 @@ ABI_SYMBOLS = (
     "sq_linear_workspace_size",
     "sq_linear_noalloc",
     "sq_device_status",
+    "sq_selftest_wait_timeout",
 )
 
 
@@ -84,6 +85,7 @@ def _declare(lib):
         "sq_linear_workspace_size": ([I, I, I], ctypes.c_size_t),
         "sq_linear_noalloc": ([P, E, P, P, P, I, I, I, P, E, P], E),
         "sq_device_status": ([P, ctypes.POINTER(ctypes.c_uint32)], E),
+        "sq_selftest_wait_timeout": ([ctypes.c_uint32, P], E),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -240,6 +242,10 @@ def sq_device_status(stream=None) -> Tuple[int, int]:
     code = ctypes.c_uint32(0)
     st = lib().sq_device_status(_stream(stream), ctypes.byref(code))
     return st, int(code.value)
+
+
+def sq_selftest_wait_timeout(limit_us: int, stream=None):
+    _check("sq_selftest_wait_timeout", lib().sq_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------

@@ -879,6 +879,14 @@ sq_status sq_linear_noalloc(const void *x, sq_dtype in_dt, const float *s, const
     return sq_linear(x, in_dt, s, wq, sw, M, N, K, y, out_dt, ws, need, stream);
 }
 
+sq_status sq_selftest_wait_timeout(uint32_t limit_us, sq_stream_t stream)
+{
+    if (limit_us < 1 || limit_us > 2000000)
+        return SQ_ERR_INVALID_ARG;
+    return launch_kernel(sq::wait_selftest_kernel, dim3(1), dim3(32), 0, reinterpret_cast<cudaStream_t>(stream), 0, 0,
+                         static_cast<unsigned long long>(limit_us) * 1000ull);
+}
+
 sq_status sq_device_status(sq_stream_t stream, uint32_t *code)
 {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {

@@ -259,6 +259,24 @@ __global__ void __launch_bounds__(kColThreads) col_absmax_kernel(const T *__rest
 }
 
 // ----------------------------------------------------------------------------
+// Self-test of the bounded waits: one thread waits on an mbarrier that nothing
+// arrives on, with a short limit; the wait gives up, records its location
+// code in the device error word and the kernel returns normally.
+// ----------------------------------------------------------------------------
+__global__ void wait_selftest_kernel(unsigned long long limit_ns)
+{
+    pdl_prologue();
+    __shared__ __align__(8) unsigned long long bar;
+    if (threadIdx.x == 0) {
+        const uint32_t b = smem_u32(&bar);
+        mbar_init(b, 1);
+        fence_barrier_init();
+        bounded_wait(b, 0, kErrWaitSelfTest, nullptr, limit_ns);  // phase 0 never completes
+    }
+    __syncthreads();
+}
+
+// ----------------------------------------------------------------------------
 // RMSNorm gamma with the smoothing folded in: g_j = gamma_j / s_j (one IEEE
 // fp32 division per channel).
 // ----------------------------------------------------------------------------

@@ -27,6 +27,7 @@ enum : unsigned int {
     kErrWaitCluster = 0x600,    // cross-CTA exchange inside a cluster
     kErrWaitDrain = 0x700,      // teardown drain of in-flight copies
     kErrWaitRow = 0x800,        // quantiser waiting for a staged row
+    kErrWaitSelfTest = 0x900,   // the wait-timeout self-test (nothing ever arrives)
 };
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
