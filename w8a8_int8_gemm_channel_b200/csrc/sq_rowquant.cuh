@@ -433,6 +433,66 @@ __device__ __forceinline__ int stage_factor_tables(const float *__restrict__ s, 
     return bad;
 }
 
+// Rare paths of the single-pass quantisers, kept out of the unrolled chunk
+// loops (which only record a bit per chunk): they re-read one 16-byte chunk
+// of the row (from L2) and compute exactly.
+//   exact maximum of |v| over the chunk (v = x / s or x * s)
+template <typename T, int MODE>
+__device__ __noinline__ float chunk_exact_absmax(const T *__restrict__ p, const float *__restrict__ sc)
+{
+    constexpr int V = Vec<T>::N;
+    float x[V];
+    widen<T>(__ldg(reinterpret_cast<const uint4 *>(p)), x);
+    float m = 0.0f;
+    for (int e = 0; e < V; ++e) {
+        const float sv = __ldg(sc + e);
+        m = fmaxf(m, fabsf(MODE == MODE_X ? __fdiv_rn(x[e], sv) : __fmul_rn(x[e], sv)));
+    }
+    return m;
+}
+
+__device__ __forceinline__ void store_code_words(int8_t *dst, const uint32_t *y, int n)
+{
+    if (n == 8)
+        *reinterpret_cast<uint2 *>(dst) =
+            make_uint2(pack_code_bytes(y[0], y[1], y[2], y[3]), pack_code_bytes(y[4], y[5], y[6], y[7]));
+    else
+        *reinterpret_cast<uint32_t *>(dst) = pack_code_bytes(y[0], y[1], y[2], y[3]);
+}
+
+//   exact codes of the chunk, overwriting what the fast path stored
+template <typename T, int MODE>
+__device__ __noinline__ void chunk_store_exact_codes(const T *__restrict__ p, const float *__restrict__ sc, float scale,
+                                                     int8_t *dst)
+{
+    constexpr int V = Vec<T>::N;
+    float x[V];
+    widen<T>(__ldg(reinterpret_cast<const uint4 *>(p)), x);
+    uint32_t y[8];
+    for (int e = 0; e < V; ++e) {
+        const float sv = __ldg(sc + e);
+        const float v = MODE == MODE_X ? __fdiv_rn(x[e], sv) : __fmul_rn(x[e], sv);
+        y[e] = scale != 0.0f ? exact_code_bits(v, scale) : code_bits(0.0f);
+    }
+    store_code_words(dst, y, V);
+}
+
+//   exact codes of a chunk of the normalised, smoothed row a = (h * rinv) * g
+template <typename T>
+__device__ __noinline__ void chunk_store_exact_codes_norm(const T *__restrict__ p, const float *g, float rinv,
+                                                          float scale, int8_t *dst)
+{
+    constexpr int V = Vec<T>::N;
+    float x[V];
+    widen<T>(__ldg(reinterpret_cast<const uint4 *>(p)), x);
+    uint32_t y[8];
+    for (int e = 0; e < V; ++e) {
+        const float a = __fmul_rn(__fmul_rn(x[e], rinv), g[e]);
+        y[e] = scale != 0.0f ? exact_code_bits(a, scale) : code_bits(0.0f);
+    }
+    store_code_words(dst, y, V);
+}
+
 // bytes of shared memory the factor tables of a K-column row take
 __host__ __device__ constexpr int64_t row_quant_smem(int64_t K, bool bf) { return K * 4 + (bf ? K * 2 : 0); }
 
@@ -541,20 +601,18 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
         if (BF || MODE == MODE_X) {
             const bool exact_all = bad_divisor || !(A >= kTinyQuotient) || !(A <= 0x1.fffffep127f);
             const float thr = __fmul_rn(A, BF ? 0.96875f : kCandidateScale);
-            float em = 0.0f;
+            uint32_t cand = 0;  // chunks that may hold the exact maximum
 #pragma unroll
             for (int i = 0; i < CH; ++i) {
                 const int c = c0 + cstep * i;
-                if ((FIT || c < nch) && (exact_all || hm[i] >= thr)) {
-                    Chunk8 xv;
-                    float x[V];
-                    widen<T>(raw[i], x);
-#pragma unroll
-                    for (int e = 0; e < V; ++e)
-                        xv.v[e] = x[e];
-                    const float *sc = s + static_cast<int64_t>(c) * V;
-                    em = fmaxf(em, MODE == MODE_X ? chunk_absmax_div(xv, sc, V) : chunk_absmax_mul(xv, sc, V));
-                }
+                cand |= ((FIT || c < nch) && (exact_all || hm[i] >= thr)) ? (1u << i) : 0u;
+            }
+            float em = 0.0f;
+            while (cand != 0u) {  // rare: re-read those chunks and compute exactly
+                const int i = __ffs(cand) - 1;
+                cand &= cand - 1u;
+                const int64_t c = c0 + cstep * i;
+                em = fmaxf(em, chunk_exact_absmax<T, MODE>(in + row * K + c * V, s + c * V));
             }
             E = group_max(em);
         }
@@ -570,49 +628,39 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
         const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
         const float2 nmagic2 = make_float2(-kRoundMagic, -kRoundMagic);
         int8_t *dst = q + row * K;
+        uint32_t ties = 0;  // chunks whose codes need the exact path
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
             const int c = c0 + cstep * i;
             if (FIT || c < nch) {
                 float x[V];
                 uint32_t y[V];
+                float2 f2[V / 2];
                 widen<T>(raw[i], x);
-                bool tie = !fast;
-                if (fast) {
-                    float2 f2[V / 2];
-                    factor_pairs(c, f2);
-                    float dmax = 0.0f;
+                factor_pairs(c, f2);
+                float dmax = 0.0f;
 #pragma unroll
-                    for (int e = 0; e < V; e += 2) {
-                        // yy = RN(a * rsc + 1.5*2^23): a*rsc rounded half-even to an
-                        // integer r (the code is yy's low byte); dd = r - a*rsc
-                        const float2 a = f2_mul(make_float2(x[e], x[e + 1]), f2[e / 2]);
-                        const float2 yy = f2_fma(a, rsc2, magic2);
-                        const float2 rr = f2_add(yy, nmagic2);
-                        const float2 dd = f2_fma(a, nrsc2, rr);
-                        dmax = fmaxf(dmax, fmaxf(fabsf(dd.x), fabsf(dd.y)));
-                        y[e] = __float_as_uint(yy.x);
-                        y[e + 1] = __float_as_uint(yy.y);
-                    }
-                    tie = !(dmax < kTieLimit);  // NaN (scale too small) also takes the exact path
+                for (int e = 0; e < V; e += 2) {
+                    // yy = RN(a * rsc + 1.5*2^23): a*rsc rounded half-even to an
+                    // integer r (the code is yy's low byte); dd = r - a*rsc
+                    const float2 a = f2_mul(make_float2(x[e], x[e + 1]), f2[e / 2]);
+                    const float2 yy = f2_fma(a, rsc2, magic2);
+                    const float2 rr = f2_add(yy, nmagic2);
+                    const float2 dd = f2_fma(a, nrsc2, rr);
+                    dmax = fmaxf(dmax, fmaxf(fabsf(dd.x), fabsf(dd.y)));
+                    y[e] = __float_as_uint(yy.x);
+                    y[e + 1] = __float_as_uint(yy.y);
                 }
-                if (tie) {
-                    Chunk8 xv;
-#pragma unroll
-                    for (int e = 0; e < V; ++e)
-                        xv.v[e] = x[e];
-                    const Chunk8 yy = chunk_codes_exact(xv, s + static_cast<int64_t>(c) * V, V, MODE == MODE_X, scale);
-#pragma unroll
-                    for (int e = 0; e < V; ++e)
-                        y[e] = __float_as_uint(yy.v[e]);
-                }
-                int8_t *d = dst + static_cast<int64_t>(c) * V;
-                if constexpr (V == 8)
-                    *reinterpret_cast<uint2 *>(d) = make_uint2(pack_code_bytes(y[0], y[1], y[2], y[3]),
-                                                               pack_code_bytes(y[4], y[5], y[6], y[7]));
-                else
-                    *reinterpret_cast<uint32_t *>(d) = pack_code_bytes(y[0], y[1], y[2], y[3]);
+                // NaN (scale too small) and scales outside the fast range also go exact
+                ties |= (!fast || !(dmax < kTieLimit)) ? (1u << i) : 0u;
+                store_code_words(dst + static_cast<int64_t>(c) * V, y, V);
             }
+        }
+        while (ties != 0u) {  // rare: near ties; every chunk when the scale is outside the fast range
+            const int i = __ffs(ties) - 1;
+            ties &= ties - 1u;
+            const int64_t c = c0 + cstep * i;
+            chunk_store_exact_codes<T, MODE>(in + row * K + c * V, s + c * V, scale, dst + c * V);
         }
         row += rstride;
         if (row < rows)
@@ -762,40 +810,33 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
         const float rsc = rcp_approx(scale);
         const bool fast = scale_in_fast_range(scale);
         int8_t *dst = q + row * K;
+        uint32_t ties = 0;  // chunks whose codes need the exact path
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
             const int c = c0 + cstep * i;
             if (c < nch) {
-                float x[V], f[V], a[V];
+                float x[V], f[V];
                 uint32_t y[V];
                 widen<T>(raw[i], x);
                 gvals(c, f);
                 float dmax = 0.0f;
 #pragma unroll
                 for (int e = 0; e < V; ++e) {
-                    a[e] = __fmul_rn(__fmul_rn(x[e], rinv), f[e]);
-                    const float yy = __fmaf_rn(a[e], rsc, kRoundMagic);
+                    const float a = __fmul_rn(__fmul_rn(x[e], rinv), f[e]);
+                    const float yy = __fmaf_rn(a, rsc, kRoundMagic);
                     const float rr = __fsub_rn(yy, kRoundMagic);
-                    dmax = fmaxf(dmax, fabsf(__fmaf_rn(a[e], -rsc, rr)));
+                    dmax = fmaxf(dmax, fabsf(__fmaf_rn(a, -rsc, rr)));
                     y[e] = __float_as_uint(yy);
                 }
-                if (!fast || !(dmax < kTieLimit)) {
-                    Chunk8 av;
-#pragma unroll
-                    for (int e = 0; e < V; ++e)
-                        av.v[e] = a[e];
-                    const Chunk8 yy = chunk_codes_of_values(av, V, scale);
-#pragma unroll
-                    for (int e = 0; e < V; ++e)
-                        y[e] = __float_as_uint(yy.v[e]);
-                }
-                int8_t *dd = dst + static_cast<int64_t>(c) * V;
-                if constexpr (V == 8)
-                    *reinterpret_cast<uint2 *>(dd) = make_uint2(pack_code_bytes(y[0], y[1], y[2], y[3]),
-                                                                pack_code_bytes(y[4], y[5], y[6], y[7]));
-                else
-                    *reinterpret_cast<uint32_t *>(dd) = pack_code_bytes(y[0], y[1], y[2], y[3]);
+                ties |= (!fast || !(dmax < kTieLimit)) ? (1u << i) : 0u;
+                store_code_words(dst + static_cast<int64_t>(c) * V, y, V);
             }
+        }
+        while (ties != 0u) {  // rare: near ties; every chunk when the scale is outside the fast range
+            const int i = __ffs(ties) - 1;
+            ties &= ties - 1u;
+            const int64_t c = c0 + cstep * i;
+            chunk_store_exact_codes_norm<T>(in + row * K + c * V, g_sm + c * V, rinv, scale, dst + c * V);
         }
         row += rstride;
         if (row < rows)
