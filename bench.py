@@ -217,7 +217,8 @@ class Step:
         of 8 warps, else a scale kernel and a code kernel."""
         esize = 2 if self.in_code == self.sq.SQ_BF16 else 4
         nch = self.K * esize // 16
-        smem = self.K * 4 + (self.K * 2 if esize == 2 else 0)
+        bb = esize == 2 and self.K * 6 <= 64 * 1024
+        smem = self.K * 4 + (self.K * 2 if bb else 0)
         if os.environ.get("SQ_QUANT_KIND") == "2":
             return 2
         return 1 if smem <= 232448 - 1024 and nch <= 32 * 16 * 8 else 2

@@ -226,12 +226,12 @@ sq_status launch_row_scale(const T *in, int64_t rows, int64_t K, const float *s,
 
 // Single-pass quantiser (row in registers): 2^log2g warps per row, CH chunks
 // per lane.
-template <typename T, int MODE, int CH, bool FIT>
+template <typename T, int MODE, int CH, bool FIT, bool BB>
 sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
                                float *scale, int log2g, cudaStream_t st, const DeviceInfo &di)
 {
-    auto kernel = sq::row_quant_kernel<T, MODE, CH, FIT>;
-    const int smem = static_cast<int>(sq::row_quant_smem(K, sq::Vec<T>::N == 8));
+    auto kernel = sq::row_quant_kernel<T, MODE, CH, FIT, BB>;
+    const int smem = static_cast<int>(sq::row_quant_smem(K, BB));
     static std::atomic<uint64_t> attr_done{0};
     // the kernel also has a little static shared memory (the group maxima)
     if (!ensure_smem_attr(kernel, kMaxDynSmem - 1024, attr_done))
@@ -283,7 +283,9 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
     static const int force_kind = std::getenv("SQ_QUANT_KIND") ? std::atoi(std::getenv("SQ_QUANT_KIND")) : 0;
     constexpr int V = sq::Vec<T>::N;
     const int64_t nch = K / V;
-    if (force_kind != 2 && sq::row_quant_smem(K, V == 8) <= kMaxDynSmem - 1024) {
+    // the bf16 bound while both factor tables stay small (about 3 CTAs per SM)
+    const bool bb = V == 8 && sq::row_quant_smem(K, true) <= 64 * 1024;
+    if (force_kind != 2 && sq::row_quant_smem(K, bb) <= kMaxDynSmem - 1024) {
         // 8 chunks per lane (three CTAs per SM), 16 for rows too long for that
         for (int ch : {8, 16}) {
             int log2g = 0;
@@ -294,11 +296,18 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
             // an exact fit drops the bounds checks; few rows rather spread over more warps
             const bool fit = ((int64_t)32 * ch << log2g) == nch &&
                              rows * (1 << log2g) >= (int64_t)di.sms * 2 * (sq::kQuantThreads / 32);
+            if (bb) {
+                if (ch == 8)
+                    return fit ? launch_row_quant_cfg<T, MODE, 8, true, true>(in, rows, K, s, q, scale, log2g, st, di)
+                               : launch_row_quant_cfg<T, MODE, 8, false, true>(in, rows, K, s, q, scale, log2g, st, di);
+                return fit ? launch_row_quant_cfg<T, MODE, 16, true, true>(in, rows, K, s, q, scale, log2g, st, di)
+                           : launch_row_quant_cfg<T, MODE, 16, false, true>(in, rows, K, s, q, scale, log2g, st, di);
+            }
             if (ch == 8)
-                return fit ? launch_row_quant_cfg<T, MODE, 8, true>(in, rows, K, s, q, scale, log2g, st, di)
-                           : launch_row_quant_cfg<T, MODE, 8, false>(in, rows, K, s, q, scale, log2g, st, di);
-            return fit ? launch_row_quant_cfg<T, MODE, 16, true>(in, rows, K, s, q, scale, log2g, st, di)
-                       : launch_row_quant_cfg<T, MODE, 16, false>(in, rows, K, s, q, scale, log2g, st, di);
+                return fit ? launch_row_quant_cfg<T, MODE, 8, true, false>(in, rows, K, s, q, scale, log2g, st, di)
+                           : launch_row_quant_cfg<T, MODE, 8, false, false>(in, rows, K, s, q, scale, log2g, st, di);
+            return fit ? launch_row_quant_cfg<T, MODE, 16, true, false>(in, rows, K, s, q, scale, log2g, st, di)
+                       : launch_row_quant_cfg<T, MODE, 16, false, false>(in, rows, K, s, q, scale, log2g, st, di);
         }
     }
     sq_status r = (K * (int64_t)sizeof(float) <= kSmemFactorBytes)

@@ -493,19 +493,22 @@ __device__ __noinline__ void chunk_store_exact_codes_norm(const T *__restrict__ 
     store_code_words(dst, y, V);
 }
 
-// bytes of shared memory the factor tables of a K-column row take
+// bytes of shared memory the factor tables of a K-column row take (bf: with
+// the bf16 table)
 __host__ __device__ constexpr int64_t row_quant_smem(int64_t K, bool bf) { return K * 4 + (bf ? K * 2 : 0); }
 
 // FIT: the G warps of a row cover its chunks exactly (32 CH G = K / V), so
-// no chunk needs a bounds check.
-template <typename T, int MODE, int CH, bool FIT>
+// no chunk needs a bounds check.  BB (bf16 rows only): bound |v| in packed
+// bf16 arithmetic (fewer instructions, a wider candidate window and a second
+// factor table in shared memory) instead of fp32.
+template <typename T, int MODE, int CH, bool FIT, bool BB>
 __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
     row_quant_kernel(const T *__restrict__ in, int64_t rows, int64_t K, const float *__restrict__ s,
                      int log2g, int8_t *__restrict__ q, float *__restrict__ scale_out)
 {
     pdl_prologue();
     constexpr int V = Vec<T>::N;
-    constexpr bool BF = (V == 8);  // bf16 rows
+    constexpr bool BF = BB && (V == 8);  // the bf16 bound
     constexpr int WARPS = kQuantThreads / 32;
     extern __shared__ float4 smem_f4[];
     float *f_sm = reinterpret_cast<float *>(smem_f4);
@@ -597,7 +600,7 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
             }
         }
         const float A = group_max(am);
-        float E = A;  // fp32 weights: the bounds are the values themselves
+        float E = A;  // fp32-bounded weights: the bounds are the values themselves
         if (BF || MODE == MODE_X) {
             const bool exact_all = bad_divisor || !(A >= kTinyQuotient) || !(A <= 0x1.fffffep127f);
             const float thr = __fmul_rn(A, BF ? 0.96875f : kCandidateScale);
