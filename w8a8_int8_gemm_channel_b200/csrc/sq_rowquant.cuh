@@ -434,15 +434,15 @@ __device__ __forceinline__ int stage_factor_tables(const float *__restrict__ s, 
 }
 
 // Rare paths of the single-pass quantisers, kept out of the unrolled chunk
-// loops (which only record a bit per chunk): they re-read one 16-byte chunk
-// of the row (from L2) and compute exactly.
-//   exact maximum of |v| over the chunk (v = x / s or x * s)
+// loops (which only record a bit per chunk); they compute one 16-byte chunk
+// exactly.
+//   exact maximum of |v| over the chunk (v = x / s or x * s), given its raw bits
 template <typename T, int MODE>
-__device__ __noinline__ float chunk_exact_absmax(const T *__restrict__ p, const float *__restrict__ sc)
+__device__ __noinline__ float chunk_exact_absmax(uint4 raw, const float *__restrict__ sc)
 {
     constexpr int V = Vec<T>::N;
     float x[V];
-    widen<T>(__ldg(reinterpret_cast<const uint4 *>(p)), x);
+    widen<T>(raw, x);
     float m = 0.0f;
     for (int e = 0; e < V; ++e) {
         const float sv = __ldg(sc + e);
@@ -460,7 +460,7 @@ __device__ __forceinline__ void store_code_words(int8_t *dst, const uint32_t *y,
         *reinterpret_cast<uint32_t *>(dst) = pack_code_bytes(y[0], y[1], y[2], y[3]);
 }
 
-//   exact codes of the chunk, overwriting what the fast path stored
+//   exact codes of the chunk (re-read from L2), overwriting what the fast path stored
 template <typename T, int MODE>
 __device__ __noinline__ void chunk_store_exact_codes(const T *__restrict__ p, const float *__restrict__ sc, float scale,
                                                      int8_t *dst)
@@ -611,11 +611,16 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
                 cand |= ((FIT || c < nch) && (exact_all || hm[i] >= thr)) ? (1u << i) : 0u;
             }
             float em = 0.0f;
-            while (cand != 0u) {  // rare: re-read those chunks and compute exactly
+            while (cand != 0u) {  // rare: those chunks exactly, taken from the registers
                 const int i = __ffs(cand) - 1;
                 cand &= cand - 1u;
+                uint4 v = raw[0];
+#pragma unroll
+                for (int j = 1; j < CH; ++j)
+                    if (j == i)
+                        v = raw[j];
                 const int64_t c = c0 + cstep * i;
-                em = fmaxf(em, chunk_exact_absmax<T, MODE>(in + row * K + c * V, s + c * V));
+                em = fmaxf(em, chunk_exact_absmax<T, MODE>(v, s + c * V));
             }
             E = group_max(em);
         }
