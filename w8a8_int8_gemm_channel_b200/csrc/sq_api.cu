@@ -189,9 +189,13 @@ sq_status launch_col_absmax(const T *x, int64_t R, int64_t K, int64_t ld, float 
     constexpr int CL = sq::kColClusterRows;
     const int64_t chunks = K / V;
     const int64_t col_blocks = (chunks + sq::kColThreads - 1) / sq::kColThreads;
-    // one wave of about 4 CTAs of 256 threads per SM, in clusters of CL row
-    // bands; bands are whole multiples of the 16 rows a thread keeps in flight
-    const int64_t want = std::max<int64_t>(CL, (int64_t)di.sms * 4 / col_blocks);
+    // one wave of about 4 CTAs of 256 threads per SM (measured best from 1 to
+    // 12 for calibration batches and weights alike), in clusters of CL row
+    // bands; bands are whole multiples of the 16 rows a thread keeps in
+    // flight.  SQ_COL_PER_SM overrides the CTAs per SM.
+    static const int force_per_sm = std::getenv("SQ_COL_PER_SM") ? std::atoi(std::getenv("SQ_COL_PER_SM")) : 0;
+    const int per_sm = force_per_sm > 0 ? force_per_sm : 4;
+    const int64_t want = std::max<int64_t>(CL, (int64_t)di.sms * per_sm / col_blocks);
     int64_t rows_per_block = std::max<int64_t>(16, ((R + want - 1) / want + 15) / 16 * 16);
     int64_t row_blocks = (R + rows_per_block - 1) / rows_per_block;
     while (row_blocks > 65528) {
