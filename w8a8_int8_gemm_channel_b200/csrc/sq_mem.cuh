@@ -315,27 +315,6 @@ __global__ void smooth_factors_kernel(const float *__restrict__ ax, float *s, fl
     s[j] = r;
 }
 
-// ----------------------------------------------------------------------------
-// Block-wide max of non-negative floats (all threads receive the result).
-// ----------------------------------------------------------------------------
-__device__ __forceinline__ float block_max(float v, float *red /* >= 32 floats */)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nwarps = (blockDim.x + 31) >> 5;
-    __syncthreads();  // red may still be read by a previous call
-    if (lane == 0)
-        red[warp] = v;
-    __syncthreads();
-    float r = lane < nwarps ? red[lane] : 0.0f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        r = fmaxf(r, __shfl_xor_sync(0xFFFFFFFFu, r, o));
-    return r;
-}
-
 // Store the codes of one 16-byte input vector: 8 codes (bf16 input) as 8
 // bytes or 4 codes (fp32 input) as 4 bytes.
 template <int V>
@@ -417,25 +396,6 @@ __device__ __noinline__ float chunk_absmax_div(Chunk8 x, const float *__restrict
     for (int e = 0; e < n; ++e)
         m = fmaxf(m, fabsf(__fdiv_rn(x.v[e], __ldg(s_chunk + e))));
     return m;
-}
-
-// Exact max of |x * s| over one chunk (weights: the smoothed values).
-__device__ __noinline__ float chunk_absmax_mul(Chunk8 x, const float *__restrict__ s_chunk, int n)
-{
-    float m = 0.0f;
-    for (int e = 0; e < n; ++e)
-        m = fmaxf(m, fabsf(__fmul_rn(x.v[e], __ldg(s_chunk + e))));
-    return m;
-}
-
-// Exact codes of one chunk of known values (rare: near ties, scales outside
-// the fast range).
-__device__ __noinline__ Chunk8 chunk_codes_of_values(Chunk8 a, int n, float scale)
-{
-    Chunk8 y;
-    for (int e = 0; e < n; ++e)
-        y.v[e] = __uint_as_float(scale != 0.0f ? exact_code_bits(a.v[e], scale) : code_bits(0.0f));
-    return y;
 }
 
 // Approximate magnitudes a = RN(|x| * r) of one chunk and their maximum.

@@ -218,16 +218,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
-// Contiguous copy global -> shared of `bytes` (multiple of 16, both addresses
-// 16-byte aligned); completion is signalled on `bar` as transaction bytes.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     dst),
-                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-
 // ----------------------------------------------------------------------------
 // packed fp32 pairs (sm_100): two independent IEEE round-to-nearest
 // operations per instruction, exactly the scalar _rn results.  The pairs are
