@@ -70,6 +70,12 @@ def _load():
             lib.sqo_fold_gamma.argtypes = [P, P, I, P]
             lib.sqo_rmsnorm_quant.argtypes = [P, ctypes.c_int, I, I, P, ctypes.c_float, P, P, P, P]
             lib.sqo_f32_to_bf16.argtypes = [ctypes.c_float]
+            lib.sqo_exp_f32.argtypes = [ctypes.c_float]
+            lib.sqo_exp_f32.restype = ctypes.c_float
+            lib.sqo_silu_f32.argtypes = [ctypes.c_float]
+            lib.sqo_silu_f32.restype = ctypes.c_float
+            lib.sqo_exp_silu_vec.argtypes = [P, I, ctypes.c_int, P]
+            lib.sqo_silu_mul_quant.argtypes = [P, ctypes.c_int, I, I, P, P, P, P]
             lib.sqo_f32_to_bf16.restype = ctypes.c_uint16
             lib.sqo_num_threads.restype = ctypes.c_int
             _lib = lib
@@ -203,6 +209,39 @@ def rmsnorm_rinv_fp64(h: np.ndarray, eps: float) -> np.ndarray:
     ms = (h64 * h64).sum(axis=1) / h64.shape[1] + np.float64(np.float32(eps))
     with np.errstate(divide="ignore"):
         return np.where(ms > 0, 1.0 / np.sqrt(ms), 0.0)
+
+
+def exp_f32(x: np.ndarray) -> np.ndarray:
+    """e^x per element by the fixed fp32 sequence of ``sqo_exp_f32``."""
+    x = _c(x, np.float32)
+    y = np.empty_like(x)
+    _load().sqo_exp_silu_vec(_ptr(x), x.size, 0, _ptr(y))
+    return y
+
+
+def silu_f32(x: np.ndarray) -> np.ndarray:
+    """SiLU(x) = x / (1 + e^-x) per element in fp32 (``sqo_silu_f32``)."""
+    x = _c(x, np.float32)
+    y = np.empty_like(x)
+    _load().sqo_exp_silu_vec(_ptr(x), x.size, 1, _ptr(y))
+    return y
+
+
+def silu_mul_quant(gu: np.ndarray, s: np.ndarray):
+    """Gated feed-forward activation h = SiLU(gate) * up (gu = [gate | up], [M, 2I]),
+    rounded to gu's storage type, then per-token int8 quantisation of h / s.
+    Returns (xq int8 [M, I], sx fp32 [M], h fp32 [M, I])."""
+    gu = _c(gu)
+    s = _c(s, np.float32)
+    M, I2 = gu.shape
+    assert I2 % 2 == 0
+    I = I2 // 2
+    assert s.shape == (I,)
+    xq = np.empty((M, I), np.int8)
+    sx = np.empty(M, np.float32)
+    h = np.empty((M, I), np.float32)
+    _load().sqo_silu_mul_quant(_ptr(gu), _dt(gu), M, I, _ptr(s), _ptr(xq), _ptr(sx), _ptr(h))
+    return xq, sx, h
 
 
 def gemm_i32(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:

@@ -39,6 +39,14 @@
  *        outlier actually comes from": RMSNorm (divide by the vector's
  *        root-mean-square, multiply by gamma) and SmoothQuant's division of
  *        gamma by s.
+ *   [F]  "Understanding W8A8 INT8 LLM Quantization", section "Inter-Token
+ *        Latency (ITL)": per layer and token, the dynamic activation
+ *        quantisation is memory-bound work; and "How does SmoothQuant int8
+ *        LLM calibration work...", section "Hardware Acceleration and
+ *        Inference Optimization Strategies": fusing the feed-forward network
+ *        with its neighbours saves memory traffic.  The pages do not define
+ *        the feed-forward network itself; the gated SiLU form below is the
+ *        one of the Llama-3-8B layers whose shapes the workloads use.
  *
  * The smoothing-factor equation itself did not survive the page's text
  * extraction; this oracle uses s_j = A_j^alpha / B_j^(1-alpha), with A_j the
@@ -47,6 +55,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 #include <stddef.h>
 #ifdef _OPENMP
@@ -322,6 +331,104 @@ void sqo_rmsnorm_quant(const void *h, int dt, int64_t M, int64_t K, const float 
             }
             xq[m * K + k] = q;
         }
+    }
+}
+
+/* [F] e^x in binary32, as a fixed sequence of IEEE operations (fmaf is one
+ * correctly rounded fused multiply-add), so that every implementation that
+ * follows the same steps gets the same bits.  Method: Cody and Waite's
+ * argument reduction, then the Taylor series of e^r to degree 7.
+ *   x < -87: 0 (e^-87 is about 1.6e-38; below it the result would leave the
+ *            normal range; for SiLU only 1 + e^x matters, which is then 1);
+ *   x >  88: +infinity;
+ *   else     n = the integer nearest to x * L2E (L2E = RN(log2 e)), taken
+ *            from fmaf(x, L2E, 1.5 * 2^23) - 1.5 * 2^23;
+ *            r = fmaf(-n, LN2_LO, fmaf(-n, LN2_HI, x)), with LN2_HI = RN(ln 2)
+ *            and LN2_LO = RN(ln 2 - LN2_HI);
+ *            p = 1 + r (1 + r (1/2! + r (1/3! + ... + r / 7!))) by Horner's
+ *            rule, one fmaf per step, each coefficient RN(1/k!);
+ *            e^x = p * 2^n (exact: the result is normal). */
+float sqo_exp_f32(float x)
+{
+    if (x < -87.0f)
+        return 0.0f;
+    if (x > 88.0f)
+        return INFINITY;
+    const float magic = 12582912.0f; /* 1.5 * 2^23 */
+    const float n = fmaf(x, 0x1.715476p+0f, magic) - magic;
+    float r = fmaf(-n, 0x1.62e430p-1f, x);
+    r = fmaf(-n, -0x1.05c610p-29f, r);
+    float p = 0x1.a01a02p-13f;         /* 1/7! */
+    p = fmaf(p, r, 0x1.6c16c2p-10f);   /* 1/6! */
+    p = fmaf(p, r, 0x1.111112p-7f);    /* 1/5! */
+    p = fmaf(p, r, 0x1.555556p-5f);    /* 1/4! */
+    p = fmaf(p, r, 0x1.555556p-3f);    /* 1/3! */
+    p = fmaf(p, r, 0.5f);              /* 1/2! */
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    return ldexpf(p, (int)n);
+}
+
+/* [F] SiLU(z) = z * sigmoid(z) = z / (1 + e^-z): one fp32 addition and one
+ * IEEE fp32 division, e^-z from sqo_exp_f32. */
+float sqo_silu_f32(float z)
+{
+    const float d = 1.0f + sqo_exp_f32(-z);
+    return z / d;
+}
+
+/* elementwise over arrays (for the tests): y[i] = sqo_exp_f32(x[i]) when
+ * which == 0, sqo_silu_f32(x[i]) when which == 1 */
+void sqo_exp_silu_vec(const float *x, int64_t n, int which, float *y)
+{
+    for (int64_t i = 0; i < n; ++i)
+        y[i] = which == 0 ? sqo_exp_f32(x[i]) : sqo_silu_f32(x[i]);
+}
+
+/* [F] then [S] then [A]: the gated feed-forward activation of token m,
+ *   h[m, j] = SiLU(gu[m, j]) * gu[m, I + j]   (gate, then up, in one row of
+ *             2I values), one fp32 multiply, then rounded to the storage type
+ *             of gu (bf16 by round-half-to-even; fp32 unchanged) -- the value
+ *             an unfused feed-forward step would store for the next layer;
+ * then exactly sqo_quant_act on h: x^ = h / s, sx = max |x^| / 127, codes.
+ * h_out (may be NULL) receives h as fp32 [M, I]. */
+void sqo_silu_mul_quant(const void *gu, int dt, int64_t M, int64_t I, const float *s, int8_t *xq,
+                        float *sx, float *h_out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        float *h = (float *)malloc((size_t)I * sizeof(float));
+        for (int64_t j = 0; j < I; ++j) {
+            const float g = elem(gu, dt, (size_t)(m * 2 * I + j));
+            const float u = elem(gu, dt, (size_t)(m * 2 * I + I + j));
+            float v = sqo_silu_f32(g) * u;
+            if (dt == SQO_BF16)
+                v = widen_bf16(sqo_f32_to_bf16(v));
+            h[j] = v;
+            if (h_out)
+                h_out[m * I + j] = v;
+        }
+        float amax = 0.0f;
+        for (int64_t j = 0; j < I; ++j) {
+            const float v = fabsf(h[j] / s[j]);
+            if (v > amax)
+                amax = v;
+        }
+        const float scale = amax / 127.0f;
+        sx[m] = scale;
+        for (int64_t j = 0; j < I; ++j) {
+            int8_t q = 0;
+            if (amax != 0.0f) {
+                float r = nearbyintf((h[j] / s[j]) / scale);
+                if (r > 127.0f)
+                    r = 127.0f;
+                if (r < -127.0f)
+                    r = -127.0f;
+                q = (int8_t)r;
+            }
+            xq[m * I + j] = q;
+        }
+        free(h);
     }
 }
 

@@ -483,3 +483,114 @@ def test_rmsnorm_fold_matches_unfused_composition(oracle):
     q_ref, _ = oracle.quant_act(x, s)
     d = np.abs(q_fold.astype(np.int32) - q_ref.astype(np.int32))
     assert d.max() <= 1 and (d == 0).mean() > 0.995
+
+
+# ---------------------------------------------------------------------------
+# The gated feed-forward activation SiLU(gate) * up, quantised for the down
+# projection ("Understanding W8A8 INT8 LLM Quantization", section
+# "Inter-Token Latency (ITL)": the per-token quantisation is memory-bound work
+# worth fusing into the op before it)
+# ---------------------------------------------------------------------------
+
+def _bf16_rne_bits(x):
+    """Round-half-to-even of finite fp32 values to bf16 bit patterns (numpy)."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((b + 0x7FFF + ((b >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def _bf16_bits_f32(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def test_exp_f32_within_one_ulp_of_fp64(oracle):
+    rng = np.random.default_rng(50)
+    x = np.concatenate([np.linspace(-87.0, 88.0, 400001),
+                        rng.uniform(-87.0, 88.0, 200000),
+                        rng.uniform(-1e-3, 1e-3, 20000)]).astype(np.float32)
+    y = oracle.exp_f32(x).astype(np.float64)
+    ref = np.exp(x.astype(np.float64))
+    ulp = np.spacing(ref.astype(np.float32)).astype(np.float64)
+    assert (np.abs(y - ref) / ulp).max() <= 1.0
+    e = oracle.exp_f32(f32([0.0, -0.0, 1.0, -87.5, -1e30, 88.5, 1e30]))
+    assert e[0] == 1.0 and e[1] == 1.0
+    assert abs(float(e[2]) - math.e) <= 2.5e-7
+    assert e[3] == 0.0 and e[4] == 0.0
+    assert np.isinf(e[5]) and np.isinf(e[6]) and e[5] > 0
+
+
+def test_silu_closed_forms(oracle):
+    """SiLU(0) = 0 with the sign of zero kept; SiLU(z) = z once 1 + e^-z rounds
+    to 1 (z >= 17); -0 once e^-z overflows; SiLU(z) - SiLU(-z) = z."""
+    z = f32([0.0, -0.0])
+    s0 = oracle.silu_f32(z)
+    assert s0[0] == 0.0 and not np.signbit(s0[0]) and s0[1] == 0.0 and np.signbit(s0[1])
+    big = f32(np.concatenate([np.linspace(17.0, 87.0, 5001), [1e3, 1e20, 3e38]]))
+    assert np.array_equal(oracle.silu_f32(big), big)
+    neg = f32([-88.5, -1e3, -3e38])
+    sn = oracle.silu_f32(neg)
+    assert np.all(sn == 0.0) and np.all(np.signbit(sn))
+    rng = np.random.default_rng(51)
+    z = f32(rng.uniform(-10.0, 10.0, 100000))
+    d = oracle.silu_f32(z).astype(np.float64) - oracle.silu_f32(-z).astype(np.float64)
+    assert np.allclose(d, z.astype(np.float64), rtol=4e-7, atol=1e-6)
+
+
+def test_silu_within_three_ulp_of_fp64(oracle):
+    rng = np.random.default_rng(52)
+    z = f32(np.concatenate([np.linspace(-80.0, 80.0, 400001), rng.standard_normal(100000) * 4.0]))
+    got = oracle.silu_f32(z).astype(np.float64)
+    z64 = z.astype(np.float64)
+    ref = z64 / (1.0 + np.exp(-z64))
+    ok = ref != 0.0
+    ulp = np.spacing(np.abs(ref[ok]).astype(np.float32)).astype(np.float64)
+    assert (np.abs(got[ok] - ref[ok]) / ulp).max() <= 3.0
+
+
+def test_silu_mul_quant_saturated_gate_is_the_product(oracle):
+    """For gate >= 17 SiLU(gate) = gate exactly, so h = RN_bf16(gate * up) and
+    the codes are those of the plain quantiser on that product: pins the
+    [gate | up] order, the rounding of h to bf16 and the division by s."""
+    rng = np.random.default_rng(53)
+    M, I = 8, 64
+    g = _bf16_rne_bits(rng.uniform(17.0, 60.0, (M, I)))
+    u = _bf16_rne_bits(rng.standard_normal((M, I)))
+    s = f32(rng.uniform(0.5, 2.0, I))
+    xq, sx, h = oracle.silu_mul_quant(np.concatenate([g, u], axis=1), s)
+    prod_bits = _bf16_rne_bits(_bf16_bits_f32(g) * _bf16_bits_f32(u))  # the fp32 product is exact
+    assert np.array_equal(h, _bf16_bits_f32(prod_bits))
+    q_ref, sx_ref = oracle.quant_act(prod_bits, s)
+    assert np.array_equal(xq, q_ref) and np.array_equal(sx, sx_ref)
+    # with gate and up swapped the activation is SiLU(up) * gate, not the same codes
+    xq_sw, _, _ = oracle.silu_mul_quant(np.concatenate([u, g], axis=1), s)
+    assert not np.array_equal(xq_sw, xq)
+
+
+def test_silu_mul_quant_against_fp64(oracle):
+    """h lies within half a bf16 ulp (plus the fp32 steps) of the fp64 value
+    SiLU(gate) * up, and the codes quantise exactly that h."""
+    rng = np.random.default_rng(54)
+    M, I = 16, 256
+    g = _bf16_rne_bits(rng.standard_normal((M, I)) * 3.0)
+    u = _bf16_rne_bits(rng.standard_normal((M, I)))
+    s = f32(rng.uniform(0.5, 2.0, I))
+    xq, sx, h = oracle.silu_mul_quant(np.concatenate([g, u], axis=1), s)
+    g64 = _bf16_bits_f32(g).astype(np.float64)
+    ref = g64 / (1.0 + np.exp(-g64)) * _bf16_bits_f32(u).astype(np.float64)
+    assert np.all(np.abs(h - ref) <= np.abs(ref) * (2.0 ** -8) * (1.0 + 2.0 ** -18) + 1e-38)
+    q_ref, sx_ref = oracle.quant_act(_bf16_rne_bits(h), s)
+    assert np.array_equal(xq, q_ref) and np.array_equal(sx, sx_ref)
+
+
+def test_silu_mul_quant_zero_rows_and_fp32(oracle):
+    """A zero gate, or a gate whose e^-gate overflows, gives a zero row (scale 0,
+    codes 0); fp32 rows keep h = SiLU(gate) * up unrounded."""
+    I = 32
+    s = np.ones(I, np.float32)
+    gu = np.zeros((3, 2 * I), np.float32)
+    gu[:, I:] = 1.5
+    gu[1, :I] = -100.0
+    gu[2, :I] = np.linspace(-3.0, 3.0, I, dtype=np.float32)
+    xq, sx, h = oracle.silu_mul_quant(gu, s)
+    assert sx[0] == 0.0 and sx[1] == 0.0 and not xq[:2].any()
+    assert np.array_equal(h[2], oracle.silu_f32(gu[2, :I]) * np.float32(1.5))
+    assert sx[2] == np.float32(np.abs(h[2]).max() / np.float32(127.0))
