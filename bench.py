@@ -465,7 +465,7 @@ def workload_config(wl):
 def run_case(spec, steps, warmup, flush_l2=True, settle_us=0.0):
     """Time one C-ABI call on synthetic data.  spec is one of
     gemm:M,N,K  linear:M,N,K  quant_act:M,K  quant_w:N,K  calib:T,K
-    smooth_factors:N,K  rmsnorm_quant:M,K.  Prints one JSON line with the median time."""
+    smooth_factors:N,K  rmsnorm_quant:M,K  silu_mul_quant:M,I.  Prints one JSON line with the median time."""
     import w8a8_int8_gemm_channel_b200 as sq
 
     lib = sq.lib()
@@ -512,6 +512,13 @@ def run_case(spec, steps, warmup, flush_l2=True, settle_us=0.0):
         fn = lambda: lib.sq_rmsnorm_quant(h.data_ptr(), sq.SQ_BF16, M, K, g.data_ptr(), 1e-5, xq.data_ptr(),
                                           sx.data_ptr(), None, st)
         nbytes = 3 * M * K + 4 * K + 4 * M
+    elif kind == "silu_mul_quant":
+        M, I = d
+        gu, s = r(M, 2 * I), torch.rand(I, device=dev) + 0.5
+        xq, sx = torch.empty(M, I, dtype=i8, device=dev), torch.empty(M, device=dev)
+        fn = lambda: lib.sq_silu_mul_quant(gu.data_ptr(), sq.SQ_BF16, M, I, s.data_ptr(), xq.data_ptr(),
+                                           sx.data_ptr(), None, st)
+        nbytes = 4 * M * I + M * I + 4 * I + 4 * M
     elif kind == "quant_w":
         N, K = d
         w, s = r(N, K, sc=0.02), torch.rand(K, device=dev) + 0.5

@@ -170,6 +170,33 @@ SQ_API sq_status sq_rmsnorm_quant(const void *h, sq_dtype dt, int64_t M, int64_t
                                   float eps, int8_t *xq, float *sx, float *rinv, sq_stream_t stream);
 
 /*
+ * The gated feed-forward activation of the down projection, quantised in the
+ * same pass that computes it, so that it never travels through HBM in bf16
+ * ("Understanding W8A8 INT8 LLM Quantization", section "Inter-Token Latency
+ * (ITL)": the per-token quantisation is memory-bound work; "How does
+ * SmoothQuant int8 LLM calibration work...", section "Hardware Acceleration
+ * and Inference Optimization Strategies": fuse the feed-forward network with
+ * its neighbours).  The pages do not define the activation; this is the
+ * gated SiLU of the Llama layers:
+ *   E(x)    = e^x by a fixed fp32 sequence: 0 for x < -87, +inf for x > 88,
+ *             else Cody-Waite reduction with RN(log2 e), RN(ln 2) and
+ *             RN(ln 2 - RN(ln 2)), then the degree-7 Taylor series by
+ *             Horner's rule with fused multiply-adds and coefficients
+ *             RN(1/k!), times 2^n (within 1 ulp of e^x);
+ *   h[m, j] = RN(RN(g / RN(1 + E(-g))) * u), g = gu[m, j], u = gu[m, I + j],
+ *             rounded to dt (bf16 by round-half-to-even): the value an
+ *             unfused feed-forward step would store;
+ *   then exactly sq_quant_act on h: sx[m] = max_j |h / s_j| / 127, codes.
+ *   gu [M, 2I] dtype dt (each row: the I gate values, then the I up values);
+ *   s [I] fp32; xq [M, I] int8 out; sx [M] fp32 out; h [M, I] dtype dt out
+ *   (may be NULL: then h is not stored).
+ * I a multiple of 16, at most 32768 (bf16) or 16384 (fp32).  Inputs must be
+ * finite, and so must h (|SiLU(gate) * up| within dt's range).
+ */
+SQ_API sq_status sq_silu_mul_quant(const void *gu, sq_dtype dt, int64_t M, int64_t I, const float *s,
+                                   int8_t *xq, float *sx, void *h, sq_stream_t stream);
+
+/*
  * W8A8 GEMM with the dequantising epilogue ("quant_llm_int8": int32
  * accumulation, outer product of row and column scales):
  *   acc[m, n] = sum_k xq[m, k] * wq[n, k]   (exact int32; K * 127^2 < 2^31,

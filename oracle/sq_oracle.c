@@ -391,7 +391,8 @@ void sqo_exp_silu_vec(const float *x, int64_t n, int which, float *y)
  *             of gu (bf16 by round-half-to-even; fp32 unchanged) -- the value
  *             an unfused feed-forward step would store for the next layer;
  * then exactly sqo_quant_act on h: x^ = h / s, sx = max |x^| / 127, codes.
- * h_out (may be NULL) receives h as fp32 [M, I]. */
+ * h_out (may be NULL) receives h as fp32 [M, I].  h must be finite (like
+ * every input of the quantisers). */
 void sqo_silu_mul_quant(const void *gu, int dt, int64_t M, int64_t I, const float *s, int8_t *xq,
                         float *sx, float *h_out)
 {

@@ -154,6 +154,18 @@ def test_rmsnorm_entry_points_reject_bad_arguments(lib):
     assert g(A, 1, 4, 65536, B, 1e-5, C, D, None, None) == UNS   # row too long for one pass
 
 
+def test_silu_mul_quant_rejects_bad_arguments(lib):
+    f = lib.sq_silu_mul_quant
+    assert f(None, 1, 4, 64, B, C, D, None, None) == INV
+    assert f(A, 1, 0, 64, B, C, D, None, None) == INV           # M < 1
+    assert f(A, 1, 4, 40, B, C, D, None, None) == INV           # I not a multiple of 16
+    assert f(A, 1, 4, 64, MIS, C, D, None, None) == INV         # misaligned s
+    assert f(A, 1, 4, 64, B, C, D, MIS, None) == INV            # misaligned h
+    assert f(A, 7, 4, 64, B, C, D, None, None) == INV           # bad dtype
+    assert f(A, 1, 4, 65536, B, C, D, None, None) == UNS        # row longer than one pass takes
+    assert f(A, 0, 4, 32768, B, C, D, None, None) == UNS        # fp32 rows: at most 16384
+
+
 def test_selftest_rejects_limits_out_of_range(lib):
     f = lib.sq_selftest_wait_timeout
     assert f(0, None) == INV

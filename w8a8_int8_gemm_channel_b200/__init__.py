@@ -46,6 +46,7 @@ ABI_SYMBOLS = (
     "sq_quant_act",
     "sq_fold_gamma",
     "sq_rmsnorm_quant",
+    "sq_silu_mul_quant",
     "sq_w8a8_gemm",
     "sq_w8a8_gemm_s32",
     "sq_linear",
@@ -79,6 +80,7 @@ def _declare(lib):
         "sq_quant_act": ([P, E, I, I, P, P, P, P], E),
         "sq_fold_gamma": ([P, P, I, P, P], E),
         "sq_rmsnorm_quant": ([P, E, I, I, P, F, P, P, P, P], E),
+        "sq_silu_mul_quant": ([P, E, I, I, P, P, P, P, P], E),
         "sq_w8a8_gemm": ([P, P, P, P, I, I, I, P, E, P], E),
         "sq_w8a8_gemm_s32": ([P, P, I, I, I, P, P], E),
         "sq_linear": ([P, E, P, P, P, I, I, I, P, E, P, ctypes.c_size_t, P], E),
@@ -191,6 +193,15 @@ def sq_rmsnorm_quant(h, g, eps, xq, sx, rinv=None, stream=None):
     _check("sq_rmsnorm_quant",
            lib().sq_rmsnorm_quant(_ptr(h), _dtype_code(h), M, K, _ptr(g), float(eps), _ptr(xq), _ptr(sx),
                                   None if rinv is None else _ptr(rinv), _stream(stream)))
+
+
+def sq_silu_mul_quant(gu, s, xq, sx, h=None, stream=None):
+    """gu [M, 2I] = [gate | up] rows; xq [M, I] int8 and sx [M] fp32 out; h [M, I]
+    (gu's dtype) receives SiLU(gate) * up when given."""
+    M, I2 = gu.shape
+    _check("sq_silu_mul_quant",
+           lib().sq_silu_mul_quant(_ptr(gu), _dtype_code(gu), M, I2 // 2, _ptr(s), _ptr(xq), _ptr(sx),
+                                   None if h is None else _ptr(h), _stream(stream)))
 
 
 def sq_w8a8_gemm(xq, sx, wq, sw, y, stream=None):

@@ -230,11 +230,11 @@ sq_status launch_row_scale(const T *in, int64_t rows, int64_t K, const float *s,
 
 // Single-pass quantiser (row in registers): 2^log2g warps per row, CH chunks
 // per lane.
-template <typename T, int MODE, int CH, bool FIT, bool BB>
+template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false>
 sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
-                               float *scale, int log2g, cudaStream_t st, const DeviceInfo &di)
+                               float *scale, int log2g, cudaStream_t st, const DeviceInfo &di, T *hout = nullptr)
 {
-    auto kernel = sq::row_quant_kernel<T, MODE, CH, FIT, BB>;
+    auto kernel = sq::row_quant_kernel<T, MODE, CH, FIT, BB, GLU>;
     const int smem = static_cast<int>(sq::row_quant_smem(K, BB));
     static std::atomic<uint64_t> attr_done{0};
     // the kernel also has a little static shared memory (the group maxima)
@@ -270,7 +270,46 @@ sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float
         std::fprintf(stderr, "sq quant rows=%lld K=%lld: single pass CH=%d G=%d per_sm=%d blocks=%lld\n",
                      (long long)rows, (long long)K, CH, 1 << log2g, per_sm, (long long)blocks);
     return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(sq::kQuantThreads), smem, st, 0, 0, in, rows,
-                         K, s, log2g, q, scale);
+                         K, s, log2g, q, scale, hout);
+}
+
+// The quantiser with the gated feed-forward activation in front (rows of
+// [gate | up], 2K values each): single pass only, 8 chunks per lane (two CTAs
+// per SM: the up half doubles the registers a row takes) or 16 for rows too
+// long for that (one CTA per SM).
+template <typename T>
+sq_status launch_glu_quant(const T *gu, int64_t rows, int64_t K, const float *s, int8_t *q, float *scale, T *hout,
+                           cudaStream_t st)
+{
+    DeviceInfo di;
+    if (!device_info(di))
+        return SQ_ERR_CUDA;
+    if (rows > 2147483647LL)
+        return SQ_ERR_UNSUPPORTED;
+    constexpr int V = sq::Vec<T>::N;
+    const int64_t nch = K / V;
+    const bool bb = V == 8 && sq::row_quant_smem(K, true) <= 64 * 1024;
+    if (sq::row_quant_smem(K, bb) > kMaxDynSmem - 1024)
+        return SQ_ERR_UNSUPPORTED;
+    for (int ch : {8, 16}) {
+        int log2g = 0;
+        while (log2g < 3 && ((int64_t)32 * ch << log2g) < nch)
+            ++log2g;
+        if (((int64_t)32 * ch << log2g) < nch)
+            continue;
+        const bool fit = ((int64_t)32 * ch << log2g) == nch &&
+                         rows * (1 << log2g) >= (int64_t)di.sms * 2 * (sq::kQuantThreads / 32);
+#define SQ_GLU_CFG(CH_, FIT_, BB_) \
+    launch_row_quant_cfg<T, sq::MODE_X, CH_, FIT_, BB_, true>(gu, rows, K, s, q, scale, log2g, st, di, hout)
+        if (ch == 8) {
+            if (bb)
+                return fit ? SQ_GLU_CFG(8, true, true) : SQ_GLU_CFG(8, false, true);
+            return fit ? SQ_GLU_CFG(8, true, false) : SQ_GLU_CFG(8, false, false);
+        }
+        return fit ? SQ_GLU_CFG(16, true, false) : SQ_GLU_CFG(16, false, false);
+#undef SQ_GLU_CFG
+    }
+    return SQ_ERR_UNSUPPORTED;
 }
 
 template <typename T, int MODE>
@@ -796,6 +835,23 @@ sq_status sq_rmsnorm_quant(const void *h, sq_dtype dt, int64_t M, int64_t K, con
     if (dt == SQ_BF16)
         return launch_rmsnorm_quant(static_cast<const __nv_bfloat16 *>(h), M, K, g, eps, xq, sx, rinv, st);
     return launch_rmsnorm_quant(static_cast<const float *>(h), M, K, g, eps, xq, sx, rinv, st);
+}
+
+sq_status sq_silu_mul_quant(const void *gu, sq_dtype dt, int64_t M, int64_t I, const float *s, int8_t *xq,
+                            float *sx, void *h, sq_stream_t stream)
+{
+    if (gu == nullptr || s == nullptr || xq == nullptr || sx == nullptr || !valid_dtype(dt) || M < 1 || I < 16 ||
+        I % 16 != 0 || !aligned16(gu) || !aligned16(s) || !aligned16(xq) || !aligned16(sx) ||
+        (h != nullptr && !aligned16(h)))
+        return SQ_ERR_INVALID_ARG;
+    const int64_t imax = dt == SQ_BF16 ? 32768 : 16384;
+    if (I > imax || M > kMaxDim)
+        return SQ_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dt == SQ_BF16)
+        return launch_glu_quant(static_cast<const __nv_bfloat16 *>(gu), M, I, s, xq, sx, static_cast<__nv_bfloat16 *>(h),
+                                st);
+    return launch_glu_quant(static_cast<const float *>(gu), M, I, s, xq, sx, static_cast<float *>(h), st);
 }
 
 sq_status sq_w8a8_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,

@@ -16,6 +16,7 @@
 #include <cstdint>
 
 #include "sq_div.cuh"
+#include "sq_glu.cuh"
 #include "sq_mem.cuh"
 
 namespace sq {
@@ -460,14 +461,13 @@ __device__ __forceinline__ void store_code_words(int8_t *dst, const uint32_t *y,
         *reinterpret_cast<uint32_t *>(dst) = pack_code_bytes(y[0], y[1], y[2], y[3]);
 }
 
-//   exact codes of the chunk (re-read from L2), overwriting what the fast path stored
+//   exact codes of the chunk (raw bits from the registers), overwriting what the fast path stored
 template <typename T, int MODE>
-__device__ __noinline__ void chunk_store_exact_codes(const T *__restrict__ p, const float *__restrict__ sc, float scale,
-                                                     int8_t *dst)
+__device__ __noinline__ void chunk_store_exact_codes(uint4 raw, const float *__restrict__ sc, float scale, int8_t *dst)
 {
     constexpr int V = Vec<T>::N;
     float x[V];
-    widen<T>(__ldg(reinterpret_cast<const uint4 *>(p)), x);
+    widen<T>(raw, x);
     uint32_t y[8];
     for (int e = 0; e < V; ++e) {
         const float sv = __ldg(sc + e);
@@ -500,11 +500,13 @@ __host__ __device__ constexpr int64_t row_quant_smem(int64_t K, bool bf) { retur
 // FIT: the G warps of a row cover its chunks exactly (32 CH G = K / V), so
 // no chunk needs a bounds check.  BB (bf16 rows only): bound |v| in packed
 // bf16 arithmetic (fewer instructions, a wider candidate window and a second
-// factor table in shared memory) instead of fp32.
-template <typename T, int MODE, int CH, bool FIT, bool BB>
-__global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
+// factor table in shared memory) instead of fp32.  GLU: each input row is
+// [gate | up] (2K values) and the row quantised is h = SiLU(gate) * up
+// (sq_glu.cuh), written to hout as well when hout is not null.
+template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false>
+__global__ void __launch_bounds__(kQuantThreads, (GLU ? (CH <= 8 ? 2 : 1) : (CH <= 8 ? 3 : 2)))
     row_quant_kernel(const T *__restrict__ in, int64_t rows, int64_t K, const float *__restrict__ s,
-                     int log2g, int8_t *__restrict__ q, float *__restrict__ scale_out)
+                     int log2g, int8_t *__restrict__ q, float *__restrict__ scale_out, T *__restrict__ hout)
 {
     pdl_prologue();
     constexpr int V = Vec<T>::N;
@@ -526,13 +528,23 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
     int64_t row = static_cast<int64_t>(blockIdx.x) * slots + slot;
     const int64_t rstride = static_cast<int64_t>(gridDim.x) * slots;
 
+    const int64_t ld = GLU ? 2 * K : K;  // input row stride
     uint4 raw[CH];
+    uint4 uraw[GLU ? CH : 1];  // GLU: the up half of the row
     auto load_row = [&](int64_t r) {
-        const T *src = in + r * K;
+        const T *src = in + r * ld;
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
             const int c = c0 + cstep * i;
             raw[i] = (FIT || c < nch) ? ld_chunk<T>(src + static_cast<int64_t>(c) * V) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        if constexpr (GLU) {
+#pragma unroll
+            for (int i = 0; i < CH; ++i) {
+                const int c = c0 + cstep * i;
+                uraw[i] = (FIT || c < nch) ? ld_chunk<T>(src + K + static_cast<int64_t>(c) * V)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+            }
         }
     };
     if (row < rows)
@@ -568,6 +580,43 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
     };
 
     while (row < rows) {
+        if constexpr (GLU) {
+            // 0. h = SiLU(gate) * up into raw[]: the fast path for bf16 rows,
+            // the definition for fp32 rows and for the chunks the fast path
+            // cannot decide (re-read from L2, outside the unrolled loop)
+            uint32_t redo = 0;
+#pragma unroll
+            for (int i = 0; i < CH; ++i) {
+                const int c = c0 + cstep * i;
+                if (FIT || c < nch) {
+                    if constexpr (V == 8) {
+                        bool r;
+                        raw[i] = glu_chunk_fast(raw[i], uraw[i], r);
+                        redo |= r ? (1u << i) : 0u;
+                    } else {
+                        raw[i] = glu_chunk_exact<T>(raw[i], uraw[i]);
+                    }
+                }
+            }
+            while (redo != 0u) {
+                const int i = __ffs(redo) - 1;
+                redo &= redo - 1u;
+                const int64_t c = c0 + cstep * i;
+                const uint4 hv = glu_chunk_exact_at<T>(in + row * ld + c * V, in + row * ld + K + c * V);
+#pragma unroll
+                for (int j = 0; j < CH; ++j)
+                    if (j == i)
+                        raw[j] = hv;
+            }
+            if (hout != nullptr) {
+#pragma unroll
+                for (int i = 0; i < CH; ++i) {
+                    const int c = c0 + cstep * i;
+                    if (FIT || c < nch)
+                        *reinterpret_cast<uint4 *>(hout + row * K + static_cast<int64_t>(c) * V) = raw[i];
+                }
+            }
+        }
         // 1. bounds of |v| per chunk, the row's largest bound A, the exact maximum E
         float hm[CH];
         float am = 0.0f;
@@ -668,7 +717,17 @@ __global__ void __launch_bounds__(kQuantThreads, (CH <= 8 ? 3 : 2))
             const int i = __ffs(ties) - 1;
             ties &= ties - 1u;
             const int64_t c = c0 + cstep * i;
-            chunk_store_exact_codes<T, MODE>(in + row * K + c * V, s + c * V, scale, dst + c * V);
+            uint4 v;
+            if constexpr (GLU) {  // h exists only in the registers
+                v = raw[0];
+#pragma unroll
+                for (int j = 1; j < CH; ++j)
+                    if (j == i)
+                        v = raw[j];
+            } else {  // re-read from L2: keeps raw[] dead after the code loop
+                v = __ldg(reinterpret_cast<const uint4 *>(in + row * K + c * V));
+            }
+            chunk_store_exact_codes<T, MODE>(v, s + c * V, scale, dst + c * V);
         }
         row += rstride;
         if (row < rows)

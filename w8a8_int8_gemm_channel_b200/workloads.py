@@ -12,6 +12,8 @@ name, the tensor name and a base seed):
     bf16 tensors are rounded to bf16 after the scaling;
   * the MLP down-projection input is SiLU(g) * u with g, u ~ N(0, 1) in fp32,
     then the outlier scaling, then bf16;
+  * the same input before the gated activation, [gate | up] (2K values a
+    row): g, u ~ N(0, 1) in fp32 with u's outlier channels scaled, then bf16;
   * weights: N(0, sigma) with sigma 0.02 (8B shapes, small case) or 0.015
     (70B shapes).
 The outlier count is round(0.001 * K): 4 at K=4096, 8 at 8192, 14 at 14336 and
@@ -181,6 +183,26 @@ def activations(
     idx = torch.tensor(outlier_channels(wl, K, base_seed), device=device, dtype=torch.long)
     x[:, idx] *= wl.outlier_scale
     return x.to(_torch_dtype(dtype or wl.dtype))
+
+
+def gate_up(
+    wl: Workload,
+    lin: Linear,
+    rows: int,
+    tensor: str,
+    device="cpu",
+    base_seed: int = 0,
+    dtype: Optional[str] = None,
+) -> torch.Tensor:
+    """[rows, 2K] = [gate | up], the feed-forward projections before the gated
+    activation of the down projection (K = lin.K): N(0, 1) each, the up half
+    scaled at the workload's outlier channels."""
+    K = lin.K
+    g = _gen(device, seed_for(wl.name, f"{tensor}/{lin.name}/gate_up/{rows}", base_seed))
+    gu = torch.randn(rows, 2 * K, generator=g, device=device, dtype=torch.float32)
+    idx = torch.tensor(outlier_channels(wl, K, base_seed), device=device, dtype=torch.long)
+    gu[:, K + idx] *= wl.outlier_scale
+    return gu.to(_torch_dtype(dtype or wl.dtype))
 
 
 def calibration(wl: Workload, lin: Linear, device="cpu", base_seed: int = 0, tokens: Optional[int] = None):
