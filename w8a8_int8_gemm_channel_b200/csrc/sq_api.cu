@@ -230,6 +230,16 @@ sq_status launch_row_scale(const T *in, int64_t rows, int64_t K, const float *s,
 
 // Single-pass quantiser (row in registers): 2^log2g warps per row, CH chunks
 // per lane.
+// log2 of the warps per row for an exact fit of `ch` chunks a lane (-1: none),
+// taken only when the rows fill the SMs at that width
+inline int exact_fit_log2g(int64_t nch, int ch, int64_t rows, const DeviceInfo &di)
+{
+    for (int log2g = 0; log2g <= 3; ++log2g)
+        if (((int64_t)32 * ch << log2g) == nch)
+            return rows * (1 << log2g) >= (int64_t)di.sms * 2 * (sq::kQuantThreads / 32) ? log2g : -1;
+    return -1;
+}
+
 template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false>
 sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
                                float *scale, int log2g, cudaStream_t st, const DeviceInfo &di, T *hout = nullptr)
@@ -291,6 +301,13 @@ sq_status launch_glu_quant(const T *gu, int64_t rows, int64_t K, const float *s,
     const bool bb = V == 8 && sq::row_quant_smem(K, true) <= 64 * 1024;
     if (sq::row_quant_smem(K, bb) > kMaxDynSmem - 1024)
         return SQ_ERR_UNSUPPORTED;
+#define SQ_GLU_CFG(CH_, FIT_, BB_) \
+    launch_row_quant_cfg<T, sq::MODE_X, CH_, FIT_, BB_, true>(gu, rows, K, s, q, scale, log2g, st, di, hout)
+    if constexpr (V == 8) {  // 7 chunks a lane where that fits exactly and 8 does not
+        const int log2g = exact_fit_log2g(nch, 8, rows, di) < 0 ? exact_fit_log2g(nch, 7, rows, di) : -1;
+        if (log2g >= 0)
+            return bb ? SQ_GLU_CFG(7, true, true) : SQ_GLU_CFG(7, true, false);
+    }
     for (int ch : {8, 16}) {
         int log2g = 0;
         while (log2g < 3 && ((int64_t)32 * ch << log2g) < nch)
@@ -299,8 +316,6 @@ sq_status launch_glu_quant(const T *gu, int64_t rows, int64_t K, const float *s,
             continue;
         const bool fit = ((int64_t)32 * ch << log2g) == nch &&
                          rows * (1 << log2g) >= (int64_t)di.sms * 2 * (sq::kQuantThreads / 32);
-#define SQ_GLU_CFG(CH_, FIT_, BB_) \
-    launch_row_quant_cfg<T, sq::MODE_X, CH_, FIT_, BB_, true>(gu, rows, K, s, q, scale, log2g, st, di, hout)
         if (ch == 8) {
             if (bb)
                 return fit ? SQ_GLU_CFG(8, true, true) : SQ_GLU_CFG(8, false, true);
