@@ -119,11 +119,36 @@ __device__ __forceinline__ uint4 glu_chunk_exact(const uint4 &g, const uint4 &u)
     }
 }
 
-// the rare path, out of line: the chunk's gate and up re-read (from L2)
-template <typename T>
-__device__ __noinline__ uint4 glu_chunk_exact_at(const T *__restrict__ gp, const T *__restrict__ up)
+// a bf16 rounding midpoint within kGluWindow patterns of b:
+// ((b + 0x8000 + W) mod 2^16) <= 2W, tested in the high half-word
+__device__ __forceinline__ bool glu_near_midpoint(uint32_t b)
 {
-    return glu_chunk_exact<T>(__ldg(reinterpret_cast<const uint4 *>(gp)), __ldg(reinterpret_cast<const uint4 *>(up)));
+    constexpr uint32_t add = (0x8000u + kGluWindow) << 16;
+    constexpr uint32_t lim = (2u * kGluWindow) << 16;
+    return (b * 65536u + add) <= lim;
+}
+
+// v' of the fast path for one element
+__device__ __forceinline__ float glu_value_fast(float g, float u)
+{
+    const float d = __fadd_rn(ex2_approx(__fmul_rn(g, -kLog2e)), 1.0f);
+    return __fmul_rn(__fmul_rn(g, rcp_approx(d)), u);
+}
+
+// The rare path, out of line, for a bf16 chunk the fast path could not
+// decide (its raw gate and up, still in registers): each element keeps its
+// fast value unless it is the one (or ones) that needs the definition.
+__device__ __noinline__ uint4 glu_chunk_fix(uint4 g, uint4 u)
+{
+    float gv[8], uv[8], hv[8];
+    widen<__nv_bfloat16>(g, gv);
+    widen<__nv_bfloat16>(u, uv);
+    for (int e = 0; e < 8; ++e) {
+        const float v = glu_value_fast(gv[e], uv[e]);
+        hv[e] = (glu_near_midpoint(__float_as_uint(v)) || !(gv[e] >= kGluGateMin)) ? glu_value(gv[e], uv[e]) : v;
+    }
+    return make_uint4(bf16x2_rn(hv[0], hv[1]), bf16x2_rn(hv[2], hv[3]), bf16x2_rn(hv[4], hv[5]),
+                      bf16x2_rn(hv[6], hv[7]));
 }
 
 // h of one bf16 chunk by the fast path; `redo` is set when the chunk must take
@@ -135,10 +160,6 @@ __device__ __forceinline__ uint4 glu_chunk_fast(const uint4 &g, const uint4 &u, 
     uint32_t hw[4];
     const float2 nl2e = make_float2(-kLog2e, -kLog2e);
     const float2 one2 = make_float2(1.0f, 1.0f);
-    // a rounding midpoint of bf16 within kGluWindow patterns of b:
-    // ((b + 0x8000 + W) mod 2^16) <= 2W, tested in the high half-word
-    constexpr uint32_t add = (0x8000u + kGluWindow) << 16;
-    constexpr uint32_t lim = (2u * kGluWindow) << 16;
     bool near = false;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -148,8 +169,8 @@ __device__ __forceinline__ uint4 glu_chunk_fast(const uint4 &g, const uint4 &u, 
         const float2 d = f2_add(make_float2(ex2_approx(t.x), ex2_approx(t.y)), one2);
         const float2 v = f2_mul(f2_mul(g2, make_float2(rcp_approx(d.x), rcp_approx(d.y))), u2);
         const uint32_t bx = __float_as_uint(v.x), by = __float_as_uint(v.y);
-        near |= (bx * 65536u + add) <= lim;
-        near |= (by * 65536u + add) <= lim;
+        near |= glu_near_midpoint(bx);
+        near |= glu_near_midpoint(by);
         hw[k] = bf16x2_rn(v.x, v.y);
     }
     // the smallest gate of the chunk

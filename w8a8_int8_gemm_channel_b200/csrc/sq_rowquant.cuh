@@ -582,8 +582,9 @@ __global__ void __launch_bounds__(kQuantThreads, (GLU ? (CH <= 8 ? 2 : 1) : (CH 
     while (row < rows) {
         if constexpr (GLU) {
             // 0. h = SiLU(gate) * up into raw[]: the fast path for bf16 rows,
-            // the definition for fp32 rows and for the chunks the fast path
-            // cannot decide (re-read from L2, outside the unrolled loop)
+            // the definition for fp32 rows and for the elements the fast path
+            // cannot decide (their chunks keep the gate in raw[] until a loop
+            // outside the unrolled one fixes them from the registers)
             uint32_t redo = 0;
 #pragma unroll
             for (int i = 0; i < CH; ++i) {
@@ -591,22 +592,31 @@ __global__ void __launch_bounds__(kQuantThreads, (GLU ? (CH <= 8 ? 2 : 1) : (CH 
                 if (FIT || c < nch) {
                     if constexpr (V == 8) {
                         bool r;
-                        raw[i] = glu_chunk_fast(raw[i], uraw[i], r);
+                        const uint4 hv = glu_chunk_fast(raw[i], uraw[i], r);
+                        raw[i] = r ? raw[i] : hv;
                         redo |= r ? (1u << i) : 0u;
                     } else {
                         raw[i] = glu_chunk_exact<T>(raw[i], uraw[i]);
                     }
                 }
             }
-            while (redo != 0u) {
-                const int i = __ffs(redo) - 1;
-                redo &= redo - 1u;
-                const int64_t c = c0 + cstep * i;
-                const uint4 hv = glu_chunk_exact_at<T>(in + row * ld + c * V, in + row * ld + K + c * V);
+            if constexpr (V == 8) {
+                while (redo != 0u) {
+                    const int i = __ffs(redo) - 1;
+                    redo &= redo - 1u;
+                    uint4 gq = raw[0], uq = uraw[0];
 #pragma unroll
-                for (int j = 0; j < CH; ++j)
-                    if (j == i)
-                        raw[j] = hv;
+                    for (int j = 1; j < CH; ++j)
+                        if (j == i) {
+                            gq = raw[j];
+                            uq = uraw[j];
+                        }
+                    const uint4 hv = glu_chunk_fix(gq, uq);
+#pragma unroll
+                    for (int j = 0; j < CH; ++j)
+                        if (j == i)
+                            raw[j] = hv;
+                }
             }
             if (hout != nullptr) {
 #pragma unroll
