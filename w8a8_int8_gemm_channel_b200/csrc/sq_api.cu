@@ -230,13 +230,12 @@ sq_status launch_row_scale(const T *in, int64_t rows, int64_t K, const float *s,
 
 // Single-pass quantiser (row in registers): 2^log2g warps per row, CH chunks
 // per lane.
-// log2 of the warps per row for an exact fit of `ch` chunks a lane (-1: none),
-// taken only when the rows fill the SMs at that width
-inline int exact_fit_log2g(int64_t nch, int ch, int64_t rows, const DeviceInfo &di)
+// log2 of the warps per row for an exact fit of `ch` chunks a lane (-1: none)
+inline int exact_fit_log2g(int64_t nch, int ch)
 {
     for (int log2g = 0; log2g <= 3; ++log2g)
         if (((int64_t)32 * ch << log2g) == nch)
-            return rows * (1 << log2g) >= (int64_t)di.sms * 2 * (sq::kQuantThreads / 32) ? log2g : -1;
+            return log2g;
     return -1;
 }
 
@@ -303,9 +302,13 @@ sq_status launch_glu_quant(const T *gu, int64_t rows, int64_t K, const float *s,
         return SQ_ERR_UNSUPPORTED;
 #define SQ_GLU_CFG(CH_, FIT_, BB_) \
     launch_row_quant_cfg<T, sq::MODE_X, CH_, FIT_, BB_, true>(gu, rows, K, s, q, scale, log2g, st, di, hout)
+    // an exact fit once the rows give every SM 4 warps or more; fewer rows
+    // rather spread over more warps (the SiLU step makes a row's work heavier
+    // than in sq_quant_act: measured at M = 128 and 1024, I = 4096)
+    const int64_t min_warps = (int64_t)di.sms * 4;
     if constexpr (V == 8) {  // 7 chunks a lane where that fits exactly and 8 does not
-        const int log2g = exact_fit_log2g(nch, 8, rows, di) < 0 ? exact_fit_log2g(nch, 7, rows, di) : -1;
-        if (log2g >= 0)
+        int log2g = exact_fit_log2g(nch, 8) < 0 ? exact_fit_log2g(nch, 7) : -1;
+        if (log2g >= 0 && rows * (1 << log2g) >= min_warps)
             return bb ? SQ_GLU_CFG(7, true, true) : SQ_GLU_CFG(7, true, false);
     }
     for (int ch : {8, 16}) {
@@ -314,8 +317,7 @@ sq_status launch_glu_quant(const T *gu, int64_t rows, int64_t K, const float *s,
             ++log2g;
         if (((int64_t)32 * ch << log2g) < nch)
             continue;
-        const bool fit = ((int64_t)32 * ch << log2g) == nch &&
-                         rows * (1 << log2g) >= (int64_t)di.sms * 2 * (sq::kQuantThreads / 32);
+        const bool fit = ((int64_t)32 * ch << log2g) == nch && rows * (1 << log2g) >= min_warps;
         if (ch == 8) {
             if (bb)
                 return fit ? SQ_GLU_CFG(8, true, true) : SQ_GLU_CFG(8, false, true);
@@ -344,6 +346,25 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
     // the bf16 bound while both factor tables stay small (about 3 CTAs per SM)
     const bool bb = V == 8 && sq::row_quant_smem(K, true) <= 64 * 1024;
     if (force_kind != 2 && sq::row_quant_smem(K, bb) <= kMaxDynSmem - 1024) {
+        // tuning override: SQ_QUANT_CH=2|4|8 takes that many chunks a lane
+        // wherever it fits a row exactly (same arithmetic, another shape)
+        static const int force_ch = std::getenv("SQ_QUANT_CH") ? std::atoi(std::getenv("SQ_QUANT_CH")) : 0;
+        if (force_ch == 2 || force_ch == 4 || force_ch == 8) {
+            int g = -1;
+            for (int l = 0; l <= 3 && g < 0; ++l)
+                if (((int64_t)32 * force_ch << l) == nch)
+                    g = l;
+            if (g >= 0) {
+#define SQ_Q_CFG(CH_) (bb ? launch_row_quant_cfg<T, MODE, CH_, true, true>(in, rows, K, s, q, scale, g, st, di) \
+                          : launch_row_quant_cfg<T, MODE, CH_, true, false>(in, rows, K, s, q, scale, g, st, di))
+                if (force_ch == 2)
+                    return SQ_Q_CFG(2);
+                if (force_ch == 4)
+                    return SQ_Q_CFG(4);
+                return SQ_Q_CFG(8);
+#undef SQ_Q_CFG
+            }
+        }
         // 8 chunks per lane (three CTAs per SM), 16 for rows too long for that
         for (int ch : {8, 16}) {
             int log2g = 0;
@@ -351,9 +372,10 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
                 ++log2g;
             if (((int64_t)32 * ch << log2g) < nch)
                 continue;
-            // an exact fit drops the bounds checks; few rows rather spread over more warps
-            const bool fit = ((int64_t)32 * ch << log2g) == nch &&
-                             rows * (1 << log2g) >= (int64_t)di.sms * 2 * (sq::kQuantThreads / 32);
+            // an exact fit drops the bounds checks and idle lanes; it is taken
+            // however few the rows (measured: at M = 128 and 1024, K = 4096, as
+            // fast as or faster than spreading each row over more warps)
+            const bool fit = ((int64_t)32 * ch << log2g) == nch;
             if (bb) {
                 if (ch == 8)
                     return fit ? launch_row_quant_cfg<T, MODE, 8, true, true>(in, rows, K, s, q, scale, log2g, st, di)
