@@ -225,12 +225,13 @@ class Step:
 
     def launches_per_step(self):
         """Kernels of this library one step launches: the calibration absmax
-        (1); per linear the weight's input-channel absmax and the factors (2)
-        and the weight quantiser; per token count and linear either the fused
-        linear (1) or the activation quantiser and the GEMM (1)."""
+        (1); per linear the zeroing of the factors' accumulator, the weight's
+        input-channel absmax and the factors (3) and the weight quantiser; per
+        token count and linear either the fused linear (1) or the activation
+        quantiser and the GEMM (1)."""
         q = self.quant_kernels()
         n = 1
-        n += (2 + q) * len(self.lins)
+        n += (3 + q) * len(self.lins)
         for M in self.wl.Ms:
             n += len(self.lins) * (1 if self.fused(M) else q + 1)
         return n

@@ -800,15 +800,16 @@ sq_status sq_smooth_factors(const float *ax, const void *w, sq_dtype dt, int64_t
         return SQ_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // B_j accumulates into s (as fp32 bit patterns), then s is overwritten in place.
-    if (cudaMemsetAsync(s, 0, static_cast<size_t>(K) * sizeof(float), st) != cudaSuccess)
-        return SQ_ERR_CUDA;
-    sq_status r = (dt == SQ_BF16)
+    const int threads = 256;
+    const unsigned blocks = static_cast<unsigned>((K + threads - 1) / threads);
+    sq_status r = launch_kernel(sq::zero_f32_kernel, dim3(blocks), dim3(threads), 0, st, 0, 0, s, K);
+    if (r != SQ_OK)
+        return r;
+    r = (dt == SQ_BF16)
                       ? launch_col_absmax(static_cast<const __nv_bfloat16 *>(w), N, K, K, s, st)
                       : launch_col_absmax(static_cast<const float *>(w), N, K, K, s, st);
     if (r != SQ_OK)
         return r;
-    const int threads = 256;
-    const unsigned blocks = static_cast<unsigned>((K + threads - 1) / threads);
     return launch_kernel(sq::smooth_factors_kernel, dim3(blocks), dim3(threads), 0, st, 0, 0, ax, s, aw, K, alpha);
 }
 

@@ -289,6 +289,16 @@ __global__ void fold_gamma_kernel(const float *__restrict__ gamma, const float *
         g[j] = __fdiv_rn(gamma[j], s[j]);
 }
 
+// Zero n floats: the accumulator of a column maximum, as a kernel so that it
+// takes part in the launch overlap of the stream (a memset does not).
+__global__ void zero_f32_kernel(float *__restrict__ p, int64_t n)
+{
+    pdl_prologue();
+    const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (j < n)
+        p[j] = 0.0f;
+}
+
 // ----------------------------------------------------------------------------
 // Smoothing factors, in place: on entry s holds B_j (as written by the
 // column-absmax kernel); on exit s_j = A_j^alpha / B_j^(1-alpha) evaluated in
