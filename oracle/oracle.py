@@ -70,6 +70,11 @@ def _load():
             lib.sqo_fold_gamma.argtypes = [P, P, I, P]
             lib.sqo_rmsnorm_quant.argtypes = [P, ctypes.c_int, I, I, P, ctypes.c_float, P, P, P, P]
             lib.sqo_f32_to_bf16.argtypes = [ctypes.c_float]
+            lib.sqo_gptq_hessian.argtypes = [P, ctypes.c_int, I, I, P, P]
+            lib.sqo_gptq_damp.argtypes = [P, I, ctypes.c_float]
+            lib.sqo_gptq_factor.argtypes = [P, I, P]
+            lib.sqo_gptq_factor.restype = ctypes.c_int
+            lib.sqo_gptq_quant_weight.argtypes = [P, ctypes.c_int, I, I, P, P, P, P]
             lib.sqo_exp_f32.argtypes = [ctypes.c_float]
             lib.sqo_exp_f32.restype = ctypes.c_float
             lib.sqo_silu_f32.argtypes = [ctypes.c_float]
@@ -242,6 +247,54 @@ def silu_mul_quant(gu: np.ndarray, s: np.ndarray):
     h = np.empty((M, I), np.float32)
     _load().sqo_silu_mul_quant(_ptr(gu), _dt(gu), M, I, _ptr(s), _ptr(xq), _ptr(sx), _ptr(h))
     return xq, sx, h
+
+
+def gptq_hessian(x: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """H = sum_t xh_t xh_t^T in fp64 (xh = X / s per element in fp32), [K, K]."""
+    x = _c(x)
+    s = _c(s, np.float32)
+    T, K = x.shape
+    H = np.empty((K, K), np.float64)
+    _load().sqo_gptq_hessian(_ptr(x), _dt(x), T, K, _ptr(s), _ptr(H))
+    return H
+
+
+def gptq_damp(H: np.ndarray, damp_frac: float) -> np.ndarray:
+    """A damped copy of H: damp_frac times the mean diagonal added to the diagonal."""
+    Hd = np.array(H, np.float64, order="C", copy=True)
+    _load().sqo_gptq_damp(_ptr(Hd), Hd.shape[0], float(damp_frac))
+    return Hd
+
+
+def gptq_factor(H: np.ndarray) -> np.ndarray:
+    """U, the upper Cholesky factor of H^-1 (H^-1 = U^T U); raises if H is not
+    positive definite."""
+    H = _c(H, np.float64)
+    K = H.shape[0]
+    U = np.empty((K, K), np.float64)
+    if _load().sqo_gptq_factor(_ptr(H), K, _ptr(U)) != 0:
+        raise ValueError("H is not positive definite")
+    return U
+
+
+def gptq_quant_weight(w: np.ndarray, s: np.ndarray, U: np.ndarray):
+    """GPTQ codes and per-channel scales of the smoothed weight W * s:
+    (wq int8 [N, K], sw fp32 [N])."""
+    w = _c(w)
+    s = _c(s, np.float32)
+    U = _c(U, np.float64)
+    N, K = w.shape
+    wq = np.empty((N, K), np.int8)
+    sw = np.empty(N, np.float32)
+    _load().sqo_gptq_quant_weight(_ptr(w), _dt(w), N, K, _ptr(s), _ptr(U), _ptr(wq), _ptr(sw))
+    return wq, sw
+
+
+def gptq(xcal: np.ndarray, w: np.ndarray, s: np.ndarray, damp_frac: float = 0.01):
+    """The whole GPTQ weight rounding: Hessian, damping, factor, rows."""
+    U = gptq_factor(gptq_damp(gptq_hessian(xcal, s), damp_frac))
+    wq, sw = gptq_quant_weight(w, s, U)
+    return wq, sw, U
 
 
 def gemm_i32(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:

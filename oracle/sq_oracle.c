@@ -48,6 +48,12 @@
  *        the feed-forward network itself; the gated SiLU form below is the
  *        one of the Llama-3-8B layers whose shapes the workloads use.
  *
+ *   [G]  "Understanding W8A8 INT8 LLM Quantization", section "How GPTQ
+ *        improves on naive quantization": quantise the weights of a channel
+ *        one at a time, and after each one push its rounding error onto the
+ *        channel's not yet quantised weights, weighted by the Hessian computed
+ *        from the calibration activations.
+ *
  * The smoothing-factor equation itself did not survive the page's text
  * extraction; this oracle uses s_j = A_j^alpha / B_j^(1-alpha), with A_j the
  * calibration absmax of input channel j and B_j the absmax of input channel j
@@ -430,6 +436,155 @@ void sqo_silu_mul_quant(const void *gu, int dt, int64_t M, int64_t I, const floa
             xq[m * I + j] = q;
         }
         free(h);
+    }
+}
+
+/* ------------------------------------------------------------------------
+ * [G] GPTQ.  Every step below is a fixed sequence of IEEE binary64
+ * operations (fma is one correctly rounded fused multiply-add), in the index
+ * order written, so that any implementation following it gets the same bits.
+ * ------------------------------------------------------------------------ */
+
+/* [G] the Hessian of the layer's squared output error over the calibration
+ * tokens, without the constant factor (which cancels in every use below):
+ *   H[i][j] = sum over t = 0, 1, ... of xh[t][i] * xh[t][j],
+ * with xh[t][k] = X[t][k] / s[k] (the smoothed activation, one fp32
+ * division, as in sqo_quant_act) widened to fp64; each step
+ * acc = fma(xh[t][i], xh[t][j], acc) from acc = 0. */
+void sqo_gptq_hessian(const void *x, int dt, int64_t T, int64_t K, const float *s, double *H)
+{
+    float *xh = (float *)malloc((size_t)(T * K) * sizeof(float));
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t k = 0; k < K; ++k)
+            xh[t * K + k] = elem(x, dt, (size_t)(t * K + k)) / s[k];
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t i = 0; i < K; ++i)
+        for (int64_t j = 0; j < K; ++j) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < T; ++t)
+                acc = fma((double)xh[t * K + i], (double)xh[t * K + j], acc);
+            H[i * K + j] = acc;
+        }
+    free(xh);
+}
+
+/* [G] damping, in place: d = RN(RN(sum_i H[i][i] / K) * damp_frac), the sum
+ * taken in index order; d = 1 when that sum is 0 (an all-zero Hessian);
+ * then H[i][i] = H[i][i] + d. */
+void sqo_gptq_damp(double *H, int64_t K, float damp_frac)
+{
+    double sum = 0.0;
+    for (int64_t i = 0; i < K; ++i)
+        sum = sum + H[i * K + i];
+    double d = (sum / (double)K) * (double)damp_frac;
+    if (sum == 0.0)
+        d = 1.0;
+    for (int64_t i = 0; i < K; ++i)
+        H[i * K + i] = H[i * K + i] + d;
+}
+
+/* [G] U, the upper triangular Cholesky factor of H^-1 (H^-1 = U^T U), which
+ * carries the error feedback: U[k][j] / U[k][k] is the share of weight k's
+ * error that weight j > k takes.  It is computed through the identity
+ * U = J L^-1 J, with J the index reversal and L the lower Cholesky factor of
+ * J H J (so no inverse of H itself is formed):
+ *   G[a][b] = H[K-1-a][K-1-b];
+ *   L (left-looking, column by column):
+ *     p = G[j][j]; p = fma(-L[j][k], L[j][k], p) for k = 0..j-1;
+ *     L[j][j] = sqrt(p)  (p <= 0: not positive definite, return -1);
+ *     for i > j: q = G[i][j]; q = fma(-L[i][k], L[j][k], q) for k = 0..j-1;
+ *                L[i][j] = q / L[j][j];
+ *   N = L^-1 (forward substitution, row by row):
+ *     N[i][i] = 1 / L[i][i];
+ *     for c < i: q = 0; q = fma(L[i][k], N[k][c], q) for k = c..i-1;
+ *                N[i][c] = -(q / L[i][i]);
+ *   U[a][b] = N[K-1-a][K-1-b] (zero below the diagonal).
+ * Returns 0, or -1 when a pivot is not positive. */
+int sqo_gptq_factor(const double *H, int64_t K, double *U)
+{
+    double *L = (double *)calloc((size_t)(K * K), sizeof(double));
+    double *N = (double *)calloc((size_t)(K * K), sizeof(double));
+    int bad = 0;
+    for (int64_t j = 0; j < K && !bad; ++j) {
+        double p = H[(K - 1 - j) * K + (K - 1 - j)];
+        for (int64_t k = 0; k < j; ++k)
+            p = fma(-L[j * K + k], L[j * K + k], p);
+        if (!(p > 0.0)) {
+            bad = 1;
+            break;
+        }
+        const double ljj = sqrt(p);
+        L[j * K + j] = ljj;
+#pragma omp parallel for schedule(static)
+        for (int64_t i = j + 1; i < K; ++i) {
+            double q = H[(K - 1 - i) * K + (K - 1 - j)];
+            for (int64_t k = 0; k < j; ++k)
+                q = fma(-L[i * K + k], L[j * K + k], q);
+            L[i * K + j] = q / ljj;
+        }
+    }
+    if (!bad) {
+        for (int64_t i = 0; i < K; ++i) {
+            N[i * K + i] = 1.0 / L[i * K + i];
+#pragma omp parallel for schedule(static)
+            for (int64_t c = 0; c < i; ++c) {
+                double q = 0.0;
+                for (int64_t k = c; k < i; ++k)
+                    q = fma(L[i * K + k], N[k * K + c], q);
+                N[i * K + c] = -(q / L[i * K + i]);
+            }
+        }
+        for (int64_t a = 0; a < K; ++a)
+            for (int64_t b = 0; b < K; ++b)
+                U[a * K + b] = b >= a ? N[(K - 1 - a) * K + (K - 1 - b)] : 0.0;
+    }
+    free(L);
+    free(N);
+    return bad ? -1 : 0;
+}
+
+/* [G] then [W]: GPTQ rounding of the smoothed weight, one output channel
+ * (row n) at a time:
+ *   w[k]  = W[n][k] * s[k] (one fp32 multiply, as in
+ *           sqo_smooth_quant_weight), widened to fp64;
+ *   sw[n] = max_k |w[k]| / 127 in fp32: the same per-channel scale as the
+ *           plain rounding, found once from the unmodified row;
+ *   for k = 0..K-1 in order:
+ *     q      = clamp(rint(w[k] / sw), -127, 127)  (fp64 division, rounding
+ *              half to even; q = 0 throughout when sw = 0)
+ *     e      = fma(-q, sw, w[k]) / U[k][k]
+ *     w[j]   = fma(-e, U[k][j], w[j]) for every j > k. */
+void sqo_gptq_quant_weight(const void *w, int dt, int64_t N, int64_t K, const float *s, const double *U,
+                           int8_t *wq, float *sw)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t n = 0; n < N; ++n) {
+        double *r = (double *)malloc((size_t)K * sizeof(double));
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            const float v = elem(w, dt, (size_t)(n * K + k)) * s[k];
+            r[k] = (double)v;
+            if (fabsf(v) > amax)
+                amax = fabsf(v);
+        }
+        const float scale = amax / 127.0f;
+        sw[n] = scale;
+        const double sd = (double)scale;
+        for (int64_t k = 0; k < K; ++k) {
+            double q = 0.0;
+            if (scale != 0.0f) {
+                q = nearbyint(r[k] / sd);
+                if (q > 127.0)
+                    q = 127.0;
+                if (q < -127.0)
+                    q = -127.0;
+                const double e = fma(-q, sd, r[k]) / U[k * K + k];
+                for (int64_t j = k + 1; j < K; ++j)
+                    r[j] = fma(-e, U[k * K + j], r[j]);
+            }
+            wq[n * K + k] = (int8_t)q;
+        }
+        free(r);
     }
 }
 

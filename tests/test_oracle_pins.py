@@ -594,3 +594,129 @@ def test_silu_mul_quant_zero_rows_and_fp32(oracle):
     assert sx[0] == 0.0 and sx[1] == 0.0 and not xq[:2].any()
     assert np.array_equal(h[2], oracle.silu_f32(gu[2, :I]) * np.float32(1.5))
     assert sx[2] == np.float32(np.abs(h[2]).max() / np.float32(127.0))
+
+
+# ---------------------------------------------------------------------------
+# GPTQ weight rounding ("Understanding W8A8 INT8 LLM Quantization", section
+# "How GPTQ improves on naive quantization")
+# ---------------------------------------------------------------------------
+
+def _correlated_calibration(rng, T, K):
+    """Calibration tokens with correlated channels (a few shared factors)."""
+    f = rng.standard_normal((T, 6))
+    mix = rng.standard_normal((6, K))
+    return (f @ mix + 0.3 * rng.standard_normal((T, K))).astype(np.float32)
+
+
+def test_gptq_hessian_is_the_gram_matrix(oracle):
+    rng = np.random.default_rng(70)
+    T, K = 96, 48
+    x = _correlated_calibration(rng, T, K)
+    s = f32(rng.uniform(0.5, 2.0, K))
+    H = oracle.gptq_hessian(x, s)
+    xh = (x / s).astype(np.float32).astype(np.float64)   # one fp32 division per element
+    assert np.allclose(H, xh.T @ xh, rtol=1e-12, atol=1e-12)
+    assert np.array_equal(H, H.T)
+
+
+def test_gptq_damping_closed_forms(oracle):
+    rng = np.random.default_rng(71)
+    A = rng.standard_normal((20, 20))
+    H = A @ A.T
+    Hd = oracle.gptq_damp(H, 0.01)
+    d = np.diag(Hd) - np.diag(H)
+    assert np.allclose(d, 0.01 * np.trace(H) / 20, rtol=1e-14)
+    assert np.array_equal(Hd - np.diag(np.diag(Hd)), H - np.diag(np.diag(H)))
+    assert np.array_equal(oracle.gptq_damp(np.zeros((5, 5)), 0.01), np.eye(5))
+
+
+def test_gptq_factor_is_the_cholesky_factor_of_the_inverse(oracle):
+    rng = np.random.default_rng(72)
+    K = 40
+    x = _correlated_calibration(rng, 200, K)
+    Hd = oracle.gptq_damp(oracle.gptq_hessian(x, np.ones(K, np.float32)), 0.01)
+    U = oracle.gptq_factor(Hd)
+    assert np.array_equal(U, np.triu(U)) and (np.diag(U) > 0).all()
+    assert np.allclose(U.T @ U @ Hd, np.eye(K), atol=1e-9)
+    ref = np.linalg.cholesky(np.linalg.inv(Hd)).T          # numpy / LAPACK, another route
+    assert np.allclose(U, ref, rtol=1e-8, atol=1e-12)
+    with pytest.raises(ValueError):
+        oracle.gptq_factor(-np.eye(4))
+
+
+def test_gptq_without_correlation_is_plain_rounding(oracle):
+    """No calibration signal (H = 0, so U = I after the unit damping), or
+    channels that never co-occur (diagonal H): no error is passed on and the
+    codes are the plain per-channel rounding's."""
+    rng = np.random.default_rng(73)
+    N, K = 24, 32
+    w = f32(rng.standard_normal((N, K)) * 0.02)
+    s = f32(rng.uniform(0.5, 2.0, K))
+    q_rtn, sw_rtn = oracle.smooth_quant_weight(w, s)
+    for x in (np.zeros((16, K), np.float32),
+              np.eye(K, dtype=np.float32) * f32(rng.uniform(0.5, 3.0, K))[:, None]):
+        q, sw, U = oracle.gptq(x, w, s)
+        assert np.array_equal(U, np.diag(np.diag(U)))
+        assert np.array_equal(q, q_rtn) and np.array_equal(sw, sw_rtn)
+
+
+def test_gptq_against_brute_force_obs(oracle):
+    """Tiny layers against the explicit form of the method: after rounding
+    weight k, spread its error over the remaining weights with the inverse of
+    the Hessian restricted to them, inverted afresh by numpy at every step."""
+    rng = np.random.default_rng(74)
+    N, K = 12, 10
+    x = _correlated_calibration(rng, 64, K)
+    w = f32(rng.standard_normal((N, K)) * 0.05)
+    s = np.ones(K, np.float32)
+    q, sw, _ = oracle.gptq(x, w, s)
+    Hd = oracle.gptq_damp(oracle.gptq_hessian(x, s), 0.01)
+    for n in range(N):
+        r = w[n].astype(np.float64).copy()
+        sc = float(np.float32(np.abs(w[n]).max() / np.float32(127.0)))
+        codes = []
+        for k in range(K):
+            qk = float(np.clip(np.rint(r[k] / sc), -127, 127))
+            codes.append(int(qk))
+            Hi = np.linalg.inv(Hd[k:, k:])
+            e = (r[k] - qk * sc) / Hi[0, 0]
+            r[k + 1:] -= e * Hi[0, 1:]
+        assert codes == q[n].tolist(), n
+        assert sw[n] == np.float32(sc)
+
+
+def test_gptq_reduces_output_error(oracle):
+    """The point of the method: on the calibration tokens the layer's output
+    error X (W' - Q)^T is smaller than plain rounding's."""
+    rng = np.random.default_rng(75)
+    N, K = 64, 96
+    x = _correlated_calibration(rng, 512, K)
+    w = f32(rng.standard_normal((N, K)) * 0.02)
+    s = f32(rng.uniform(0.7, 1.5, K))
+    q, sw, _ = oracle.gptq(x, w, s)
+    q_rtn, sw_rtn = oracle.smooth_quant_weight(w, s)
+    xh = (x / s).astype(np.float64)
+    wp = (w * s).astype(np.float64)
+    err = lambda qq, ss: np.linalg.norm(xh @ (wp - qq.astype(np.float64) * ss.astype(np.float64)[:, None]).T)
+    assert err(q, sw) < 0.8 * err(q_rtn, sw_rtn)
+
+
+def test_gptq_page_example_first_weight(oracle, golden):
+    """The page's channel: the first weight is rounded exactly as plain
+    rounding does (0.31 -> code 43, 0.3088 reconstructed), and with the page's
+    input as the calibration token the channel's output ends closer to the
+    original than plain rounding's."""
+    g = golden("weight_rtn_example.json")
+    w = f32([g["w_page_columns"]["ch0"], g["w_page_columns"]["ch1"]])
+    x = f32([g["x_page"]])
+    s = np.ones(3, F32)
+    q, sw, _ = oracle.gptq(x, w, s)
+    q_rtn, _ = oracle.smooth_quant_weight(w, s)
+    assert q[:, 0].tolist() == q_rtn[:, 0].tolist()
+    assert float(q[0, 0]) * float(sw[0]) == pytest.approx(0.3088, abs=6e-5)
+    xv = np.asarray(g["x_page"], np.float64)
+    for i in range(2):
+        y0 = float(w[i].astype(np.float64) @ xv)
+        yg = float((q[i] * np.float64(sw[i])) @ xv)
+        yr = float((q_rtn[i] * np.float64(sw[i])) @ xv)
+        assert abs(yg - y0) <= abs(yr - y0)
