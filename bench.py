@@ -466,7 +466,8 @@ def workload_config(wl):
 def run_case(spec, steps, warmup, flush_l2=True, settle_us=0.0):
     """Time one C-ABI call on synthetic data.  spec is one of
     gemm:M,N,K  linear:M,N,K  quant_act:M,K  quant_w:N,K  calib:T,K
-    smooth_factors:N,K  rmsnorm_quant:M,K  silu_mul_quant:M,I.  Prints one JSON line with the median time."""
+    smooth_factors:N,K  rmsnorm_quant:M,K  silu_mul_quant:M,I  gptq_hessian:T,K  gptq_factor:K
+    gptq_rows:N,K.  Prints one JSON line with the median time."""
     import w8a8_int8_gemm_channel_b200 as sq
 
     lib = sq.lib()
@@ -520,6 +521,39 @@ def run_case(spec, steps, warmup, flush_l2=True, settle_us=0.0):
         fn = lambda: lib.sq_silu_mul_quant(gu.data_ptr(), sq.SQ_BF16, M, I, s.data_ptr(), xq.data_ptr(),
                                            sx.data_ptr(), None, st)
         nbytes = 4 * M * I + M * I + 4 * I + 4 * M
+    elif kind in ("gptq_hessian", "gptq_factor", "gptq_rows"):
+        # GPTQ stages (offline): gptq_hessian:T,K  gptq_factor:K  gptq_rows:N,K
+        f64 = torch.float64
+        if kind == "gptq_hessian":
+            T_, K = d
+            x, s = r(T_, K), torch.rand(K, device=dev) + 0.5
+            H = torch.empty(K, K, dtype=f64, device=dev)
+            fn = lambda: lib.sq_gptq_hessian(x.data_ptr(), sq.SQ_BF16, T_, K, s.data_ptr(), H.data_ptr(), st)
+            nbytes = 2 * T_ * K + 8 * K * K
+        elif kind == "gptq_factor":
+            (K,) = d
+            xc = torch.randn(2 * K, K, device=dev, dtype=f64)
+            H0 = xc.T @ xc
+            H = H0.clone()
+            U = torch.empty_like(H)
+            ws = torch.empty(int(lib.sq_gptq_workspace_size(K)), dtype=torch.uint8, device=dev)
+
+            def fn():
+                H.copy_(H0)
+                return lib.sq_gptq_factor(H.data_ptr(), K, 0.01, U.data_ptr(), ws.data_ptr(), ws.numel(), st)
+            nbytes = 3 * 8 * K * K
+        else:
+            N, K = d
+            w, s = r(N, K, sc=0.02), torch.rand(K, device=dev) + 0.5
+            xc = torch.randn(2 * K, K, device=dev, dtype=f64)
+            H = xc.T @ xc
+            U = torch.empty_like(H)
+            ws = torch.empty(int(lib.sq_gptq_workspace_size(K)), dtype=torch.uint8, device=dev)
+            assert lib.sq_gptq_factor(H.data_ptr(), K, 0.01, U.data_ptr(), ws.data_ptr(), ws.numel(), st) == 0
+            wq, sw = torch.empty(N, K, dtype=i8, device=dev), torch.empty(N, device=dev)
+            fn = lambda: lib.sq_gptq_quant_weight(w.data_ptr(), sq.SQ_BF16, N, K, s.data_ptr(), U.data_ptr(),
+                                                  wq.data_ptr(), sw.data_ptr(), st)
+            nbytes = 2 * N * K + N * K + 4 * N
     elif kind == "quant_w":
         N, K = d
         w, s = r(N, K, sc=0.02), torch.rand(K, device=dev) + 0.5

@@ -197,6 +197,48 @@ SQ_API sq_status sq_silu_mul_quant(const void *gu, sq_dtype dt, int64_t M, int64
                                    int8_t *xq, float *sx, void *h, sq_stream_t stream);
 
 /*
+ * GPTQ weight rounding, offline, in place of sq_smooth_quant_weight's plain
+ * rounding ("Understanding W8A8 INT8 LLM Quantization", section "How GPTQ
+ * improves on naive quantization": quantise a channel's weights one at a
+ * time and push each rounding error onto the channel's not yet quantised
+ * weights, weighted by the Hessian from the calibration activations).  Three
+ * calls, each a fixed sequence of IEEE fp64 operations in a fixed order (so
+ * the results do not depend on the thread layout):
+ *
+ * sq_gptq_hessian: H[i][j] = sum over tokens t (ascending) of
+ *   xh[t][i] * xh[t][j], one fp64 FMA a term, with xh = RN_f32(x / s) (the
+ *   smoothed activation, as in sq_quant_act).  x [T, K] dtype dt (calibration
+ *   tokens); s [K]; H [K, K] fp64 out (overwritten; symmetric).
+ *
+ * sq_gptq_factor: damps H in place, H[i][i] += d with d =
+ *   RN(RN(sum_i H[i][i] / K) * damp_frac) (the sum in index order; d = 1 when
+ *   the sum is 0), then writes U [K, K] fp64, the upper Cholesky factor of
+ *   H^-1 (zero below the diagonal), through U = J L^-1 J: J reverses the
+ *   index order and L is the lower Cholesky factor of J H J, computed column
+ *   by column with every dot product in ascending index order; L^-1 by forward
+ *   substitution, row by row, the same way.  workspace: device scratch of at
+ *   least sq_gptq_workspace_size(K) bytes (K * K fp64).  A non-positive pivot
+ *   leaves U NaN and sets the device error word (sq_device_status returns
+ *   SQ_ERR_INVALID_ARG).  Takes 2K + 2 kernel launches.
+ *
+ * sq_gptq_quant_weight: per output channel n, w = RN_f32(W[n] * s) widened to
+ *   fp64 and sw[n] = RN_f32(max |w| / 127) (sq_smooth_quant_weight's scale);
+ *   then for k = 0 .. K-1 in order: q = clamp(rint(w[k] / sw[n]), -127, 127)
+ *   (fp64, half to even), e = fma(-q, sw[n], w[k]) / U[k][k], and
+ *   w[j] = fma(-e, U[k][j], w[j]) for every j > k.  w [N, K] dtype dt;
+ *   s [K]; U from sq_gptq_factor; wq [N, K] int8 out; sw [N] fp32 out.
+ *
+ * K a multiple of 16, at most 16384.
+ */
+SQ_API size_t sq_gptq_workspace_size(int64_t K);
+SQ_API sq_status sq_gptq_hessian(const void *x, sq_dtype dt, int64_t T, int64_t K, const float *s,
+                                 double *H, sq_stream_t stream);
+SQ_API sq_status sq_gptq_factor(double *H, int64_t K, float damp_frac, double *U, void *workspace,
+                                size_t ws_bytes, sq_stream_t stream);
+SQ_API sq_status sq_gptq_quant_weight(const void *w, sq_dtype dt, int64_t N, int64_t K, const float *s,
+                                      const double *U, int8_t *wq, float *sw, sq_stream_t stream);
+
+/*
  * W8A8 GEMM with the dequantising epilogue ("quant_llm_int8": int32
  * accumulation, outer product of row and column scales):
  *   acc[m, n] = sum_k xq[m, k] * wq[n, k]   (exact int32; K * 127^2 < 2^31,
@@ -271,9 +313,11 @@ SQ_API sq_status sq_linear_noalloc(const void *x, sq_dtype in_dt, const float *s
 
 /*
  * Device error word: synchronises `stream`, then reads and clears the error
- * word the kernels set when a bounded on-chip wait gives up.  Returns SQ_OK,
- * SQ_ERR_TIMEOUT (with the kernel's location code in *code when code is not
- * NULL) or SQ_ERR_CUDA if the synchronisation itself failed.
+ * word the kernels set when a bounded on-chip wait gives up, or when
+ * sq_gptq_factor meets a non-positive pivot.  Returns SQ_OK, SQ_ERR_TIMEOUT
+ * (a wait gave up), SQ_ERR_INVALID_ARG (code 0xA00: the GPTQ Hessian was not
+ * positive definite), with the kernel's location code in *code when code is
+ * not NULL, or SQ_ERR_CUDA if the synchronisation itself failed.
  */
 SQ_API sq_status sq_device_status(sq_stream_t stream, uint32_t *code);
 

@@ -453,19 +453,21 @@ void sqo_silu_mul_quant(const void *gu, int dt, int64_t M, int64_t I, const floa
  * acc = fma(xh[t][i], xh[t][j], acc) from acc = 0. */
 void sqo_gptq_hessian(const void *x, int dt, int64_t T, int64_t K, const float *s, double *H)
 {
-    float *xh = (float *)malloc((size_t)(T * K) * sizeof(float));
+    /* xh stored channel by channel (xt[k][t]) so that each sum reads memory
+     * in order; the arithmetic is as written above */
+    float *xt = (float *)malloc((size_t)(T * K) * sizeof(float));
     for (int64_t t = 0; t < T; ++t)
         for (int64_t k = 0; k < K; ++k)
-            xh[t * K + k] = elem(x, dt, (size_t)(t * K + k)) / s[k];
+            xt[k * T + t] = elem(x, dt, (size_t)(t * K + k)) / s[k];
 #pragma omp parallel for schedule(dynamic, 4)
     for (int64_t i = 0; i < K; ++i)
         for (int64_t j = 0; j < K; ++j) {
             double acc = 0.0;
             for (int64_t t = 0; t < T; ++t)
-                acc = fma((double)xh[t * K + i], (double)xh[t * K + j], acc);
+                acc = fma((double)xt[i * T + t], (double)xt[j * T + t], acc);
             H[i * K + j] = acc;
         }
-    free(xh);
+    free(xt);
 }
 
 /* [G] damping, in place: d = RN(RN(sum_i H[i][i] / K) * damp_frac), the sum
@@ -524,19 +526,22 @@ int sqo_gptq_factor(const double *H, int64_t K, double *U)
         }
     }
     if (!bad) {
+        /* N stored column by column (Nt[c][k] = N[k][c]) so that each sum reads
+         * memory in order; the arithmetic is as written above */
+        double *Nt = N;
         for (int64_t i = 0; i < K; ++i) {
-            N[i * K + i] = 1.0 / L[i * K + i];
+            Nt[i * K + i] = 1.0 / L[i * K + i];
 #pragma omp parallel for schedule(static)
             for (int64_t c = 0; c < i; ++c) {
                 double q = 0.0;
                 for (int64_t k = c; k < i; ++k)
-                    q = fma(L[i * K + k], N[k * K + c], q);
-                N[i * K + c] = -(q / L[i * K + i]);
+                    q = fma(L[i * K + k], Nt[c * K + k], q);
+                Nt[c * K + i] = -(q / L[i * K + i]);
             }
         }
         for (int64_t a = 0; a < K; ++a)
             for (int64_t b = 0; b < K; ++b)
-                U[a * K + b] = b >= a ? N[(K - 1 - a) * K + (K - 1 - b)] : 0.0;
+                U[a * K + b] = b >= a ? Nt[(K - 1 - b) * K + (K - 1 - a)] : 0.0;
     }
     free(L);
     free(N);

@@ -166,6 +166,30 @@ def test_silu_mul_quant_rejects_bad_arguments(lib):
     assert f(A, 0, 4, 32768, B, C, D, None, None) == UNS        # fp32 rows: at most 16384
 
 
+def test_gptq_entry_points_reject_bad_arguments(lib):
+    assert lib.sq_gptq_workspace_size(4096) == 4096 * 4096 * 8
+    assert lib.sq_gptq_workspace_size(40) == 0                     # not a multiple of 16
+    assert lib.sq_gptq_workspace_size(32768) == 0                  # beyond the limit
+    h = lib.sq_gptq_hessian
+    assert h(None, 1, 8, 64, B, C, None) == INV
+    assert h(A, 1, 0, 64, B, C, None) == INV                       # no tokens
+    assert h(A, 1, 8, 40, B, C, None) == INV                       # K not a multiple of 16
+    assert h(A, 7, 8, 64, B, C, None) == INV                       # bad dtype
+    assert h(A, 1, 8, 32768, B, C, None) == UNS
+    f = lib.sq_gptq_factor
+    assert f(A, 64, 0.01, B, None, 1 << 20, None) == INV           # no workspace
+    assert f(A, 64, 0.01, B, C, 64 * 64 * 8 - 1, None) == INV      # workspace too small
+    assert f(A, 64, -0.5, B, C, 1 << 20, None) == INV              # negative damping
+    assert f(A, 64, float("nan"), B, C, 1 << 20, None) == INV
+    assert f(A, 64, 0.01, A, C, 1 << 20, None) == INV              # U aliases H
+    assert f(A, 64, 0.01, MIS, C, 1 << 20, None) == INV
+    q = lib.sq_gptq_quant_weight
+    assert q(None, 1, 4, 64, B, C, D, E, None) == INV
+    assert q(A, 1, 0, 64, B, C, D, E, None) == INV
+    assert q(A, 1, 4, 24, B, C, D, E, None) == INV
+    assert q(A, 1, 4, 64, B, C, D, MIS, None) == INV
+
+
 def test_selftest_rejects_limits_out_of_range(lib):
     f = lib.sq_selftest_wait_timeout
     assert f(0, None) == INV

@@ -1,0 +1,125 @@
+"""Parity of the GPTQ weight rounding (sq_gptq_hessian, sq_gptq_factor,
+sq_gptq_quant_weight) against the CPU oracle on the same seeded bytes.
+
+Source: "Understanding W8A8 INT8 LLM Quantization", section "How GPTQ
+improves on naive quantization".
+
+Both sides follow one fixed sequence of IEEE fp64 operations, so everything
+is bit-exact: the Hessian, the damped Hessian, the factor U, the codes and the
+scales.
+"""
+import numpy as np
+import pytest
+import torch
+
+import w8a8_int8_gemm_channel_b200 as sq
+from w8a8_int8_gemm_channel_b200 import workloads as wlmod
+from tests.gpu_util import assert_bits_equal, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from w8a8_int8_gemm_channel_b200 import _build
+
+    _build.build()
+    yield
+    st, code = sq.sq_device_status()
+    assert st == sq.SQ_OK, f"device error word {code:#x}"
+
+
+def _case(T, K, N, dtype, seed):
+    """Calibration tokens with the workloads' outlier channels, a weight and
+    smoothing factors."""
+    wl = wlmod.WORKLOADS["llama3_8b_attn"]
+    lin = wlmod.Linear("gptq", N, K)
+    x = wlmod.activations(wl, lin, T, f"gptq{seed}", dtype=dtype)
+    w = wlmod.weight(wl, lin, rows=N, base_seed=seed).to(torch.float32)
+    w = w.to(torch.bfloat16 if dtype == "bf16" else torch.float32)
+    g = torch.Generator().manual_seed(seed)
+    s = (torch.rand(K, generator=g) * 1.5 + 0.5).numpy().astype(np.float32)
+    return to_np(x), to_np(w), s
+
+
+def _run(x_np, w_np, s_np, tdt, damp=0.01):
+    x, w, s = to_dev(x_np, tdt), to_dev(w_np, tdt), to_dev(s_np)
+    K = w.shape[1]
+    H = torch.empty(K, K, dtype=torch.float64, device="cuda")
+    U = torch.empty_like(H)
+    sq.sq_gptq_hessian(x, s, H)
+    H0 = H.clone()
+    sq.sq_gptq_factor(H, U, damp)
+    wq = torch.empty(w.shape, dtype=torch.int8, device="cuda")
+    sw = torch.empty(w.shape[0], device="cuda")
+    sq.sq_gptq_quant_weight(w, s, U, wq, sw)
+    torch.cuda.synchronize()
+    return to_np(H0), to_np(H), to_np(U), to_np(wq), to_np(sw)
+
+
+@pytest.mark.parametrize("T,K,N,dtype", [(16, 16, 8, "f32"), (64, 48, 20, "f32"), (200, 256, 96, "bf16"),
+                                         (1024, 512, 300, "bf16"), (33, 320, 17, "bf16")])
+def test_gptq_parity(T, K, N, dtype, oracle):
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    x, w, s = _case(T, K, N, dtype, seed=T + K)
+    H0, Hd, U, wq, sw = _run(x, w, s, tdt)
+    H0_o = oracle.gptq_hessian(x, s)
+    assert_bits_equal(H0.view(np.uint64), H0_o.view(np.uint64), "H")
+    Hd_o = oracle.gptq_damp(H0_o, 0.01)
+    assert_bits_equal(Hd.view(np.uint64), Hd_o.view(np.uint64), "damped H")
+    U_o = oracle.gptq_factor(Hd_o)
+    assert_bits_equal(U.view(np.uint64), U_o.view(np.uint64), "U")
+    q_o, sw_o = oracle.gptq_quant_weight(w, s, U_o)
+    assert_bits_equal(sw, sw_o, "scales")
+    assert_bits_equal(wq, q_o, "codes")
+
+
+def test_gptq_zero_calibration_is_plain_rounding(oracle):
+    """No calibration signal: H = 0, unit damping, U = I, and the codes are
+    those of sq_smooth_quant_weight."""
+    K, N = 128, 40
+    _, w_np, s_np = _case(8, K, N, "bf16", seed=5)
+    x_np = np.zeros((8, K), np.uint16)
+    _, _, U, wq, sw = _run(x_np, w_np, s_np, torch.bfloat16)
+    assert np.array_equal(U, np.eye(K))
+    w, s = to_dev(w_np, torch.bfloat16), to_dev(s_np)
+    q2 = torch.empty(N, K, dtype=torch.int8, device="cuda")
+    s2 = torch.empty(N, device="cuda")
+    sq.sq_smooth_quant_weight(w, s, q2, s2)
+    torch.cuda.synchronize()
+    assert np.array_equal(wq, to_np(q2)) and np.array_equal(sw, to_np(s2))
+
+
+def test_gptq_not_positive_definite_reports_and_recovers(oracle):
+    """A Hessian that is not positive definite (here -I, undamped): U is NaN,
+    the device status reports SQ_ERR_INVALID_ARG with code 0xA00, and the
+    context stays usable."""
+    K = 32
+    H = -torch.eye(K, dtype=torch.float64, device="cuda")
+    U = torch.empty_like(H)
+    sq.sq_gptq_factor(H, U, 0.0)
+    st, code = sq.sq_device_status()
+    assert st == sq.SQ_ERR_INVALID_ARG and code == 0xA00
+    assert torch.isnan(U.diagonal()).any()
+    st, code = sq.sq_device_status()
+    assert st == sq.SQ_OK and code == 0
+    x, w, s = _case(64, 64, 16, "f32", seed=9)
+    _, _, U2, wq, sw = _run(x, w, s, torch.float32)
+    q_o, sw_o, U_o = oracle.gptq(x, w, s)
+    assert_bits_equal(wq, q_o, "codes after the error")
+
+
+def test_gptq_full_width_sampled(oracle):
+    """K = 4096 (the attention projections' width) with 512 calibration
+    tokens: the factor and sampled rows against the oracle."""
+    T, K, N = 512, 4096, 64
+    x, w, s = _case(T, K, N, "bf16", seed=11)
+    H0, Hd, U, wq, sw = _run(x, w, s, torch.bfloat16)
+    U_o = oracle.gptq_factor(oracle.gptq_damp(oracle.gptq_hessian(x, s), 0.01))
+    assert_bits_equal(U.view(np.uint64), U_o.view(np.uint64), "U (K = 4096)")
+    rows = np.arange(0, N, 8)
+    q_o, sw_o = oracle.gptq_quant_weight(w[rows], s, U_o)
+    assert_bits_equal(sw[rows], sw_o, "scales (K = 4096)")
+    assert_bits_equal(wq[rows], q_o, "codes (K = 4096)")

@@ -47,6 +47,10 @@ ABI_SYMBOLS = (
     "sq_fold_gamma",
     "sq_rmsnorm_quant",
     "sq_silu_mul_quant",
+    "sq_gptq_workspace_size",
+    "sq_gptq_hessian",
+    "sq_gptq_factor",
+    "sq_gptq_quant_weight",
     "sq_w8a8_gemm",
     "sq_w8a8_gemm_s32",
     "sq_linear",
@@ -81,6 +85,10 @@ def _declare(lib):
         "sq_fold_gamma": ([P, P, I, P, P], E),
         "sq_rmsnorm_quant": ([P, E, I, I, P, F, P, P, P, P], E),
         "sq_silu_mul_quant": ([P, E, I, I, P, P, P, P, P], E),
+        "sq_gptq_workspace_size": ([I], ctypes.c_size_t),
+        "sq_gptq_hessian": ([P, E, I, I, P, P, P], E),
+        "sq_gptq_factor": ([P, I, F, P, P, ctypes.c_size_t, P], E),
+        "sq_gptq_quant_weight": ([P, E, I, I, P, P, P, P, P], E),
         "sq_w8a8_gemm": ([P, P, P, P, I, I, I, P, E, P], E),
         "sq_w8a8_gemm_s32": ([P, P, I, I, I, P, P], E),
         "sq_linear": ([P, E, P, P, P, I, I, I, P, E, P, ctypes.c_size_t, P], E),
@@ -202,6 +210,47 @@ def sq_silu_mul_quant(gu, s, xq, sx, h=None, stream=None):
     _check("sq_silu_mul_quant",
            lib().sq_silu_mul_quant(_ptr(gu), _dtype_code(gu), M, I2 // 2, _ptr(s), _ptr(xq), _ptr(sx),
                                    None if h is None else _ptr(h), _stream(stream)))
+
+
+def sq_gptq_hessian(x, s, H, stream=None):
+    """H [K, K] fp64 = xh^T xh over the calibration tokens x [T, K] (xh = x / s)."""
+    T, K = x.shape
+    _check("sq_gptq_hessian", lib().sq_gptq_hessian(_ptr(x), _dtype_code(x), T, K, _ptr(s), _ptr(H), _stream(stream)))
+
+
+def sq_gptq_factor(H, U, damp_frac=0.01, workspace=None, stream=None):
+    """Damps H in place and writes U, the upper Cholesky factor of H^-1."""
+    import torch
+
+    K = H.shape[0]
+    need = int(lib().sq_gptq_workspace_size(K))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=H.device)
+    _check("sq_gptq_factor", lib().sq_gptq_factor(_ptr(H), K, float(damp_frac), _ptr(U), _ptr(workspace),
+                                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def sq_gptq_quant_weight(w, s, U, wq, sw, stream=None):
+    """GPTQ codes wq [N, K] and per-channel scales sw [N] of the smoothed weight."""
+    N, K = w.shape
+    _check("sq_gptq_quant_weight", lib().sq_gptq_quant_weight(_ptr(w), _dtype_code(w), N, K, _ptr(s), _ptr(U),
+                                                              _ptr(wq), _ptr(sw), _stream(stream)))
+
+
+def gptq_weight(xcal, w, s, damp_frac=0.01, stream=None):
+    """GPTQ in place of prepare_weight's plain rounding: (wq, sw) for the
+    smoothed weight w * s, with the Hessian from the calibration tokens xcal."""
+    import torch
+
+    K = w.shape[1]
+    H = torch.empty(K, K, dtype=torch.float64, device=w.device)
+    U = torch.empty_like(H)
+    sq_gptq_hessian(xcal, s, H, stream)
+    sq_gptq_factor(H, U, damp_frac, stream=stream)
+    wq = torch.empty(w.shape, dtype=torch.int8, device=w.device)
+    sw = torch.empty(w.shape[0], dtype=torch.float32, device=w.device)
+    sq_gptq_quant_weight(w, s, U, wq, sw, stream)
+    return wq, sw
 
 
 def sq_w8a8_gemm(xq, sx, wq, sw, y, stream=None):

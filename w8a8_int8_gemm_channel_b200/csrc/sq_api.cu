@@ -22,6 +22,7 @@
 #include "sq_gemm_pair.cuh"
 #include "sq_mem.cuh"
 #include "sq_ptx.cuh"
+#include "sq_gptq.cuh"
 #include "sq_splitk.cuh"
 
 namespace {
@@ -756,6 +757,35 @@ sq_status launch_rmsnorm_quant(const T *h, int64_t rows, int64_t K, const float 
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// GPTQ (offline weight rounding)
+// ---------------------------------------------------------------------------
+constexpr int64_t kGptqMaxK = 16384;  // H is K x K fp64 (2 GiB at the limit)
+
+template <typename T>
+sq_status launch_gptq_hessian(const T *x, int64_t ntok, int64_t K, const float *s, double *H, cudaStream_t st)
+{
+    const unsigned nb = static_cast<unsigned>(K / sq::kGptqTile);
+    return launch_kernel(sq::gptq_hessian_kernel<T>, dim3(nb, nb), dim3(sq::kGptqTile * sq::kGptqTile), 0, st, 0, 0, x,
+                         ntok, K, s, H);
+}
+
+template <typename T>
+sq_status launch_gptq_rows(const T *w, int64_t N, int64_t K, const float *s, const double *U, int8_t *wq, float *sw,
+                           cudaStream_t st)
+{
+    auto kernel = sq::gptq_rows_kernel<T>;
+    static std::atomic<uint64_t> attr_done{0};
+    if (!ensure_smem_attr(kernel, kMaxDynSmem - 1024, attr_done))
+        return SQ_ERR_CUDA;
+    // one warp per row, the rows in shared memory as fp64
+    const int64_t per_cta = std::max<int64_t>(1, std::min<int64_t>(8, (kMaxDynSmem - 1024) / (K * 8)));
+    const int smem = static_cast<int>(per_cta * K * 8);
+    const unsigned blocks = static_cast<unsigned>((N + per_cta - 1) / per_cta);
+    return launch_kernel(kernel, dim3(blocks), dim3(static_cast<unsigned>(32 * per_cta)), smem, st, 0, 0, w, N, K, s,
+                         U, wq, sw);
+}
+
 extern "C" {
 
 const char *sq_status_string(sq_status st)
@@ -892,6 +922,77 @@ sq_status sq_silu_mul_quant(const void *gu, sq_dtype dt, int64_t M, int64_t I, c
     return launch_glu_quant(static_cast<const float *>(gu), M, I, s, xq, sx, static_cast<float *>(h), st);
 }
 
+size_t sq_gptq_workspace_size(int64_t K)
+{
+    if (K < 16 || K % 16 != 0 || K > kGptqMaxK)
+        return 0;
+    return static_cast<size_t>(K) * static_cast<size_t>(K) * sizeof(double);
+}
+
+sq_status sq_gptq_hessian(const void *x, sq_dtype dt, int64_t T, int64_t K, const float *s, double *H,
+                          sq_stream_t stream)
+{
+    if (x == nullptr || s == nullptr || H == nullptr || !valid_dtype(dt) || T < 1 || K < 16 || K % 16 != 0 ||
+        !aligned16(x) || !aligned16(s) || !aligned16(H))
+        return SQ_ERR_INVALID_ARG;
+    if (K > kGptqMaxK || T > kMaxDim || (K / sq::kGptqTile) > 65535)
+        return SQ_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dt == SQ_BF16)
+        return launch_gptq_hessian(static_cast<const __nv_bfloat16 *>(x), T, K, s, H, st);
+    return launch_gptq_hessian(static_cast<const float *>(x), T, K, s, H, st);
+}
+
+sq_status sq_gptq_factor(double *H, int64_t K, float damp_frac, double *U, void *workspace, size_t ws_bytes,
+                         sq_stream_t stream)
+{
+    if (H == nullptr || U == nullptr || workspace == nullptr || K < 16 || K % 16 != 0 || !aligned16(H) ||
+        !aligned16(U) || !aligned16(workspace) || !(damp_frac >= 0.0f) || !(damp_frac <= 1.0e30f) || H == U)
+        return SQ_ERR_INVALID_ARG;
+    if (K > kGptqMaxK)
+        return SQ_ERR_UNSUPPORTED;
+    if (ws_bytes < sq_gptq_workspace_size(K))
+        return SQ_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    double *Lt = static_cast<double *>(workspace);
+    static std::atomic<uint64_t> attr_damp{0}, attr_chol{0};
+    // both kernels also hold a little static shared memory
+    if (!ensure_smem_attr(sq::gptq_damp_kernel, kMaxDynSmem - 1024, attr_damp) ||
+        !ensure_smem_attr(sq::gptq_chol_col_kernel, kMaxDynSmem - 1024, attr_chol))
+        return SQ_ERR_CUDA;
+    const int T = sq::kGptqThreads;
+    sq_status r = launch_kernel(sq::gptq_damp_kernel, dim3(1), dim3(T), static_cast<int>(K * 8), st, 0, 0, H, K,
+                                damp_frac);
+    if (r == SQ_OK)
+        r = launch_kernel(sq::gptq_zero_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(4096, (K * K + T - 1) / T))),
+                          dim3(T), 0, st, 0, 0, U, K * K);
+    // the Cholesky factor of the reversed H, one column a launch
+    for (int64_t j = 0; j < K && r == SQ_OK; ++j)
+        r = launch_kernel(sq::gptq_chol_col_kernel, dim3(static_cast<unsigned>((K - j + T - 1) / T)), dim3(T),
+                          static_cast<int>(std::max<int64_t>(j, 1) * 8), st, 0, 0, static_cast<const double *>(H), K,
+                          j, Lt);
+    // its inverse, one row a launch, into U at the reversed positions
+    for (int64_t i = 0; i < K && r == SQ_OK; ++i)
+        r = launch_kernel(sq::gptq_inv_row_kernel, dim3(static_cast<unsigned>((i + 1 + T - 1) / T)), dim3(T), 0, st, 0,
+                          0, static_cast<const double *>(Lt), K, i, U);
+    return r;
+}
+
+sq_status sq_gptq_quant_weight(const void *w, sq_dtype dt, int64_t N, int64_t K, const float *s, const double *U,
+                               int8_t *wq, float *sw, sq_stream_t stream)
+{
+    if (w == nullptr || s == nullptr || U == nullptr || wq == nullptr || sw == nullptr || !valid_dtype(dt) || N < 1 ||
+        K < 16 || K % 16 != 0 || !aligned16(w) || !aligned16(s) || !aligned16(U) || !aligned16(wq) ||
+        !aligned16(sw))
+        return SQ_ERR_INVALID_ARG;
+    if (K > kGptqMaxK || N > kMaxDim)
+        return SQ_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dt == SQ_BF16)
+        return launch_gptq_rows(static_cast<const __nv_bfloat16 *>(w), N, K, s, U, wq, sw, st);
+    return launch_gptq_rows(static_cast<const float *>(w), N, K, s, U, wq, sw, st);
+}
+
 sq_status sq_w8a8_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
                        int64_t M, int64_t N, int64_t K, void *y, sq_dtype out_dt,
                        sq_stream_t stream)
@@ -1008,7 +1109,9 @@ sq_status sq_device_status(sq_stream_t stream, uint32_t *code)
     }
     if (code != nullptr)
         *code = v;
-    return v == 0 ? SQ_OK : SQ_ERR_TIMEOUT;
+    if (v == 0)
+        return SQ_OK;
+    return v == sq::kErrGptqPivot ? SQ_ERR_INVALID_ARG : SQ_ERR_TIMEOUT;
 }
 
 }  // extern "C"
