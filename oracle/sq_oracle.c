@@ -485,21 +485,41 @@ void sqo_gptq_damp(double *H, int64_t K, float damp_frac)
         H[i * K + i] = H[i * K + i] + d;
 }
 
+/* [G] the dot product sum_{k = kb}^{ke - 1} a[k] b[k] in the fixed order the
+ * factorisation uses: 32 partial sums, partial l taking k = kb + l, kb + l +
+ * 32, ... in ascending order (p_l = fma(a[k], b[k], p_l) from 0), then, for
+ * o = 16, 8, 4, 2, 1 in turn, every p_l replaced by p_l + p_(l xor o) (all
+ * from the previous values); the result is p_0. */
+static double dot32(const double *a, const double *b, int64_t kb, int64_t ke)
+{
+    double p[32], t[32];
+    for (int l = 0; l < 32; ++l) {
+        p[l] = 0.0;
+        for (int64_t k = kb + l; k < ke; k += 32)
+            p[l] = fma(a[k], b[k], p[l]);
+    }
+    for (int o = 16; o >= 1; o >>= 1) {
+        for (int l = 0; l < 32; ++l)
+            t[l] = p[l] + p[l ^ o];
+        for (int l = 0; l < 32; ++l)
+            p[l] = t[l];
+    }
+    return p[0];
+}
+
 /* [G] U, the upper triangular Cholesky factor of H^-1 (H^-1 = U^T U), which
  * carries the error feedback: U[k][j] / U[k][k] is the share of weight k's
  * error that weight j > k takes.  It is computed through the identity
  * U = J L^-1 J, with J the index reversal and L the lower Cholesky factor of
  * J H J (so no inverse of H itself is formed):
  *   G[a][b] = H[K-1-a][K-1-b];
- *   L (left-looking, column by column):
- *     p = G[j][j]; p = fma(-L[j][k], L[j][k], p) for k = 0..j-1;
- *     L[j][j] = sqrt(p)  (p <= 0: not positive definite, return -1);
- *     for i > j: q = G[i][j]; q = fma(-L[i][k], L[j][k], q) for k = 0..j-1;
- *                L[i][j] = q / L[j][j];
+ *   L (left-looking, column by column), with dot32 over k = 0..j-1:
+ *     p = G[j][j] - dot32(L[j], L[j]);  L[j][j] = sqrt(p)
+ *       (p <= 0: not positive definite, return -1);
+ *     for i > j: L[i][j] = (G[i][j] - dot32(L[i], L[j])) / L[j][j];
  *   N = L^-1 (forward substitution, row by row):
  *     N[i][i] = 1 / L[i][i];
- *     for c < i: q = 0; q = fma(L[i][k], N[k][c], q) for k = c..i-1;
- *                N[i][c] = -(q / L[i][i]);
+ *     for c < i: N[i][c] = -(dot32(L[i][k], N[k][c] over k = c..i-1) / L[i][i]);
  *   U[a][b] = N[K-1-a][K-1-b] (zero below the diagonal).
  * Returns 0, or -1 when a pivot is not positive. */
 int sqo_gptq_factor(const double *H, int64_t K, double *U)
@@ -508,9 +528,7 @@ int sqo_gptq_factor(const double *H, int64_t K, double *U)
     double *N = (double *)calloc((size_t)(K * K), sizeof(double));
     int bad = 0;
     for (int64_t j = 0; j < K && !bad; ++j) {
-        double p = H[(K - 1 - j) * K + (K - 1 - j)];
-        for (int64_t k = 0; k < j; ++k)
-            p = fma(-L[j * K + k], L[j * K + k], p);
+        const double p = H[(K - 1 - j) * K + (K - 1 - j)] - dot32(L + j * K, L + j * K, 0, j);
         if (!(p > 0.0)) {
             bad = 1;
             break;
@@ -518,12 +536,8 @@ int sqo_gptq_factor(const double *H, int64_t K, double *U)
         const double ljj = sqrt(p);
         L[j * K + j] = ljj;
 #pragma omp parallel for schedule(static)
-        for (int64_t i = j + 1; i < K; ++i) {
-            double q = H[(K - 1 - i) * K + (K - 1 - j)];
-            for (int64_t k = 0; k < j; ++k)
-                q = fma(-L[i * K + k], L[j * K + k], q);
-            L[i * K + j] = q / ljj;
-        }
+        for (int64_t i = j + 1; i < K; ++i)
+            L[i * K + j] = (H[(K - 1 - i) * K + (K - 1 - j)] - dot32(L + i * K, L + j * K, 0, j)) / ljj;
     }
     if (!bad) {
         /* N stored column by column (Nt[c][k] = N[k][c]) so that each sum reads
@@ -532,12 +546,8 @@ int sqo_gptq_factor(const double *H, int64_t K, double *U)
         for (int64_t i = 0; i < K; ++i) {
             Nt[i * K + i] = 1.0 / L[i * K + i];
 #pragma omp parallel for schedule(static)
-            for (int64_t c = 0; c < i; ++c) {
-                double q = 0.0;
-                for (int64_t k = c; k < i; ++k)
-                    q = fma(L[i * K + k], Nt[c * K + k], q);
-                Nt[c * K + i] = -(q / L[i * K + i]);
-            }
+            for (int64_t c = 0; c < i; ++c)
+                Nt[c * K + i] = -(dot32(L + i * K, Nt + c * K, c, i) / L[i * K + i]);
         }
         for (int64_t a = 0; a < K; ++a)
             for (int64_t b = 0; b < K; ++b)
