@@ -215,9 +215,12 @@ SQ_API sq_status sq_silu_mul_quant(const void *gu, sq_dtype dt, int64_t M, int64
  *   the sum is 0), then writes U [K, K] fp64, the upper Cholesky factor of
  *   H^-1 (zero below the diagonal), through U = J L^-1 J: J reverses the
  *   index order and L is the lower Cholesky factor of J H J, computed column
- *   by column with every dot product in ascending index order; L^-1 by forward
- *   substitution, row by row, the same way.  workspace: device scratch of at
- *   least sq_gptq_workspace_size(K) bytes (K * K fp64).  A non-positive pivot
+ *   by column; L^-1 by forward
+ *   substitution, row by row, the same way.  Every dot product there is 32
+ *   interleaved partial sums (partial l over the terms l, l + 32, ... from
+ *   the first, ascending, one FMA a term) combined by the xor butterfly over
+ *   offsets 16, 8, 4, 2, 1.  workspace: device scratch of at least
+ *   sq_gptq_workspace_size(K) bytes (2 K * K fp64).  A non-positive pivot
  *   leaves U NaN and sets the device error word (sq_device_status returns
  *   SQ_ERR_INVALID_ARG).  Takes 2K + 2 kernel launches.
  *

@@ -167,7 +167,7 @@ def test_silu_mul_quant_rejects_bad_arguments(lib):
 
 
 def test_gptq_entry_points_reject_bad_arguments(lib):
-    assert lib.sq_gptq_workspace_size(4096) == 4096 * 4096 * 8
+    assert lib.sq_gptq_workspace_size(4096) == 2 * 4096 * 4096 * 8
     assert lib.sq_gptq_workspace_size(40) == 0                     # not a multiple of 16
     assert lib.sq_gptq_workspace_size(32768) == 0                  # beyond the limit
     h = lib.sq_gptq_hessian
@@ -178,7 +178,7 @@ def test_gptq_entry_points_reject_bad_arguments(lib):
     assert h(A, 1, 8, 32768, B, C, None) == UNS
     f = lib.sq_gptq_factor
     assert f(A, 64, 0.01, B, None, 1 << 20, None) == INV           # no workspace
-    assert f(A, 64, 0.01, B, C, 64 * 64 * 8 - 1, None) == INV      # workspace too small
+    assert f(A, 64, 0.01, B, C, 2 * 64 * 64 * 8 - 1, None) == INV  # workspace too small
     assert f(A, 64, -0.5, B, C, 1 << 20, None) == INV              # negative damping
     assert f(A, 64, float("nan"), B, C, 1 << 20, None) == INV
     assert f(A, 64, 0.01, A, C, 1 << 20, None) == INV              # U aliases H

@@ -123,3 +123,37 @@ def test_gptq_full_width_sampled(oracle):
     q_o, sw_o = oracle.gptq_quant_weight(w[rows], s, U_o)
     assert_bits_equal(sw[rows], sw_o, "scales (K = 4096)")
     assert_bits_equal(wq[rows], q_o, "codes (K = 4096)")
+
+
+CHILD_UNSTAGED = r'''
+import numpy as np, torch
+import w8a8_int8_gemm_channel_b200 as sq
+from oracle import oracle
+from tests.gpu_util import to_np, to_dev, assert_bits_equal
+g = torch.Generator().manual_seed(3)
+K, N = 512, 40
+x = torch.randn(300, K, generator=g).to(torch.bfloat16)
+w = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+s = (torch.rand(K, generator=g) + 0.5).numpy().astype(np.float32)
+wq, sw = sq.gptq_weight(x.cuda(), w.cuda(), to_dev(s))
+q_o, sw_o, _ = oracle.gptq(to_np(x), to_np(w), s)
+assert_bits_equal(to_np(sw), sw_o, "scales")
+assert_bits_equal(to_np(wq), q_o, "codes")
+st, code = sq.sq_device_status()
+assert st == sq.SQ_OK, hex(code)
+print("unstaged-ok")
+'''
+
+
+def test_gptq_rows_reading_u_from_l2_child_process():
+    """Rows too long to stage U in shared memory read it from L2; the same
+    kernel with SQ_GPTQ_STAGE=0 (read once per process, so in a child)."""
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SQ_GPTQ_STAGE="0", PYTHONPATH=root)
+    r = subprocess.run([sys.executable, "-c", CHILD_UNSTAGED], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0 and "unstaged-ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]

@@ -770,20 +770,33 @@ sq_status launch_gptq_hessian(const T *x, int64_t ntok, int64_t K, const float *
                          ntok, K, s, H);
 }
 
+template <typename T, bool STAGE>
+sq_status launch_gptq_rows_cfg(const T *w, int64_t N, int64_t K, const float *s, const double *U, int8_t *wq,
+                               float *sw, cudaStream_t st)
+{
+    auto kernel = sq::gptq_rows_kernel<T, STAGE>;
+    static std::atomic<uint64_t> attr_done{0};
+    if (!ensure_smem_attr(kernel, kMaxDynSmem - 1024, attr_done))
+        return SQ_ERR_CUDA;
+    // one warp per row, the rows (and with STAGE two rows of U) in shared memory as fp64
+    const int64_t avail = kMaxDynSmem - 1024 - (STAGE ? 2 * K * 8 : 0);
+    const int64_t per_cta = std::max<int64_t>(1, std::min<int64_t>(8, avail / (K * 8)));
+    const int smem = static_cast<int>((per_cta + (STAGE ? 2 : 0)) * K * 8);
+    const unsigned blocks = static_cast<unsigned>((N + per_cta - 1) / per_cta);
+    return launch_kernel(kernel, dim3(blocks), dim3(static_cast<unsigned>(32 * per_cta)), smem, st, 0, 0, w, N, K, s,
+                         U, wq, sw);
+}
+
 template <typename T>
 sq_status launch_gptq_rows(const T *w, int64_t N, int64_t K, const float *s, const double *U, int8_t *wq, float *sw,
                            cudaStream_t st)
 {
-    auto kernel = sq::gptq_rows_kernel<T>;
-    static std::atomic<uint64_t> attr_done{0};
-    if (!ensure_smem_attr(kernel, kMaxDynSmem - 1024, attr_done))
-        return SQ_ERR_CUDA;
-    // one warp per row, the rows in shared memory as fp64
-    const int64_t per_cta = std::max<int64_t>(1, std::min<int64_t>(8, (kMaxDynSmem - 1024) / (K * 8)));
-    const int smem = static_cast<int>(per_cta * K * 8);
-    const unsigned blocks = static_cast<unsigned>((N + per_cta - 1) / per_cta);
-    return launch_kernel(kernel, dim3(blocks), dim3(static_cast<unsigned>(32 * per_cta)), smem, st, 0, 0, w, N, K, s,
-                         U, wq, sw);
+    // staging U needs room for a row of the weight and two rows of U
+    // (SQ_GPTQ_STAGE=0 reads U from L2 instead, as longer rows must)
+    static const bool no_stage = std::getenv("SQ_GPTQ_STAGE") && std::atoi(std::getenv("SQ_GPTQ_STAGE")) == 0;
+    if (!no_stage && 3 * K * 8 <= kMaxDynSmem - 1024)
+        return launch_gptq_rows_cfg<T, true>(w, N, K, s, U, wq, sw, st);
+    return launch_gptq_rows_cfg<T, false>(w, N, K, s, U, wq, sw, st);
 }
 
 extern "C" {
@@ -926,7 +939,7 @@ size_t sq_gptq_workspace_size(int64_t K)
 {
     if (K < 16 || K % 16 != 0 || K > kGptqMaxK)
         return 0;
-    return static_cast<size_t>(K) * static_cast<size_t>(K) * sizeof(double);
+    return 2 * static_cast<size_t>(K) * static_cast<size_t>(K) * sizeof(double);
 }
 
 sq_status sq_gptq_hessian(const void *x, sq_dtype dt, int64_t T, int64_t K, const float *s, double *H,
@@ -954,27 +967,28 @@ sq_status sq_gptq_factor(double *H, int64_t K, float damp_frac, double *U, void 
     if (ws_bytes < sq_gptq_workspace_size(K))
         return SQ_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    double *Lt = static_cast<double *>(workspace);
-    static std::atomic<uint64_t> attr_damp{0}, attr_chol{0};
-    // both kernels also hold a little static shared memory
-    if (!ensure_smem_attr(sq::gptq_damp_kernel, kMaxDynSmem - 1024, attr_damp) ||
-        !ensure_smem_attr(sq::gptq_chol_col_kernel, kMaxDynSmem - 1024, attr_chol))
+    double *Lr = static_cast<double *>(workspace);  // L, row-major
+    double *Nt = Lr + K * K;                         // L^-1, column-major
+    static std::atomic<uint64_t> attr_damp{0};
+    // the damping kernel also holds a little static shared memory
+    if (!ensure_smem_attr(sq::gptq_damp_kernel, kMaxDynSmem - 1024, attr_damp))
         return SQ_ERR_CUDA;
-    const int T = sq::kGptqThreads;
-    sq_status r = launch_kernel(sq::gptq_damp_kernel, dim3(1), dim3(T), static_cast<int>(K * 8), st, 0, 0, H, K,
-                                damp_frac);
-    if (r == SQ_OK)
-        r = launch_kernel(sq::gptq_zero_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(4096, (K * K + T - 1) / T))),
-                          dim3(T), 0, st, 0, 0, U, K * K);
-    // the Cholesky factor of the reversed H, one column a launch
+    const int W = sq::kGptqWarps;
+    sq_status r = launch_kernel(sq::gptq_damp_kernel, dim3(1), dim3(sq::kGptqThreads), static_cast<int>(K * 8), st, 0,
+                                0, H, K, damp_frac);
+    // the Cholesky factor of the reversed H, one column a launch, one warp a row
     for (int64_t j = 0; j < K && r == SQ_OK; ++j)
-        r = launch_kernel(sq::gptq_chol_col_kernel, dim3(static_cast<unsigned>((K - j + T - 1) / T)), dim3(T),
-                          static_cast<int>(std::max<int64_t>(j, 1) * 8), st, 0, 0, static_cast<const double *>(H), K,
-                          j, Lt);
-    // its inverse, one row a launch, into U at the reversed positions
+        r = launch_kernel(sq::gptq_chol_col_kernel, dim3(static_cast<unsigned>((K - j + W - 1) / W)), dim3(32 * W), 0,
+                          st, 0, 0, static_cast<const double *>(H), K, j, Lr);
+    // its inverse, one row a launch, one warp a column
     for (int64_t i = 0; i < K && r == SQ_OK; ++i)
-        r = launch_kernel(sq::gptq_inv_row_kernel, dim3(static_cast<unsigned>((i + 1 + T - 1) / T)), dim3(T), 0, st, 0,
-                          0, static_cast<const double *>(Lt), K, i, U);
+        r = launch_kernel(sq::gptq_inv_row_kernel, dim3(static_cast<unsigned>((i + 1 + W - 1) / W)), dim3(32 * W), 0,
+                          st, 0, 0, static_cast<const double *>(Lr), K, i, Nt);
+    // U = the inverse, reversed and transposed
+    const unsigned tiles = static_cast<unsigned>((K + 31) / 32);
+    if (r == SQ_OK)
+        r = launch_kernel(sq::gptq_u_from_n_kernel, dim3(tiles, tiles), dim3(256), 0, st, 0, 0,
+                          static_cast<const double *>(Nt), K, U);
     return r;
 }
 

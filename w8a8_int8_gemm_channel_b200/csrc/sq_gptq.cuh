@@ -13,15 +13,18 @@
 //             (d = 1 when the sum is 0), added to the diagonal;
 //   U       = the upper Cholesky factor of H^-1, through U = J L^-1 J with J
 //             the index reversal and L the lower Cholesky factor of J H J:
-//             L left-looking, column by column, each dot product in ascending
-//             k; L^-1 by forward substitution, row by row, each dot product in
-//             ascending k;
+//             L left-looking, column by column; L^-1 by forward substitution,
+//             row by row; every dot product as 32 interleaved partial sums
+//             (partial l over k = kb + l, kb + l + 32, ..., ascending, one FMA
+//             a term) combined by the xor butterfly o = 16, 8, 4, 2, 1 -- what
+//             one warp computes, lane l holding partial l;
 //   rows    w = RN_f32(W * s) widened; sw = RN_f32(max |w| / 127); for k in
 //             order: q = clamp(rint(w[k] / sw)), e = RN(fma(-q, sw, w[k]) /
 //             U[k][k]), w[j] = fma(-e, U[k][j], w[j]) for j > k.
 // The Cholesky and the inverse take one launch per column (per row), since
 // each depends on all before it; the parallelism is over the rows (columns)
-// of that step.  This is offline work, done once per layer.
+// of that step, one warp per element.  This is offline work, done once per
+// layer.
 #pragma once
 
 #include <cstdint>
@@ -104,123 +107,174 @@ __global__ void __launch_bounds__(kGptqThreads) gptq_damp_kernel(double *__restr
         H[i * K + i] = __dadd_rn(diag[i], d);
 }
 
-// zero a K x K fp64 matrix (U's lower triangle stays zero)
-__global__ void gptq_zero_kernel(double *__restrict__ p, int64_t n)
+// The fixed-order dot product: lane l sums k = kb + l, kb + l + 32, ... (< ke)
+// in ascending order, then the xor butterfly; every lane returns the result.
+__device__ __forceinline__ double warp_dot32(const double *__restrict__ a, const double *__restrict__ b, int64_t kb,
+                                             int64_t ke, int lane)
 {
-    pdl_prologue();
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-        p[i] = 0.0;
+    double p = 0.0;
+    int64_t k = kb + lane;
+    for (; k + 96 < ke; k += 128) {  // four loads in flight, the sum in order
+        const double a0 = a[k], a1 = a[k + 32], a2 = a[k + 64], a3 = a[k + 96];
+        const double b0 = b[k], b1 = b[k + 32], b2 = b[k + 64], b3 = b[k + 96];
+        p = __fma_rn(a0, b0, p);
+        p = __fma_rn(a1, b1, p);
+        p = __fma_rn(a2, b2, p);
+        p = __fma_rn(a3, b3, p);
+    }
+    for (; k < ke; k += 32)
+        p = __fma_rn(a[k], b[k], p);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1)
+        p = __dadd_rn(p, __shfl_xor_sync(0xFFFFFFFFu, p, o));
+    return p;
 }
+
+constexpr int kGptqWarps = 8;  // warps (elements) per CTA in the factor steps
 
 // Column j of L, the lower Cholesky factor of G = J H J (G[a][b] =
-// H[K-1-a][K-1-b]).  L is stored transposed, Lt[k][i] = L[i][k], so that the
-// rows i of one step read consecutive addresses.  Every CTA stages row j of L
-// and computes the pivot itself (the same operations, so the same bits).
-__global__ void __launch_bounds__(kGptqThreads)
-    gptq_chol_col_kernel(const double *__restrict__ H, int64_t K, int64_t j, double *__restrict__ Lt)
+// H[K-1-a][K-1-b]), row-major in Lr.  One warp per row i >= j; every warp
+// computes the pivot itself (the same operations, so the same bits).
+__global__ void __launch_bounds__(kGptqWarps * 32)
+    gptq_chol_col_kernel(const double *__restrict__ H, int64_t K, int64_t j, double *__restrict__ Lr)
 {
     pdl_prologue();
-    extern __shared__ double lj[];  // L[j][0..j-1]
-    __shared__ double piv;
-    for (int64_t k = threadIdx.x; k < j; k += blockDim.x)
-        lj[k] = Lt[k * K + j];
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        double p = H[(K - 1 - j) * K + (K - 1 - j)];
-        for (int64_t k = 0; k < j; ++k)
-            p = __fma_rn(-lj[k], lj[k], p);
-        if (!(p > 0.0)) {
-            record_error(kErrGptqPivot);
-            piv = __longlong_as_double(0x7FF8000000000000LL);  // NaN from here on
-        } else {
-            piv = __dsqrt_rn(p);
-        }
-    }
-    __syncthreads();
-    const double ljj = piv;
-    const int64_t i = j + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t i = j + static_cast<int64_t>(blockIdx.x) * kGptqWarps + warp;
     if (i >= K)
         return;
-    if (i == j) {
-        Lt[j * K + j] = ljj;
+    const double *lj = Lr + j * K;
+    const double p = __dsub_rn(H[(K - 1 - j) * K + (K - 1 - j)], warp_dot32(lj, lj, 0, j, lane));
+    if (!(p > 0.0)) {
+        if (lane == 0) {
+            record_error(kErrGptqPivot);
+            Lr[i * K + j] = __longlong_as_double(0x7FF8000000000000LL);  // NaN from here on
+        }
         return;
     }
-    double q = H[(K - 1 - i) * K + (K - 1 - j)];
-    for (int64_t k = 0; k < j; ++k)
-        q = __fma_rn(-Lt[k * K + i], lj[k], q);
-    Lt[j * K + i] = __ddiv_rn(q, ljj);
+    const double ljj = __dsqrt_rn(p);
+    if (i == j) {
+        if (lane == 0)
+            Lr[j * K + j] = ljj;
+        return;
+    }
+    const double q = __dsub_rn(H[(K - 1 - i) * K + (K - 1 - j)], warp_dot32(Lr + i * K, lj, 0, j, lane));
+    if (lane == 0)
+        Lr[i * K + j] = __ddiv_rn(q, ljj);
 }
 
-// Row i of N = L^-1, written straight into U at the reversed positions:
-// N[i][c] -> U[K-1-i][K-1-c].  Thread c sums L[i][k] N[k][c] over k = c..i-1
-// in ascending k; all threads walk k together (a thread joins at k = c), so
-// that each step reads one row of N at consecutive addresses.
-__global__ void __launch_bounds__(kGptqThreads)
-    gptq_inv_row_kernel(const double *__restrict__ Lt, int64_t K, int64_t i, double *__restrict__ U)
+// Row i of N = L^-1, column-major in Nt (Nt[c][k] = N[k][c]).  One warp per
+// column c <= i.
+__global__ void __launch_bounds__(kGptqWarps * 32)
+    gptq_inv_row_kernel(const double *__restrict__ Lr, int64_t K, int64_t i, double *__restrict__ Nt)
 {
     pdl_prologue();
-    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const double lii = Lt[i * K + i];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * kGptqWarps + warp;
     if (c > i)
         return;
+    const double lii = Lr[i * K + i];
     if (c == i) {
-        U[(K - 1 - i) * K + (K - 1 - i)] = __ddiv_rn(1.0, lii);
+        if (lane == 0)
+            Nt[i * K + i] = __ddiv_rn(1.0, lii);
         return;
     }
-    // the CTA's first column: its threads join from there
-    const int64_t k0 = static_cast<int64_t>(blockIdx.x) * blockDim.x;
-    double q = 0.0;
-    for (int64_t k = k0; k < i; ++k) {
-        const double lik = Lt[k * K + i];
-        const double nkc = U[(K - 1 - k) * K + (K - 1 - c)];
-        if (k >= c)
-            q = __fma_rn(lik, nkc, q);
+    const double q = warp_dot32(Lr + i * K, Nt + c * K, c, i, lane);
+    if (lane == 0)
+        Nt[c * K + i] = -__ddiv_rn(q, lii);
+}
+
+// U[a][b] = N[K-1-a][K-1-b] = Nt[K-1-b][K-1-a] for b >= a, 0 below the
+// diagonal: a transpose through 32 x 32 tiles in shared memory.
+__global__ void __launch_bounds__(32 * 8) gptq_u_from_n_kernel(const double *__restrict__ Nt, int64_t K,
+                                                               double *__restrict__ U)
+{
+    pdl_prologue();
+    __shared__ double tile[32][33];
+    const int64_t a0 = static_cast<int64_t>(blockIdx.y) * 32, b0 = static_cast<int64_t>(blockIdx.x) * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    // the source block: rows K-1-b (b in [b0, b0+32)), columns K-1-a
+    for (int r = ty; r < 32; r += 8) {
+        const int64_t b = b0 + r, a = a0 + 31 - tx;  // ascending source addresses across the warp
+        tile[r][31 - tx] = (a < K && b < K) ? Nt[(K - 1 - b) * K + (K - 1 - a)] : 0.0;
     }
-    U[(K - 1 - i) * K + (K - 1 - c)] = -__ddiv_rn(q, lii);
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {
+        const int64_t a = a0 + r, b = b0 + tx;
+        if (a < K && b < K)
+            U[a * K + b] = b >= a ? tile[tx][r] : 0.0;
+    }
 }
 
 // GPTQ rounding of the smoothed rows: one warp per row, the row in shared
 // memory as fp64.  Every lane computes the code and the error of weight k
 // itself (the same operations, so the same bits); lanes then update the
-// weights j > k that they own.
-template <typename T>
+// weights j > k that they own.  STAGE: the CTA copies row k + 1 of U into
+// shared memory (cp.async, double-buffered) while its warps apply row k, so
+// each row of U crosses from L2 once per CTA instead of once per warp, ahead
+// of its use.
+template <typename T, bool STAGE>
 __global__ void gptq_rows_kernel(const T *__restrict__ w, int64_t N, int64_t K, const float *__restrict__ s,
                                  const double *__restrict__ U, int8_t *__restrict__ wq, float *__restrict__ sw)
 {
     pdl_prologue();
-    extern __shared__ double rows_sm[];
+    extern __shared__ __align__(16) double rows_sm[];  // [warps][K] rows, then (STAGE) [2][K] rows of U
+    const int warps = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
-    if (n >= N)
-        return;
+    const int64_t n = static_cast<int64_t>(blockIdx.x) * warps + warp;
+    const bool active = n < N;  // idle warps still take part in the copies and barriers
     double *r = rows_sm + static_cast<int64_t>(warp) * K;
+    double *ubuf = rows_sm + static_cast<int64_t>(warps) * K;
+    // U[k][k..K) -> dst[k..K), 16-byte copies from the even index at or below k
+    auto stage = [&](int64_t k, double *dst) {
+        for (int64_t q2 = (k >> 1) + threadIdx.x; q2 < (K >> 1); q2 += blockDim.x)
+            cp_async_16(smem_u32(dst + 2 * q2), U + k * K + 2 * q2, true);
+    };
     float amax = 0.0f;
-    for (int64_t k = lane; k < K; k += 32) {
-        const float v = __fmul_rn(load_widen<T>(w + n * K + k), s[k]);
-        r[k] = static_cast<double>(v);
-        amax = fmaxf(amax, fabsf(v));
+    if (active) {
+        for (int64_t k = lane; k < K; k += 32) {
+            const float v = __fmul_rn(load_widen<T>(w + n * K + k), s[k]);
+            r[k] = static_cast<double>(v);
+            amax = fmaxf(amax, fabsf(v));
+        }
     }
     amax = warp_max(amax);
     const float scale = __fdiv_rn(amax, 127.0f);
-    if (lane == 0)
+    if (active && lane == 0)
         sw[n] = scale;
-    __syncwarp();
+    if constexpr (STAGE) {
+        stage(0, ubuf);
+        cp_async_wait_all();
+        __syncthreads();
+    } else {
+        __syncwarp();
+    }
     const double sd = static_cast<double>(scale);
     int8_t *dst = wq + n * K;
     for (int64_t k = 0; k < K; ++k) {
-        double q = 0.0;
-        if (scale != 0.0f) {
-            const double rk = r[k];
-            q = fmin(fmax(rint(__ddiv_rn(rk, sd)), -127.0), 127.0);
-            const double e = __ddiv_rn(__fma_rn(-q, sd, rk), U[k * K + k]);
-            const double *uk = U + k * K;
-            for (int64_t j = k + 1 + lane; j < K; j += 32)
-                r[j] = __fma_rn(-e, uk[j], r[j]);
+        const double *uk = STAGE ? ubuf + (k & 1) * K : U + k * K;
+        if constexpr (STAGE) {
+            if (k + 1 < K)  // the next row of U, into the buffer every warp has finished with
+                stage(k + 1, ubuf + ((k + 1) & 1) * K);
         }
-        if (lane == 0)
-            dst[k] = static_cast<int8_t>(q);
-        __syncwarp();
+        if (active) {
+            double q = 0.0;
+            if (scale != 0.0f) {
+                const double rk = r[k];
+                q = fmin(fmax(rint(__ddiv_rn(rk, sd)), -127.0), 127.0);
+                const double e = __ddiv_rn(__fma_rn(-q, sd, rk), uk[k]);
+                for (int64_t j = k + 1 + lane; j < K; j += 32)
+                    r[j] = __fma_rn(-e, uk[j], r[j]);
+            }
+            if (lane == 0)
+                dst[k] = static_cast<int8_t>(q);
+        }
+        if constexpr (STAGE) {
+            cp_async_wait_all();
+            __syncthreads();
+        } else {
+            __syncwarp();
+        }
     }
 }
 
