@@ -9,6 +9,11 @@
  *             W'    = W diag(s), quantised per output channel (row n) to int8
  *   online    X^    = X diag(s)^-1, quantised per token (row m) to int8
  *             acc   = Xq Wq^T in int32, Y = (acc * sx[m]) * sw[n]
+ * and, around it: RMSNorm with gamma / s folded in and fused with the
+ * per-token quantiser (sq_fold_gamma, sq_rmsnorm_quant); the gated SiLU
+ * activation of the down projection fused with its quantiser
+ * (sq_silu_mul_quant); GPTQ rounding of the weight in place of the plain one
+ * (sq_gptq_*).
  *
  * Sources (page title, section):
  *   "Understanding W8A8 INT8 LLM Quantization": "Why Naive Weight Quantization
@@ -24,8 +29,11 @@
  *   "How does SmoothQuant int8 LLM calibration work...": "The Technical
  *     Workflow for Int8 Quantization Deployment" (absmax per channel over
  *     calibration samples; alpha between 0 and 1).
+ *   The sources of the fused and offline extras are cited at each of them.
  *
- * Numerics (every entry point): fp32 IEEE arithmetic, round-to-nearest-even,
+ * Numerics (every entry point; GPTQ and the gated activation's e^x state
+ * their own sequences of fused multiply-adds): fp32 IEEE arithmetic,
+ * round-to-nearest-even,
  * no fused multiply-add in any step whose result is rounded; codes are
  * clamp(round_half_even(v / scale), -127, 127) (-128 is never produced); a
  * zero absolute maximum gives scale 0 and all-zero codes; s_j is evaluated in

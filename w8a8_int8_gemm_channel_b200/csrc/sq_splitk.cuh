@@ -136,7 +136,6 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     float *pmax = reinterpret_cast<float *>(g + L.pmax);
     float *wpmax = reinterpret_cast<float *>(g + L.wpmax);
     float *sxs = reinterpret_cast<float *>(g + L.sxs);
-    float *rsxs = sxs + BNX;
     const uint32_t bars = base + L.bars;
     auto full_bar = [&](int i) { return bars + 8u * i; };
     auto empty_bar = [&](int i) { return bars + 8u * (stages + i); };
