@@ -81,6 +81,7 @@ def test_gptq_zero_calibration_is_plain_rounding(oracle):
     those of sq_smooth_quant_weight."""
     K, N = 128, 40
     _, w_np, s_np = _case(8, K, N, "bf16", seed=5)
+    w_np[3] = 0  # an all-zero channel: scale 0, codes 0
     x_np = np.zeros((8, K), np.uint16)
     _, _, U, wq, sw = _run(x_np, w_np, s_np, torch.bfloat16)
     assert np.array_equal(U, np.eye(K))
@@ -109,6 +110,17 @@ def test_gptq_not_positive_definite_reports_and_recovers(oracle):
     _, _, U2, wq, sw = _run(x, w, s, torch.float32)
     q_o, sw_o, U_o = oracle.gptq(x, w, s)
     assert_bits_equal(wq, q_o, "codes after the error")
+
+
+def test_gptq_zero_rows_with_calibration(oracle):
+    """All-zero output channels among ordinary ones, with a real Hessian."""
+    x, w, s = _case(128, 96, 24, "f32", seed=13)
+    w[[0, 7, 23]] = 0.0
+    _, _, U, wq, sw = _run(x, w, s, torch.float32)
+    q_o, sw_o = oracle.gptq_quant_weight(w, s, oracle.gptq_factor(oracle.gptq_damp(oracle.gptq_hessian(x, s), 0.01)))
+    assert_bits_equal(sw, sw_o, "scales")
+    assert_bits_equal(wq, q_o, "codes")
+    assert not wq[[0, 7, 23]].any()
 
 
 def test_gptq_full_width_sampled(oracle):
