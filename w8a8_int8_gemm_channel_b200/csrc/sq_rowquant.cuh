@@ -461,7 +461,8 @@ __device__ __forceinline__ void store_code_words(int8_t *dst, const uint32_t *y,
         *reinterpret_cast<uint32_t *>(dst) = pack_code_bytes(y[0], y[1], y[2], y[3]);
 }
 
-//   exact codes of the chunk (raw bits from the registers), overwriting what the fast path stored
+//   exact codes of the chunk from its raw bits (the caller takes them from the
+//   registers or re-reads them from L2), overwriting what the fast path stored
 template <typename T, int MODE>
 __device__ __noinline__ void chunk_store_exact_codes(uint4 raw, const float *__restrict__ sc, float scale, int8_t *dst)
 {
