@@ -765,9 +765,8 @@ constexpr int64_t kGptqMaxK = 16384;  // H is K x K fp64 (2 GiB at the limit)
 template <typename T>
 sq_status launch_gptq_hessian(const T *x, int64_t ntok, int64_t K, const float *s, double *H, cudaStream_t st)
 {
-    const unsigned nb = static_cast<unsigned>(K / sq::kGptqTile);
-    return launch_kernel(sq::gptq_hessian_kernel<T>, dim3(nb, nb), dim3(sq::kGptqTile * sq::kGptqTile), 0, st, 0, 0, x,
-                         ntok, K, s, H);
+    const unsigned nb = static_cast<unsigned>((K + sq::kGptqHT - 1) / sq::kGptqHT);
+    return launch_kernel(sq::gptq_hessian_kernel<T>, dim3(nb, nb), dim3(256), 0, st, 0, 0, x, ntok, K, s, H);
 }
 
 template <typename T, bool STAGE>
@@ -948,7 +947,7 @@ sq_status sq_gptq_hessian(const void *x, sq_dtype dt, int64_t T, int64_t K, cons
     if (x == nullptr || s == nullptr || H == nullptr || !valid_dtype(dt) || T < 1 || K < 16 || K % 16 != 0 ||
         !aligned16(x) || !aligned16(s) || !aligned16(H))
         return SQ_ERR_INVALID_ARG;
-    if (K > kGptqMaxK || T > kMaxDim || (K / sq::kGptqTile) > 65535)
+    if (K > kGptqMaxK || T > kMaxDim)
         return SQ_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (dt == SQ_BF16)

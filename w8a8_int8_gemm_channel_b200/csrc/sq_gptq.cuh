@@ -53,11 +53,14 @@ __device__ __forceinline__ float load_widen<__nv_bfloat16>(const __nv_bfloat16 *
     return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(p)) << 16);
 }
 
-// H = xh^T xh over T tokens, one 16 x 16 tile of H per CTA (only tiles on or
-// above the diagonal; each also writes its mirror, which holds the same
-// sums since a * b = b * a).  Tokens past T contribute fma(0, 0, acc) = acc.
+// H = xh^T xh over T tokens: one 64 x 64 tile of H per CTA (only tiles on or
+// above the diagonal; each also writes its mirror, which holds the same sums
+// since a * b = b * a), a 4 x 4 block of it per thread.  Every output's sum
+// runs over the tokens in ascending order, 16 tokens a stage; tokens past T
+// and columns past K contribute fma(0, b, acc) = acc.
+constexpr int kGptqHT = 64;  // Hessian tile edge
 template <typename T>
-__global__ void __launch_bounds__(kGptqTile *kGptqTile)
+__global__ void __launch_bounds__(256)
     gptq_hessian_kernel(const T *__restrict__ x, int64_t ntok, int64_t K, const float *__restrict__ s,
                         double *__restrict__ H)
 {
@@ -65,24 +68,61 @@ __global__ void __launch_bounds__(kGptqTile *kGptqTile)
     const int bi = blockIdx.y, bj = blockIdx.x;
     if (bi > bj)
         return;
-    __shared__ double xa[kGptqTile][kGptqTile + 1];  // [token][column of the i tile]
-    __shared__ double xb[kGptqTile][kGptqTile + 1];  // [token][column of the j tile]
-    const int tx = threadIdx.x % kGptqTile, ty = threadIdx.x / kGptqTile;
-    const int64_t i0 = static_cast<int64_t>(bi) * kGptqTile, j0 = static_cast<int64_t>(bj) * kGptqTile;
-    const float si = s[i0 + tx], sj = s[j0 + tx];
-    double acc = 0.0;
+    __shared__ double xa[kGptqTile][kGptqHT];  // [token][column of the i tile]
+    __shared__ double xb[kGptqTile][kGptqHT];  // [token][column of the j tile]
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    const int64_t i0 = static_cast<int64_t>(bi) * kGptqHT, j0 = static_cast<int64_t>(bj) * kGptqHT;
+    // loads: thread (lt, lc) fetches token lt, columns lc and lc + 16, 32, 48
+    const int lt = threadIdx.x / 16, lc = threadIdx.x % 16;
+    float si[4], sj[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        si[q] = i0 + lc + 16 * q < K ? s[i0 + lc + 16 * q] : 1.0f;
+        sj[q] = j0 + lc + 16 * q < K ? s[j0 + lc + 16 * q] : 1.0f;
+    }
+    double acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            acc[a][b] = 0.0;
     for (int64_t t0 = 0; t0 < ntok; t0 += kGptqTile) {
-        const int64_t t = t0 + ty;
-        xa[ty][tx] = t < ntok ? static_cast<double>(__fdiv_rn(load_widen<T>(x + t * K + i0 + tx), si)) : 0.0;
-        xb[ty][tx] = t < ntok ? static_cast<double>(__fdiv_rn(load_widen<T>(x + t * K + j0 + tx), sj)) : 0.0;
+        const int64_t t = t0 + lt;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int64_t ci = i0 + lc + 16 * q, cj = j0 + lc + 16 * q;
+            xa[lt][lc + 16 * q] =
+                (t < ntok && ci < K) ? static_cast<double>(__fdiv_rn(load_widen<T>(x + t * K + ci), si[q])) : 0.0;
+            xb[lt][lc + 16 * q] =
+                (t < ntok && cj < K) ? static_cast<double>(__fdiv_rn(load_widen<T>(x + t * K + cj), sj[q])) : 0.0;
+        }
         __syncthreads();
 #pragma unroll
-        for (int u = 0; u < kGptqTile; ++u)
-            acc = __fma_rn(xa[u][ty], xb[u][tx], acc);
+        for (int u = 0; u < kGptqTile; ++u) {
+            double av[4], bv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                av[q] = xa[u][ty + 16 * q];
+                bv[q] = xb[u][tx + 16 * q];
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    acc[a][b] = __fma_rn(av[a], bv[b], acc[a][b]);
+        }
         __syncthreads();
     }
-    H[(i0 + ty) * K + j0 + tx] = acc;
-    H[(j0 + tx) * K + i0 + ty] = acc;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int64_t i = i0 + ty + 16 * a, j = j0 + tx + 16 * b;
+            if (i < K && j < K) {
+                H[i * K + j] = acc[a][b];
+                H[j * K + i] = acc[a][b];
+            }
+        }
 }
 
 // damping, in place (one CTA): the diagonal staged in shared memory, summed
