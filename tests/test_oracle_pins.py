@@ -660,17 +660,19 @@ def test_gptq_without_correlation_is_plain_rounding(oracle):
         assert np.array_equal(q, q_rtn) and np.array_equal(sw, sw_rtn)
 
 
-def test_gptq_against_brute_force_obs(oracle):
+@pytest.mark.parametrize("damp", [0.01, 0.0])
+def test_gptq_against_brute_force_obs(oracle, damp):
     """Tiny layers against the explicit form of the method: after rounding
     weight k, spread its error over the remaining weights with the inverse of
-    the Hessian restricted to them, inverted afresh by numpy at every step."""
+    the Hessian restricted to them, inverted afresh by numpy at every step.
+    Undamped too (64 tokens of 10 channels: H is positive definite)."""
     rng = np.random.default_rng(74)
     N, K = 12, 10
     x = _correlated_calibration(rng, 64, K)
     w = f32(rng.standard_normal((N, K)) * 0.05)
     s = np.ones(K, np.float32)
-    q, sw, _ = oracle.gptq(x, w, s)
-    Hd = oracle.gptq_damp(oracle.gptq_hessian(x, s), 0.01)
+    q, sw, _ = oracle.gptq(x, w, s, damp_frac=damp)
+    Hd = oracle.gptq_damp(oracle.gptq_hessian(x, s), damp)
     for n in range(N):
         r = w[n].astype(np.float64).copy()
         sc = float(np.float32(np.abs(w[n]).max() / np.float32(127.0)))
