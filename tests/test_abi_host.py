@@ -194,3 +194,34 @@ def test_selftest_rejects_limits_out_of_range(lib):
     f = lib.sq_selftest_wait_timeout
     assert f(0, None) == INV
     assert f(2000001, None) == INV
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "sq.h"
+int main(void)
+{
+    if (sq_version() < 100) return 1;
+    if (strcmp(sq_status_string(SQ_ERR_INVALID_ARG), "SQ_ERR_INVALID_ARG") != 0) return 2;
+    if (sq_gptq_workspace_size(64) != (size_t)2 * 64 * 64 * 8) return 3;
+    /* rejected on the host before anything reaches CUDA */
+    if (sq_quant_act(NULL, SQ_BF16, 4, 64, NULL, NULL, NULL, NULL) != SQ_ERR_INVALID_ARG) return 4;
+    if (sq_silu_mul_quant(NULL, SQ_BF16, 4, 64, NULL, NULL, NULL, NULL, NULL) != SQ_ERR_INVALID_ARG) return 5;
+    puts("c-client-ok");
+    return 0;
+}
+"""
+
+
+def test_plain_c_client_compiles_links_and_runs(tmp_path, lib):
+    """include/sq.h is plain C (C11, -pedantic) and a C program links against
+    libsq.so and calls it; only host-side entry points are exercised."""
+    src = tmp_path / "client.c"
+    exe = tmp_path / "client"
+    src.write_text(C_CLIENT)
+    libdir = os.path.dirname(sq.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), f"-L{libdir}", "-l:libsq.so", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0 and "c-client-ok" in out.stdout, (out.returncode, out.stderr)
