@@ -230,7 +230,7 @@ SQ_API sq_status sq_silu_mul_quant(const void *gu, sq_dtype dt, int64_t M, int64
  *   offsets 16, 8, 4, 2, 1.  workspace: device scratch of at least
  *   sq_gptq_workspace_size(K) bytes (2 K * K fp64).  A non-positive pivot
  *   leaves U NaN and sets the device error word (sq_device_status returns
- *   SQ_ERR_INVALID_ARG).  Takes 2K + 2 kernel launches.
+ *   SQ_ERR_INVALID_ARG).  Takes K + 3 kernel launches.
  *
  * sq_gptq_quant_weight: per output channel n, w = RN_f32(W[n] * s) widened to
  *   fp64 and sw[n] = RN_f32(max |w| / 127) (sq_smooth_quant_weight's scale);

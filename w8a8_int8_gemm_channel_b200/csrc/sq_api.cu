@@ -975,14 +975,14 @@ sq_status sq_gptq_factor(double *H, int64_t K, float damp_frac, double *U, void 
     const int W = sq::kGptqWarps;
     sq_status r = launch_kernel(sq::gptq_damp_kernel, dim3(1), dim3(sq::kGptqThreads), static_cast<int>(K * 8), st, 0,
                                 0, H, K, damp_frac);
-    // the Cholesky factor of the reversed H, one column a launch, one warp a row
-    for (int64_t j = 0; j < K && r == SQ_OK; ++j)
-        r = launch_kernel(sq::gptq_chol_col_kernel, dim3(static_cast<unsigned>((K - j + W - 1) / W)), dim3(32 * W), 0,
-                          st, 0, 0, static_cast<const double *>(H), K, j, Lr);
-    // its inverse, one row a launch, one warp a column
-    for (int64_t i = 0; i < K && r == SQ_OK; ++i)
-        r = launch_kernel(sq::gptq_inv_row_kernel, dim3(static_cast<unsigned>((i + 1 + W - 1) / W)), dim3(32 * W), 0,
-                          st, 0, 0, static_cast<const double *>(Lr), K, i, Nt);
+    // step t: column t of the Cholesky factor of the reversed H (one warp a
+    // row) and row t - 1 of its inverse (one warp a column), one launch
+    for (int64_t t = 0; t <= K && r == SQ_OK; ++t) {
+        const int64_t chol_blocks = t < K ? (K - t + W - 1) / W : 0;
+        const int64_t inv_blocks = t >= 1 ? (t + W - 1) / W : 0;
+        r = launch_kernel(sq::gptq_factor_step_kernel, dim3(static_cast<unsigned>(chol_blocks + inv_blocks)),
+                          dim3(32 * W), 0, st, 0, 0, static_cast<const double *>(H), K, t, chol_blocks, Lr, Nt);
+    }
     // U = the inverse, reversed and transposed
     const unsigned tiles = static_cast<unsigned>((K + 31) / 32);
     if (r == SQ_OK)

@@ -175,12 +175,11 @@ constexpr int kGptqWarps = 8;  // warps (elements) per CTA in the factor steps
 // Column j of L, the lower Cholesky factor of G = J H J (G[a][b] =
 // H[K-1-a][K-1-b]), row-major in Lr.  One warp per row i >= j; every warp
 // computes the pivot itself (the same operations, so the same bits).
-__global__ void __launch_bounds__(kGptqWarps * 32)
-    gptq_chol_col_kernel(const double *__restrict__ H, int64_t K, int64_t j, double *__restrict__ Lr)
+__device__ __forceinline__ void gptq_chol_col(const double *__restrict__ H, int64_t K, int64_t j,
+                                              double *__restrict__ Lr, int64_t blk)
 {
-    pdl_prologue();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t i = j + static_cast<int64_t>(blockIdx.x) * kGptqWarps + warp;
+    const int64_t i = j + blk * kGptqWarps + warp;
     if (i >= K)
         return;
     const double *lj = Lr + j * K;
@@ -205,12 +204,11 @@ __global__ void __launch_bounds__(kGptqWarps * 32)
 
 // Row i of N = L^-1, column-major in Nt (Nt[c][k] = N[k][c]).  One warp per
 // column c <= i.
-__global__ void __launch_bounds__(kGptqWarps * 32)
-    gptq_inv_row_kernel(const double *__restrict__ Lr, int64_t K, int64_t i, double *__restrict__ Nt)
+__device__ __forceinline__ void gptq_inv_row(const double *__restrict__ Lr, int64_t K, int64_t i,
+                                             double *__restrict__ Nt, int64_t blk)
 {
-    pdl_prologue();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t c = static_cast<int64_t>(blockIdx.x) * kGptqWarps + warp;
+    const int64_t c = blk * kGptqWarps + warp;
     if (c > i)
         return;
     const double lii = Lr[i * K + i];
@@ -222,6 +220,22 @@ __global__ void __launch_bounds__(kGptqWarps * 32)
     const double q = warp_dot32(Lr + i * K, Nt + c * K, c, i, lane);
     if (lane == 0)
         Nt[c * K + i] = -__ddiv_rn(q, lii);
+}
+
+// Step t of the factorisation, in one launch: column t of L (CTAs
+// [0, chol_blocks)) and row t - 1 of L^-1 (the CTAs after them).  Row t - 1 of
+// the inverse reads only rows and columns of L up to t - 1, finished by the
+// steps before, so the two halves share nothing within the launch.
+__global__ void __launch_bounds__(kGptqWarps * 32)
+    gptq_factor_step_kernel(const double *__restrict__ H, int64_t K, int64_t t, int64_t chol_blocks,
+                            double *__restrict__ Lr, double *__restrict__ Nt)
+{
+    pdl_prologue();
+    const int64_t b = blockIdx.x;
+    if (b < chol_blocks)
+        gptq_chol_col(H, K, t, Lr, b);
+    else
+        gptq_inv_row(Lr, K, t - 1, Nt, b - chol_blocks);
 }
 
 // U[a][b] = N[K-1-a][K-1-b] = Nt[K-1-b][K-1-a] for b >= a, 0 below the
