@@ -68,13 +68,14 @@ def _load():
             lib.sqo_dequant.argtypes = [P, P, P, I, I, P, P]
             lib.sqo_dequant_pairs.argtypes = [P, P, P, I, P, P]
             lib.sqo_fold_gamma.argtypes = [P, P, I, P]
-            lib.sqo_rmsnorm_quant.argtypes = [P, ctypes.c_int, I, I, P, ctypes.c_float, P, P, P, P]
+            lib.sqo_rmsnorm_quant.argtypes = [P, ctypes.c_int, I, I, P, ctypes.c_float, ctypes.c_double, P, P, P,
+                                              P, P, P, P]
             lib.sqo_f32_to_bf16.argtypes = [ctypes.c_float]
             lib.sqo_gptq_hessian.argtypes = [P, ctypes.c_int, I, I, P, P]
             lib.sqo_gptq_damp.argtypes = [P, I, ctypes.c_float]
             lib.sqo_gptq_factor.argtypes = [P, I, P]
             lib.sqo_gptq_factor.restype = ctypes.c_int
-            lib.sqo_gptq_quant_weight.argtypes = [P, ctypes.c_int, I, I, P, P, P, P]
+            lib.sqo_gptq_quant_weight.argtypes = [P, ctypes.c_int, I, I, P, P, ctypes.c_double, P, P, P]
             lib.sqo_exp_f32.argtypes = [ctypes.c_float]
             lib.sqo_exp_f32.restype = ctypes.c_float
             lib.sqo_silu_f32.argtypes = [ctypes.c_float]
@@ -189,31 +190,33 @@ def fold_gamma(gamma: np.ndarray, s: np.ndarray) -> np.ndarray:
     return g
 
 
-def rmsnorm_quant(h: np.ndarray, g: np.ndarray, eps: float, rinv_in=None):
+def rmsnorm_quant(h: np.ndarray, g: np.ndarray, eps: float):
     """RMSNorm of each token row with the folded gamma g, then per-token int8
-    quantisation.  Returns (xq int8 [M, K], sx fp32 [M], rinv fp32 [M]).
-    rinv_in (fp32 [M]) replaces the computed 1/RMS when given."""
+    quantisation.  Returns (xq int8 [M, K], sx fp32 [M], rinv fp32 [M])."""
+    c = rmsnorm_quant_candidates(h, g, eps)
+    return c["xq"], c["sx"], c["rinv"]
+
+
+def rmsnorm_quant_candidates(h: np.ndarray, g: np.ndarray, eps: float, window: float = -1.0):
+    """The RMSNorm quantiser's result, plus, for every token whose fp64 1/RMS
+    lies within ``window`` (relative; negative: the summation-order bound
+    (K + 16) 2^-52) of an fp32 rounding midpoint, the whole result for the
+    fp32 neighbour across that midpoint.  Returns a dict of numpy arrays:
+    xq, sx, rinv (the result), near (bool [M], flagged tokens), and xq_alt,
+    sx_alt, rinv_alt (the alternate result; equal to the result where not
+    flagged)."""
     h = _c(h)
     g = _c(g, np.float32)
     M, K = h.shape
     assert g.shape == (K,)
-    ri = None if rinv_in is None else _c(rinv_in, np.float32)
-    assert ri is None or ri.shape == (M,)
-    xq = np.empty((M, K), np.int8)
-    sx = np.empty(M, np.float32)
-    rinv = np.empty(M, np.float32)
-    _load().sqo_rmsnorm_quant(_ptr(h), _dt(h), M, K, _ptr(g), float(eps), _ptr(ri), _ptr(xq), _ptr(sx), _ptr(rinv))
-    return xq, sx, rinv
-
-
-def rmsnorm_rinv_fp64(h: np.ndarray, eps: float) -> np.ndarray:
-    """1 / sqrt(mean(h^2) + eps) per row in fp64 (numpy's summation order), before
-    the rounding to fp32: used to check that two rinv values one fp32 ulp apart
-    both come from an fp64 value at the rounding midpoint."""
-    h64 = _c(h).astype(np.float64) if _c(h).dtype != np.uint16 else bf16_bits_to_f32(h).astype(np.float64)
-    ms = (h64 * h64).sum(axis=1) / h64.shape[1] + np.float64(np.float32(eps))
-    with np.errstate(divide="ignore"):
-        return np.where(ms > 0, 1.0 / np.sqrt(ms), 0.0)
+    out = {"xq": np.empty((M, K), np.int8), "sx": np.empty(M, np.float32), "rinv": np.empty(M, np.float32),
+           "near": np.empty(M, np.uint8), "xq_alt": np.empty((M, K), np.int8), "sx_alt": np.empty(M, np.float32),
+           "rinv_alt": np.empty(M, np.float32)}
+    _load().sqo_rmsnorm_quant(_ptr(h), _dt(h), M, K, _ptr(g), float(eps), float(window), _ptr(out["xq"]),
+                              _ptr(out["sx"]), _ptr(out["rinv"]), _ptr(out["near"]), _ptr(out["xq_alt"]),
+                              _ptr(out["sx_alt"]), _ptr(out["rinv_alt"]))
+    out["near"] = out["near"].astype(bool)
+    return out
 
 
 def exp_f32(x: np.ndarray) -> np.ndarray:
@@ -280,14 +283,23 @@ def gptq_factor(H: np.ndarray) -> np.ndarray:
 def gptq_quant_weight(w: np.ndarray, s: np.ndarray, U: np.ndarray):
     """GPTQ codes and per-channel scales of the smoothed weight W * s:
     (wq int8 [N, K], sw fp32 [N])."""
+    wq, sw, _ = gptq_quant_weight_ties(w, s, U)
+    return wq, sw
+
+
+def gptq_quant_weight_ties(w: np.ndarray, s: np.ndarray, U: np.ndarray, tau: float = 2.0 ** -20):
+    """As gptq_quant_weight, plus per row the first weight index whose
+    quotient lies within tau of a rounding tie (-1 if none): (wq, sw, tie_pos)."""
     w = _c(w)
     s = _c(s, np.float32)
     U = _c(U, np.float64)
     N, K = w.shape
     wq = np.empty((N, K), np.int8)
     sw = np.empty(N, np.float32)
-    _load().sqo_gptq_quant_weight(_ptr(w), _dt(w), N, K, _ptr(s), _ptr(U), _ptr(wq), _ptr(sw))
-    return wq, sw
+    tie = np.empty(N, np.int64)
+    _load().sqo_gptq_quant_weight(_ptr(w), _dt(w), N, K, _ptr(s), _ptr(U), float(tau), _ptr(wq), _ptr(sw),
+                                  _ptr(tie))
+    return wq, sw, tie
 
 
 def gptq(xcal: np.ndarray, w: np.ndarray, s: np.ndarray, damp_frac: float = 0.01):

@@ -289,20 +289,56 @@ void sqo_fold_gamma(const float *gamma, const float *s, int64_t K, float *g)
 }
 
 /* [R] then [A], per token m:
- *   ms   = (sum_k h[m, k]^2) / K in fp64 (every square is exact in fp64; the
- *          sum runs in index order);
- *   rinv = 1 / sqrt(ms + eps) with IEEE fp64 sqrt and division, rounded once
- *          to fp32 (0 when ms + eps is 0: a zero row stays zero);
+ *   ms   = (sum_k h[m, k]^2) / K + eps in fp64 (every square is exact in
+ *          fp64; the sum runs in index order);
+ *   rinv = 1 / sqrt(ms) with IEEE fp64 sqrt and division, rounded once to
+ *          fp32 (0 when ms is 0: a zero row stays zero);
  *   a    = (h[m, k] * rinv) * g[k], two fp32 multiplies;
  *   sx   = max_k |a| / 127;  xq = clamp(round(a / sx), -127, 127).
- * rinv_out (may be NULL) receives rinv per token.  rinv_in (may be NULL)
- * replaces the computed rinv: the pages fix no summation order for the
- * squares, so another order may round rinv the other way when the fp64
- * value lies at an fp32 rounding midpoint; given the same rinv, everything
- * after it is fixed. */
-void sqo_rmsnorm_quant(const void *h, int dt, int64_t M, int64_t K, const float *g, float eps,
-                       const float *rinv_in, int8_t *xq, float *sx, float *rinv_out)
+ * rinv_out (may be NULL) receives rinv per token.
+ *
+ * The pages fix no summation order for the squares.  Any order of the fp64
+ * sum of K non-negative terms lies within (K - 1) 2^-53 (relative) of the
+ * exact sum, so any implementation's fp64 value of 1 / sqrt(ms) lies within
+ * about (K + 16) 2^-53 of this one's, and only where this one's lies that
+ * close to an fp32 rounding midpoint can another order round rinv to the
+ * other neighbour.  For such a token the oracle flags it (alt_flag[m] = 1)
+ * and also computes the whole result for the neighbour on the far side of
+ * that midpoint (alt_rinv, alt_sx, alt_xq); otherwise alt_flag[m] = 0 and the
+ * alternate outputs repeat the primary ones.  `window` is the relative
+ * distance to a midpoint that flags a token; window < 0 takes
+ * (K + 16) 2^-52, twice the bound above.  The alt_* pointers may be NULL. */
+static void rmsnorm_quant_row(const void *h, int dt, int64_t m, int64_t K, const float *g, float rinv,
+                              int8_t *xq_row, float *sx_out)
 {
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        float a = fabsf((elem(h, dt, (size_t)(m * K + k)) * rinv) * g[k]);
+        if (a > amax)
+            amax = a;
+    }
+    float scale = amax / 127.0f;
+    *sx_out = scale;
+    for (int64_t k = 0; k < K; ++k) {
+        int8_t q = 0;
+        if (amax != 0.0f) {
+            float a = (elem(h, dt, (size_t)(m * K + k)) * rinv) * g[k];
+            float r = nearbyintf(a / scale);
+            if (r > 127.0f)
+                r = 127.0f;
+            if (r < -127.0f)
+                r = -127.0f;
+            q = (int8_t)r;
+        }
+        xq_row[k] = q;
+    }
+}
+
+void sqo_rmsnorm_quant(const void *h, int dt, int64_t M, int64_t K, const float *g, float eps, double window,
+                       int8_t *xq, float *sx, float *rinv_out, uint8_t *alt_flag, int8_t *alt_xq, float *alt_sx,
+                       float *alt_rinv)
+{
+    const double win = window < 0.0 ? ((double)K + 16.0) * ldexp(1.0, -52) : window;
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m) {
         double ss = 0.0;
@@ -311,31 +347,31 @@ void sqo_rmsnorm_quant(const void *h, int dt, int64_t M, int64_t K, const float 
             ss += v * v;
         }
         double ms = ss / (double)K + (double)eps;
-        float rinv = ms > 0.0 ? (float)(1.0 / sqrt(ms)) : 0.0f;
-        if (rinv_in)
-            rinv = rinv_in[m];
+        double r64 = ms > 0.0 ? 1.0 / sqrt(ms) : 0.0;
+        float rinv = (float)r64;
         if (rinv_out)
             rinv_out[m] = rinv;
-        float amax = 0.0f;
-        for (int64_t k = 0; k < K; ++k) {
-            float a = fabsf((elem(h, dt, (size_t)(m * K + k)) * rinv) * g[k]);
-            if (a > amax)
-                amax = a;
+        rmsnorm_quant_row(h, dt, m, K, g, rinv, xq + m * K, sx + m);
+        /* the neighbour across the midpoint on r64's side of rinv (the
+         * nearer one), if that midpoint lies within the window */
+        float other = rinv;
+        if (r64 > 0.0) {
+            const float nb = r64 >= (double)rinv ? nextafterf(rinv, INFINITY) : nextafterf(rinv, 0.0f);
+            const double mid = ((double)rinv + (double)nb) / 2.0;
+            if (fabs(r64 - mid) <= win * r64)
+                other = nb;
         }
-        float scale = amax / 127.0f;
-        sx[m] = scale;
-        for (int64_t k = 0; k < K; ++k) {
-            int8_t q = 0;
-            if (amax != 0.0f) {
-                float a = (elem(h, dt, (size_t)(m * K + k)) * rinv) * g[k];
-                float r = nearbyintf(a / scale);
-                if (r > 127.0f)
-                    r = 127.0f;
-                if (r < -127.0f)
-                    r = -127.0f;
-                q = (int8_t)r;
+        if (alt_flag)
+            alt_flag[m] = other != rinv;
+        if (alt_rinv)
+            alt_rinv[m] = other;
+        if (alt_xq && alt_sx) {
+            if (other != rinv) {
+                rmsnorm_quant_row(h, dt, m, K, g, other, alt_xq + m * K, alt_sx + m);
+            } else {
+                memcpy(alt_xq + m * K, xq + m * K, (size_t)K);
+                alt_sx[m] = sx[m];
             }
-            xq[m * K + k] = q;
         }
     }
 }
@@ -440,9 +476,12 @@ void sqo_silu_mul_quant(const void *gu, int dt, int64_t M, int64_t I, const floa
 }
 
 /* ------------------------------------------------------------------------
- * [G] GPTQ.  Every step below is a fixed sequence of IEEE binary64
- * operations (fma is one correctly rounded fused multiply-add), in the index
- * order written, so that any implementation following it gets the same bits.
+ * [G] GPTQ.  Every step below is a sequence of IEEE binary64 operations (fma
+ * is one correctly rounded fused multiply-add), with every sum in plain index
+ * order.  The page describes the algorithm, not an order of summation: an
+ * implementation that sums in another order reaches the same values up to
+ * rounding, and its codes may then differ where a quotient lies at a
+ * rounding tie (the tests bound both).
  * ------------------------------------------------------------------------ */
 
 /* [G] the Hessian of the layer's squared output error over the calibration
@@ -485,42 +524,21 @@ void sqo_gptq_damp(double *H, int64_t K, float damp_frac)
         H[i * K + i] = H[i * K + i] + d;
 }
 
-/* [G] the dot product sum_{k = kb}^{ke - 1} a[k] b[k] in the fixed order the
- * factorisation uses: 32 partial sums, partial l taking k = kb + l, kb + l +
- * 32, ... in ascending order (p_l = fma(a[k], b[k], p_l) from 0), then, for
- * o = 16, 8, 4, 2, 1 in turn, every p_l replaced by p_l + p_(l xor o) (all
- * from the previous values); the result is p_0. */
-static double dot32(const double *a, const double *b, int64_t kb, int64_t ke)
-{
-    double p[32], t[32];
-    for (int l = 0; l < 32; ++l) {
-        p[l] = 0.0;
-        for (int64_t k = kb + l; k < ke; k += 32)
-            p[l] = fma(a[k], b[k], p[l]);
-    }
-    for (int o = 16; o >= 1; o >>= 1) {
-        for (int l = 0; l < 32; ++l)
-            t[l] = p[l] + p[l ^ o];
-        for (int l = 0; l < 32; ++l)
-            p[l] = t[l];
-    }
-    return p[0];
-}
-
 /* [G] U, the upper triangular Cholesky factor of H^-1 (H^-1 = U^T U), which
  * carries the error feedback: U[k][j] / U[k][k] is the share of weight k's
  * error that weight j > k takes.  It is computed through the identity
  * U = J L^-1 J, with J the index reversal and L the lower Cholesky factor of
- * J H J (so no inverse of H itself is formed):
+ * J H J (so no inverse of H itself is formed).  Every sum below runs in index
+ * order, one fma a term:
  *   G[a][b] = H[K-1-a][K-1-b];
- *   L (left-looking, column by column), with dot32 over k = 0..j-1:
- *     p = G[j][j] - dot32(L[j], L[j]);  L[j][j] = sqrt(p)
- *       (p <= 0: not positive definite, return -1);
- *     for i > j: L[i][j] = (G[i][j] - dot32(L[i], L[j])) / L[j][j];
- *   N = L^-1 (forward substitution, row by row):
+ *   L, column by column (j = 0, 1, ...):
+ *     p = G[j][j] - L[j][0]^2 - L[j][1]^2 - ... - L[j][j-1]^2;
+ *       L[j][j] = sqrt(p)  (p <= 0: not positive definite, return -1);
+ *     for i > j: L[i][j] = (G[i][j] - L[i][0] L[j][0] - ... - L[i][j-1] L[j][j-1]) / L[j][j];
+ *   N = L^-1, row by row (forward substitution):
  *     N[i][i] = 1 / L[i][i];
- *     for c < i: N[i][c] = -(dot32(L[i][k], N[k][c] over k = c..i-1) / L[i][i]);
- *   U[a][b] = N[K-1-a][K-1-b] (zero below the diagonal).
+ *     for c < i: N[i][c] = -((L[i][c] N[c][c] + L[i][c+1] N[c+1][c] + ... + L[i][i-1] N[i-1][c]) / L[i][i]);
+ *   U[a][b] = N[K-1-a][K-1-b] for b >= a, 0 below the diagonal.
  * Returns 0, or -1 when a pivot is not positive. */
 int sqo_gptq_factor(const double *H, int64_t K, double *U)
 {
@@ -528,7 +546,9 @@ int sqo_gptq_factor(const double *H, int64_t K, double *U)
     double *N = (double *)calloc((size_t)(K * K), sizeof(double));
     int bad = 0;
     for (int64_t j = 0; j < K && !bad; ++j) {
-        const double p = H[(K - 1 - j) * K + (K - 1 - j)] - dot32(L + j * K, L + j * K, 0, j);
+        double p = H[(K - 1 - j) * K + (K - 1 - j)];
+        for (int64_t k = 0; k < j; ++k)
+            p = fma(-L[j * K + k], L[j * K + k], p);
         if (!(p > 0.0)) {
             bad = 1;
             break;
@@ -536,18 +556,26 @@ int sqo_gptq_factor(const double *H, int64_t K, double *U)
         const double ljj = sqrt(p);
         L[j * K + j] = ljj;
 #pragma omp parallel for schedule(static)
-        for (int64_t i = j + 1; i < K; ++i)
-            L[i * K + j] = (H[(K - 1 - i) * K + (K - 1 - j)] - dot32(L + i * K, L + j * K, 0, j)) / ljj;
+        for (int64_t i = j + 1; i < K; ++i) {
+            double q = H[(K - 1 - i) * K + (K - 1 - j)];
+            for (int64_t k = 0; k < j; ++k)
+                q = fma(-L[i * K + k], L[j * K + k], q);
+            L[i * K + j] = q / ljj;
+        }
     }
     if (!bad) {
-        /* N stored column by column (Nt[c][k] = N[k][c]) so that each sum reads
-         * memory in order; the arithmetic is as written above */
+        /* N is stored column by column (Nt[c][k] = N[k][c]) so that each sum
+         * reads memory in order; the arithmetic is as written above */
         double *Nt = N;
         for (int64_t i = 0; i < K; ++i) {
             Nt[i * K + i] = 1.0 / L[i * K + i];
 #pragma omp parallel for schedule(static)
-            for (int64_t c = 0; c < i; ++c)
-                Nt[c * K + i] = -(dot32(L + i * K, Nt + c * K, c, i) / L[i * K + i]);
+            for (int64_t c = 0; c < i; ++c) {
+                double q = 0.0;
+                for (int64_t k = c; k < i; ++k)
+                    q = fma(L[i * K + k], Nt[c * K + k], q);
+                Nt[c * K + i] = -(q / L[i * K + i]);
+            }
         }
         for (int64_t a = 0; a < K; ++a)
             for (int64_t b = 0; b < K; ++b)
@@ -568,9 +596,14 @@ int sqo_gptq_factor(const double *H, int64_t K, double *U)
  *     q      = clamp(rint(w[k] / sw), -127, 127)  (fp64 division, rounding
  *              half to even; q = 0 throughout when sw = 0)
  *     e      = fma(-q, sw, w[k]) / U[k][k]
- *     w[j]   = fma(-e, U[k][j], w[j]) for every j > k. */
+ *     w[j]   = fma(-e, U[k][j], w[j]) for every j > k.
+ * tie_pos (may be NULL) receives, per row, the first k whose quotient
+ * w[k] / sw lies within `tau` of a rounding tie (a half-integer of magnitude
+ * below 127.5), or -1.  A U that differs from this one by rounding moves the
+ * quotients slightly, so from such a k on another implementation's codes of
+ * that row may differ. */
 void sqo_gptq_quant_weight(const void *w, int dt, int64_t N, int64_t K, const float *s, const double *U,
-                           int8_t *wq, float *sw)
+                           double tau, int8_t *wq, float *sw, int64_t *tie_pos)
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t n = 0; n < N; ++n) {
@@ -585,10 +618,15 @@ void sqo_gptq_quant_weight(const void *w, int dt, int64_t N, int64_t K, const fl
         const float scale = amax / 127.0f;
         sw[n] = scale;
         const double sd = (double)scale;
+        int64_t tie = -1;
         for (int64_t k = 0; k < K; ++k) {
             double q = 0.0;
             if (scale != 0.0f) {
-                q = nearbyint(r[k] / sd);
+                const double t = r[k] / sd;
+                const double a = fabs(t);
+                if (tie < 0 && a < 127.5 + tau && fabs(a - floor(a) - 0.5) <= tau)
+                    tie = k;
+                q = nearbyint(t);
                 if (q > 127.0)
                     q = 127.0;
                 if (q < -127.0)
@@ -599,6 +637,8 @@ void sqo_gptq_quant_weight(const void *w, int dt, int64_t N, int64_t K, const fl
             }
             wq[n * K + k] = (int8_t)q;
         }
+        if (tie_pos)
+            tie_pos[n] = tie;
         free(r);
     }
 }

@@ -4,9 +4,19 @@ sq_gptq_quant_weight) against the CPU oracle on the same seeded bytes.
 Source: "Understanding W8A8 INT8 LLM Quantization", section "How GPTQ
 improves on naive quantization".
 
-Both sides follow one fixed sequence of IEEE fp64 operations, so everything
-is bit-exact: the Hessian, the damped Hessian, the factor U, the codes and the
-scales.
+* The Hessian and the damped Hessian: bit-exact (both sum over the tokens in
+  order).
+* U, the upper Cholesky factor of the inverse: the oracle sums every dot
+  product in index order and the device in another order, so U agrees within
+  the classical forward-error bound of a Cholesky factorisation and a
+  triangular inverse, max|dU| <= 8 K 2^-53 kappa(H) max|U| (kappa from numpy's
+  eigenvalues of the damped H).
+* The rows kernel given the oracle's U: codes and scales bit-exact (one fixed
+  sequence of fp64 operations per row).
+* End to end (the device's own U): scales bit-exact, codes bit-exact except
+  in rows where the oracle's own quotient w/sw comes within 2^-20 of a
+  rounding tie; there the codes agree up to that weight, and such rows are
+  few (counted and bounded).
 """
 import numpy as np
 import pytest
@@ -59,6 +69,39 @@ def _run(x_np, w_np, s_np, tdt, damp=0.01):
     return to_np(H0), to_np(H), to_np(U), to_np(wq), to_np(sw)
 
 
+def _rows_given_u(w_np, s_np, U_np, tdt):
+    """The device's rows kernel run on the oracle's U."""
+    w, s = to_dev(w_np, tdt), to_dev(s_np)
+    wq = torch.empty(w.shape, dtype=torch.int8, device="cuda")
+    sw = torch.empty(w.shape[0], device="cuda")
+    sq.sq_gptq_quant_weight(w, s, to_dev(np.ascontiguousarray(U_np)), wq, sw)
+    torch.cuda.synchronize()
+    return to_np(wq), to_np(sw)
+
+
+def assert_u_close(U, U_o, Hd_o, what):
+    K = U_o.shape[0]
+    ev = np.linalg.eigvalsh(Hd_o)
+    kappa = ev[-1] / ev[0]
+    tol = 8.0 * K * 2.0 ** -53 * kappa * np.abs(U_o).max()
+    err = np.abs(U - U_o).max()
+    assert err <= tol, f"{what}: max |dU| {err:.3e} above {tol:.3e} (kappa {kappa:.3e})"
+    assert np.array_equal(np.tril(U, -1), np.zeros_like(U)), f"{what}: U not upper triangular"
+
+
+def assert_codes_up_to_ties(wq, q_o, tie, what):
+    """Codes equal the oracle's, except from a row's first near-tie on."""
+    exempt = 0
+    for n in np.flatnonzero((wq != q_o).any(axis=1)):
+        assert tie[n] >= 0, f"{what}: row {n} differs and has no near-tie quotient"
+        first = np.flatnonzero(wq[n] != q_o[n])[0]
+        assert first >= tie[n], f"{what}: row {n} differs at {first}, before its first near-tie at {tie[n]}"
+        exempt += 1
+    N = wq.shape[0]
+    assert exempt <= max(3, N // 20), f"{what}: {exempt} of {N} rows differ"
+    return exempt
+
+
 @pytest.mark.parametrize("T,K,N,dtype", [(16, 16, 8, "f32"), (64, 48, 20, "f32"), (200, 256, 96, "bf16"),
                                          (1024, 512, 300, "bf16"), (33, 320, 17, "bf16")])
 def test_gptq_parity(T, K, N, dtype, oracle):
@@ -70,10 +113,13 @@ def test_gptq_parity(T, K, N, dtype, oracle):
     Hd_o = oracle.gptq_damp(H0_o, 0.01)
     assert_bits_equal(Hd.view(np.uint64), Hd_o.view(np.uint64), "damped H")
     U_o = oracle.gptq_factor(Hd_o)
-    assert_bits_equal(U.view(np.uint64), U_o.view(np.uint64), "U")
-    q_o, sw_o = oracle.gptq_quant_weight(w, s, U_o)
+    assert_u_close(U, U_o, Hd_o, "U")
+    q_o, sw_o, tie = oracle.gptq_quant_weight_ties(w, s, U_o)
+    q_u, sw_u = _rows_given_u(w, s, U_o, tdt)
+    assert_bits_equal(sw_u, sw_o, "scales (oracle U)")
+    assert_bits_equal(q_u, q_o, "codes (oracle U)")
     assert_bits_equal(sw, sw_o, "scales")
-    assert_bits_equal(wq, q_o, "codes")
+    assert_codes_up_to_ties(wq, q_o, tie, "codes")
 
 
 def test_gptq_zero_calibration_is_plain_rounding(oracle):
@@ -108,8 +154,9 @@ def test_gptq_not_positive_definite_reports_and_recovers(oracle):
     assert st == sq.SQ_OK and code == 0
     x, w, s = _case(64, 64, 16, "f32", seed=9)
     _, _, U2, wq, sw = _run(x, w, s, torch.float32)
-    q_o, sw_o, U_o = oracle.gptq(x, w, s)
-    assert_bits_equal(wq, q_o, "codes after the error")
+    Hd_o = oracle.gptq_damp(oracle.gptq_hessian(x, s), 0.01)
+    q_o, sw_o, tie = oracle.gptq_quant_weight_ties(w, s, oracle.gptq_factor(Hd_o))
+    assert_codes_up_to_ties(wq, q_o, tie, "codes after the error")
 
 
 def test_gptq_zero_rows_with_calibration(oracle):
@@ -117,9 +164,10 @@ def test_gptq_zero_rows_with_calibration(oracle):
     x, w, s = _case(128, 96, 24, "f32", seed=13)
     w[[0, 7, 23]] = 0.0
     _, _, U, wq, sw = _run(x, w, s, torch.float32)
-    q_o, sw_o = oracle.gptq_quant_weight(w, s, oracle.gptq_factor(oracle.gptq_damp(oracle.gptq_hessian(x, s), 0.01)))
+    q_o, sw_o, tie = oracle.gptq_quant_weight_ties(
+        w, s, oracle.gptq_factor(oracle.gptq_damp(oracle.gptq_hessian(x, s), 0.01)))
     assert_bits_equal(sw, sw_o, "scales")
-    assert_bits_equal(wq, q_o, "codes")
+    assert_codes_up_to_ties(wq, q_o, tie, "codes")
     assert not wq[[0, 7, 23]].any()
 
 
@@ -129,12 +177,15 @@ def test_gptq_full_width_sampled(oracle):
     T, K, N = 512, 4096, 64
     x, w, s = _case(T, K, N, "bf16", seed=11)
     H0, Hd, U, wq, sw = _run(x, w, s, torch.bfloat16)
-    U_o = oracle.gptq_factor(oracle.gptq_damp(oracle.gptq_hessian(x, s), 0.01))
-    assert_bits_equal(U.view(np.uint64), U_o.view(np.uint64), "U (K = 4096)")
+    Hd_o = oracle.gptq_damp(oracle.gptq_hessian(x, s), 0.01)
+    U_o = oracle.gptq_factor(Hd_o)
+    assert_u_close(U, U_o, Hd_o, "U (K = 4096)")
     rows = np.arange(0, N, 8)
-    q_o, sw_o = oracle.gptq_quant_weight(w[rows], s, U_o)
+    q_o, sw_o, tie = oracle.gptq_quant_weight_ties(w[rows], s, U_o)
     assert_bits_equal(sw[rows], sw_o, "scales (K = 4096)")
-    assert_bits_equal(wq[rows], q_o, "codes (K = 4096)")
+    assert_codes_up_to_ties(wq[rows], q_o, tie, "codes (K = 4096)")
+    q_u, _ = _rows_given_u(w[rows], s, U_o, torch.bfloat16)
+    assert_bits_equal(q_u, q_o, "codes (K = 4096, oracle U)")
 
 
 CHILD_UNSTAGED = r'''
@@ -147,10 +198,15 @@ K, N = 512, 40
 x = torch.randn(300, K, generator=g).to(torch.bfloat16)
 w = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
 s = (torch.rand(K, generator=g) + 0.5).numpy().astype(np.float32)
-wq, sw = sq.gptq_weight(x.cuda(), w.cuda(), to_dev(s))
-q_o, sw_o, _ = oracle.gptq(to_np(x), to_np(w), s)
+xn, wn = to_np(x), to_np(w)
+U_o = oracle.gptq_factor(oracle.gptq_damp(oracle.gptq_hessian(xn, s), 0.01))
+q_o, sw_o = oracle.gptq_quant_weight(wn, s, U_o)
+wq = torch.empty(N, K, dtype=torch.int8, device="cuda")
+sw = torch.empty(N, device="cuda")
+sq.sq_gptq_quant_weight(w.cuda(), to_dev(s), to_dev(U_o), wq, sw)
+torch.cuda.synchronize()
 assert_bits_equal(to_np(sw), sw_o, "scales")
-assert_bits_equal(to_np(wq), q_o, "codes")
+assert_bits_equal(to_np(wq), q_o, "codes (oracle U, unstaged rows)")
 st, code = sq.sq_device_status()
 assert st == sq.SQ_OK, hex(code)
 print("unstaged-ok")

@@ -485,6 +485,60 @@ def test_rmsnorm_fold_matches_unfused_composition(oracle):
     assert d.max() <= 1 and (d == 0).mean() > 0.995
 
 
+def test_rmsnorm_midpoint_candidate_constructed(oracle):
+    """The row [4 - 2^-22, 0, ..., 0] of 16 values: its mean square is
+    (1 - 2^-24)^2 exactly, so 1/RMS = 1 / (1 - 2^-24) = 1 + 2^-24 + 2^-48 + ...,
+    which lies 2^-48 above the fp32 midpoint between 1 and 1 + 2^-23.  Round
+    to nearest gives 1 + 2^-23; another summation order could give 1.  The
+    oracle flags the token, and its alternate result is the same definition
+    with 1/RMS = 1 (then a = h g exactly, so sx = RN(|h_0 g_0| / 127))."""
+    K = 16
+    h = np.zeros((2, K), np.float32)
+    h[0, 0] = np.float32(4.0 - 2.0 ** -22)
+    h[1] = np.linspace(-1.0, 2.0, K, dtype=np.float32)
+    g = np.linspace(0.5, 2.0, K, dtype=np.float32)
+    c = oracle.rmsnorm_quant_candidates(h, g, 0.0)
+    assert c["near"].tolist() == [True, False]
+    assert c["rinv"][0] == np.float32(1.0 + 2.0 ** -23)
+    assert c["rinv_alt"][0] == np.float32(1.0)
+    assert c["sx_alt"][0] == np.float32(np.float32(h[0, 0] * g[0]) / np.float32(127.0))
+    assert c["sx"][0] == np.float32(np.float32(np.float32(h[0, 0] * c["rinv"][0]) * g[0]) / np.float32(127.0))
+    assert c["xq"][0, 0] == 127 and c["xq_alt"][0, 0] == 127 and not c["xq"][0, 1:].any()
+    # an unflagged token's alternate repeats its result
+    assert c["rinv_alt"][1] == c["rinv"][1] and np.array_equal(c["xq_alt"][1], c["xq"][1])
+    # with a window of 2^-49 the same token is not flagged: the flag follows the stated bound
+    c2 = oracle.rmsnorm_quant_candidates(h, g, 0.0, window=2.0 ** -49)
+    assert c2["near"].tolist() == [False, False]
+
+
+def test_rmsnorm_midpoint_candidates_are_the_neighbouring_rounding(oracle):
+    """With the window opened to 1 every token is flagged: the alternate 1/RMS
+    is the fp32 neighbour on the side of the fp64 value, and the alternate
+    codes and scale are the definition evaluated with it (numpy, element by
+    element).  With the default window, random tokens are almost never
+    flagged (a window that accepted both roundings everywhere would fail)."""
+    rng = np.random.default_rng(45)
+    M, K = 40, 384
+    h = (rng.standard_normal((M, K)) * rng.uniform(0.1, 10.0, (M, 1))).astype(np.float32)
+    g = rng.uniform(0.2, 3.0, K).astype(np.float32)
+    c = oracle.rmsnorm_quant_candidates(h, g, 1e-5, window=1.0)
+    assert c["near"].all()
+    h64 = h.astype(np.float64)
+    r64 = 1.0 / np.sqrt((h64 * h64).sum(axis=1) / K + np.float64(np.float32(1e-5)))
+    up = c["rinv"].astype(np.float64) < r64
+    want = np.where(up, np.nextafter(c["rinv"], np.float32(np.inf)), np.nextafter(c["rinv"], np.float32(0)))
+    assert np.array_equal(c["rinv_alt"], want.astype(np.float32))
+    for m in range(M):
+        a = ((h[m] * c["rinv_alt"][m]).astype(np.float32) * g).astype(np.float32)
+        sx = np.float32(np.abs(a).max() / np.float32(127.0))
+        assert c["sx_alt"][m] == sx
+        q = np.clip(np.rint((a / sx).astype(np.float32)), -127, 127).astype(np.int8)
+        assert np.array_equal(c["xq_alt"][m], q)
+    hb = rng.standard_normal((4000, 512)).astype(np.float32)
+    cb = oracle.rmsnorm_quant_candidates(hb, np.ones(512, np.float32), 1e-5)
+    assert cb["near"].sum() <= 2
+
+
 # ---------------------------------------------------------------------------
 # The gated feed-forward activation SiLU(gate) * up, quantised for the down
 # projection ("Understanding W8A8 INT8 LLM Quantization", section

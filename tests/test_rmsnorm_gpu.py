@@ -5,10 +5,12 @@ Source: "Understanding W8A8 INT8 LLM Quantization", section "Where the
 outlier actually comes from" (RMSNorm, and SmoothQuant dividing gamma by s).
 
 * the folded gamma g = gamma / s: bit-exact;
-* 1/RMS per token: bit-exact, or one fp32 ulp apart where the fp64 value
-  lies at an fp32 rounding midpoint (the summation order of the squares is
-  not fixed);
-* given the device's 1/RMS, the scales and codes: bit-exact.
+* per token, 1/RMS, the scale and the codes: bit-exact against the oracle's
+  result.  The summation order of the squares is not fixed, so for a token
+  whose fp64 1/RMS lies within the order-independence bound of an fp32
+  rounding midpoint the oracle also computes the whole result for the other
+  rounding, and the device may match either.  Every expected value comes from
+  the oracle on the input bytes alone.
 """
 import numpy as np
 import pytest
@@ -45,16 +47,26 @@ def _rows(M, K, dtype, seed):
     return h.to(dtype)
 
 
-def _check_rinv(r_dev, r_ora, h, eps, oracle):
-    same = r_dev.view(np.uint32) == r_ora.view(np.uint32)
-    if same.all():
-        return
-    ref = oracle.rmsnorm_rinv_fp64(to_np(h)[~same], eps)
-    lo = np.minimum(r_dev[~same], r_ora[~same]).astype(np.float64)
-    hi = np.maximum(r_dev[~same], r_ora[~same]).astype(np.float64)
-    assert (np.nextafter(lo.astype(np.float32), np.float32(np.inf)).astype(np.float64) == hi).all()
-    mid = (lo + hi) / 2
-    assert (np.abs(ref - mid) <= mid * 2.0 ** -40).all(), "1/RMS differs away from a rounding midpoint"
+def _match_candidates(cand, xq, sx, rinv=None):
+    """Every token of the device result equals the oracle's result, or, for a
+    flagged token, the oracle's alternate result.  Returns the number of
+    tokens that matched the alternate."""
+    M = sx.shape[0]
+    alt_rows = 0
+    for m in range(M):
+        prim = np.array_equal(xq[m], cand["xq"][m]) and sx[m].view(np.uint32) == cand["sx"][m].view(np.uint32)
+        if rinv is not None:
+            prim = prim and rinv[m].view(np.uint32) == cand["rinv"][m].view(np.uint32)
+        if prim:
+            continue
+        assert cand["near"][m], f"token {m}: differs from the oracle and 1/RMS is not near a rounding midpoint"
+        alt = np.array_equal(xq[m], cand["xq_alt"][m]) and \
+            sx[m].view(np.uint32) == cand["sx_alt"][m].view(np.uint32)
+        if rinv is not None:
+            alt = alt and rinv[m].view(np.uint32) == cand["rinv_alt"][m].view(np.uint32)
+        assert alt, f"token {m}: matches neither rounding of 1/RMS"
+        alt_rows += 1
+    return alt_rows
 
 
 @pytest.mark.parametrize("M,K,dtype,eps", [(1, 16, torch.float32, 1e-5), (6, 256, torch.float32, 0.0),
@@ -76,12 +88,9 @@ def test_rmsnorm_quant(oracle, M, K, dtype, eps):
     sx = torch.empty(M, device="cuda")
     rinv = torch.empty(M, device="cuda")
     sq.sq_rmsnorm_quant(h.cuda(), g, eps, xq, sx, rinv)
-    h_np = to_np(h)
-    _, _, r_o = oracle.rmsnorm_quant(h_np, g_o, eps)
-    _check_rinv(to_np(rinv), r_o, h, eps, oracle)
-    q_o, sx_o, _ = oracle.rmsnorm_quant(h_np, g_o, eps, rinv_in=to_np(rinv))
-    assert_bits_equal(to_np(sx), sx_o, "sx")
-    assert_bits_equal(to_np(xq), q_o, "xq")
+    cand = oracle.rmsnorm_quant_candidates(to_np(h), g_o, eps)
+    assert cand["near"].mean() < 0.05  # flagged tokens are rare: about (K + 16) 2^-27 each
+    _match_candidates(cand, to_np(xq), to_np(sx), to_np(rinv))
 
 
 def test_rmsnorm_quant_without_rinv_output(oracle):
@@ -96,5 +105,25 @@ def test_rmsnorm_quant_without_rinv_output(oracle):
     sx2 = torch.empty_like(sx)
     sq.sq_rmsnorm_quant(h.cuda(), to_dev(g_o), 1e-5, xq2, sx2, rinv)
     assert torch.equal(xq, xq2) and torch.equal(sx, sx2)
-    q_o, sx_o, _ = oracle.rmsnorm_quant(to_np(h), g_o, 1e-5, rinv_in=to_np(rinv))
-    assert_bits_equal(to_np(xq), q_o, "xq")
+    _match_candidates(oracle.rmsnorm_quant_candidates(to_np(h), g_o, 1e-5), to_np(xq), to_np(sx), to_np(rinv))
+
+
+def test_rmsnorm_quant_at_a_rounding_midpoint(oracle):
+    """A token whose 1/RMS sits 2^-48 above the fp32 midpoint 1 + 2^-24: the
+    row [4 - 2^-22, 0, ..., 0] of 16 values has mean square (1 - 2^-24)^2
+    exactly, so 1/RMS = 1 + 2^-24 + 2^-48 + ... (flagged by the oracle, which
+    also supplies the result for rinv = 1).  The device must give one of the
+    two oracle results; the rows around it are ordinary."""
+    K = 16
+    h = np.zeros((3, K), np.float32)
+    h[0] = np.linspace(-2.0, 3.0, K, dtype=np.float32)
+    h[1, 0] = np.float32(4.0 - 2.0 ** -22)
+    h[2] = np.linspace(0.5, -7.0, K, dtype=np.float32)
+    g_o = np.linspace(0.5, 2.0, K, dtype=np.float32)
+    cand = oracle.rmsnorm_quant_candidates(h, g_o, 0.0)
+    assert cand["near"].tolist() == [False, True, False]
+    xq = torch.empty(3, K, dtype=torch.int8, device="cuda")
+    sx = torch.empty(3, device="cuda")
+    rinv = torch.empty(3, device="cuda")
+    sq.sq_rmsnorm_quant(to_dev(h), to_dev(g_o), 0.0, xq, sx, rinv)
+    _match_candidates(cand, to_np(xq), to_np(sx), to_np(rinv))
