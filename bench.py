@@ -1,44 +1,53 @@
 #!/usr/bin/env python3
-"""Benchmark of the SmoothQuant W8A8 INT8 linear-layer hot path on B200.
+"""Benchmark of the SmoothQuant W8A8 INT8 linear layer on B200.
 
-One step is one pass of the whole hot path over one batch of synthetic input
-of the Llama-3-8B attention-projection workload (K = 4096; fused QKV N = 6144
-and O-projection N = 4096; bf16 activations with 0.1% outlier channels x60;
-calibration batch 128 x 512 tokens; alpha 0.5; token counts 16/128/1024/4096;
-bf16 out):
+The headline step is the online linear of the Llama-3-70B-shaped workload
+(the largest configuration): for M = 2048 and 8192 tokens, each of the four
+linears (QKV 8192 -> 10240, O 8192 -> 8192, gate/up 8192 -> 57344, down
+28672 -> 8192; bf16 activations with 0.1% outlier channels x80, alpha 0.85,
+bf16 out) runs ``sq_linear`` -- dynamic per-token int8 quantisation of
+X / s, then the int8 x int8 -> int32 tcgen05 GEMM with its dequantising
+epilogue -- on weights that were calibrated, smoothed and quantised
+beforehand.
 
-  1. calibration absmax over the 65536-token batch      (sq_calib_absmax)
-  2. smoothing factors for each linear                    (sq_smooth_factors)
-  3. smoothed per-output-channel int8 weights             (sq_smooth_quant_weight)
-  4. for every token count M and linear: the online linear, sq_quant_act
-     then sq_w8a8_gemm (the two kernels sq_linear runs, called separately so
-     the GEMM kernel can be timed on its own; with SQ_LINEAR_FUSED=1 up to 32
-     tokens run sq_linear's fused kernel instead)
+    value = sum over the step's calls of 2 M N K int8 operations / step time,
+            in TOPS, every input resident in HBM.
 
-value = int8 operations of all GEMMs in the step (2 M N K each) / step time,
-in TOPS, inputs resident in HBM.  e2e = the same through the same C-ABI calls
-with the step's inputs copied from pinned host memory and the outputs read
-back inside the timed region.
+The same run also measures, each as its own block of the JSON line:
+  * roofline  the dominant kernel (the tcgen05 pair GEMM): a second pass of
+              the same steps issues the two calls sq_linear makes
+              (sq_quant_act, sq_w8a8_gemm) with CUDA events around every GEMM
+              launch; achieved = ops per launch / average launch time;
+  * configs   every workload (small, Llama-3-8B attention, MLP and decode,
+              Llama-3-70B): per (linear, M) sq_linear and its two kernels,
+              each call timed alone with L2 flushed before it; for the decode
+              workload also the calls back to back;
+  * offline   the preparation stages of every workload (calibration absmax,
+              smoothing factors, smoothed int8 weights), each timed alone
+              with L2 flushed;
+  * e2e       the headline step through sq_linear with the activations
+              uploaded from pinned host memory and the outputs read back
+              inside the timed region;
+  * cpu_baseline  the CPU oracle on a bounded sample of the headline step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sq|reference]
 
-Under torchrun (N > 1) every rank runs an independent replica of the step on
-its own GPU (the path has no exchange step); value is the aggregate over ranks
-with the time taken as the maximum over ranks.
+Under torchrun (N > 1) every rank runs an independent replica of the
+headline step on its own GPU (the path has no exchange step); value is the
+aggregate over ranks, the time the maximum over ranks.  ``--case`` times
+single calls (used for the profiler captures).
 """
 from __future__ import annotations
 
 import argparse
-import ctypes
 import datetime
+import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
 import sys
 import tempfile
-import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -51,22 +60,20 @@ from w8a8_int8_gemm_channel_b200 import workloads as wls  # noqa: E402
 
 METRIC = "sq_linear INT8 TOPS & GB/s on 1 B200; % of INT8 tensor peak / HBM roofline"
 UNIT = "TOPS"
-DEFAULT_WORKLOAD = "llama3_8b_attn"
+DEFAULT_WORKLOAD = "llama3_70b"
+CONFIG_ORDER = ("small", "llama3_8b_attn", "llama3_8b_mlp", "llama3_8b_decode", "llama3_70b")
 
 # int8 dense tensor peak = measured bf16 peak x the nominal int8:bf16 ratio (4.5 : 2.25)
 INT8_PER_BF16 = 2.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
 
-# DRAM traffic per launch of the prefill GEMM kernel (dram__bytes_read.sum +
-# dram__bytes_write.sum), keyed by (M, N, K), from the ncu capture summarised
-# in the profile named below.
-GEMM_TRAFFIC_BYTES = {
-    (1024, 6144, 4096): 29417216 + 256,
-    (1024, 4096, 4096): 21018880 + 0,
-    (4096, 6144, 4096): 42038528 + 3244032,
-    (4096, 4096, 4096): 33625600 + 16128,
-}
-GEMM_TRAFFIC_SOURCE = "profiles/gemm_i8_pair_4096x6144x4096.md"
+# DRAM bytes (read + write) per launch of the pair GEMM, keyed by (M, N, K),
+# from one ncu capture each (--metrics dram__bytes_read.sum,dram__bytes_write.sum)
+# of `bench.py --case gemm:M,N,K`, taken on the kernel sources whose digest is
+# GEMM_TRAFFIC_DIGEST; reported only while the sources still have that digest.
+GEMM_TRAFFIC = {}
+GEMM_TRAFFIC_DIGEST = None
 
 
 # ---------------------------------------------------------------------------
@@ -86,6 +93,17 @@ def load_peaks():
         }
     except Exception:
         return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def kernel_digest():
+    """Digest of the CUDA sources (kernels and launchers)."""
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "w8a8_int8_gemm_channel_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
 
 
 class ClockSampler:
@@ -155,189 +173,318 @@ def visible_gpu_index(local_rank):
     return [local_rank]
 
 
+def _esize(name):
+    return 2 if name == "bf16" else 4
+
+
+def linear_bytes(M, N, K, ein, eout):
+    """Algorithmic HBM bytes of one sq_linear call: X read, s, Wq, sw read, Y written."""
+    return M * K * ein + 4 * K + N * K + 4 * N + M * N * eout
+
+
+def gemm_bytes(M, N, K, eout):
+    return M * K + N * K + 4 * (M + N) + M * N * eout
+
+
+def quant_bytes(M, K, ein):
+    return M * K * ein + 4 * K + M * K + 4 * M
+
+
+def bound_of(ops, nbytes, peaks):
+    """Tensor-bound where the arithmetic intensity is above the ridge of the
+    measured peaks, else HBM-bound."""
+    ridge = INT8_PER_BF16 * peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    return "tensor" if nbytes and ops / nbytes > ridge else "hbm"
+
+
+def rates(us, ops, nbytes, peaks):
+    """TOPS, GB/s and the fraction of the bounding roofline (burst int8 peak
+    for tensor-bound calls, measured copy bandwidth for HBM-bound ones)."""
+    s = us * 1e-6
+    gbs = nbytes / s / 1e9
+    ent = {"us": round(us, 2), "GB/s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 3)}
+    if ops:
+        tops = ops / s / 1e12
+        ent["TOPS"] = round(tops, 1)
+        ent["tensor_frac"] = round(tops / (INT8_PER_BF16 * peaks["bf16_tflops"]), 3)
+    b = bound_of(ops, nbytes, peaks)
+    ent["bound"] = b
+    ent["frac"] = ent["tensor_frac"] if b == "tensor" else ent["hbm_frac"]
+    return ent
+
+
 # ---------------------------------------------------------------------------
-# the step (CUDA path, through the C ABI)
+# one workload, prepared on the device through the C ABI
 # ---------------------------------------------------------------------------
 
-class Step:
-    """Inputs, outputs and the C-ABI call sequence of one step of a workload."""
+class Prepared:
+    """Inputs, prepared weights and outputs of one workload.
 
-    def __init__(self, wl: wls.Workload, device, base_seed=0):
+    Per linear: its calibration batch and bf16/fp32 weight (kept for the
+    offline block), the smoothing factors, the int8 weight and its scales
+    (computed once here by sq_calib_absmax, sq_smooth_factors and
+    sq_smooth_quant_weight), and per token count M the activations X and the
+    output Y."""
+
+    def __init__(self, wl: wls.Workload, device, base_seed=0, keep_offline_inputs=True):
         import w8a8_int8_gemm_channel_b200 as sq
 
         self.sq = sq
         self.lib = sq.lib()
         self.wl = wl
         self.device = device
-        self.in_dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-        self.out_dt = torch.bfloat16 if wl.out_dtype == "bf16" else torch.float32
+        self.ein = _esize(wl.dtype)
+        self.eout = _esize(wl.out_dtype)
         self.in_code = sq.SQ_BF16 if wl.dtype == "bf16" else sq.SQ_F32
         self.out_code = sq.SQ_BF16 if wl.out_dtype == "bf16" else sq.SQ_F32
-        lin0 = wl.linears[0]
-        K = lin0.K
-        assert all(l.K == K for l in wl.linears), "one shared calibration batch needs one K"
-        self.K = K
-        self.xcal = wls.calibration(wl, lin0, device=device, base_seed=base_seed)
-        self.ax = torch.zeros(K, dtype=torch.float32, device=device)
+        out_dt = torch.bfloat16 if wl.out_dtype == "bf16" else torch.float32
+        st = torch.cuda.current_stream(device).cuda_stream
         self.lins = []
         for lin in wl.linears:
-            d = {"lin": lin, "w": wls.weight(wl, lin, device=device, base_seed=base_seed),
+            K, N = lin.K, lin.N
+            d = {"lin": lin, "xcal": wls.calibration(wl, lin, device=device, base_seed=base_seed),
+                 "w": wls.weight(wl, lin, device=device, base_seed=base_seed),
+                 "ax": torch.zeros(K, dtype=torch.float32, device=device),
                  "s": torch.empty(K, dtype=torch.float32, device=device),
-                 "wq": torch.empty(lin.N, K, dtype=torch.int8, device=device),
-                 "sw": torch.empty(lin.N, dtype=torch.float32, device=device),
+                 "wq": torch.empty(N, K, dtype=torch.int8, device=device),
+                 "sw": torch.empty(N, dtype=torch.float32, device=device),
                  "x": {}, "y": {}}
+            self._ok("sq_calib_absmax", self.lib.sq_calib_absmax(
+                d["xcal"].data_ptr(), self.in_code, d["xcal"].shape[0], K, K, d["ax"].data_ptr(), st))
+            self._ok("sq_smooth_factors", self.lib.sq_smooth_factors(
+                d["ax"].data_ptr(), d["w"].data_ptr(), self.in_code, N, K, wl.alpha, d["s"].data_ptr(), None, st))
+            self._ok("sq_smooth_quant_weight", self.lib.sq_smooth_quant_weight(
+                d["w"].data_ptr(), self.in_code, N, K, d["s"].data_ptr(), d["wq"].data_ptr(), d["sw"].data_ptr(),
+                st))
             for M in wl.Ms:
                 d["x"][M] = wls.inputs(wl, lin, M, device=device, base_seed=base_seed)
-                d["y"][M] = torch.empty(M, lin.N, dtype=self.out_dt, device=device)
+                d["y"][M] = torch.empty(M, N, dtype=out_dt, device=device)
+            if not keep_offline_inputs:
+                d["xcal"] = None
+                d["w"] = None
             self.lins.append(d)
+        self.ws_bytes = max(sq.sq_linear_workspace_size(M, d["lin"].N, d["lin"].K)
+                            for M in wl.Ms for d in self.lins)
+        self.ws = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=device)
         Mmax = max(wl.Ms)
-        self.xq = torch.empty(Mmax, K, dtype=torch.int8, device=device)
+        Kmax = max(l.K for l in wl.linears)
+        self.xq = torch.empty(Mmax * Kmax, dtype=torch.int8, device=device)
         self.sx = torch.empty(Mmax, dtype=torch.float32, device=device)
-        self.ws_bytes = max(sq.sq_linear_workspace_size(M, l.N, K) for M in wl.Ms for l in wl.linears)
-        self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=device)
-        torch.cuda.synchronize()
+        torch.cuda.synchronize(device)
 
-    # -- algorithmic work ------------------------------------------------------
-    def gemm_ops(self):
-        return sum(2 * M * d["lin"].N * self.K for d in self.lins for M in self.wl.Ms)
+    def _ok(self, name, r):
+        if r != 0:
+            raise RuntimeError(f"{name}: {self.sq.status_string(r)}")
 
-    def input_bytes(self):
-        b = self.xcal.numel() * self.xcal.element_size()
-        for d in self.lins:
-            b += d["w"].numel() * d["w"].element_size()
-            b += sum(x.numel() * x.element_size() for x in d["x"].values())
-        return b
+    # -- the calls ---------------------------------------------------------------
+    def calls(self):
+        """(linear entry, M) in step order: every linear for each token count."""
+        return [(d, M) for M in self.wl.Ms for d in self.lins]
 
-    def output_bytes(self):
-        return sum(y.numel() * y.element_size() for d in self.lins for y in d["y"].values())
+    def linear(self, d, M, st):
+        lin = d["lin"]
+        self._ok(f"sq_linear[{lin.name},M={M}]", self.lib.sq_linear(
+            d["x"][M].data_ptr(), self.in_code, d["s"].data_ptr(), d["wq"].data_ptr(), d["sw"].data_ptr(),
+            M, lin.N, lin.K, d["y"][M].data_ptr(), self.out_code,
+            self.ws.data_ptr() if self.ws_bytes else None, self.ws_bytes, st))
 
-    def quant_kernels(self):
+    def quant(self, d, M, st):
+        lin = d["lin"]
+        self._ok("sq_quant_act", self.lib.sq_quant_act(
+            d["x"][M].data_ptr(), self.in_code, M, lin.K, d["s"].data_ptr(), self.xq.data_ptr(),
+            self.sx.data_ptr(), st))
+
+    def gemm(self, d, M, st):
+        lin = d["lin"]
+        self._ok("sq_w8a8_gemm", self.lib.sq_w8a8_gemm(
+            self.xq.data_ptr(), self.sx.data_ptr(), d["wq"].data_ptr(), d["sw"].data_ptr(), M, lin.N, lin.K,
+            d["y"][M].data_ptr(), self.out_code, st))
+
+    # offline stages of one linear (the weights are re-derived in place)
+    def calib(self, d, st):
+        lin = d["lin"]
+        d["ax"].zero_()
+        self._ok("sq_calib_absmax", self.lib.sq_calib_absmax(
+            d["xcal"].data_ptr(), self.in_code, d["xcal"].shape[0], lin.K, lin.K, d["ax"].data_ptr(), st))
+
+    def factors(self, d, st):
+        lin = d["lin"]
+        self._ok("sq_smooth_factors", self.lib.sq_smooth_factors(
+            d["ax"].data_ptr(), d["w"].data_ptr(), self.in_code, lin.N, lin.K, self.wl.alpha, d["s"].data_ptr(),
+            None, st))
+
+    def quant_weight(self, d, st):
+        lin = d["lin"]
+        self._ok("sq_smooth_quant_weight", self.lib.sq_smooth_quant_weight(
+            d["w"].data_ptr(), self.in_code, lin.N, lin.K, d["s"].data_ptr(), d["wq"].data_ptr(),
+            d["sw"].data_ptr(), st))
+
+    # -- work --------------------------------------------------------------------
+    def ops(self, d, M):
+        return 2 * M * d["lin"].N * d["lin"].K
+
+    def step_ops(self):
+        return sum(self.ops(d, M) for d, M in self.calls())
+
+    def step_linear_bytes(self):
+        return sum(linear_bytes(M, d["lin"].N, d["lin"].K, self.ein, self.eout) for d, M in self.calls())
+
+    def quant_kernels(self, K):
         """Kernels one quantiser call launches: one single-pass kernel while
-        the factor tables fit shared memory and a row fits 16 chunks per lane
-        of 8 warps, else a scale kernel and a code kernel."""
-        esize = 2 if self.in_code == self.sq.SQ_BF16 else 4
-        nch = self.K * esize // 16
-        bb = esize == 2 and self.K * 6 <= 64 * 1024
-        smem = self.K * 4 + (self.K * 2 if bb else 0)
-        if os.environ.get("SQ_QUANT_KIND") == "2":
-            return 2
+        the factor tables fit shared memory and a row fits 16 chunks a lane
+        over 8 warps, else a scale kernel and a code kernel."""
+        nch = K * self.ein // 16
+        bb = self.ein == 2 and K * 6 <= 64 * 1024
+        smem = K * 4 + (K * 2 if bb else 0)
         return 1 if smem <= 232448 - 1024 and nch <= 32 * 16 * 8 else 2
 
-    def launches_per_step(self):
-        """Kernels of this library one step launches: the calibration absmax
-        (1); per linear the zeroing of the factors' accumulator, the weight's
-        input-channel absmax and the factors (3) and the weight quantiser; per
-        token count and linear either the fused linear (1) or the activation
-        quantiser and the GEMM (1)."""
-        q = self.quant_kernels()
-        n = 1
-        n += (3 + q) * len(self.lins)
-        for M in self.wl.Ms:
-            n += len(self.lins) * (1 if self.fused(M) else q + 1)
-        return n
+    def linear_kernels(self, d, M):
+        if self.sq.sq_linear_workspace_size(M, d["lin"].N, d["lin"].K) == 0:
+            return 1  # the fused decode kernel
+        return self.quant_kernels(d["lin"].K) + 1
 
-    def fused(self, M):
-        return self.sq.sq_linear_workspace_size(M, self.lins[0]["lin"].N, self.K) == 0
+    def step_launches(self):
+        return sum(self.linear_kernels(d, M) for d, M in self.calls())
 
-    # -- the call sequence -------------------------------------------------------
-    def run(self, stream, gemm_events=None, stage_events=None, capturing=False):
-        """Enqueue one step on `stream`.  gemm_events: list receiving
-        (M, N, start, end) around each prefill GEMM; stage_events: list
-        receiving (name, start, end) around every call.  capturing: the
-        stream is being captured into a CUDA graph (events become graph
-        nodes that record on every replay)."""
-        lib, K = self.lib, self.K
-        st = stream.cuda_stream
+    def input_bytes(self):
+        return sum(d["x"][M].numel() * d["x"][M].element_size() for d, M in self.calls())
 
-        def ev():
-            e = torch.cuda.Event(enable_timing=True, external=capturing)
-            e.record(stream)
-            return e
+    def output_bytes(self):
+        return sum(d["y"][M].numel() * d["y"][M].element_size() for d, M in self.calls())
 
-        def call(name, fn, *args):
-            s0 = ev() if stage_events is not None else None
-            r = fn(*args)
-            if r != 0:
-                raise RuntimeError(f"{name}: {self.sq.status_string(r)}")
-            if stage_events is not None:
-                stage_events.append((name, s0, ev()))
-
-        self.ax.zero_()
-        call("calib_absmax", lib.sq_calib_absmax, self.xcal.data_ptr(), self.in_code,
-             self.xcal.shape[0], K, K, self.ax.data_ptr(), st)
+    def free_offline_inputs(self):
         for d in self.lins:
-            lin = d["lin"]
-            call(f"smooth_factors[{lin.name}]", lib.sq_smooth_factors, self.ax.data_ptr(),
-                 d["w"].data_ptr(), self.in_code, lin.N, K, self.wl.alpha, d["s"].data_ptr(), None, st)
-            call(f"smooth_quant_weight[{lin.name}]", lib.sq_smooth_quant_weight, d["w"].data_ptr(),
-                 self.in_code, lin.N, K, d["s"].data_ptr(), d["wq"].data_ptr(), d["sw"].data_ptr(), st)
-        for M in self.wl.Ms:
-            for d in self.lins:
-                lin = d["lin"]
-                x, y = d["x"][M], d["y"][M]
-                if self.fused(M):
-                    call(f"linear[{lin.name},M={M}]", lib.sq_linear, x.data_ptr(), self.in_code,
-                         d["s"].data_ptr(), d["wq"].data_ptr(), d["sw"].data_ptr(), M, lin.N, K,
-                         y.data_ptr(), self.out_code, None, 0, st)
-                    continue
-                call(f"quant_act[{lin.name},M={M}]", lib.sq_quant_act, x.data_ptr(), self.in_code,
-                     M, K, d["s"].data_ptr(), self.xq.data_ptr(), self.sx.data_ptr(), st)
-                g0 = ev() if gemm_events is not None and stage_events is None else None
-                call(f"gemm[{lin.name},M={M}]", lib.sq_w8a8_gemm, self.xq.data_ptr(),
-                     self.sx.data_ptr(), d["wq"].data_ptr(), d["sw"].data_ptr(), M, lin.N, K,
-                     y.data_ptr(), self.out_code, st)
-                if g0 is not None:
-                    gemm_events.append((M, lin.N, g0, ev()))
-
-    # -- per-stage algorithmic bytes / ops ---------------------------------------------
-    def stage_work(self, name):
-        """(ops, bytes, bound) for a stage name produced by run()."""
-        K = self.K
-        ein = 2 if self.in_code == self.sq.SQ_BF16 else 4
-        eout = 2 if self.out_code == self.sq.SQ_BF16 else 4
-        if name == "calib_absmax":
-            return 0, self.xcal.numel() * ein + 8 * K, "hbm"
-        lname = name[name.index("[") + 1:name.index("]")].split(",")[0]
-        N = next(d["lin"].N for d in self.lins if d["lin"].name == lname)
-        if name.startswith("smooth_factors"):
-            return 0, N * K * ein + 12 * K, "hbm"
-        if name.startswith("smooth_quant_weight"):
-            return 0, N * K * ein + 4 * K + N * K + 4 * N, "hbm"
-        M = int(name.split("M=")[1].rstrip("]"))
-        if name.startswith("quant_act"):
-            return 0, M * K * ein + 4 * K + M * K + 4 * M, "hbm"
-        ops = 2 * M * N * K
-        if name.startswith("gemm"):
-            b = M * K + N * K + 4 * (M + N) + M * N * eout
-        else:  # fused linear
-            b = M * K * ein + 4 * K + N * K + 4 * N + M * N * eout
-        bound = "tensor" if ops / b > 600 else "hbm"
-        return ops, b, bound
+            d["xcal"] = None
+            d["w"] = None
 
 
 # ---------------------------------------------------------------------------
-# CPU oracle baseline (a bounded sample of the same step, scaled to the step)
+# timing helpers
+# ---------------------------------------------------------------------------
+
+class Flusher:
+    def __init__(self, device):
+        self.buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def __call__(self):
+        self.buf.zero_()
+
+
+def time_alone(fn, stream, flush, reps=7, warm=2):
+    """Median CUDA-event time (us) of fn(st) on `stream`, L2 flushed before
+    every timed call."""
+    st = stream.cuda_stream
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            fn(st)
+        evs = []
+        for _ in range(reps):
+            flush()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn(st)
+            e1.record(stream)
+            evs.append((e0, e1))
+    stream.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+
+
+def config_block(p: Prepared, stream, flush, peaks, reps=7):
+    """Every (linear, M) call of a workload timed alone: sq_linear and its two
+    kernels (the fused decode kernel has no separate parts)."""
+    wl = p.wl
+    out = {"workload": wl.name, "description": wl.description, "calls": {}}
+    t_lin = 0.0
+    ops_all = 0
+    bytes_all = 0
+    for d, M in p.calls():
+        lin = d["lin"]
+        N, K = lin.N, lin.K
+        ops = p.ops(d, M)
+        lb = linear_bytes(M, N, K, p.ein, p.eout)
+        us = time_alone(lambda st: p.linear(d, M, st), stream, flush, reps)
+        ent = {"M": M, "N": N, "K": K, "linear": rates(us, ops, lb, peaks)}
+        if p.sq.sq_linear_workspace_size(M, N, K) > 0:
+            uq = time_alone(lambda st: p.quant(d, M, st), stream, flush, reps)
+            p.quant(d, M, stream.cuda_stream)  # the codes the GEMM below reads
+            ug = time_alone(lambda st: p.gemm(d, M, st), stream, flush, reps)
+            ent["quant_act"] = rates(uq, 0, quant_bytes(M, K, p.ein), peaks)
+            ent["gemm"] = rates(ug, ops, gemm_bytes(M, N, K, p.eout), peaks)
+        else:
+            ent["fused"] = True
+        out["calls"][f"{lin.name},M={M}"] = ent
+        t_lin += us
+        ops_all += ops
+        bytes_all += lb
+    out["sum_alone"] = {"TOPS": round(ops_all / (t_lin * 1e-6) / 1e12, 2),
+                        "GB/s": round(bytes_all / (t_lin * 1e-6) / 1e9, 1), "us": round(t_lin, 2)}
+    return out
+
+
+def back_to_back(p: Prepared, stream, steps=20, warm=3):
+    """The workload's calls back to back (launches overlapped), `steps` times:
+    (us per pass, GB/s of algorithmic bytes, TOPS)."""
+    st = stream.cuda_stream
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            for d, M in p.calls():
+                p.linear(d, M, st)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            for d, M in p.calls():
+                p.linear(d, M, st)
+        e1.record(stream)
+    stream.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / steps
+    return {"us_per_pass": round(us, 2), "GB/s": round(p.step_linear_bytes() / (us * 1e-6) / 1e9, 1),
+            "TOPS": round(p.step_ops() / (us * 1e-6) / 1e12, 2), "passes": steps}
+
+
+def offline_block(p: Prepared, stream, flush, peaks, reps=5):
+    """Preparation stages of a workload, each timed alone with L2 flushed."""
+    out = {}
+    for d in p.lins:
+        lin = d["lin"]
+        N, K = lin.N, lin.K
+        T = d["xcal"].shape[0]
+        us = time_alone(lambda st: p.calib(d, st), stream, flush, reps)
+        out[f"calib_absmax[{lin.name}]"] = dict(rates(us, 0, T * K * p.ein + 4 * K, peaks), T=T, K=K)
+        us = time_alone(lambda st: p.factors(d, st), stream, flush, reps)
+        out[f"smooth_factors[{lin.name}]"] = dict(rates(us, 0, N * K * p.ein + 12 * K, peaks), N=N, K=K)
+        us = time_alone(lambda st: p.quant_weight(d, st), stream, flush, reps)
+        out[f"smooth_quant_weight[{lin.name}]"] = dict(rates(us, 0, N * K * p.ein + 4 * K + N * K + 4 * N, peaks),
+                                                       N=N, K=K)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample of the headline step
 # ---------------------------------------------------------------------------
 
 class CpuSample:
-    """Times the CPU oracle on a bounded sample of every stage of the step and
-    scales each stage's time by (full work / sampled work)."""
+    """The online linear of every (linear, M) of a workload, run by the CPU
+    oracle on `rows` tokens (all K channels) against `cols` output channels:
+    per-token quantisation, int32 GEMM and dequantisation.  The smoothing
+    factors come from the oracle on a small calibration sample (untimed)."""
 
-    def __init__(self, wl: wls.Workload, base_seed=0):
+    def __init__(self, wl: wls.Workload, rows=8, cols=256, base_seed=0):
         from oracle import oracle
 
         self.o = oracle
         self.wl = wl
-        lin0 = wl.linears[0]
-        self.K = lin0.K
-        self.calib_rows = 2048
-        self.w_rows = 256
-        self.lin_rows = 8
-        # seeded CPU draws with the workload's distributions (same recipe, fewer rows)
-        self.xcal = self._np(wls.activations(wl, lin0, self.calib_rows, "calib", base_seed=base_seed))
-        self.w = {l.name: self._np(wls.weight(wl, l, rows=self.w_rows, base_seed=base_seed))
-                  for l in wl.linears}
-        self.x = {l.name: self._np(wls.inputs(wl, l, self.lin_rows, base_seed=base_seed)) for l in wl.linears}
+        self.rows = rows
+        self.cols = cols
+        self.data = []
+        for lin in wl.linears:
+            xcal = self._np(wls.activations(wl, lin, 256, "calib_sample", base_seed=base_seed))
+            w = self._np(wls.weight(wl, lin, rows=cols, base_seed=base_seed))
+            _, _, s, wq, sw = oracle.prepare(xcal, w, wl.alpha)
+            x = {M: self._np(wls.activations(wl, lin, min(M, rows), f"x_sample{M}", base_seed=base_seed))
+                 for M in wl.Ms}
+            self.data.append((lin, s, wq, sw, x))
 
     @staticmethod
     def _np(t):
@@ -349,66 +496,49 @@ class CpuSample:
         return t.numpy()
 
     def step(self):
-        """Returns (sampled seconds, estimated full-step seconds, ops of the full step)."""
-        import numpy as np
-
-        o, wl, K = self.o, self.wl, self.K
-        T = wl.calib_tokens
-        spent = 0.0
-        est = 0.0
-        t0 = time.perf_counter()
-        ax = o.calib_absmax(self.xcal)
-        dt = time.perf_counter() - t0
-        spent += dt
-        est += dt * T / self.calib_rows
+        """Runs one sampled step; returns (seconds, int8 ops computed)."""
+        o = self.o
         ops = 0
-        for lin in wl.linears:
-            w = self.w[lin.name]
-            t0 = time.perf_counter()
-            aw = o.weight_in_absmax(w)
-            s = o.smooth_factors(ax, aw, wl.alpha)
-            dt = time.perf_counter() - t0
-            spent += dt
-            est += dt * lin.N / self.w_rows
-            t0 = time.perf_counter()
-            wq, sw = o.smooth_quant_weight(w, s)
-            dt = time.perf_counter() - t0
-            spent += dt
-            est += dt * lin.N / self.w_rows
-            # the online path for lin_rows tokens against w_rows output channels
-            for M in wl.Ms:
-                rows = min(M, self.lin_rows)
-                t0 = time.perf_counter()
-                xq, sx = o.quant_act(self.x[lin.name][:rows], s)
+        t0 = time.perf_counter()
+        for M in self.wl.Ms:
+            for lin, s, wq, sw, x in self.data:
+                xq, sx = o.quant_act(x[M], s)
                 acc = o.gemm_i32(xq, wq)
-                o.dequant(acc, sx, sw, wl.out_dtype)
-                dt = time.perf_counter() - t0
-                spent += dt
-                est += dt * (M / rows) * (lin.N / self.w_rows)
-                ops += 2 * M * lin.N * K
-        return spent, est, ops
+                o.dequant(acc, sx, sw, self.wl.out_dtype)
+                ops += 2 * xq.shape[0] * wq.shape[0] * lin.K
+        return time.perf_counter() - t0, ops
 
     def describe(self):
-        return (f"oracle on {self.calib_rows} of {self.wl.calib_tokens} calibration tokens, "
-                f"{self.w_rows} weight rows per linear, and up to {self.lin_rows} tokens per token "
-                "count against those rows; each stage's time scaled by full/sampled work")
+        return (f"the oracle's online linear (per-token quantisation, int32 GEMM, dequantisation) for every "
+                f"(linear, M) of {self.wl.name} on {self.rows} tokens (all K channels) against {self.cols} "
+                f"output channels; throughput = the sample's int8 ops / its wall time")
 
 
 def cpu_baseline(wl, target_s=12.0):
     samp = CpuSample(wl)
-    samp.step()  # warm (builds/loads the oracle)
-    spent_total, est_total, ops = 0.0, 0.0, 0
-    n = 0
-    while spent_total < target_s and n < 5000:
-        spent, est, ops = samp.step()
-        spent_total += spent
-        est_total += est
+    samp.step()  # warm (loads the oracle)
+    spent, ops, n = 0.0, 0, 0
+    while spent < target_s and n < 10000:
+        t, o = samp.step()
+        spent += t
+        ops += o
         n += 1
-    est_step = est_total / n
-    return {"value": ops / est_step / 1e12, "unit": UNIT, "cores": samp.o.num_threads(),
-            "kind": "oracle", "sample": samp.describe() + f"; {n} sampled steps, "
-                                                           f"{spent_total:.1f} s of CPU time",
-            "est_full_step_s": est_step}
+    return {"value": ops / spent / 1e12, "unit": UNIT, "cores": samp.o.num_threads(), "kind": "oracle",
+            "sample": samp.describe() + f"; {n} sampled steps, {spent:.1f} s"}
+
+
+def workload_config(wl, step_desc=True):
+    cfg = {"workload": wl.name, "description": wl.description,
+           "linears": {l.name: {"N": l.N, "K": l.K} for l in wl.linears},
+           "M": list(wl.Ms), "calib_tokens": wl.calib_tokens, "alpha": wl.alpha,
+           "in_dtype": wl.dtype, "out_dtype": wl.out_dtype, "parallelism": "replicas", "launch": "eager"}
+    if step_desc:
+        cfg["step"] = ("sq_linear for every (linear, M), weights calibrated, smoothed and quantised "
+                       "beforehand (their stages are timed in `offline`)")
+        cfg["l2"] = ("inputs larger than L2: a step reads "
+                     f"{sum(l.N * l.K for l in wl.linears) / 1e6:.0f} MB of int8 weights per token count "
+                     "and the calls' activations and outputs, so every call starts with its operands cold")
+    return cfg
 
 
 # ---------------------------------------------------------------------------
@@ -422,41 +552,25 @@ def run_reference(args, rank, world):
     samp = CpuSample(wl)
     for _ in range(args.warmup):
         samp.step()
-    spent_total, est_total, ops = 0.0, 0.0, 0
-    budget = 150.0
-    steps = 0
-    for i in range(args.steps):
-        spent, est, ops = samp.step()
-        spent_total += spent
-        est_total += est
-        steps += 1
-        if spent_total > budget:
-            break
-    est_step = est_total / steps
-    value = ops / est_step / 1e12
+    spent, ops = 0.0, 0
+    for _ in range(args.steps):
+        t, o = samp.step()
+        spent += t
+        ops += o
+    value = ops / spent / 1e12
+    cfg = workload_config(wl)
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": steps,
-        "warmup": args.warmup, "ms_per_step": est_step * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "impl": "reference",
-        "config": workload_config(wl),
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": spent / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic", "impl": "reference",
+        "config": cfg,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": samp.o.num_threads(), "kind": "oracle",
-                         "sample": samp.describe() + f"; {steps} sampled steps"},
+                         "sample": samp.describe()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
     print(json.dumps(line), flush=True)
     return 0
-
-
-def workload_config(wl):
-    lin_desc = {l.name: {"N": l.N, "K": l.K} for l in wl.linears}
-    return {"workload": wl.name, "description": wl.description, "linears": lin_desc,
-            "M": list(wl.Ms), "calib_tokens": wl.calib_tokens, "alpha": wl.alpha,
-            "in_dtype": wl.dtype, "out_dtype": wl.out_dtype,
-            "l2": "inputs larger than L2: every step streams the calibration batch "
-                  f"({wl.calib_tokens} x {wl.linears[0].K} {wl.dtype}) first",
-            "parallelism": "replicas"}
 
 
 # ---------------------------------------------------------------------------
@@ -476,7 +590,7 @@ def run_case(spec, steps, warmup, flush_l2=True, settle_us=0.0):
     dev = torch.device("cuda", 0)
     st = torch.cuda.current_stream().cuda_stream
     peaks = load_peaks()
-    bf, i8, f32 = torch.bfloat16, torch.int8, torch.float32
+    bf, i8 = torch.bfloat16, torch.int8
     r = lambda *shape, dt=bf, sc=1.0: (torch.randn(*shape, device=dev) * sc).to(dt)
     ops, nbytes = 0, 0
     if kind in ("gemm", "linear"):
@@ -490,7 +604,7 @@ def run_case(spec, steps, warmup, flush_l2=True, settle_us=0.0):
             sx = torch.rand(M, device=dev)
             fn = lambda: lib.sq_w8a8_gemm(xq.data_ptr(), sx.data_ptr(), wq.data_ptr(), sw.data_ptr(),
                                           M, N, K, y.data_ptr(), sq.SQ_BF16, st)
-            nbytes = M * K + N * K + 4 * (M + N) + 2 * M * N
+            nbytes = gemm_bytes(M, N, K, 2)
         else:
             x = r(M, K)
             s = torch.rand(K, device=dev) + 0.5
@@ -499,21 +613,21 @@ def run_case(spec, steps, warmup, flush_l2=True, settle_us=0.0):
             fn = lambda: lib.sq_linear(x.data_ptr(), sq.SQ_BF16, s.data_ptr(), wq.data_ptr(),
                                        sw.data_ptr(), M, N, K, y.data_ptr(), sq.SQ_BF16,
                                        ws.data_ptr() if ws_n else None, ws_n, st)
-            nbytes = 2 * M * K + 4 * K + N * K + 4 * N + 2 * M * N
+            nbytes = linear_bytes(M, N, K, 2, 2)
     elif kind == "quant_act":
         M, K = d
         x, s = r(M, K), torch.rand(K, device=dev) + 0.5
         xq, sx = torch.empty(M, K, dtype=i8, device=dev), torch.empty(M, device=dev)
         fn = lambda: lib.sq_quant_act(x.data_ptr(), sq.SQ_BF16, M, K, s.data_ptr(), xq.data_ptr(),
                                       sx.data_ptr(), st)
-        nbytes = 3 * M * K + 4 * K + 4 * M
+        nbytes = quant_bytes(M, K, 2)
     elif kind == "rmsnorm_quant":
         M, K = d
         h, g = r(M, K), torch.rand(K, device=dev) + 0.5
         xq, sx = torch.empty(M, K, dtype=i8, device=dev), torch.empty(M, device=dev)
         fn = lambda: lib.sq_rmsnorm_quant(h.data_ptr(), sq.SQ_BF16, M, K, g.data_ptr(), 1e-5, xq.data_ptr(),
                                           sx.data_ptr(), None, st)
-        nbytes = 3 * M * K + 4 * K + 4 * M
+        nbytes = quant_bytes(M, K, 2)
     elif kind == "silu_mul_quant":
         M, I = d
         gu, s = r(M, 2 * I), torch.rand(I, device=dev) + 0.5
@@ -574,7 +688,7 @@ def run_case(spec, steps, warmup, flush_l2=True, settle_us=0.0):
         nbytes = 2 * N * K + 8 * K
     else:
         raise SystemExit(f"unknown case {spec}")
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush_l2 else None
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush_l2 else None
     for _ in range(warmup):
         assert fn() == 0
     torch.cuda.synchronize()
@@ -593,11 +707,8 @@ def run_case(spec, steps, warmup, flush_l2=True, settle_us=0.0):
         times.append((e0, e1))
     torch.cuda.synchronize()
     us = statistics.median(a.elapsed_time(b) for a, b in times) * 1e3
-    out = {"case": spec, "us": round(us, 2), "settle_us": settle_us, "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1),
-           "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3), "l2_flushed": flush_l2}
-    if ops:
-        out["TOPS"] = round(ops / (us * 1e-6) / 1e12, 1)
-        out["tensor_frac_burst"] = round(out["TOPS"] / (INT8_PER_BF16 * peaks["bf16_tflops"]), 3)
+    out = {"case": spec, "settle_us": settle_us, "l2_flushed": flush_l2}
+    out.update(rates(us, ops, nbytes, peaks))
     stc, code = sq.sq_device_status()
     assert stc == 0, f"device error {code:#x}"
     print(json.dumps(out), flush=True)
@@ -631,21 +742,19 @@ def aggregate_tops(world, ops_per_step, steps, ms):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="sq", choices=["sq", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wls.WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--breakdown-steps", type=int, default=20)
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-workload and offline blocks")
     ap.add_argument("--case", action="append", default=None,
                     help="time single calls instead of the step, e.g. gemm:4096,6144,4096")
     ap.add_argument("--no-flush", action="store_true")
     ap.add_argument("--settle-us", type=float, default=0.0,
                     help="--case: GPU idle time between the L2 flush and the timed call")
-    ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=False,
-                    help="replay the step as a CUDA graph in the timed region")
     args = ap.parse_args()
     if args.case:
         for c in args.case:
@@ -670,169 +779,183 @@ def main():
     torch.cuda.set_device(device)
     wl = wls.WORKLOADS[args.workload]
     peaks = load_peaks()
-    step = Step(wl, device)
+    step = Prepared(wl, device)
+    step.free_offline_inputs()
     stream = torch.cuda.Stream(device)
+    st = stream.cuda_stream
 
     def barrier():
         if world > 1:
             dist.barrier()
 
+    def run_step(call_events=None):
+        for d, M in step.calls():
+            if call_events is not None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            step.linear(d, M, st)
+            if call_events is not None:
+                e1 = torch.cuda.Event(enable_timing=True)
+                e1.record(stream)
+                call_events.append((d, M, e0, e1))
+
     # warm-up
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            step.run(stream)
+            run_step()
     stream.synchronize()
-    st, code = step.sq.sq_device_status(stream)
-    if st != 0:
+    stc, code = step.sq.sq_device_status(stream)
+    if stc != 0:
         raise RuntimeError(f"device error word {code:#x} after warm-up")
 
-    # The step as a CUDA graph: S steps per graph (S divides the step count),
-    # replayed steps / S times.  The GEMM events inside the graph record on
-    # every replay, so after the timed region they hold the last replay's S
-    # steps.  Without --graph the steps are enqueued eagerly and every GEMM
-    # launch of the timed region is bracketed by its own events.
-    graph = None
-    gemm_events = []
-    per_graph = 1
-    if args.graph:
-        per_graph = max(d for d in range(1, min(args.steps, 10) + 1) if args.steps % d == 0)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            for _ in range(per_graph):
-                step.run(stream, gemm_events=gemm_events, capturing=True)
-        for _ in range(2):
-            graph.replay()
-        stream.synchronize()
-
-    # timed region
+    # timed region: `steps` steps of sq_linear over every (linear, M)
     sampler = ClockSampler() if rank == 0 else None
     barrier()
     torch.cuda.synchronize()
     if sampler:
         sampler.start()
         time.sleep(0.2)
+    call_events = []
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         t_start.record(stream)
-        if graph is not None:
-            for _ in range(args.steps // per_graph):
-                graph.replay()
-        else:
-            for _ in range(args.steps):
-                step.run(stream, gemm_events=gemm_events)
+        for _ in range(args.steps):
+            run_step(call_events)
         t_end.record(stream)
     stream.synchronize()
     torch.cuda.synchronize()
     clocks = sampler.stop(visible_gpu_index(local_rank)) if sampler else None
     barrier()
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world, device)
-    st, code = step.sq.sq_device_status(stream)
-    if st != 0:
+    stc, code = step.sq.sq_device_status(stream)
+    if stc != 0:
         raise RuntimeError(f"device error word {code:#x} after the timed region")
-
     ms_per_step = elapsed_ms / args.steps
-    ops_step = step.gemm_ops()
+    ops_step = step.step_ops()
     value = aggregate_tops(world, ops_step, args.steps, elapsed_ms)
+    burst = INT8_PER_BF16 * peaks["bf16_tflops"]
 
-    # roofline of the dominant kernel: the prefill tcgen05 GEMM (M >= 1024)
-    g_ops = 0
-    g_ms = 0.0
-    g_n = 0
-    g_traffic = []
-    for (M, N, e0, e1) in gemm_events:
-        if M < 1024:
-            continue
-        g_ops += 2 * M * N * step.K
-        g_ms += e0.elapsed_time(e1)
-        g_n += 1
-        key = (M, N, step.K)
-        if key in GEMM_TRAFFIC_BYTES:
-            g_traffic.append(GEMM_TRAFFIC_BYTES[key])
-    int8_peak = INT8_PER_BF16 * peaks["bf16_tflops_sustained"]
+    # sq_linear calls of the timed region (each bracketed by its own events)
+    lin_ms = sum(e0.elapsed_time(e1) for _, _, e0, e1 in call_events)
+    lin_ops = sum(step.ops(d, M) for d, M, _, _ in call_events)
+    linear_calls = {"calls": len(call_events), "avg_call_us": lin_ms / len(call_events) * 1e3,
+                    "TOPS": lin_ops / (lin_ms * 1e-3) / 1e12,
+                    "frac_of_burst_int8": lin_ops / (lin_ms * 1e-3) / 1e12 / burst}
+
+    # the dominant kernel: a second pass of the same steps issuing the two
+    # calls sq_linear makes, with events around every GEMM launch
+    gemm_events = []
+    quant_ms = 0.0
+    with torch.cuda.stream(stream):
+        qev = []
+        for _ in range(args.steps):
+            for d, M in step.calls():
+                q0 = torch.cuda.Event(enable_timing=True)
+                q0.record(stream)
+                step.quant(d, M, st)
+                g0 = torch.cuda.Event(enable_timing=True)
+                g0.record(stream)
+                step.gemm(d, M, st)
+                g1 = torch.cuda.Event(enable_timing=True)
+                g1.record(stream)
+                gemm_events.append((d, M, g0, g1))
+                qev.append((q0, g0))
+    stream.synchronize()
+    quant_ms = sum(a.elapsed_time(b) for a, b in qev)
+    g_ops = sum(step.ops(d, M) for d, M, _, _ in gemm_events if M >= 1024)
+    g_ms = sum(e0.elapsed_time(e1) for d, M, e0, e1 in gemm_events if M >= 1024)
+    g_n = sum(1 for _, M, _, _ in gemm_events if M >= 1024)
     achieved = g_ops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
+    digest = kernel_digest()
+    traffic = None
+    if GEMM_TRAFFIC_DIGEST == digest and g_n:
+        t = [GEMM_TRAFFIC.get((M, d["lin"].N, d["lin"].K)) for d, M, _, _ in gemm_events if M >= 1024]
+        if all(v is not None for v in t):
+            traffic = sum(t) / len(t)
     roofline = {
         "kernel": "gemm_i8_pair_kernel (tcgen05.mma.cta_group::2 kind::i8, 256-row tiles on CTA pairs)",
-        "bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s",
-        "frac": (achieved / int8_peak) if achieved else None,
-        "traffic": (sum(g_traffic) / len(g_traffic)) if len(g_traffic) == g_n and g_n else None,
-        "traffic_source": GEMM_TRAFFIC_SOURCE,
-        "peak_note": f"int8 dense = 2 x {peaks['source']} sustained bf16 cuBLAS "
-                     f"({peaks['bf16_tflops_sustained']:.0f} TFLOP/s); 'TFLOP/s' here counts int8 ops",
-        "launches": g_n, "avg_launch_us": g_ms / max(g_n, 1) * 1e3,
-        "events": (f"the timed region's last graph replay ({per_graph} steps)" if graph is not None
-                   else "every launch of the timed region"),
-        "ops_per_launch": g_ops / max(g_n, 1),
+        "bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+        "frac": (achieved / burst) if achieved else None,
+        "traffic": traffic,
+        "traffic_note": ("ncu dram bytes per launch of this kernel version" if traffic is not None else
+                         "null: no ncu capture recorded for the current kernel sources"),
+        "kernel_digest": digest,
+        "peak_note": (f"int8 dense = 2 x {peaks['source']} burst bf16 cuBLAS ({peaks['bf16_tflops']:.1f} "
+                      "TFLOP/s); the timed region is well under a second; 'TFLOP/s' counts int8 ops"),
+        "launches": g_n, "avg_launch_us": g_ms / max(g_n, 1) * 1e3, "ops_per_launch": g_ops / max(g_n, 1),
+        "events": ("a second pass of the timed steps issuing sq_quant_act and sq_w8a8_gemm (the two calls "
+                   "sq_linear makes) with CUDA events on the launching stream around every GEMM launch"),
+        "share_of_split_pass": g_ms / (g_ms + quant_ms) if g_ms + quant_ms > 0 else None,
     }
 
-    # per-stage breakdown (separate, untimed pass with an event around every call)
-    stages = {}
-    if rank == 0 and args.breakdown_steps > 0:
-        ev = []
-        with torch.cuda.stream(stream):
-            for _ in range(args.breakdown_steps):
-                step.run(stream, stage_events=ev)
-        stream.synchronize()
-        acc = {}
-        for name, e0, e1 in ev:
-            acc.setdefault(name, []).append(e0.elapsed_time(e1))
-        for name, ts in acc.items():
-            us = statistics.median(ts) * 1e3
-            ops, b, bound = step.stage_work(name)
-            ent = {"us": round(us, 2), "bound": bound, "GB/s": round(b / (us * 1e-6) / 1e9, 1),
-                   "hbm_frac": round(b / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3)}
-            if ops:
-                ent["TOPS"] = round(ops / (us * 1e-6) / 1e12, 1)
-                ent["tensor_frac"] = round(ops / (us * 1e-6) / 1e12 /
-                                           (INT8_PER_BF16 * peaks["bf16_tflops"]), 3)
-            stages[name] = ent
+    # per-workload and offline blocks (one GPU only)
+    configs = None
+    offline = None
+    if rank == 0 and world == 1 and not args.no_configs:
+        flush = Flusher(device)
+        configs = {}
+        offline = {}
+        for name in CONFIG_ORDER:
+            if name == wl.name:
+                p = Prepared(wl, device)
+            else:
+                p = Prepared(wls.WORKLOADS[name], device)
+            blk = config_block(p, stream, flush, peaks)
+            if name == "llama3_8b_decode":
+                blk["back_to_back"] = back_to_back(p, stream)
+                blk["back_to_back"]["l2"] = (
+                    f"{sum(l.N * l.K for l in p.wl.linears) / 1e6:.0f} MB of int8 weights rotate through "
+                    "every token count, more than L2 holds")
+            configs[name] = blk
+            offline[name] = offline_block(p, stream, flush, peaks)
+            del p
+            torch.cuda.empty_cache()
+        del flush
+        torch.cuda.empty_cache()
 
-    # end to end: every step's inputs copied from pinned host memory and its
-    # outputs read back.  Two device buffer sets alternate, so the upload of
-    # step i+1 (one copy stream) and the download of step i (another) overlap
-    # the computation of step i; each buffer set is reused only after the
-    # computation and the download that used it have finished.
+    # end to end through sq_linear: every step uploads its activations from
+    # pinned host memory and reads every output back.  Two device buffer sets
+    # alternate so the upload of step i+1 and the download of step i overlap
+    # the computation of step i; a set is reused only after the computation
+    # and the download that last used it have finished.
     e2e = None
     if not args.no_e2e:
-        e2e_steps = args.e2e_steps or max(4, min(args.steps, 20))
-        sets = [step, Step(wl, device)]
-        h_xcal = step.xcal.cpu().pin_memory()
-        h_w = [d["w"].cpu().pin_memory() for d in step.lins]
-        h_x = [{M: x.cpu().pin_memory() for M, x in d["x"].items()} for d in step.lins]
-        h_y = [[{M: torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for M, y in d["y"].items()}
-                for d in step.lins] for _ in range(2)]
+        e2e_steps = args.e2e_steps or max(3, min(args.steps, 6))
+        sets = [step, Prepared(wl, device, keep_offline_inputs=False)]
+        h_x = [d["x"][M].cpu().pin_memory() for d, M in step.calls()]
+        h_y = [[torch.empty(d["y"][M].shape, dtype=d["y"][M].dtype, pin_memory=True) for d, M in step.calls()]
+               for _ in range(2)]
         h2d = step.input_bytes()
         d2h = step.output_bytes()
         s_in = torch.cuda.Stream(device)
         s_out = torch.cuda.Stream(device)
         ev = lambda: torch.cuda.Event(enable_timing=False)
-        done = [ev(), ev()]      # computation on set b finished
-        drained = [ev(), ev()]   # download of set b's outputs finished
+        done = [ev(), ev()]
+        drained = [ev(), ev()]
 
         def e2e_step(i):
             b = i % 2
-            st = sets[b]
+            p = sets[b]
+            calls = p.calls()
             loaded = ev()
             with torch.cuda.stream(s_in):
                 if i >= 2:
                     s_in.wait_event(done[b])
-                st.xcal.copy_(h_xcal, non_blocking=True)
-                for j, d in enumerate(st.lins):
-                    d["w"].copy_(h_w[j], non_blocking=True)
-                    for M in wl.Ms:
-                        d["x"][M].copy_(h_x[j][M], non_blocking=True)
+                for j, (d, M) in enumerate(calls):
+                    d["x"][M].copy_(h_x[j], non_blocking=True)
                 loaded.record(s_in)
             with torch.cuda.stream(stream):
                 stream.wait_event(loaded)
                 if i >= 2:
                     stream.wait_event(drained[b])
-                st.run(stream)
+                for d, M in calls:
+                    p.linear(d, M, st)
                 done[b].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(done[b])
-                for j, d in enumerate(st.lins):
-                    for M in wl.Ms:
-                        h_y[b][j][M].copy_(d["y"][M], non_blocking=True)
+                for j, (d, M) in enumerate(calls):
+                    h_y[b][j].copy_(d["y"][M], non_blocking=True)
                 drained[b].record(s_out)
 
         for i in range(2):
@@ -852,6 +975,7 @@ def main():
         e2e = {"value": aggregate_tops(world, ops_step, e2e_steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps,
+               "copies": "activations X of every call uploaded, outputs Y of every call downloaded, each step",
                "pipelining": "two device buffer sets; uploads, computation and downloads on three streams"}
         del sets
 
@@ -864,18 +988,20 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": dict(workload_config(wl),
-                           launch="cuda_graph" if graph is not None else "eager"),
+            "config": workload_config(wl),
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": step.launches_per_step() * args.steps,
+            "gpu_launches": step.step_launches() * args.steps,
             "clocks": clocks,
             "peaks": peaks,
-            "stages": stages,
+            "step_linear": {"GB/s": step.step_linear_bytes() * args.steps / (elapsed_ms * 1e-3) / 1e9,
+                            "frac_of_burst_int8": value / world / burst},
+            "linear_calls": linear_calls,
+            "configs": configs,
+            "offline": offline,
         }
         print(json.dumps(line), flush=True)
-    graph = None
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
