@@ -310,8 +310,10 @@ SQ_API size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K);
  *     SQ_LINEAR_NOALLOC_SCRATCH_BYTES are rejected with SQ_ERR_UNSUPPORTED
  *     before anything is enqueued.
  *   - The first call on a device (with that device current) looks up the
- *     device address of the scratch array once; make that first call before
- *     any stream capture on the device.
+ *     device address of the scratch array once and keeps it for the process;
+ *     make that first call before any stream capture on the device.  The
+ *     kept address is not valid after cudaDeviceReset on that device: do not
+ *     call this entry point on a device after resetting it.
  *   - All calls on a device share the one scratch array, which keeps the
  *     previous call's contents (nothing in it needs to start at zero).  Calls
  *     that can overlap on the GPU (different streams without ordering between

@@ -152,7 +152,8 @@ def test_smooth_factors(oracle, alpha, N, K, dtype):
 QUANT_SHAPES = [(1, 16, torch.float32), (3, 48, torch.bfloat16), (37, 4096, torch.bfloat16),
                 (130, 4112, torch.bfloat16), (5, 14336, torch.bfloat16), (2, 28672, torch.bfloat16),
                 (9, 8192, torch.float32), (4, 65536, torch.bfloat16), (2, 32768, torch.float32),
-                (2048, 4096, torch.bfloat16), (320, 14336, torch.bfloat16)]
+                (2048, 4096, torch.bfloat16), (320, 14336, torch.bfloat16), (300, 8192, torch.bfloat16),
+                (513, 2048, torch.bfloat16), (257, 28672, torch.bfloat16), (260, 16384, torch.bfloat16)]
 
 
 @pytest.mark.parametrize("R,K,dtype", QUANT_SHAPES)

@@ -46,15 +46,28 @@ def test_noalloc_matches_sq_linear_on_two_calls_in_a_row():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     _build.build()
-    shapes = [(300, 512, 2048, 101), (77, 272, 4112, 202)]
+    # a prefill-sized call, a few-token call (the weight-streaming GEMM, whose
+    # tile counters and partial sums also live in the scratch array) and one in between
+    shapes = [(300, 512, 2048, 101), (16, 1040, 4096, 303), (77, 272, 4112, 202)]
     cases = [_case(M, N, K, seed) for (M, N, K, seed) in shapes]
-    # two allocation-free calls back to back, sharing the library's scratch array
-    outs = []
-    for (x, s, wq, sw) in cases:
-        y = torch.empty(x.shape[0], wq.shape[0], dtype=torch.bfloat16, device="cuda")
+    outs = [torch.empty(x.shape[0], wq.shape[0], dtype=torch.bfloat16, device="cuda") for (x, s, wq, sw) in cases]
+    # first round: the calls back to back, sharing the library's scratch array
+    for (x, s, wq, sw), y in zip(cases, outs):
         sq.sq_linear_noalloc(x, s, wq, sw, y)
-        outs.append(y)
     torch.cuda.synchronize()
+    # second round: nothing is allocated, on the device or in torch's cache
+    outs2 = [torch.empty_like(y) for y in outs]
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    for (x, s, wq, sw), y in zip(cases, outs2):
+        sq.sq_linear_noalloc(x, s, wq, sw, y)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == alloc0, "torch memory changed across allocation-free calls"
+    assert free1 == free0, f"device free memory changed across allocation-free calls: {free0} -> {free1}"
+    for y, y2 in zip(outs, outs2):
+        assert torch.equal(y, y2)
     for (x, s, wq, sw), y in zip(cases, outs):
         ref = sq.linear(x, s, wq, sw, out_dtype=torch.bfloat16)  # caller workspace
         torch.cuda.synchronize()

@@ -13,6 +13,7 @@
 #include <cstdlib>
 #include <mutex>
 #include <tuple>
+#include <type_traits>
 #include <vector>
 #include <utility>
 #include <climits>
@@ -24,6 +25,8 @@
 #include "sq_ptx.cuh"
 #include "sq_gptq.cuh"
 #include "sq_splitk.cuh"
+#include "sq_decode.cuh"
+#include "sq_quant_staged.cuh"
 
 namespace {
 
@@ -33,6 +36,7 @@ using sq::OUT_S32;
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxDynSmem = 232448;  // 227 KB of dynamic shared memory per CTA on sm_100
+constexpr int kSmSmemBytes = 233472;  // shared memory of one SM (228 KB)
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -242,7 +246,8 @@ inline int exact_fit_log2g(int64_t nch, int ch)
 
 template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false>
 sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
-                               float *scale, int log2g, cudaStream_t st, const DeviceInfo &di, T *hout = nullptr)
+                               float *scale, int log2g, cudaStream_t st, const DeviceInfo &di, T *hout = nullptr,
+                               int *zero = nullptr, int nzero = 0)
 {
     auto kernel = sq::row_quant_kernel<T, MODE, CH, FIT, BB, GLU>;
     const int smem = static_cast<int>(sq::row_quant_smem(K, BB));
@@ -280,7 +285,7 @@ sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float
         std::fprintf(stderr, "sq quant rows=%lld K=%lld: single pass CH=%d G=%d per_sm=%d blocks=%lld\n",
                      (long long)rows, (long long)K, CH, 1 << log2g, per_sm, (long long)blocks);
     return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(sq::kQuantThreads), smem, st, 0, 0, in, rows,
-                         K, s, log2g, q, scale, hout);
+                         K, s, log2g, q, scale, hout, zero, nzero);
 }
 
 // The quantiser with the gated feed-forward activation in front (rows of
@@ -330,15 +335,90 @@ sq_status launch_glu_quant(const T *gu, int64_t rows, int64_t K, const float *s,
     return SQ_ERR_UNSUPPORTED;
 }
 
+// The staged quantiser (bf16 rows brought into shared memory by bulk
+// copies): rows of exactly 32 * CH * G chunks, CH in {7, 8, 14} and G in
+// {1, 2, 4, 8}.  Returns false (nothing launched) for other rows.
+template <int MODE, int CH, bool BF>
+sq_status launch_staged_cfg(const __nv_bfloat16 *in, int64_t rows, int64_t K, const float *s, int8_t *q,
+                            float *scale, int log2g, cudaStream_t st, const DeviceInfo &di, int *zero, int nzero)
+{
+    auto kernel = sq::row_quant_staged_kernel<MODE, CH, BF>;
+    static std::atomic<uint64_t> attr_done{0};
+    if (!ensure_smem_attr(kernel, kMaxDynSmem - 1024, attr_done))
+        return SQ_ERR_CUDA;
+    const int groups = 8 >> log2g;
+    // two CTAs an SM with two row buffers a group where that fits, else one
+    // CTA with as many buffers (up to 4) as fit
+    int nslots = 0, per_sm = 0;
+    const int64_t per_cta2 = kSmSmemBytes / 2 - 1024 - 256;
+    if (sq::staged_smem_bytes(K, BF, groups, 2) <= per_cta2) {
+        nslots = 2;
+        per_sm = 2;
+        if (sq::staged_smem_bytes(K, BF, groups, 3) <= per_cta2)
+            nslots = 3;
+    } else {
+        for (int n = 4; n >= 2 && nslots == 0; --n)
+            if (sq::staged_smem_bytes(K, BF, groups, n) <= kMaxDynSmem - 1024)
+                nslots = n;
+        per_sm = 1;
+    }
+    if (nslots == 0)
+        return SQ_ERR_UNSUPPORTED;
+    const int smem = static_cast<int>(sq::staged_smem_bytes(K, BF, groups, nslots));
+    const int64_t blocks = std::min<int64_t>((rows + groups - 1) / groups, (int64_t)per_sm * di.sms);
+    if (debug_plan())
+        std::fprintf(stderr, "sq staged quant rows=%lld K=%lld: CH=%d G=%d BF=%d slots=%d per_sm=%d blocks=%lld smem=%d\n",
+                     (long long)rows, (long long)K, CH, 1 << log2g, (int)BF, nslots, per_sm, (long long)blocks, smem);
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(sq::kQuantThreads), smem, st, 0, 0, in, rows,
+                         K, s, log2g, nslots, q, scale, zero, nzero);
+}
+
+template <int MODE>
+bool launch_staged(const __nv_bfloat16 *in, int64_t rows, int64_t K, const float *s, int8_t *q, float *scale,
+                   cudaStream_t st, const DeviceInfo &di, int *zero, int nzero, sq_status &r)
+{
+    // for few rows the quantiser is latency-bound and the register-resident
+    // kernel (smaller shared memory, so it shares an SM with the few-token
+    // GEMM that follows it in sq_linear) is used; SQ_QUANT_STAGED=0 turns the
+    // staged kernel off, =2 takes it for any row count (same arithmetic)
+    static const int mode = std::getenv("SQ_QUANT_STAGED") ? std::atoi(std::getenv("SQ_QUANT_STAGED")) : 1;
+    if (mode == 0 || (mode == 1 && rows < 256))
+        return false;
+    const int64_t nch = K / 8;
+    const bool bb = sq::row_quant_smem(K, true) <= 64 * 1024;
+    for (int ch : {8, 7, 14}) {
+        for (int log2g = 0; log2g <= 3; ++log2g) {
+            if ((int64_t)32 * ch << log2g != nch)
+                continue;
+            if (ch == 8)
+                r = bb ? launch_staged_cfg<MODE, 8, true>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero)
+                       : launch_staged_cfg<MODE, 8, false>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero);
+            else if (ch == 7)
+                r = bb ? launch_staged_cfg<MODE, 7, true>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero)
+                       : launch_staged_cfg<MODE, 7, false>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero);
+            else
+                r = launch_staged_cfg<MODE, 14, false>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero);
+            return r != SQ_ERR_UNSUPPORTED;
+        }
+    }
+    return false;
+}
+
+// `zero` (may be null): nzero ints the quantiser kernel clears on the side.
 template <typename T, int MODE>
 sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
-                            float *scale, cudaStream_t st)
+                            float *scale, cudaStream_t st, int *zero = nullptr, int nzero = 0)
 {
     DeviceInfo di;
     if (!device_info(di))
         return SQ_ERR_CUDA;
     if (rows > 2147483647LL)
         return SQ_ERR_UNSUPPORTED;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        sq_status r = SQ_OK;
+        if (launch_staged<MODE>(in, rows, K, s, q, scale, st, di, zero, nzero, r))
+            return r;
+    }
     // tuning override (same arithmetic, other kernels): SQ_QUANT_KIND=2 takes
     // the two-kernel path for every K
     static const int force_kind = std::getenv("SQ_QUANT_KIND") ? std::atoi(std::getenv("SQ_QUANT_KIND")) : 0;
@@ -356,8 +436,8 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
                 if (((int64_t)32 * force_ch << l) == nch)
                     g = l;
             if (g >= 0) {
-#define SQ_Q_CFG(CH_) (bb ? launch_row_quant_cfg<T, MODE, CH_, true, true>(in, rows, K, s, q, scale, g, st, di) \
-                          : launch_row_quant_cfg<T, MODE, CH_, true, false>(in, rows, K, s, q, scale, g, st, di))
+#define SQ_Q_CFG(CH_) (bb ? launch_row_quant_cfg<T, MODE, CH_, true, true>(in, rows, K, s, q, scale, g, st, di, nullptr, zero, nzero) \
+                          : launch_row_quant_cfg<T, MODE, CH_, true, false>(in, rows, K, s, q, scale, g, st, di, nullptr, zero, nzero))
                 if (force_ch == 2)
                     return SQ_Q_CFG(2);
                 if (force_ch == 4)
@@ -379,16 +459,16 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
             const bool fit = ((int64_t)32 * ch << log2g) == nch;
             if (bb) {
                 if (ch == 8)
-                    return fit ? launch_row_quant_cfg<T, MODE, 8, true, true>(in, rows, K, s, q, scale, log2g, st, di)
-                               : launch_row_quant_cfg<T, MODE, 8, false, true>(in, rows, K, s, q, scale, log2g, st, di);
-                return fit ? launch_row_quant_cfg<T, MODE, 16, true, true>(in, rows, K, s, q, scale, log2g, st, di)
-                           : launch_row_quant_cfg<T, MODE, 16, false, true>(in, rows, K, s, q, scale, log2g, st, di);
+                    return fit ? launch_row_quant_cfg<T, MODE, 8, true, true>(in, rows, K, s, q, scale, log2g, st, di, nullptr, zero, nzero)
+                               : launch_row_quant_cfg<T, MODE, 8, false, true>(in, rows, K, s, q, scale, log2g, st, di, nullptr, zero, nzero);
+                return fit ? launch_row_quant_cfg<T, MODE, 16, true, true>(in, rows, K, s, q, scale, log2g, st, di, nullptr, zero, nzero)
+                           : launch_row_quant_cfg<T, MODE, 16, false, true>(in, rows, K, s, q, scale, log2g, st, di, nullptr, zero, nzero);
             }
             if (ch == 8)
-                return fit ? launch_row_quant_cfg<T, MODE, 8, true, false>(in, rows, K, s, q, scale, log2g, st, di)
-                           : launch_row_quant_cfg<T, MODE, 8, false, false>(in, rows, K, s, q, scale, log2g, st, di);
-            return fit ? launch_row_quant_cfg<T, MODE, 16, true, false>(in, rows, K, s, q, scale, log2g, st, di)
-                       : launch_row_quant_cfg<T, MODE, 16, false, false>(in, rows, K, s, q, scale, log2g, st, di);
+                return fit ? launch_row_quant_cfg<T, MODE, 8, true, false>(in, rows, K, s, q, scale, log2g, st, di, nullptr, zero, nzero)
+                           : launch_row_quant_cfg<T, MODE, 8, false, false>(in, rows, K, s, q, scale, log2g, st, di, nullptr, zero, nzero);
+            return fit ? launch_row_quant_cfg<T, MODE, 16, true, false>(in, rows, K, s, q, scale, log2g, st, di, nullptr, zero, nzero)
+                       : launch_row_quant_cfg<T, MODE, 16, false, false>(in, rows, K, s, q, scale, log2g, st, di, nullptr, zero, nzero);
         }
     }
     sq_status r = (K * (int64_t)sizeof(float) <= kSmemFactorBytes)
@@ -408,7 +488,7 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
     }
     dim3 grid(static_cast<unsigned>(col_blocks), static_cast<unsigned>(row_blocks));
     return launch_kernel(sq::row_codes_kernel<T, MODE>, grid, dim3(threads), 0, st, 0, 0, in, rows, K, s,
-                         static_cast<const float *>(scale), rpb, q);
+                         static_cast<const float *>(scale), rpb, q, zero, nzero);
 }
 
 int64_t max_quant_k(sq_dtype dt) { return dt == SQ_BF16 ? 65536 : 32768; }
@@ -600,11 +680,12 @@ inline int pick_pair_bn(int64_t M, int64_t N, int pairs)
     static const int force = std::getenv("SQ_GEMM_PAIR_BN") ? std::atoi(std::getenv("SQ_GEMM_PAIR_BN")) : -1;
     if (force >= 0)
         return force;
-    constexpr int cand[3] = {256, 192, 128};
-    constexpr int64_t tile_time[3] = {271, 237, 206};
+    // 224 and 160 are interpolated between the measured widths
+    constexpr int cand[5] = {256, 224, 192, 160, 128};
+    constexpr int64_t tile_time[5] = {271, 254, 237, 222, 206};
     int best = 256;
     int64_t best_cost = INT64_MAX;
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 5; ++i) {
         const int64_t tiles = ((M + sq::kPairBM - 1) / sq::kPairBM) * ((N + cand[i] - 1) / cand[i]);
         const int64_t rounds = (tiles + pairs - 1) / std::max(pairs, 1);
         const int64_t cost = rounds * tile_time[i];
@@ -639,8 +720,12 @@ sq_status launch_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const
     switch (bn) {
     case 256:
         return launch_gemm_pair_cfg<256, 6, OUT>(xq, sx, wq, sw, M, N, K, y, st);
+    case 224:
+        return launch_gemm_pair_cfg<224, 7, OUT>(xq, sx, wq, sw, M, N, K, y, st);
     case 192:
         return launch_gemm_pair_cfg<192, 7, OUT>(xq, sx, wq, sw, M, N, K, y, st);
+    case 160:
+        return launch_gemm_pair_cfg<160, 8, OUT>(xq, sx, wq, sw, M, N, K, y, st);
     case 128:
         return launch_gemm_pair_cfg<128, 8, OUT>(xq, sx, wq, sw, M, N, K, y, st);
     default:  // single-SM 128 x 256 tiles
@@ -672,6 +757,101 @@ sq_status launch_fused_linear(const TIN *x, const float *s, const int8_t *wq, co
 
 constexpr int64_t kMaxDim = 2147483647LL;
 
+// ---- the few-token GEMM of sq_linear: a stream over the weight -------------
+// sq_linear runs it for M <= kDecodeMaxM; its int32 partials and tile
+// counters live in the workspace after the codes and scales.
+constexpr int64_t kDecodeMaxM = 128;
+constexpr int64_t kDecodeMaxCtas = 160;  // at least the SM count of every sm_100 part
+
+inline int decode_bnx(int64_t M) { return M <= 32 ? 32 : (M <= 64 ? 64 : 128); }
+
+inline int64_t decode_units(int64_t N, int64_t K) { return ((N + sq::kBM - 1) / sq::kBM) * ((K + sq::kBK - 1) / sq::kBK); }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace of sq_linear: codes [M, K], scales [M], then, for the few-token
+// GEMM, the tile counters [T] and the partial slots [G, 2, BNX, 128].
+struct LinearWs {
+    size_t xq = 0, sx = 0, cnt = 0, slots = 0, total = 0;
+};
+
+inline LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K)
+{
+    LinearWs w;
+    w.xq = 0;
+    w.sx = align_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256);
+    size_t o = w.sx + align_up(static_cast<size_t>(M) * sizeof(float), 256);
+    if (M <= kDecodeMaxM) {
+        const int64_t T = (N + sq::kBM - 1) / sq::kBM;
+        const int64_t G = std::min<int64_t>(decode_units(N, K), kDecodeMaxCtas);
+        w.cnt = o;
+        o += align_up(static_cast<size_t>(T) * sizeof(int), 256);
+        w.slots = o;
+        o += static_cast<size_t>(G) * 2 * decode_bnx(M) * sq::kBM * sizeof(int32_t);
+    }
+    w.total = o;
+    return w;
+}
+
+// Shared memory one quantiser CTA of sq_quant_act takes for rows of K values
+// (the decode GEMM leaves room for one next to it on an SM).
+inline int64_t quant_smem_estimate(int64_t K, sq_dtype dt)
+{
+    const bool bb = dt == SQ_BF16 && sq::row_quant_smem(K, true) <= 64 * 1024;
+    return sq::row_quant_smem(K, bb) + 1024;
+}
+
+template <int BNX, int OUT>
+sq_status launch_decode_cfg(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw, int64_t M,
+                            int64_t N, int64_t K, void *y, int *cnt, int32_t *slots, sq_dtype in_dt,
+                            cudaStream_t st)
+{
+    using Cfg = sq::DecCfg<BNX>;
+    DeviceInfo di;
+    if (!device_info(di))
+        return SQ_ERR_CUDA;
+    const int64_t U = decode_units(N, K);
+    const int G = static_cast<int>(std::min<int64_t>({U, (int64_t)di.sms, kDecodeMaxCtas}));
+    // the deepest ring that still leaves room for a quantiser CTA on the SM
+    // (the two kernels overlap), within the per-CTA limit
+    static const int force_stages = std::getenv("SQ_DECODE_STAGES") ? std::atoi(std::getenv("SQ_DECODE_STAGES")) : 0;
+    const int64_t budget =
+        std::min<int64_t>(kMaxDynSmem, kSmSmemBytes - 1024 - quant_smem_estimate(K, in_dt) - 1024);
+    int stages = force_stages > 1 ? force_stages : 16;
+    while (stages > 2 && sq::dec_smem_bytes(Cfg::STAGE_BYTES, stages) > budget)
+        --stages;
+    const int smem = sq::dec_smem_bytes(Cfg::STAGE_BYTES, stages);
+    if (smem > kMaxDynSmem)
+        return SQ_ERR_UNSUPPORTED;
+    auto kernel = sq::gemm_decode_kernel<BNX, OUT>;
+    static std::atomic<uint64_t> attr_done{0};
+    if (!ensure_smem_attr(kernel, kMaxDynSmem, attr_done))
+        return SQ_ERR_CUDA;
+    CUtensorMap tw, tx;
+    if (!make_tmap_i8(&tw, wq, N, K, sq::kBM) || !make_tmap_i8(&tx, xq, M, K, BNX))
+        return SQ_ERR_CUDA;
+    if (debug_plan())
+        std::fprintf(stderr, "sq decode M=%lld N=%lld K=%lld: BNX=%d units=%lld ctas=%d stages=%d smem=%d\n",
+                     (long long)M, (long long)N, (long long)K, BNX, (long long)U, G, stages, smem);
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(G)), dim3(sq::kDecThreads), smem, st, 0, 0, tw, tx, sx, sw,
+                         y, slots, cnt, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), U, G, stages,
+                         1);
+}
+
+template <int OUT>
+sq_status launch_decode(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw, int64_t M, int64_t N,
+                        int64_t K, void *y, int *cnt, int32_t *slots, sq_dtype in_dt, cudaStream_t st)
+{
+    switch (decode_bnx(M)) {
+    case 32:
+        return launch_decode_cfg<32, OUT>(xq, sx, wq, sw, M, N, K, y, cnt, slots, in_dt, st);
+    case 64:
+        return launch_decode_cfg<64, OUT>(xq, sx, wq, sw, M, N, K, y, cnt, slots, in_dt, st);
+    default:
+        return launch_decode_cfg<128, OUT>(xq, sx, wq, sw, M, N, K, y, cnt, slots, in_dt, st);
+    }
+}
+
 sq_status check_gemm_dims(int64_t M, int64_t N, int64_t K)
 {
     if (M < 1 || N < 16 || K < 16 || N % 16 != 0 || K % 16 != 0)
@@ -680,8 +860,6 @@ sq_status check_gemm_dims(int64_t M, int64_t N, int64_t K)
         return SQ_ERR_UNSUPPORTED;
     return SQ_OK;
 }
-
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // ---- fixed scratch for sq_linear_noalloc -----------------------------------
 // The array belongs to this translation unit; in host code its name only
@@ -1038,11 +1216,9 @@ sq_status sq_w8a8_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_
 
 size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K)
 {
-    (void)N;
-    if (M < 1 || K < 1 || fused_decode_applies(M, K))
+    if (M < 1 || N < 1 || K < 1 || fused_decode_applies(M, K))
         return 0;
-    return align_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256) +
-           align_up(static_cast<size_t>(M) * sizeof(float), 256);
+    return linear_ws_layout(M, N, K).total;
 }
 
 sq_status sq_linear(const void *x, sq_dtype in_dt, const float *s, const int8_t *wq,
@@ -1065,16 +1241,31 @@ sq_status sq_linear(const void *x, sq_dtype in_dt, const float *s, const int8_t 
                                        out_dt, st);
         return launch_fused_linear(static_cast<const float *>(x), s, wq, sw, M, N, K, y, out_dt, st);
     }
-    const size_t need = sq_linear_workspace_size(M, N, K);
-    if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned16(workspace)))
+    const LinearWs L = linear_ws_layout(M, N, K);
+    if (workspace == nullptr || ws_bytes < L.total || !aligned16(workspace))
         return SQ_ERR_INVALID_ARG;
-    int8_t *xq = static_cast<int8_t *>(workspace);
-    float *sx = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
-                                          align_up(static_cast<size_t>(M) * K, 256));
-    r = sq_quant_act(x, in_dt, M, K, s, xq, sx, stream);
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    int8_t *xq = reinterpret_cast<int8_t *>(wsb + L.xq);
+    float *sx = reinterpret_cast<float *>(wsb + L.sx);
+    if (M > kDecodeMaxM) {
+        r = sq_quant_act(x, in_dt, M, K, s, xq, sx, stream);
+        if (r != SQ_OK)
+            return r;
+        return sq_w8a8_gemm(xq, sx, wq, sw, M, N, K, y, out_dt, stream);
+    }
+    // few tokens: the quantiser (which also clears the GEMM's tile counters),
+    // then the weight stream, which starts before the codes are ready
+    int *cnt = reinterpret_cast<int *>(wsb + L.cnt);
+    int32_t *slots = reinterpret_cast<int32_t *>(wsb + L.slots);
+    const int ntiles = static_cast<int>((N + sq::kBM - 1) / sq::kBM);
+    r = (in_dt == SQ_BF16)
+            ? launch_quant_rows<__nv_bfloat16, sq::MODE_X>(static_cast<const __nv_bfloat16 *>(x), M, K, s, xq, sx,
+                                                             st, cnt, ntiles)
+            : launch_quant_rows<float, sq::MODE_X>(static_cast<const float *>(x), M, K, s, xq, sx, st, cnt, ntiles);
     if (r != SQ_OK)
         return r;
-    return sq_w8a8_gemm(xq, sx, wq, sw, M, N, K, y, out_dt, stream);
+    return out_dt == SQ_BF16 ? launch_decode<OUT_BF16>(xq, sx, wq, sw, M, N, K, y, cnt, slots, in_dt, st)
+                             : launch_decode<OUT_F32>(xq, sx, wq, sw, M, N, K, y, cnt, slots, in_dt, st);
 }
 
 sq_status sq_linear_noalloc(const void *x, sq_dtype in_dt, const float *s, const int8_t *wq,

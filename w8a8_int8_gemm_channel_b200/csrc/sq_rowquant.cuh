@@ -294,13 +294,25 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     }
 }
 
+// Side task of the activation quantisers inside sq_linear: clear n ints (the
+// tile counters of the GEMM that follows), spread over the grid.
+__device__ __forceinline__ void clear_ints(int *p, int n)
+{
+    if (p == nullptr)
+        return;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+        p[i] = 0;
+}
+
 template <typename T, int MODE>
 __global__ void __launch_bounds__(256) row_codes_kernel(const T *__restrict__ in, int64_t rows, int64_t K,
                                                         const float *__restrict__ s,
                                                         const float *__restrict__ scale,
-                                                        int64_t rows_per_block, int8_t *__restrict__ q)
+                                                        int64_t rows_per_block, int8_t *__restrict__ q,
+                                                        int *__restrict__ zero, int nzero)
 {
     pdl_prologue();
+    clear_ints(zero, nzero);
     constexpr int V = Vec<T>::N;
     constexpr int U = 4;  // rows in flight per thread
     const int64_t nch = K / V;
@@ -507,9 +519,11 @@ __host__ __device__ constexpr int64_t row_quant_smem(int64_t K, bool bf) { retur
 template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false>
 __global__ void __launch_bounds__(kQuantThreads, (GLU ? (CH <= 8 ? 2 : 1) : (CH <= 8 ? 3 : 2)))
     row_quant_kernel(const T *__restrict__ in, int64_t rows, int64_t K, const float *__restrict__ s,
-                     int log2g, int8_t *__restrict__ q, float *__restrict__ scale_out, T *__restrict__ hout)
+                     int log2g, int8_t *__restrict__ q, float *__restrict__ scale_out, T *__restrict__ hout,
+                     int *__restrict__ zero, int nzero)
 {
     pdl_prologue();
+    clear_ints(zero, nzero);
     constexpr int V = Vec<T>::N;
     constexpr bool BF = BB && (V == 8);  // the bf16 bound
     constexpr int WARPS = kQuantThreads / 32;
