@@ -363,11 +363,16 @@ class Prepared:
 # ---------------------------------------------------------------------------
 
 class Flusher:
+    """Evicts L2 by reading a buffer twice its size.  A read leaves only clean
+    lines behind; a write (a memset) would leave up to a full L2 of dirty
+    lines whose write-back then competes with the timed call for HBM."""
+
     def __init__(self, device):
-        self.buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.buf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+        self.out = torch.empty((), dtype=torch.int64, device=device)
 
     def __call__(self):
-        self.buf.zero_()
+        torch.sum(self.buf, dtype=torch.int64, out=self.out)
 
 
 def time_alone(fn, stream, flush, reps=7, warm=2):
@@ -581,7 +586,7 @@ def run_case(spec, steps, warmup, flush_l2=True, settle_us=0.0):
     """Time one C-ABI call on synthetic data.  spec is one of
     gemm:M,N,K  linear:M,N,K  quant_act:M,K  quant_w:N,K  calib:T,K
     smooth_factors:N,K  rmsnorm_quant:M,K  silu_mul_quant:M,I  gptq_hessian:T,K  gptq_factor:K
-    gptq_rows:N,K.  Prints one JSON line with the median time."""
+    gptq_rows:N,K  copy:bytes.  Prints one JSON line with the median time."""
     import w8a8_int8_gemm_channel_b200 as sq
 
     lib = sq.lib()
@@ -686,16 +691,23 @@ def run_case(spec, steps, warmup, flush_l2=True, settle_us=0.0):
         fn = lambda: lib.sq_smooth_factors(ax.data_ptr(), w.data_ptr(), sq.SQ_BF16, N, K, 0.5,
                                            s.data_ptr(), None, st)
         nbytes = 2 * N * K + 8 * K
+    elif kind == "copy":
+        # device-to-device copy of `bytes` bytes: the bandwidth a kernel of this size can reach
+        (n,) = d
+        a = torch.empty(n, dtype=torch.uint8, device=dev)
+        b = torch.empty_like(a)
+        fn = lambda: (b.copy_(a), 0)[1]
+        nbytes = 2 * n
     else:
         raise SystemExit(f"unknown case {spec}")
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush_l2 else None
+    flush = Flusher(dev) if flush_l2 else None
     for _ in range(warmup):
         assert fn() == 0
     torch.cuda.synchronize()
     times = []
     for _ in range(steps):
         if flush is not None:
-            flush.zero_()
+            flush()
         if settle_us > 0:
             # idle the GPU after the flush so its write-back does not overlap the call
             torch.cuda._sleep(int(settle_us * 1965))

@@ -283,14 +283,25 @@ SQ_API sq_status sq_w8a8_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M,
  *   need separate workspaces.
  * Two kernels run back to back (the second launch overlaps the first);
  * the workspace holds the int8 activations and their scales in between.
+ * For M <= 128 the GEMM streams the weight over every SM: it starts loading
+ * weight tiles while the quantiser is still running (the quantiser waits
+ * for all earlier work on the stream before it lets the GEMM start), and
+ * the workspace also holds the int32 partial sums of tiles that several SMs
+ * share and their counters (cleared by the quantiser on every call, so the
+ * workspace may hold anything beforehand).
  * With the environment variable SQ_LINEAR_FUSED=1, up to 32 tokens are
- * instead quantised inside the GEMM kernel (no workspace; slower on B200).
+ * instead quantised inside an older cluster split-K GEMM kernel (no
+ * workspace; slower on B200).
  */
 SQ_API sq_status sq_linear(const void *x, sq_dtype in_dt, const float *s, const int8_t *wq,
                     const float *sw, int64_t M, int64_t N, int64_t K, void *y, sq_dtype out_dt,
                     void *workspace, size_t ws_bytes, sq_stream_t stream);
 
-/* Bytes of workspace sq_linear needs for these sizes (0 when none). */
+/* Bytes of workspace sq_linear needs for these sizes (0 when none): M * K
+ * bytes of codes and 4 * M of scales (each rounded up to 256), and for
+ * M <= 128 also 4 * ceil(N / 128) of tile counters and
+ * min(ceil(N / 128) * ceil(K / 128), 160) * 2 * T * 512 bytes of partial
+ * sums, T = 32, 64 or 128 the token count rounded up to one of those. */
 SQ_API size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*

@@ -833,9 +833,14 @@ sq_status launch_decode_cfg(const int8_t *xq, const float *sx, const int8_t *wq,
     if (debug_plan())
         std::fprintf(stderr, "sq decode M=%lld N=%lld K=%lld: BNX=%d units=%lld ctas=%d stages=%d smem=%d\n",
                      (long long)M, (long long)N, (long long)K, BNX, (long long)U, G, stages, smem);
+    // tuning overrides (same arithmetic): SQ_DECODE_PREWAIT=0 waits for the
+    // quantiser before any weight load, SQ_DECODE_L2PF=0 drops the L2 prefetch
+    static const int prewait = std::getenv("SQ_DECODE_PREWAIT") ? std::atoi(std::getenv("SQ_DECODE_PREWAIT")) : 1;
+    static const int l2pf = std::getenv("SQ_DECODE_L2PF") ? std::atoi(std::getenv("SQ_DECODE_L2PF")) : 1;
+    const int flags = (prewait ? 1 : 0) | (prewait && l2pf ? 2 : 0);
     return launch_kernel(kernel, dim3(static_cast<unsigned>(G)), dim3(sq::kDecThreads), smem, st, 0, 0, tw, tx, sx, sw,
                          y, slots, cnt, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), U, G, stages,
-                         1);
+                         flags);
 }
 
 template <int OUT>

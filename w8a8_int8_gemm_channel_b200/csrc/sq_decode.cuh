@@ -91,6 +91,8 @@ __device__ __forceinline__ int32_t *dec_slot(int32_t *ws, int64_t c, int slot, i
     return ws + (c * 2 + slot) * static_cast<int64_t>(BNX) * kBM;
 }
 
+// pre_wait: bit 0 -- issue the first stages' weight loads before
+// griddepcontrol.wait; bit 1 -- also prefetch the rest of the range into L2.
 template <int BNX, int OUT>
 __global__ void __launch_bounds__(kDecThreads, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -149,7 +151,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // Up to here nothing touched global memory.  Every thread but the
     // producer waits for the grid before (the quantiser) now; the producer
     // first requests weight tiles when that is allowed.
-    if (!(producer && pre_wait))
+    if (!(producer && (pre_wait & 1)))
         asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             tma_prefetch_desc(&tmX);
             const int64_t nu = u1 - u0;
             // units whose weight tile is requested before the wait
-            const int pre = pre_wait ? static_cast<int>(nu < stages ? nu : stages) : 0;
+            const int pre = (pre_wait & 1) ? static_cast<int>(nu < stages ? nu : stages) : 0;
             for (int i = 0; i < pre; ++i) {
                 const int64_t u = u0 + i;
                 mbar_arrive_expect_tx(full_bar(i), Cfg::STAGE_BYTES);
@@ -170,10 +172,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                             static_cast<int32_t>(u / KB) * kBM);
                 issued_mask |= 1u << i;
             }
-            if (pre_wait) {
+            if (pre_wait & 1) {
                 // the rest of the range into L2 while the quantiser runs
-                for (int64_t u = u0 + pre; u < u1; ++u)
-                    tma_prefetch_l2_2d(&tmW, static_cast<int32_t>(u % KB) * kBK, static_cast<int32_t>(u / KB) * kBM);
+                if (pre_wait & 2)
+                    for (int64_t u = u0 + pre; u < u1; ++u)
+                        tma_prefetch_l2_2d(&tmW, static_cast<int32_t>(u % KB) * kBK,
+                                           static_cast<int32_t>(u / KB) * kBM);
                 asm volatile("griddepcontrol.wait;" ::: "memory");
             }
             for (int i = 0; i < pre; ++i)
