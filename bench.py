@@ -372,7 +372,7 @@ class Flusher:
         self.out = torch.empty((), dtype=torch.int64, device=device)
 
     def __call__(self):
-        torch.sum(self.buf, dtype=torch.int64, out=self.out)
+        torch.sum(self.buf, 0, dtype=torch.int64, out=self.out)
 
 
 def time_alone(fn, stream, flush, reps=7, warm=2):
