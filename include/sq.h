@@ -265,6 +265,34 @@ SQ_API sq_status sq_w8a8_gemm(const int8_t *xq, const float *sx, const int8_t *w
                        sq_stream_t stream);
 
 /*
+ * sq_w8a8_gemm with a workspace, which lets the GEMM use every SM whatever the
+ * shape ("quant_llm_int8", "The architecture: every piece explained": the
+ * same int32 accumulation and outer-product dequantisation):
+ *   - up to 128 tokens, the weight is streamed by one CTA per SM, each taking
+ *     an equal share of the 128-channel x 128-byte weight blocks;
+ *   - more tokens, the tiles that do not fill whole rounds of the CTA pairs
+ *     (the last full round and the partial one) are split along K over all
+ *     pairs.
+ *   A tile shared by several CTAs is summed through int32 partials in the
+ *   workspace (exact: the result is the same bits as sq_w8a8_gemm's).
+ *   workspace: device scratch of at least sq_w8a8_gemm_workspace_size(M, N,
+ *   K) bytes, 16-byte aligned, owned by the caller, any contents; calls that
+ *   run concurrently need separate workspaces.  A small kernel clears the
+ *   workspace's tile counters before the GEMM.  Errors as sq_w8a8_gemm, plus
+ *   SQ_ERR_INVALID_ARG for a missing or too small workspace.
+ */
+SQ_API sq_status sq_w8a8_gemm_ws(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
+                                 int64_t M, int64_t N, int64_t K, void *y, sq_dtype out_dt,
+                                 void *workspace, size_t ws_bytes, sq_stream_t stream);
+
+/* Bytes of workspace sq_w8a8_gemm_ws needs (0 for invalid sizes): for
+ * M <= 128, 4 * ceil(N / 128) bytes of tile counters (rounded up to 256) and
+ * min(ceil(N / 128) * ceil(K / 128), 160) * 2 * T * 512 bytes of partial sums,
+ * T = 32, 64 or 128 the token count rounded up to one of those; for more
+ * tokens, 1280 bytes of counters and 40 MiB of partial sums. */
+SQ_API size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
  * The raw int32 accumulators acc[m, n] = sum_k xq[m, k] * wq[n, k] of the same
  * tensor-core kernels (no scales), for verification.  acc is [M, N] int32.
  */
@@ -277,18 +305,21 @@ SQ_API sq_status sq_w8a8_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M,
  * "Inter-Token Latency (ITL)", charges to every generated token: find each
  * token's range and scale, cast to int8, multiply in int8, dequantise.
  *   x [M, K] dtype in_dt; s [K]; wq [N, K]; sw [N]; y [M, N] dtype out_dt.
- *   workspace: device scratch of at least sq_linear_workspace_size(M, N, K)
- *   bytes (may be NULL when that size is 0), 16-byte aligned, owned by the
- *   caller and not read by the caller afterwards; calls that run concurrently
- *   need separate workspaces.
+ *   workspace: device scratch, 16-byte aligned, owned by the caller and not
+ *   read by the caller afterwards (may be NULL when
+ *   sq_linear_workspace_size(M, N, K) is 0); calls that run concurrently
+ *   need separate workspaces.  It must hold at least the int8 codes and
+ *   scales, M * K + 4 * M bytes (each rounded up to 256); with
+ *   sq_linear_workspace_size(M, N, K) bytes it also holds the GEMM's own
+ *   workspace, and the GEMM runs as sq_w8a8_gemm_ws (every SM busy whatever
+ *   the shape) instead of as sq_w8a8_gemm.
  * Two kernels run back to back (the second launch overlaps the first);
- * the workspace holds the int8 activations and their scales in between.
- * For M <= 128 the GEMM streams the weight over every SM: it starts loading
+ * the workspace holds the int8 activations and their scales in between, and
+ * the GEMM's tile counters and partial sums (the quantiser clears the
+ * counters on every call, so the workspace may hold anything beforehand).
+ * For M <= 128 the GEMM streams the weight over every SM and starts loading
  * weight tiles while the quantiser is still running (the quantiser waits
- * for all earlier work on the stream before it lets the GEMM start), and
- * the workspace also holds the int32 partial sums of tiles that several SMs
- * share and their counters (cleared by the quantiser on every call, so the
- * workspace may hold anything beforehand).
+ * for all earlier work on the stream before it lets the GEMM start).
  * With the environment variable SQ_LINEAR_FUSED=1, up to 32 tokens are
  * instead quantised inside an older cluster split-K GEMM kernel (no
  * workspace; slower on B200).
@@ -297,11 +328,9 @@ SQ_API sq_status sq_linear(const void *x, sq_dtype in_dt, const float *s, const 
                     const float *sw, int64_t M, int64_t N, int64_t K, void *y, sq_dtype out_dt,
                     void *workspace, size_t ws_bytes, sq_stream_t stream);
 
-/* Bytes of workspace sq_linear needs for these sizes (0 when none): M * K
- * bytes of codes and 4 * M of scales (each rounded up to 256), and for
- * M <= 128 also 4 * ceil(N / 128) of tile counters and
- * min(ceil(N / 128) * ceil(K / 128), 160) * 2 * T * 512 bytes of partial
- * sums, T = 32, 64 or 128 the token count rounded up to one of those. */
+/* Bytes of workspace sq_linear needs for these sizes to run at its best (0
+ * when it needs none): M * K bytes of codes and 4 * M of scales (each
+ * rounded up to 256), then sq_w8a8_gemm_workspace_size(M, N, K). */
 SQ_API size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
@@ -317,9 +346,11 @@ SQ_API size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K);
  * array of SQ_LINEAR_NOALLOC_SCRATCH_BYTES bytes, held by every GPU that loads
  * the library until the process exits).  The call makes no cudaMalloc or
  * cudaFree and calls no allocating library routine.
- *   - Sizes whose sq_linear_workspace_size(M, N, K) exceeds
- *     SQ_LINEAR_NOALLOC_SCRATCH_BYTES are rejected with SQ_ERR_UNSUPPORTED
- *     before anything is enqueued.
+ *   - Sizes whose int8 codes and scales (M * K + 4 * M bytes, each rounded
+ *     up to 256) exceed SQ_LINEAR_NOALLOC_SCRATCH_BYTES are rejected with
+ *     SQ_ERR_UNSUPPORTED before anything is enqueued.  When the GEMM's own
+ *     workspace does not fit next to them, the GEMM runs without one (as
+ *     sq_w8a8_gemm).
  *   - The first call on a device (with that device current) looks up the
  *     device address of the scratch array once and keeps it for the process;
  *     make that first call before any stream capture on the device.  The

@@ -123,7 +123,9 @@ def test_linear_rejects_and_workspace_size(lib):
     assert need >= M * K + 4 * M and need % 16 == 0
     f = lib.sq_linear
     assert need > 0 and f(A, 1, B, C, D, M, N, K, E, 1, None, 0, None) == INV
-    assert f(A, 1, B, C, D, M, N, K, E, 1, A + 0x100000, need - 1, None) == INV
+    a256 = lambda v: (v + 255) // 256 * 256
+    minimum = a256(M * K) + a256(4 * M)  # the codes and scales; the rest only speeds the GEMM
+    assert f(A, 1, B, C, D, M, N, K, E, 1, A + 0x100000, minimum - 1, None) == INV
     assert f(A, 1, B, C, D, M, N, K, E, 1, MIS, need, None) == INV
     assert f(A, 1, B, C, D, 0, N, K, E, 1, A, need, None) == INV
     assert f(A, 1, B, C, D, M, 24, K, E, 1, A, need, None) == INV
@@ -164,6 +166,25 @@ def test_silu_mul_quant_rejects_bad_arguments(lib):
     assert f(A, 7, 4, 64, B, C, D, None, None) == INV           # bad dtype
     assert f(A, 1, 4, 65536, B, C, D, None, None) == UNS        # row longer than one pass takes
     assert f(A, 0, 4, 32768, B, C, D, None, None) == UNS        # fp32 rows: at most 16384
+
+
+def test_gemm_ws_rejects_bad_arguments(lib):
+    f = lib.sq_w8a8_gemm_ws
+    M, N, K = 300, 512, 1024
+    need = lib.sq_w8a8_gemm_workspace_size(M, N, K)
+    # 4 x 80 tile counters (1280 bytes), then 2 x 80 CTAs x 2 slots x 128 x 256 int32 partial sums
+    assert need == 1280 + 160 * 2 * 128 * 256 * 4
+    # few tokens: ceil(N / 128) counters (rounded up to 256 bytes), then
+    # min(units, 160) CTAs x 2 slots x 32 tokens x 128 int32
+    units = (6144 // 128) * (4096 // 128)
+    assert lib.sq_w8a8_gemm_workspace_size(16, 6144, 4096) == 256 + min(units, 160) * 2 * 32 * 128 * 4
+    assert lib.sq_w8a8_gemm_workspace_size(0, 6144, 4096) == 0
+    assert f(A, B, C, D, M, N, K, E, 1, None, need, None) == INV      # no workspace
+    assert f(A, B, C, D, M, N, K, E, 1, A, need - 1, None) == INV     # too small
+    assert f(A, B, C, D, M, N, K, E, 1, MIS, need, None) == INV       # misaligned
+    assert f(A, B, C, D, M, 24, K, E, 1, A, need, None) == INV        # N not a multiple of 16
+    assert f(A, B, C, D, M, N, K, E, 5, A, need, None) == INV         # bad dtype
+    assert f(None, B, C, D, M, N, K, E, 1, A, need, None) == INV
 
 
 def test_gptq_entry_points_reject_bad_arguments(lib):

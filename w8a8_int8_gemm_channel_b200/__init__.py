@@ -14,6 +14,8 @@ The raw entry points keep the C names and take caller-allocated outputs:
     sq_smooth_quant_weight(w, s, wq, sw)
     sq_quant_act(x, s, xq, sx)
     sq_w8a8_gemm(xq, sx, wq, sw, y)
+    sq_w8a8_gemm_ws(xq, sx, wq, sw, y, workspace)   every SM busy whatever the shape
+    sq_w8a8_gemm_workspace_size(M, N, K)
     sq_w8a8_gemm_s32(xq, wq, acc)
     sq_linear(x, s, wq, sw, y, workspace)
     sq_linear_workspace_size(M, N, K)
@@ -52,6 +54,8 @@ ABI_SYMBOLS = (
     "sq_gptq_factor",
     "sq_gptq_quant_weight",
     "sq_w8a8_gemm",
+    "sq_w8a8_gemm_ws",
+    "sq_w8a8_gemm_workspace_size",
     "sq_w8a8_gemm_s32",
     "sq_linear",
     "sq_linear_workspace_size",
@@ -90,6 +94,8 @@ def _declare(lib):
         "sq_gptq_factor": ([P, I, F, P, P, ctypes.c_size_t, P], E),
         "sq_gptq_quant_weight": ([P, E, I, I, P, P, P, P, P], E),
         "sq_w8a8_gemm": ([P, P, P, P, I, I, I, P, E, P], E),
+        "sq_w8a8_gemm_ws": ([P, P, P, P, I, I, I, P, E, P, ctypes.c_size_t, P], E),
+        "sq_w8a8_gemm_workspace_size": ([I, I, I], ctypes.c_size_t),
         "sq_w8a8_gemm_s32": ([P, P, I, I, I, P, P], E),
         "sq_linear": ([P, E, P, P, P, I, I, I, P, E, P, ctypes.c_size_t, P], E),
         "sq_linear_workspace_size": ([I, I, I], ctypes.c_size_t),
@@ -259,6 +265,23 @@ def sq_w8a8_gemm(xq, sx, wq, sw, y, stream=None):
     _check("sq_w8a8_gemm",
            lib().sq_w8a8_gemm(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y),
                               _dtype_code(y), _stream(stream)))
+
+
+def sq_w8a8_gemm_workspace_size(M: int, N: int, K: int) -> int:
+    return int(lib().sq_w8a8_gemm_workspace_size(M, N, K))
+
+
+def sq_w8a8_gemm_ws(xq, sx, wq, sw, y, workspace=None, stream=None):
+    """sq_w8a8_gemm with a workspace (allocated here when not given)."""
+    import torch
+
+    M, K = xq.shape
+    N = wq.shape[0]
+    if workspace is None:
+        workspace = torch.empty(sq_w8a8_gemm_workspace_size(M, N, K), dtype=torch.uint8, device=xq.device)
+    _check("sq_w8a8_gemm_ws",
+           lib().sq_w8a8_gemm_ws(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), _dtype_code(y),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def sq_w8a8_gemm_s32(xq, wq, acc, stream=None):

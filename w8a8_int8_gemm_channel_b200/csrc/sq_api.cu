@@ -644,118 +644,7 @@ sq_status launch_splitk_cfg(const TIN *x, const float *s, const int8_t *xq, cons
                          static_cast<int>(K), p.splits, p.kbps, p.stages, p.kbs);
 }
 
-// Prefill GEMM on CTA pairs: 256 x BN output tiles, persistent over tiles.
-template <int BN, int STAGES, int OUT>
-sq_status launch_gemm_pair_cfg(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
-                               int64_t M, int64_t N, int64_t K, void *y, cudaStream_t st)
-{
-    using Cfg = sq::PairCfg<BN, STAGES>;
-    CUtensorMap ta, tb;
-    if (!make_tmap_i8(&ta, xq, M, K, 128) || !make_tmap_i8(&tb, wq, N, K, BN / 2))
-        return SQ_ERR_CUDA;
-    auto kernel = sq::gemm_i8_pair_kernel<BN, STAGES, OUT>;
-    static std::atomic<uint64_t> attr_done{0};
-    if (!ensure_smem_attr(kernel, Cfg::SMEM_BYTES, attr_done))
-        return SQ_ERR_CUDA;
-    const int active = active_clusters(kernel, 2, Cfg::SMEM_BYTES, sq::kPairThreads);
-    if (active <= 0)
-        return SQ_ERR_CUDA;
-    const int64_t tiles = ((M + sq::kPairBM - 1) / sq::kPairBM) * ((N + BN - 1) / BN);
-    const int64_t pairs = std::min<int64_t>(tiles, active);
-    if (debug_plan())
-        std::fprintf(stderr, "sq gemm pair M=%lld N=%lld K=%lld: BN=%d stages=%d tiles=%lld pairs=%lld\n",
-                     (long long)M, (long long)N, (long long)K, BN, STAGES, (long long)tiles, (long long)pairs);
-    return launch_kernel(kernel, dim3(static_cast<unsigned>(2 * pairs)), dim3(sq::kPairThreads), Cfg::SMEM_BYTES, st, 2,
-                         1, ta, tb, sx, sw, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K));
-}
-
-// Tile width of the pair GEMM: the fewest rounds of tiles over the
-// co-resident pairs, each round costing one tile's time.  Narrower tiles
-// re-read more operand bytes per operation from L2, so a tile's time is not
-// proportional to its width: measured on B200 (8192 x 28672 x 4096, many
-// rounds), 256 / 192 / 128-wide tiles reach 0.94 / 0.81 / 0.62 of the int8
-// peak, i.e. relative tile times 271 : 237 : 206.
-inline int pick_pair_bn(int64_t M, int64_t N, int pairs)
-{
-    static const int force = std::getenv("SQ_GEMM_PAIR_BN") ? std::atoi(std::getenv("SQ_GEMM_PAIR_BN")) : -1;
-    if (force >= 0)
-        return force;
-    // 224 and 160 are interpolated between the measured widths
-    constexpr int cand[5] = {256, 224, 192, 160, 128};
-    constexpr int64_t tile_time[5] = {271, 254, 237, 222, 206};
-    int best = 256;
-    int64_t best_cost = INT64_MAX;
-    for (int i = 0; i < 5; ++i) {
-        const int64_t tiles = ((M + sq::kPairBM - 1) / sq::kPairBM) * ((N + cand[i] - 1) / cand[i]);
-        const int64_t rounds = (tiles + pairs - 1) / std::max(pairs, 1);
-        const int64_t cost = rounds * tile_time[i];
-        if (cost < best_cost) {
-            best_cost = cost;
-            best = cand[i];
-        }
-    }
-    return best;
-}
-
-template <int OUT>
-sq_status launch_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
-                      int64_t M, int64_t N, int64_t K, void *y, cudaStream_t st)
-{
-    const float *nf = nullptr;
-    // weight tiles through the load/store unit (cp.async) or TMA
-    static const bool lsu = std::getenv("SQ_SPLITK_LSU") && std::atoi(std::getenv("SQ_SPLITK_LSU")) == 1;
-    if (M <= 32)
-        return lsu ? launch_splitk_cfg<32, OUT, false, float, true>(nf, nf, xq, sx, wq, sw, M, N, K, y, st)
-                   : launch_splitk_cfg<32, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
-    if (M <= 64)
-        return lsu ? launch_splitk_cfg<64, OUT, false, float, true>(nf, nf, xq, sx, wq, sw, M, N, K, y, st)
-                   : launch_splitk_cfg<64, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
-    if (M <= 128)
-        return lsu ? launch_splitk_cfg<128, OUT, false, float, true>(nf, nf, xq, sx, wq, sw, M, N, K, y, st)
-                   : launch_splitk_cfg<128, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
-    DeviceInfo di;
-    if (!device_info(di))
-        return SQ_ERR_CUDA;
-    const int bn = pick_pair_bn(M, N, di.sms / 2);
-    switch (bn) {
-    case 256:
-        return launch_gemm_pair_cfg<256, 6, OUT>(xq, sx, wq, sw, M, N, K, y, st);
-    case 224:
-        return launch_gemm_pair_cfg<224, 7, OUT>(xq, sx, wq, sw, M, N, K, y, st);
-    case 192:
-        return launch_gemm_pair_cfg<192, 7, OUT>(xq, sx, wq, sw, M, N, K, y, st);
-    case 160:
-        return launch_gemm_pair_cfg<160, 8, OUT>(xq, sx, wq, sw, M, N, K, y, st);
-    case 128:
-        return launch_gemm_pair_cfg<128, 8, OUT>(xq, sx, wq, sw, M, N, K, y, st);
-    default:  // single-SM 128 x 256 tiles
-        return launch_gemm_cfg<256, 4, OUT, false>(xq, sx, wq, sw, M, N, K, y, st);
-    }
-}
-
-// The fused decode path (activation quant inside the GEMM, no workspace)
-// applies to at most 32 tokens when K fits the per-CTA token operand, and
-// only when selected.
-bool fused_decode_applies(int64_t M, int64_t K)
-{
-    // off unless SQ_LINEAR_FUSED=1: on B200 the quantiser kernel followed by
-    // the split-K GEMM (launch overlapped) is faster than quantising inside
-    // the GEMM kernel's prologue
-    static const bool on = std::getenv("SQ_LINEAR_FUSED") && std::atoi(std::getenv("SQ_LINEAR_FUSED")) == 1;
-    return on && M <= 32 && K <= sq::kMaxSplits * (kFusedSliceBytes / (32 * sq::kBK)) * sq::kBK;
-}
-
-template <typename TIN>
-sq_status launch_fused_linear(const TIN *x, const float *s, const int8_t *wq, const float *sw,
-                              int64_t M, int64_t N, int64_t K, void *y, sq_dtype out_dt,
-                              cudaStream_t st)
-{
-    if (out_dt == SQ_BF16)
-        return launch_splitk_cfg<32, OUT_BF16, true, TIN>(x, s, nullptr, nullptr, wq, sw, M, N, K, y, st);
-    return launch_splitk_cfg<32, OUT_F32, true, TIN>(x, s, nullptr, nullptr, wq, sw, M, N, K, y, st);
-}
-
-constexpr int64_t kMaxDim = 2147483647LL;
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // ---- the few-token GEMM of sq_linear: a stream over the weight -------------
 // sq_linear runs it for M <= kDecodeMaxM; its int32 partials and tile
@@ -767,12 +656,45 @@ inline int decode_bnx(int64_t M) { return M <= 32 ? 32 : (M <= 64 ? 64 : 128); }
 
 inline int64_t decode_units(int64_t N, int64_t K) { return ((N + sq::kBM - 1) / sq::kBM) * ((K + sq::kBK - 1) / sq::kBK); }
 
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Workspace of sq_linear: codes [M, K], scales [M], then, for the few-token
-// GEMM, the tile counters [T] and the partial slots [G, 2, BNX, 128].
+// Workspace of the GEMM when it has one (sq_w8a8_gemm_ws, and sq_linear after
+// its codes and scales): tile counters, then partial-sum slots.
+//   few tokens (M <= kDecodeMaxM): counters [T], slots [G, 2, BNX, 128];
+//   more: counters [4 * kMaxPairs], slots [2 * kMaxPairs, 2, 128, 256].
+constexpr int64_t kMaxPairs = 80;  // CTA pairs of the pair kernel a device can hold at once (sm_100: at most 80)
+
+struct GemmWs {
+    size_t cnt = 0, slots = 0, total = 0;
+    int ncnt = 0;  // counters to clear before each call
+};
+
+inline GemmWs gemm_ws_layout(int64_t M, int64_t N, int64_t K, size_t base)
+{
+    GemmWs w;
+    size_t o = base;
+    w.cnt = o;
+    if (M <= kDecodeMaxM) {
+        const int64_t T = (N + sq::kBM - 1) / sq::kBM;
+        const int64_t G = std::min<int64_t>(decode_units(N, K), kDecodeMaxCtas);
+        w.ncnt = static_cast<int>(T);
+        o += align_up(static_cast<size_t>(T) * sizeof(int), 256);
+        w.slots = o;
+        o += static_cast<size_t>(G) * 2 * decode_bnx(M) * sq::kBM * sizeof(int32_t);
+    } else {
+        w.ncnt = static_cast<int>(4 * kMaxPairs);
+        o += align_up(static_cast<size_t>(w.ncnt) * sizeof(int), 256);
+        w.slots = o;
+        o += static_cast<size_t>(2 * kMaxPairs) * 2 * 128 * 256 * sizeof(int32_t);
+    }
+    w.total = o;
+    return w;
+}
+
+// Workspace of sq_linear: codes [M, K] and scales [M] (the minimum), then the
+// GEMM's workspace (used when the caller's workspace holds it too).
 struct LinearWs {
-    size_t xq = 0, sx = 0, cnt = 0, slots = 0, total = 0;
+    size_t xq = 0, sx = 0, minimum = 0;
+    GemmWs g;
 };
 
 inline LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K)
@@ -780,16 +702,8 @@ inline LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K)
     LinearWs w;
     w.xq = 0;
     w.sx = align_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256);
-    size_t o = w.sx + align_up(static_cast<size_t>(M) * sizeof(float), 256);
-    if (M <= kDecodeMaxM) {
-        const int64_t T = (N + sq::kBM - 1) / sq::kBM;
-        const int64_t G = std::min<int64_t>(decode_units(N, K), kDecodeMaxCtas);
-        w.cnt = o;
-        o += align_up(static_cast<size_t>(T) * sizeof(int), 256);
-        w.slots = o;
-        o += static_cast<size_t>(G) * 2 * decode_bnx(M) * sq::kBM * sizeof(int32_t);
-    }
-    w.total = o;
+    w.minimum = w.sx + align_up(static_cast<size_t>(M) * sizeof(float), 256);
+    w.g = gemm_ws_layout(M, N, K, w.minimum);
     return w;
 }
 
@@ -856,6 +770,152 @@ sq_status launch_decode(const int8_t *xq, const float *sx, const int8_t *wq, con
         return launch_decode_cfg<128, OUT>(xq, sx, wq, sw, M, N, K, y, cnt, slots, in_dt, st);
     }
 }
+
+// Prefill GEMM on CTA pairs: 256 x BN output tiles, persistent over tiles.
+// With a workspace (slots, cnt not null) and tiles that do not fill whole
+// rounds of the co-resident pairs, the last round and the partial one are
+// done stream-K: their k blocks are cut into one equal range per pair, and
+// tiles shared by several pairs are summed through int32 partials.
+template <int BN, int STAGES, int OUT>
+sq_status launch_gemm_pair_cfg(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
+                               int64_t M, int64_t N, int64_t K, void *y, cudaStream_t st, int32_t *slots = nullptr,
+                               int *cnt = nullptr)
+{
+    using Cfg = sq::PairCfg<BN, STAGES>;
+    CUtensorMap ta, tb;
+    if (!make_tmap_i8(&ta, xq, M, K, 128) || !make_tmap_i8(&tb, wq, N, K, BN / 2))
+        return SQ_ERR_CUDA;
+    auto kernel = sq::gemm_i8_pair_kernel<BN, STAGES, OUT>;
+    static std::atomic<uint64_t> attr_done{0};
+    if (!ensure_smem_attr(kernel, Cfg::SMEM_BYTES, attr_done))
+        return SQ_ERR_CUDA;
+    const int active = std::min<int>(active_clusters(kernel, 2, Cfg::SMEM_BYTES, sq::kPairThreads),
+                                     static_cast<int>(kMaxPairs));
+    if (active <= 0)
+        return SQ_ERR_CUDA;
+    const int64_t tiles = ((M + sq::kPairBM - 1) / sq::kPairBM) * ((N + BN - 1) / BN);
+    const int64_t kb = (K + sq::kBK - 1) / sq::kBK;
+    int64_t pairs = std::min<int64_t>(tiles, active);
+    int64_t sk_first = tiles, sk_units = 0;
+    static const bool sk_off = std::getenv("SQ_GEMM_SK") && std::atoi(std::getenv("SQ_GEMM_SK")) == 0;
+    if (slots != nullptr && cnt != nullptr && !sk_off && tiles % active != 0) {
+        // the last full round and the partial one; with fewer tiles than
+        // pairs, all of them (and no more pairs than units, so that every
+        // pair has some)
+        const int64_t full = tiles / active;
+        sk_first = full >= 1 ? (full - 1) * active : 0;
+        sk_units = (tiles - sk_first) * kb;
+        pairs = full >= 1 ? active : std::min<int64_t>(active, sk_units);
+    }
+    if (debug_plan())
+        std::fprintf(stderr, "sq gemm pair M=%lld N=%lld K=%lld: BN=%d stages=%d tiles=%lld pairs=%lld sk_first=%lld sk_units=%lld\n",
+                     (long long)M, (long long)N, (long long)K, BN, STAGES, (long long)tiles, (long long)pairs,
+                     (long long)sk_first, (long long)sk_units);
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(2 * pairs)), dim3(sq::kPairThreads), Cfg::SMEM_BYTES, st, 2,
+                         1, ta, tb, sx, sw, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+                         static_cast<int>(sk_first), sk_units, slots, cnt);
+}
+
+// Tile width of the pair GEMM: the fewest rounds of tiles over the
+// co-resident pairs, each round costing one tile's time.  Narrower tiles
+// re-read more operand bytes per operation from L2, so a tile's time is not
+// proportional to its width: measured on B200 (8192 x 28672 x 4096, many
+// rounds), 256 / 192 / 128-wide tiles reach 0.94 / 0.81 / 0.62 of the int8
+// peak, i.e. relative tile times 271 : 237 : 206.
+inline int pick_pair_bn(int64_t M, int64_t N, int pairs)
+{
+    static const int force = std::getenv("SQ_GEMM_PAIR_BN") ? std::atoi(std::getenv("SQ_GEMM_PAIR_BN")) : -1;
+    if (force >= 0)
+        return force;
+    // 224 and 160 are interpolated between the measured widths
+    constexpr int cand[5] = {256, 224, 192, 160, 128};
+    constexpr int64_t tile_time[5] = {271, 254, 237, 222, 206};
+    int best = 256;
+    int64_t best_cost = INT64_MAX;
+    for (int i = 0; i < 5; ++i) {
+        const int64_t tiles = ((M + sq::kPairBM - 1) / sq::kPairBM) * ((N + cand[i] - 1) / cand[i]);
+        const int64_t rounds = (tiles + pairs - 1) / std::max(pairs, 1);
+        const int64_t cost = rounds * tile_time[i];
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = cand[i];
+        }
+    }
+    return best;
+}
+
+// The GEMM with or without a workspace (cnt, slots; null: none).  With one,
+// up to kDecodeMaxM tokens run the weight-streaming kernel and more run the
+// pair kernel with its stream-K tail; the caller has launched, right before,
+// a kernel of this library that clears the tile counters (the quantiser, or
+// the zeroing kernel of sq_w8a8_gemm_ws), which is also what lets the
+// few-token kernel request weights before its griddepcontrol.wait.
+template <int OUT>
+sq_status launch_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
+                      int64_t M, int64_t N, int64_t K, void *y, cudaStream_t st, int *cnt = nullptr,
+                      int32_t *slots = nullptr, sq_dtype in_dt = SQ_BF16)
+{
+    const float *nf = nullptr;
+    const bool ws = cnt != nullptr && slots != nullptr;
+    if (ws && M <= kDecodeMaxM)
+        return launch_decode<OUT>(xq, sx, wq, sw, M, N, K, y, cnt, slots, in_dt, st);
+    // weight tiles through the load/store unit (cp.async) or TMA
+    static const bool lsu = std::getenv("SQ_SPLITK_LSU") && std::atoi(std::getenv("SQ_SPLITK_LSU")) == 1;
+    if (M <= 32)
+        return lsu ? launch_splitk_cfg<32, OUT, false, float, true>(nf, nf, xq, sx, wq, sw, M, N, K, y, st)
+                   : launch_splitk_cfg<32, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
+    if (M <= 64)
+        return lsu ? launch_splitk_cfg<64, OUT, false, float, true>(nf, nf, xq, sx, wq, sw, M, N, K, y, st)
+                   : launch_splitk_cfg<64, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
+    if (M <= 128)
+        return lsu ? launch_splitk_cfg<128, OUT, false, float, true>(nf, nf, xq, sx, wq, sw, M, N, K, y, st)
+                   : launch_splitk_cfg<128, OUT, false, float>(nf, nf, xq, sx, wq, sw, M, N, K, y, st);
+    DeviceInfo di;
+    if (!device_info(di))
+        return SQ_ERR_CUDA;
+    // with a workspace the tail rounds are split stream-K, so the widest
+    // (most efficient) tile is used throughout
+    static const bool sk_off = std::getenv("SQ_GEMM_SK") && std::atoi(std::getenv("SQ_GEMM_SK")) == 0;
+    const int bn = (ws && !sk_off && !std::getenv("SQ_GEMM_PAIR_BN")) ? 256 : pick_pair_bn(M, N, di.sms / 2);
+    switch (bn) {
+    case 256:
+        return launch_gemm_pair_cfg<256, 6, OUT>(xq, sx, wq, sw, M, N, K, y, st, slots, cnt);
+    case 224:
+        return launch_gemm_pair_cfg<224, 7, OUT>(xq, sx, wq, sw, M, N, K, y, st, slots, cnt);
+    case 192:
+        return launch_gemm_pair_cfg<192, 7, OUT>(xq, sx, wq, sw, M, N, K, y, st, slots, cnt);
+    case 160:
+        return launch_gemm_pair_cfg<160, 8, OUT>(xq, sx, wq, sw, M, N, K, y, st, slots, cnt);
+    case 128:
+        return launch_gemm_pair_cfg<128, 8, OUT>(xq, sx, wq, sw, M, N, K, y, st, slots, cnt);
+    default:  // single-SM 128 x 256 tiles
+        return launch_gemm_cfg<256, 4, OUT, false>(xq, sx, wq, sw, M, N, K, y, st);
+    }
+}
+
+// The fused decode path (activation quant inside the GEMM, no workspace)
+// applies to at most 32 tokens when K fits the per-CTA token operand, and
+// only when selected.
+bool fused_decode_applies(int64_t M, int64_t K)
+{
+    // off unless SQ_LINEAR_FUSED=1: on B200 the quantiser kernel followed by
+    // the split-K GEMM (launch overlapped) is faster than quantising inside
+    // the GEMM kernel's prologue
+    static const bool on = std::getenv("SQ_LINEAR_FUSED") && std::atoi(std::getenv("SQ_LINEAR_FUSED")) == 1;
+    return on && M <= 32 && K <= sq::kMaxSplits * (kFusedSliceBytes / (32 * sq::kBK)) * sq::kBK;
+}
+
+template <typename TIN>
+sq_status launch_fused_linear(const TIN *x, const float *s, const int8_t *wq, const float *sw,
+                              int64_t M, int64_t N, int64_t K, void *y, sq_dtype out_dt,
+                              cudaStream_t st)
+{
+    if (out_dt == SQ_BF16)
+        return launch_splitk_cfg<32, OUT_BF16, true, TIN>(x, s, nullptr, nullptr, wq, sw, M, N, K, y, st);
+    return launch_splitk_cfg<32, OUT_F32, true, TIN>(x, s, nullptr, nullptr, wq, sw, M, N, K, y, st);
+}
+
+constexpr int64_t kMaxDim = 2147483647LL;
 
 sq_status check_gemm_dims(int64_t M, int64_t N, int64_t K)
 {
@@ -1223,7 +1283,7 @@ size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K)
 {
     if (M < 1 || N < 1 || K < 1 || fused_decode_applies(M, K))
         return 0;
-    return linear_ws_layout(M, N, K).total;
+    return linear_ws_layout(M, N, K).g.total;
 }
 
 sq_status sq_linear(const void *x, sq_dtype in_dt, const float *s, const int8_t *wq,
@@ -1247,30 +1307,60 @@ sq_status sq_linear(const void *x, sq_dtype in_dt, const float *s, const int8_t 
         return launch_fused_linear(static_cast<const float *>(x), s, wq, sw, M, N, K, y, out_dt, st);
     }
     const LinearWs L = linear_ws_layout(M, N, K);
-    if (workspace == nullptr || ws_bytes < L.total || !aligned16(workspace))
+    if (workspace == nullptr || ws_bytes < L.minimum || !aligned16(workspace))
         return SQ_ERR_INVALID_ARG;
     uint8_t *wsb = static_cast<uint8_t *>(workspace);
     int8_t *xq = reinterpret_cast<int8_t *>(wsb + L.xq);
     float *sx = reinterpret_cast<float *>(wsb + L.sx);
-    if (M > kDecodeMaxM) {
-        r = sq_quant_act(x, in_dt, M, K, s, xq, sx, stream);
-        if (r != SQ_OK)
-            return r;
-        return sq_w8a8_gemm(xq, sx, wq, sw, M, N, K, y, out_dt, stream);
-    }
-    // few tokens: the quantiser (which also clears the GEMM's tile counters),
-    // then the weight stream, which starts before the codes are ready
-    int *cnt = reinterpret_cast<int *>(wsb + L.cnt);
-    int32_t *slots = reinterpret_cast<int32_t *>(wsb + L.slots);
-    const int ntiles = static_cast<int>((N + sq::kBM - 1) / sq::kBM);
+    // the GEMM's own workspace when the caller's holds it: the quantiser
+    // clears its tile counters on the side
+    const bool gws = ws_bytes >= L.g.total;
+    int *cnt = gws ? reinterpret_cast<int *>(wsb + L.g.cnt) : nullptr;
+    int32_t *slots = gws ? reinterpret_cast<int32_t *>(wsb + L.g.slots) : nullptr;
+    const int ncnt = gws ? L.g.ncnt : 0;
     r = (in_dt == SQ_BF16)
             ? launch_quant_rows<__nv_bfloat16, sq::MODE_X>(static_cast<const __nv_bfloat16 *>(x), M, K, s, xq, sx,
-                                                             st, cnt, ntiles)
-            : launch_quant_rows<float, sq::MODE_X>(static_cast<const float *>(x), M, K, s, xq, sx, st, cnt, ntiles);
+                                                             st, cnt, ncnt)
+            : launch_quant_rows<float, sq::MODE_X>(static_cast<const float *>(x), M, K, s, xq, sx, st, cnt, ncnt);
     if (r != SQ_OK)
         return r;
-    return out_dt == SQ_BF16 ? launch_decode<OUT_BF16>(xq, sx, wq, sw, M, N, K, y, cnt, slots, in_dt, st)
-                             : launch_decode<OUT_F32>(xq, sx, wq, sw, M, N, K, y, cnt, slots, in_dt, st);
+    return out_dt == SQ_BF16 ? launch_gemm<OUT_BF16>(xq, sx, wq, sw, M, N, K, y, st, cnt, slots, in_dt)
+                             : launch_gemm<OUT_F32>(xq, sx, wq, sw, M, N, K, y, st, cnt, slots, in_dt);
+}
+
+size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 1 || N < 1 || K < 1)
+        return 0;
+    return gemm_ws_layout(M, N, K, 0).total;
+}
+
+sq_status sq_w8a8_gemm_ws(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw, int64_t M,
+                          int64_t N, int64_t K, void *y, sq_dtype out_dt, void *workspace, size_t ws_bytes,
+                          sq_stream_t stream)
+{
+    if (xq == nullptr || sx == nullptr || wq == nullptr || sw == nullptr || y == nullptr || workspace == nullptr ||
+        !valid_dtype(out_dt) || !aligned16(xq) || !aligned16(sx) || !aligned16(wq) || !aligned16(sw) ||
+        !aligned16(y) || !aligned16(workspace))
+        return SQ_ERR_INVALID_ARG;
+    sq_status r = check_gemm_dims(M, N, K);
+    if (r != SQ_OK)
+        return r;
+    const GemmWs G = gemm_ws_layout(M, N, K, 0);
+    if (ws_bytes < G.total)
+        return SQ_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    int *cnt = reinterpret_cast<int *>(wsb + G.cnt);
+    int32_t *slots = reinterpret_cast<int32_t *>(wsb + G.slots);
+    // clear the tile counters (a kernel of this library, so the GEMM after it
+    // may start on its weight before griddepcontrol.wait)
+    r = launch_kernel(sq::zero_f32_kernel, dim3(static_cast<unsigned>((G.ncnt + 255) / 256)), dim3(256), 0, st, 0, 0,
+                      reinterpret_cast<float *>(cnt), static_cast<int64_t>(G.ncnt));
+    if (r != SQ_OK)
+        return r;
+    return out_dt == SQ_BF16 ? launch_gemm<OUT_BF16>(xq, sx, wq, sw, M, N, K, y, st, cnt, slots)
+                             : launch_gemm<OUT_F32>(xq, sx, wq, sw, M, N, K, y, st, cnt, slots);
 }
 
 sq_status sq_linear_noalloc(const void *x, sq_dtype in_dt, const float *s, const int8_t *wq,
@@ -1284,7 +1374,10 @@ sq_status sq_linear_noalloc(const void *x, sq_dtype in_dt, const float *s, const
     sq_status r = check_gemm_dims(M, N, K);
     if (r != SQ_OK)
         return r;
-    const size_t need = sq_linear_workspace_size(M, N, K);
+    // the codes and scales must fit the scratch; the GEMM's own workspace is
+    // used when it fits too (else the GEMM runs without one)
+    const size_t full = sq_linear_workspace_size(M, N, K);
+    const size_t need = full == 0 ? 0 : linear_ws_layout(M, N, K).minimum;
     if (need > SQ_LINEAR_NOALLOC_SCRATCH_BYTES)
         return SQ_ERR_UNSUPPORTED;
     void *ws = nullptr;
@@ -1293,7 +1386,8 @@ sq_status sq_linear_noalloc(const void *x, sq_dtype in_dt, const float *s, const
         if (ws == nullptr)
             return SQ_ERR_CUDA;
     }
-    return sq_linear(x, in_dt, s, wq, sw, M, N, K, y, out_dt, ws, need, stream);
+    return sq_linear(x, in_dt, s, wq, sw, M, N, K, y, out_dt, ws, need == 0 ? 0 : SQ_LINEAR_NOALLOC_SCRATCH_BYTES,
+                     stream);
 }
 
 sq_status sq_selftest_wait_timeout(uint32_t limit_us, sq_stream_t stream)

@@ -30,6 +30,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "sq_decode.cuh"
 #include "sq_gemm.cuh"
 #include "sq_ptx.cuh"
 
@@ -52,11 +53,64 @@ struct PairCfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
+// The work of one pair: its data-parallel tiles t = pair, pair + pairs, ...
+// below sk_first, then its contiguous range of the stream-K units (one unit
+// = one 128-byte k block of one tile; the sk_units units of tiles sk_first,
+// sk_first + 1, ... are cut into `pairs` equal ranges, as in sq_decode.cuh).
+struct PairSeg {
+    int tile, kb0, kb1;
+    bool whole;
+};
+
+struct PairSched {
+    int pair, pairs, sk_first, KB;
+    int64_t U, u0, u1;  // stream-K units and this pair's range
+    int t;
+    int64_t u;
+    __device__ __forceinline__ PairSched(int pair_, int pairs_, int sk_first_, int KB_, int64_t U_)
+        : pair(pair_), pairs(pairs_), sk_first(sk_first_), KB(KB_), U(U_), u0(dec_start(pair_, U_, pairs_)),
+          u1(dec_start(pair_ + 1, U_, pairs_)), t(pair_), u(u0)
+    {
+    }
+    __device__ __forceinline__ bool next(PairSeg &s)
+    {
+        if (t < sk_first) {
+            s.tile = t;
+            s.kb0 = 0;
+            s.kb1 = KB;
+            s.whole = true;
+            t += pairs;
+            return true;
+        }
+        if (u < u1) {
+            const int64_t j = u / KB;
+            s.tile = sk_first + static_cast<int>(j);
+            s.kb0 = static_cast<int>(u - j * KB);
+            s.kb1 = static_cast<int>(min(static_cast<int64_t>(KB), s.kb0 + (u1 - u)));
+            s.whole = s.kb0 == 0 && s.kb1 == KB;
+            u += s.kb1 - s.kb0;
+            return true;
+        }
+        return false;
+    }
+    // first stream-K tile of this pair's range (its partial slot 0)
+    __device__ __forceinline__ int first_sk_tile() const { return sk_first + static_cast<int>(u0 / KB); }
+};
+
+// Partial-sum slot of CTA `cta` (blockIdx.x) of the pair kernel: ws holds
+// 2 slots per CTA of 128 rows x BN int32, column-chunk-major (32 columns of
+// 128 rows, the rows contiguous).
+__device__ __forceinline__ int32_t *pair_slot(int32_t *ws, int64_t cta, int slot, int BN)
+{
+    return ws + (cta * 2 + slot) * static_cast<int64_t>(BN) * 128;
+}
+
 template <int BN, int STAGES, int OUT>
 __global__ void __launch_bounds__(kPairThreads, 1)
     gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const float *__restrict__ sx, const float *__restrict__ sw, void *__restrict__ y,
-                        int M, int N, int K)
+                        int M, int N, int K, int sk_first, int64_t sk_units, int32_t *__restrict__ ws,
+                        int *__restrict__ cnt)
 {
     pdl_prologue();
     using Cfg = PairCfg<BN, STAGES>;
@@ -75,6 +129,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const uint32_t slot_off = (sBar - base) + 8u * Cfg::NUM_BARS;
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(gbase + slot_off);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + slot_off + 4);
+    volatile int *last_flag = reinterpret_cast<volatile int *>(gbase + slot_off + 8);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -111,8 +166,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     const int m_tiles = (M + kPairBM - 1) / kPairBM;
-    const int n_tiles = (N + BN - 1) / BN;
-    const int total = m_tiles * n_tiles;
     const int k_blocks = (K + kBK - 1) / kBK;
 
     uint32_t issued_mask = 0, issued_parity = 0;  // producer: last phase issued per stage
@@ -122,11 +175,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            for (int t = pair; t < total; t += pairs) {
-                const int m_blk = t % m_tiles, n_blk = t / m_tiles;
+            PairSched sch(pair, pairs, sk_first, k_blocks, sk_units);
+            PairSeg sg;
+            while (sch.next(sg)) {
+                const int m_blk = sg.tile % m_tiles, n_blk = sg.tile / m_tiles;
                 const int a_row = m_blk * kPairBM + static_cast<int>(rank) * 128;
                 const int b_row = n_blk * BN + static_cast<int>(rank) * (BN / 2);
-                for (int kb = 0; kb < k_blocks; ++kb) {
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                     if (!bounded_wait(empty_bar(stage), phase ^ 1u, kErrWaitProducer, abort_flag))
                         goto producer_done;
                     if (rank == 0)
@@ -157,13 +212,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
-            for (int t = pair; t < total; t += pairs) {
+            PairSched sch(pair, pairs, sk_first, k_blocks, sk_units);
+            PairSeg sg;
+            while (sch.next(sg)) {
                 if (!bounded_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, kErrWaitAccEmpty, abort_flag))
                     break;
                 tc_fence_after_sync();
                 const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
                 bool ok = true;
-                for (int kb = 0; kb < k_blocks; ++kb) {
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                     if (!bounded_wait(full_bar(stage), phase, kErrWaitMma, abort_flag)) {
                         ok = false;
                         break;
@@ -174,7 +231,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
                     for (int k = 0; k < kBK / 32; ++k)
                         mma_i8_pair(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k), idesc,
-                                    (kb | k) != 0 ? 1u : 0u);
+                                    (kb > sg.kb0 || k != 0) ? 1u : 0u);
                     mma_issued_any = true;
                     mma_commit_pair(empty_bar(stage), 0x3);
                     if (++stage == STAGES) {
@@ -194,11 +251,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // epilogue warps 2..5: warp w reads TMEM lanes 32 (w % 4) .. +31
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
+        const int et = threadIdx.x - 64;  // 0..127
         const uint32_t tempty_first = map_shared_rank(tempty_bar(0), 0);
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = pair; t < total; t += pairs) {
-            const int m_blk = t % m_tiles, n_blk = t / m_tiles;
+        PairSched sch(pair, pairs, sk_first, k_blocks, sk_units);
+        const int first_sk = sch.first_sk_tile();
+        PairSeg sg;
+        while (sch.next(sg)) {
+            const int m_blk = sg.tile % m_tiles, n_blk = sg.tile / m_tiles;
             const bool ok = bounded_wait(tfull_bar(acc), acc_phase, kErrWaitAccFull, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, ok))
                 break;
@@ -207,6 +268,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
             const float sxm = (m < M && OUT != OUT_S32) ? __ldg(sx + m) : 0.0f;
+            int32_t *mine = sg.whole ? nullptr : pair_slot(ws, blockIdx.x, sg.tile == first_sk ? 0 : 1, BN);
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 const int n0 = n_blk * BN + c * 32;
@@ -215,8 +277,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tbase + c * 32, r);
                 tmem_ld_wait();
-                if (m < M)
-                    store_row_chunk<OUT>(r, sxm, sw, n0, N, y, m);
+                if (sg.whole) {
+                    if (m < M)
+                        store_row_chunk<OUT>(r, sxm, sw, n0, N, y, m);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        mine[(c * 32 + j) * 128 + row] = static_cast<int32_t>(r[j]);
+                }
                 __syncwarp();
             }
             tc_fence_before_sync();
@@ -226,6 +294,46 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             acc ^= 1;
             if (acc == 0)
                 acc_phase ^= 1u;
+            if (sg.whole)
+                continue;
+            // this CTA's half of a tile shared by several pairs: count the
+            // partial in; the pair that completes the count adds every
+            // contributor's slot (same half) and stores the tile half
+            const int64_t ut = static_cast<int64_t>(sg.tile - sk_first) * k_blocks;
+            const int64_t pf = dec_owner(ut, sk_units, pairs), pl = dec_owner(ut + k_blocks - 1, sk_units, pairs);
+            __threadfence();
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            if (et == 0) {
+                const int old = atomicAdd(cnt + 2 * (sg.tile - sk_first) + static_cast<int>(rank), 1);
+                *last_flag = old == static_cast<int>(pl - pf);
+            }
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            if (*last_flag) {
+                __threadfence();
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    const int n0 = n_blk * BN + c * 32;
+                    if (n0 >= N)
+                        break;
+                    uint32_t r[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        r[j] = 0u;
+                    for (int64_t p2 = pf; p2 <= pl; ++p2) {
+                        const int s2 = (sk_first + static_cast<int>(dec_start(p2, sk_units, pairs) / k_blocks) ==
+                                        sg.tile)
+                                           ? 0
+                                           : 1;
+                        const int32_t *src = pair_slot(ws, 2 * p2 + rank, s2, BN) + (c * 32) * 128 + row;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            r[j] += static_cast<uint32_t>(__ldcg(src + j * 128));
+                    }
+                    if (m < M)
+                        store_row_chunk<OUT>(r, sxm, sw, n0, N, y, m);
+                }
+            }
+            asm volatile("bar.sync 2, 128;" ::: "memory");  // last_flag is rewritten by the next partial tile
         }
     }
 
