@@ -1,10 +1,13 @@
 """Parity of the GEMM with a workspace (sq_w8a8_gemm_ws, and sq_linear with
-a full workspace), which splits the work over every SM whatever the shape:
+a full workspace):
 
-* more than 128 tokens: the output tiles that do not fill whole rounds of
-  the CTA pairs are split along K over all pairs (stream-K), and a tile
-  shared by several pairs is summed through int32 partials;
-* up to 128 tokens: the weight-streaming kernel of sq_linear.
+* up to 128 tokens: the weight-streaming kernel, which splits the weight
+  over every SM and sums tiles shared by several CTAs through int32
+  partials;
+* more tokens: the pair kernel; with SQ_GEMM_SK=1 (off by default, tested in
+  a child process) the output tiles that do not fill whole rounds of the
+  CTA pairs are split along K over all pairs (stream-K), and a tile shared
+  by several pairs is summed through int32 partials.
 
 Integer partial sums are exact in any order, so the outputs must equal
 sq_w8a8_gemm's (data-parallel tiles) bit for bit, and the oracle's
@@ -118,3 +121,40 @@ def test_linear_full_workspace_against_oracle(oracle, M, N, K):
     cols = oracle.dequant(oracle.gemm_i32(xq_o, wq[ns]), sx_o, sw[ns], "bf16")
     assert_output_close(y_h[ms], rows, "rows")
     assert_output_close(y_h[:, ns], cols, "columns")
+
+
+CHILD_SK = r'''
+import torch
+import w8a8_int8_gemm_channel_b200 as sq
+from w8a8_int8_gemm_channel_b200 import workloads as wls
+for (M, N, K) in [(300, 528, 1040), (1024, 6144, 4096), (1000, 6160, 2064), (4096, 4096, 4096), (129, 16, 16)]:
+    xq = wls.random_int8((M, K), M).cuda()
+    wq = wls.random_int8((N, K), N).cuda()
+    sx = torch.rand(M).cuda() * 0.05 + 1e-3
+    sw = torch.rand(N).cuda() * 1e-3 + 1e-5
+    y0 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    y1 = torch.empty_like(y0)
+    sq.sq_w8a8_gemm(xq, sx, wq, sw, y0)
+    ws = torch.full((sq.sq_w8a8_gemm_workspace_size(M, N, K),), 0xFF, dtype=torch.uint8, device="cuda")
+    sq.sq_w8a8_gemm_ws(xq, sx, wq, sw, y1, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16)), (M, N, K)
+st, code = sq.sq_device_status()
+assert st == sq.SQ_OK, hex(code)
+print("stream-k-ok")
+'''
+
+
+def test_stream_k_tail_child_process():
+    """The stream-K tail of the pair GEMM (off by default, SQ_GEMM_SK=1 turns
+    it on; read once per process, so in a child): equal to the data-parallel
+    GEMM bit for bit."""
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SQ_GEMM_SK="1", PYTHONPATH=root)
+    r = subprocess.run([sys.executable, "-c", CHILD_SK], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0 and "stream-k-ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]

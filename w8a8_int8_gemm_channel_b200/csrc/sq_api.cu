@@ -771,6 +771,17 @@ sq_status launch_decode(const int8_t *xq, const float *sx, const int8_t *wq, con
     }
 }
 
+// The stream-K tail of the pair GEMM is off unless SQ_GEMM_SK=1: measured on
+// B200 it is slower than whole tiles (1024 x 6144 x 4096: 52 against 35 us;
+// 4096 x 6144 x 4096: 93 against 74 us), because the partial sums' reduction
+// (a 128 x 256 int32 slot per contributor, read back by the last one) sits at
+// the end of the critical path.
+bool gemm_sk_enabled()
+{
+    static const bool on = std::getenv("SQ_GEMM_SK") && std::atoi(std::getenv("SQ_GEMM_SK")) == 1;
+    return on;
+}
+
 // Prefill GEMM on CTA pairs: 256 x BN output tiles, persistent over tiles.
 // With a workspace (slots, cnt not null) and tiles that do not fill whole
 // rounds of the co-resident pairs, the last round and the partial one are
@@ -797,8 +808,7 @@ sq_status launch_gemm_pair_cfg(const int8_t *xq, const float *sx, const int8_t *
     const int64_t kb = (K + sq::kBK - 1) / sq::kBK;
     int64_t pairs = std::min<int64_t>(tiles, active);
     int64_t sk_first = tiles, sk_units = 0;
-    static const bool sk_off = std::getenv("SQ_GEMM_SK") && std::atoi(std::getenv("SQ_GEMM_SK")) == 0;
-    if (slots != nullptr && cnt != nullptr && !sk_off && tiles % active != 0) {
+    if (slots != nullptr && cnt != nullptr && gemm_sk_enabled() && tiles % active != 0) {
         // the last full round and the partial one; with fewer tiles than
         // pairs, all of them (and no more pairs than units, so that every
         // pair has some)
@@ -873,10 +883,8 @@ sq_status launch_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const
     DeviceInfo di;
     if (!device_info(di))
         return SQ_ERR_CUDA;
-    // with a workspace the tail rounds are split stream-K, so the widest
-    // (most efficient) tile is used throughout
-    static const bool sk_off = std::getenv("SQ_GEMM_SK") && std::atoi(std::getenv("SQ_GEMM_SK")) == 0;
-    const int bn = (ws && !sk_off && !std::getenv("SQ_GEMM_PAIR_BN")) ? 256 : pick_pair_bn(M, N, di.sms / 2);
+    // with the stream-K tail, the widest (most efficient) tile throughout
+    const int bn = (ws && gemm_sk_enabled() && !std::getenv("SQ_GEMM_PAIR_BN")) ? 256 : pick_pair_bn(M, N, di.sms / 2);
     switch (bn) {
     case 256:
         return launch_gemm_pair_cfg<256, 6, OUT>(xq, sx, wq, sw, M, N, K, y, st, slots, cnt);

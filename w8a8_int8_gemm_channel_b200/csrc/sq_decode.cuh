@@ -85,7 +85,8 @@ __host__ __device__ constexpr int dec_smem_bytes(int stage_bytes, int stages)
 __device__ __forceinline__ void dec_bar_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 // Slot of the partial that CTA c writes for tile t (0: the range's first
-// tile, 1: its last); ws holds G x 2 slots of BNX x 128 int32.
+// tile, 1: its last); ws holds G x 2 slots of 128 rows x BNX int32, each
+// row's tokens contiguous.
 __device__ __forceinline__ int32_t *dec_slot(int32_t *ws, int64_t c, int slot, int BNX)
 {
     return ws + (c * 2 + slot) * static_cast<int64_t>(BNX) * kBM;
@@ -284,9 +285,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     if (n < N)
                         store_col_chunk<OUT>(r, swn, sx, cc * 32, M, y, n, N);
                 } else {
+                    // this row's partial, the valid tokens only, 16 bytes at a time
+                    int4 *dst = reinterpret_cast<int4 *>(mine + row * BNX + cc * 32);
+                    const int nv = (min(M - cc * 32, 32) + 3) >> 2;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        mine[(cc * 32 + j) * kBM + row] = static_cast<int32_t>(r[j]);
+                    for (int v = 0; v < 8; ++v)
+                        if (v < nv)
+                            dst[v] = make_int4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
                 }
             }
             // the accumulator set is free for the next tile of the range
@@ -299,34 +304,50 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 acc_phase ^= 1u;
             if (whole)
                 continue;
-            // count this partial in; the contributor that completes the
-            // count adds every contributor's slot and stores the tile
-            __threadfence();
+            // count this partial in (one release by one thread after the
+            // barrier of the epilogue warps); the contributor that completes
+            // the count adds every contributor's slot and stores the tile
             dec_bar_sync();
+            const int64_t cf = dec_owner(t * KB, U, G), cl = dec_owner((t + 1) * KB - 1, U, G);
             if (et == 0) {
-                const int64_t cf = dec_owner(t * KB, U, G), cl = dec_owner((t + 1) * KB - 1, U, G);
-                const int contributors = static_cast<int>(cl - cf + 1);
+                __threadfence();
                 const int old = atomicAdd(cnt + t, 1);
-                *last_flag = old == contributors - 1;
+                *last_flag = old == static_cast<int>(cl - cf);
+                __threadfence();
             }
             dec_bar_sync();
             if (*last_flag) {
-                __threadfence();
-                const int64_t cf = dec_owner(t * KB, U, G), cl = dec_owner((t + 1) * KB - 1, U, G);
 #pragma unroll 1
                 for (int cc = 0; cc < BNX / 32; ++cc) {
                     if (cc * 32 >= M)
                         break;
+                    const int nv = (min(M - cc * 32, 32) + 3) >> 2;
                     uint32_t r[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         r[j] = 0u;
-                    for (int64_t c2 = cf; c2 <= cl; ++c2) {
-                        const int s2 = (dec_start(c2, U, G) / KB == t) ? 0 : 1;
-                        const int32_t *p = dec_slot(ws, c2, s2, BNX) + (cc * 32) * kBM + row;
+                    // two contributors' loads in flight at a time
+                    for (int64_t c2 = cf; c2 <= cl; c2 += 2) {
+                        int4 a[8], b[8];
+                        const bool two = c2 + 1 <= cl;
+                        const int4 *pa = reinterpret_cast<const int4 *>(
+                            dec_slot(ws, c2, dec_start(c2, U, G) / KB == t ? 0 : 1, BNX) + row * BNX + cc * 32);
+                        const int4 *pb = two ? reinterpret_cast<const int4 *>(
+                                                   dec_slot(ws, c2 + 1, dec_start(c2 + 1, U, G) / KB == t ? 0 : 1,
+                                                            BNX) + row * BNX + cc * 32)
+                                             : pa;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            r[j] += static_cast<uint32_t>(__ldcg(p + j * kBM));
+                        for (int v = 0; v < 8; ++v) {
+                            a[v] = v < nv ? __ldcg(pa + v) : make_int4(0, 0, 0, 0);
+                            b[v] = (two && v < nv) ? __ldcg(pb + v) : make_int4(0, 0, 0, 0);
+                        }
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            r[4 * v] += static_cast<uint32_t>(a[v].x) + static_cast<uint32_t>(b[v].x);
+                            r[4 * v + 1] += static_cast<uint32_t>(a[v].y) + static_cast<uint32_t>(b[v].y);
+                            r[4 * v + 2] += static_cast<uint32_t>(a[v].z) + static_cast<uint32_t>(b[v].z);
+                            r[4 * v + 3] += static_cast<uint32_t>(a[v].w) + static_cast<uint32_t>(b[v].w);
+                        }
                     }
                     if (n < N)
                         store_col_chunk<OUT>(r, swn, sx, cc * 32, M, y, n, N);

@@ -61,6 +61,68 @@ __host__ __device__ constexpr int64_t staged_smem_bytes(int64_t K, bool bf, int 
            static_cast<int64_t>(groups) * nslots * 8;
 }
 
+// Rare paths, element by element.  A chunk is flagged as a whole by the
+// cheap passes, but usually only one of its 8 elements needs the exact
+// quotient; the chunk is re-read from the row buffer in shared memory.
+//   candidates: the exact |v| of the elements whose own bound reaches thr
+//   (all of them when exact_all), maximum over those.  The element that
+//   attains the row maximum has a bound >= thr, as the chunk test assumes.
+template <int MODE, bool BF>
+__device__ __noinline__ float staged_candidates(uint32_t saddr, const uint32_t *fb, const float *f,
+                                                const float *__restrict__ sc, float thr, bool exact_all)
+{
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(saddr));
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+    float m = 0.0f;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        float b[2];
+        if constexpr (BF) {
+            const uint32_t p = bf2_mul(w[h] & 0x7FFF7FFFu, fb[h]);
+            b[0] = __uint_as_float(p << 16);
+            b[1] = __uint_as_float(p & 0xFFFF0000u);
+        } else {
+            b[0] = fabsf(__fmul_rn(__uint_as_float(w[h] << 16), f[2 * h]));
+            b[1] = fabsf(__fmul_rn(__uint_as_float(w[h] & 0xFFFF0000u), f[2 * h + 1]));
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            if (exact_all || b[k] >= thr) {
+                const float x = __uint_as_float(k == 0 ? (w[h] << 16) : (w[h] & 0xFFFF0000u));
+                const float sv = __ldg(sc + 2 * h + k);
+                m = fmaxf(m, fabsf(MODE == MODE_X ? __fdiv_rn(x, sv) : __fmul_rn(x, sv)));
+            }
+        }
+    }
+    return m;
+}
+
+//   ties: the elements whose fast code lies within 2^-13 of a rounding tie
+//   (every element when !fast) get the exact code, one byte store each; the
+//   fast path has already stored the chunk's other codes.
+template <int MODE>
+__device__ __noinline__ void staged_ties(uint32_t saddr, const float *f, const float *__restrict__ sc, float scale,
+                                         float rsc, bool fast, int8_t *dst)
+{
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(saddr));
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const float x = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+        const float a = __fmul_rn(x, f[e]);
+        const float yy = __fmaf_rn(a, rsc, kRoundMagic);
+        const float dd = __fmaf_rn(a, -rsc, __fadd_rn(yy, -kRoundMagic));
+        if (!fast || !(fabsf(dd) < kTieLimit)) {
+            const float sv = __ldg(sc + e);
+            const float v = MODE == MODE_X ? __fdiv_rn(x, sv) : __fmul_rn(x, sv);
+            const uint32_t cb = scale != 0.0f ? exact_code_bits(v, scale) : code_bits(0.0f);
+            dst[e] = static_cast<int8_t>(cb & 0xFFu);
+        }
+    }
+}
+
 template <int MODE, int CH, bool BF>
 __global__ void __launch_bounds__(kQuantThreads, CH >= 14 ? 1 : 2)
     row_quant_staged_kernel(const __nv_bfloat16 *__restrict__ in, int64_t rows, int64_t K,
@@ -199,16 +261,12 @@ __global__ void __launch_bounds__(kQuantThreads, CH >= 14 ? 1 : 2)
             for (int i = 0; i < CH; ++i)
                 cand |= (exact_all || hm[i] >= thr) ? (1u << i) : 0u;
             float em = 0.0f;
-            while (cand != 0u) {  // rare: those chunks exactly, from the registers
+            while (cand != 0u) {  // rare: the candidate elements exactly
                 const int i = __ffs(cand) - 1;
                 cand &= cand - 1u;
-                uint4 v = raw[0];
-#pragma unroll
-                for (int k = 1; k < CH; ++k)
-                    if (k == i)
-                        v = raw[k];
                 const int64_t c = c0 + cstep * i;
-                em = fmaxf(em, chunk_exact_absmax<__nv_bfloat16, MODE>(v, s + c * V));
+                em = fmaxf(em, staged_candidates<MODE, BF>(sbase + static_cast<uint32_t>(c) * 16u, fb_sm + c * 4,
+                                                           f_sm + c * V, s + c * V, thr, exact_all));
             }
             E = group_max(em);
         }
@@ -247,16 +305,12 @@ __global__ void __launch_bounds__(kQuantThreads, CH >= 14 ? 1 : 2)
             ties |= (!fast || !(dmax < kTieLimit)) ? (1u << i) : 0u;
             store_code_words(dst + static_cast<int64_t>(c) * V, y, V);
         }
-        while (ties != 0u) {  // rare: near ties; every chunk when the scale is outside the fast range
+        while (ties != 0u) {  // rare: near ties; every element when the scale is outside the fast range
             const int i = __ffs(ties) - 1;
             ties &= ties - 1u;
-            uint4 v = raw[0];
-#pragma unroll
-            for (int k = 1; k < CH; ++k)
-                if (k == i)
-                    v = raw[k];
             const int64_t c = c0 + cstep * i;
-            chunk_store_exact_codes<__nv_bfloat16, MODE>(v, s + c * V, scale, dst + c * V);
+            staged_ties<MODE>(sbase + static_cast<uint32_t>(c) * 16u, f_sm + c * V, s + c * V, scale, rsc, fast,
+                              dst + c * V);
         }
         // every warp of the group is done with the slot: refill it
         group_sync();
