@@ -715,6 +715,35 @@ inline int64_t quant_smem_estimate(int64_t K, sq_dtype dt)
     return sq::row_quant_smem(K, bb) + 1024;
 }
 
+// CTAs of the weight-streaming GEMM.  The units are cut into G equal
+// ranges; with G = S * T (T tiles, S <= KB) every range lies inside one tile,
+// so a CTA has one partial tile to sum through the workspace instead of up
+// to two.  A partial tile's epilogue (stores, a release, a count, perhaps the
+// reduction) is a chain of global-memory round trips worth about
+// kDecodeEpiUnits units of streaming, so G is the choice with the fewest
+// units per CTA plus that cost per partial tile.
+constexpr int64_t kDecodeEpiUnits = 6;
+
+inline int64_t decode_ctas(int64_t N, int64_t K, int64_t sms)
+{
+    const int64_t T = (N + sq::kBM - 1) / sq::kBM, KB = (K + sq::kBK - 1) / sq::kBK, U = T * KB;
+    static const int64_t force = std::getenv("SQ_DECODE_CTAS") ? std::atoll(std::getenv("SQ_DECODE_CTAS")) : 0;
+    if (force > 0)
+        return std::min(force, std::min(U, sms));
+    int64_t best = std::min(U, sms);
+    // the stream cut: ranges may span two tiles, so up to two partial tiles a CTA
+    int64_t best_cost = (U + best - 1) / best + (best < U ? 2 : 0) * kDecodeEpiUnits;
+    for (int64_t S = 1; S <= KB && S * T <= sms; ++S) {
+        const int64_t G = S * T;
+        const int64_t cost = (KB + S - 1) / S + (S > 1 ? kDecodeEpiUnits : 0);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = G;
+        }
+    }
+    return best;
+}
+
 template <int BNX, int OUT>
 sq_status launch_decode_cfg(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw, int64_t M,
                             int64_t N, int64_t K, void *y, int *cnt, int32_t *slots, sq_dtype in_dt,
@@ -725,7 +754,7 @@ sq_status launch_decode_cfg(const int8_t *xq, const float *sx, const int8_t *wq,
     if (!device_info(di))
         return SQ_ERR_CUDA;
     const int64_t U = decode_units(N, K);
-    const int G = static_cast<int>(std::min<int64_t>({U, (int64_t)di.sms, kDecodeMaxCtas}));
+    const int G = static_cast<int>(decode_ctas(N, K, std::min<int64_t>(di.sms, kDecodeMaxCtas)));
     // the deepest ring that still leaves room for a quantiser CTA on the SM
     // (the two kernels overlap), within the per-CTA limit
     static const int force_stages = std::getenv("SQ_DECODE_STAGES") ? std::atoi(std::getenv("SQ_DECODE_STAGES")) : 0;
