@@ -337,40 +337,42 @@ sq_status launch_glu_quant(const T *gu, int64_t rows, int64_t K, const float *s,
 
 // The staged quantiser (bf16 rows brought into shared memory by bulk
 // copies): rows of exactly 32 * CH * G chunks, CH in {7, 8, 14} and G in
-// {1, 2, 4, 8}.  Returns false (nothing launched) for other rows.
-template <int MODE, int CH, bool BF>
+// {1, 2, 4, 8} (16 with 512-thread CTAs).  Returns false (nothing launched)
+// for other rows.
+template <int MODE, int CH, int THREADS = sq::kQuantThreads>
 sq_status launch_staged_cfg(const __nv_bfloat16 *in, int64_t rows, int64_t K, const float *s, int8_t *q,
                             float *scale, int log2g, cudaStream_t st, const DeviceInfo &di, int *zero, int nzero)
 {
-    auto kernel = sq::row_quant_staged_kernel<MODE, CH, BF>;
+    auto kernel = sq::row_quant_staged_kernel<MODE, CH, THREADS>;
     static std::atomic<uint64_t> attr_done{0};
     if (!ensure_smem_attr(kernel, kMaxDynSmem - 1024, attr_done))
         return SQ_ERR_CUDA;
-    const int groups = 8 >> log2g;
-    // two CTAs an SM with two row buffers a group where that fits, else one
-    // CTA with as many buffers (up to 4) as fit
+    const int groups = (THREADS / 32) >> log2g;
+    // two CTAs an SM with two row buffers a group where that fits (256
+    // threads), else one CTA with as many buffers (up to 4) as fit
     int nslots = 0, per_sm = 0;
-    const int64_t per_cta2 = kSmSmemBytes / 2 - 1024 - 256;
-    if (sq::staged_smem_bytes(K, BF, groups, 2) <= per_cta2) {
+    // (an SM's shared memory, less 1 KB reserved a CTA and 512 bytes of static arrays)
+    const int64_t per_cta2 = kSmSmemBytes / 2 - 1024 - 512;
+    if (THREADS == sq::kQuantThreads && sq::staged_smem_bytes(K, groups, 2) <= per_cta2) {
         nslots = 2;
         per_sm = 2;
-        if (sq::staged_smem_bytes(K, BF, groups, 3) <= per_cta2)
+        if (sq::staged_smem_bytes(K, groups, 3) <= per_cta2)
             nslots = 3;
     } else {
-        for (int n = 4; n >= 2 && nslots == 0; --n)
-            if (sq::staged_smem_bytes(K, BF, groups, n) <= kMaxDynSmem - 1024)
+        for (int n = sq::kStagedMaxSlots; n >= 2 && nslots == 0; --n)
+            if (sq::staged_smem_bytes(K, groups, n) <= kMaxDynSmem - 1024)
                 nslots = n;
         per_sm = 1;
     }
     if (nslots == 0)
         return SQ_ERR_UNSUPPORTED;
-    const int smem = static_cast<int>(sq::staged_smem_bytes(K, BF, groups, nslots));
+    const int smem = static_cast<int>(sq::staged_smem_bytes(K, groups, nslots));
     const int64_t blocks = std::min<int64_t>((rows + groups - 1) / groups, (int64_t)per_sm * di.sms);
     if (debug_plan())
-        std::fprintf(stderr, "sq staged quant rows=%lld K=%lld: CH=%d G=%d BF=%d slots=%d per_sm=%d blocks=%lld smem=%d\n",
-                     (long long)rows, (long long)K, CH, 1 << log2g, (int)BF, nslots, per_sm, (long long)blocks, smem);
-    return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(sq::kQuantThreads), smem, st, 0, 0, in, rows,
-                         K, s, log2g, nslots, q, scale, zero, nzero);
+        std::fprintf(stderr, "sq staged quant rows=%lld K=%lld: CH=%d G=%d threads=%d slots=%d per_sm=%d blocks=%lld smem=%d\n",
+                     (long long)rows, (long long)K, CH, 1 << log2g, THREADS, nslots, per_sm, (long long)blocks, smem);
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(THREADS), smem, st, 0, 0, in, rows, K, s,
+                         log2g, nslots, q, scale, zero, nzero);
 }
 
 template <int MODE>
@@ -385,19 +387,25 @@ bool launch_staged(const __nv_bfloat16 *in, int64_t rows, int64_t K, const float
     if (mode == 0 || (mode == 1 && rows < 256))
         return false;
     const int64_t nch = K / 8;
-    const bool bb = sq::row_quant_smem(K, true) <= 64 * 1024;
+    // rows of 3584 chunks (K = 28672): the factor table and two rows fill an
+    // SM's shared memory, so one CTA of 16 warps (7 chunks a lane) rather
+    // than 8 warps of 14; SQ_QUANT_STAGED512=0 takes the 8-warp form
+    static const bool w512 =
+        !(std::getenv("SQ_QUANT_STAGED512") && std::atoi(std::getenv("SQ_QUANT_STAGED512")) == 0);
+    if (w512 && nch == 32 * 7 * 16) {
+        r = launch_staged_cfg<MODE, 7, 512>(in, rows, K, s, q, scale, 4, st, di, zero, nzero);
+        return r != SQ_ERR_UNSUPPORTED;
+    }
     for (int ch : {8, 7, 14}) {
         for (int log2g = 0; log2g <= 3; ++log2g) {
             if ((int64_t)32 * ch << log2g != nch)
                 continue;
             if (ch == 8)
-                r = bb ? launch_staged_cfg<MODE, 8, true>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero)
-                       : launch_staged_cfg<MODE, 8, false>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero);
+                r = launch_staged_cfg<MODE, 8>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero);
             else if (ch == 7)
-                r = bb ? launch_staged_cfg<MODE, 7, true>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero)
-                       : launch_staged_cfg<MODE, 7, false>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero);
+                r = launch_staged_cfg<MODE, 7>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero);
             else
-                r = launch_staged_cfg<MODE, 14, false>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero);
+                r = launch_staged_cfg<MODE, 14>(in, rows, K, s, q, scale, log2g, st, di, zero, nzero);
             return r != SQ_ERR_UNSUPPORTED;
         }
     }

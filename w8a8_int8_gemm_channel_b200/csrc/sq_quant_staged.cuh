@@ -12,19 +12,28 @@
 // (one scale per output channel); the smoothing division and multiplication
 // of "Where the outlier actually comes from".
 //
-// The arithmetic is that of sq_div.cuh and of row_quant_kernel: a packed
-// bf16 bound of |v| per chunk, exact quotients for the chunks within 2^-5 of
-// the row's largest bound (bf16 bound) or 2^-20 (fp32 bound), the scale by
-// Markstein's iteration, and the codes from the rounding fast path with the
-// exact IEEE path near ties.  What differs is how the rows move:
-//   * a CTA of 8 warps holds 8 / G groups of G warps; each group owns
-//     `nslots` row buffers in shared memory, and its leader thread keeps them
-//     filled with the group's next rows by 1-D bulk copies (cp.async.bulk,
-//     completion on an mbarrier), so nslots rows per group are in flight
-//     however long the arithmetic of the current one takes;
+// The arithmetic is that of sq_div.cuh and of row_quant_kernel: an fp32
+// bound a_k = RN(x_k * f_k) of |v| per element (f_k the hardware reciprocal
+// of s_k for activations, s_k itself for weights), exact quotients for the
+// elements within 2^-20 of the largest bound, the scale by Markstein's
+// iteration, and the codes from the rounding fast path with the exact IEEE
+// path near ties.  What differs is how the rows move and where a_k lives:
+//   * s is brought into shared memory whole by one bulk copy (cp.async.bulk),
+//     issued before any row, so every exact step reads s_k there;
+//   * a CTA of THREADS / 32 warps holds groups of G warps; each group owns
+//     `nslots` row buffers in shared memory, filled with the group's next rows
+//     by bulk copies (completion on an mbarrier), so nslots rows per group
+//     are in flight however long the arithmetic of the current one takes;
+//     the last warp of the group to finish with a buffer refills it, so no
+//     warp waits for another at the end of a row;
 //   * lane L of warp g of a group takes the 16-byte chunks c = 32 g + L +
-//     32 G i, i < CH, of the row: one shared-memory load each, kept in
-//     registers for every pass.
+//     32 G i, i < CH, of the row: one shared-memory load each; the products
+//     a_k of the first pass stay in registers for the second, which then
+//     only rounds them;
+//   * E = max_k |v_k|: each warp takes the exact |v| of its own elements
+//     within 2^-20 of its own largest bound (a superset of those within
+//     2^-20 of the row's largest, and every element it adds is a real |v_k|,
+//     so the maximum is unchanged), then one exchange across the group.
 #pragma once
 
 #include <cstdint>
@@ -46,54 +55,56 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
                  : "memory");
 }
 
-// shared memory of the staged quantiser: factor tables, then the row slots
-// (128-byte aligned), then one mbarrier per slot
-__host__ __device__ constexpr int64_t staged_tables_bytes(int64_t K, bool bf) { return K * 4 + (bf ? K * 2 : 0); }
+// Row buffers a group holds at most.
+constexpr int kStagedMaxSlots = 4;
 
-__host__ __device__ constexpr int64_t staged_slots_offset(int64_t K, bool bf)
+// shared memory of the staged quantiser: s (K fp32), then the row slots
+// (128-byte aligned), then one mbarrier per slot and one for s
+__host__ __device__ constexpr int64_t staged_slots_offset(int64_t K) { return (K * 4 + 127) / 128 * 128; }
+
+__host__ __device__ constexpr int64_t staged_smem_bytes(int64_t K, int groups, int nslots)
 {
-    return (staged_tables_bytes(K, bf) + 127) / 128 * 128;
+    return staged_slots_offset(K) + static_cast<int64_t>(groups) * nslots * K * 2 +
+           (static_cast<int64_t>(groups) * nslots + 1) * 8;
 }
 
-__host__ __device__ constexpr int64_t staged_smem_bytes(int64_t K, bool bf, int groups, int nslots)
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr)
 {
-    return staged_slots_offset(K, bf) + static_cast<int64_t>(groups) * nslots * K * 2 +
-           static_cast<int64_t>(groups) * nslots * 8;
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
+    return r;
+}
+
+// s_k and f_k of a chunk's eight elements, s from shared memory
+template <int MODE>
+__device__ __forceinline__ void chunk_factors(uint32_t s_addr, float (&sv)[8], float (&f)[8])
+{
+    const uint4 s0 = lds_u4(s_addr), s1 = lds_u4(s_addr + 16u);
+    const uint32_t w[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        sv[e] = __uint_as_float(w[e]);
+        f[e] = MODE == MODE_X ? rcp_approx(sv[e]) : sv[e];
+    }
 }
 
 // Rare paths, element by element.  A chunk is flagged as a whole by the
-// cheap passes, but usually only one of its 8 elements needs the exact
-// quotient; the chunk is re-read from the row buffer in shared memory.
-//   candidates: the exact |v| of the elements whose own bound reaches thr
-//   (all of them when exact_all), maximum over those.  The element that
-//   attains the row maximum has a bound >= thr, as the chunk test assumes.
-template <int MODE, bool BF>
-__device__ __noinline__ float staged_candidates(uint32_t saddr, const uint32_t *fb, const float *f,
-                                                const float *__restrict__ sc, float thr, bool exact_all)
+// register passes, but usually only one of its 8 elements needs the exact
+// quotient; the chunk is re-read from its row buffer.
+//   candidates: the exact |v| of the elements whose bound reaches thr (all of
+//   them when exact_all), maximum over those.
+template <int MODE>
+__device__ __noinline__ float staged_candidates(uint32_t raw_addr, uint32_t s_addr, float thr, bool exact_all)
 {
-    uint4 r;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(saddr));
-    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+    const uint4 r = lds_u4(raw_addr);
+    float sv[8], f[8], x[8];
+    chunk_factors<MODE>(s_addr, sv, f);
+    widen<__nv_bfloat16>(r, x);
     float m = 0.0f;
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        float b[2];
-        if constexpr (BF) {
-            const uint32_t p = bf2_mul(w[h] & 0x7FFF7FFFu, fb[h]);
-            b[0] = __uint_as_float(p << 16);
-            b[1] = __uint_as_float(p & 0xFFFF0000u);
-        } else {
-            b[0] = fabsf(__fmul_rn(__uint_as_float(w[h] << 16), f[2 * h]));
-            b[1] = fabsf(__fmul_rn(__uint_as_float(w[h] & 0xFFFF0000u), f[2 * h + 1]));
-        }
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            if (exact_all || b[k] >= thr) {
-                const float x = __uint_as_float(k == 0 ? (w[h] << 16) : (w[h] & 0xFFFF0000u));
-                const float sv = __ldg(sc + 2 * h + k);
-                m = fmaxf(m, fabsf(MODE == MODE_X ? __fdiv_rn(x, sv) : __fmul_rn(x, sv)));
-            }
-        }
+    for (int e = 0; e < 8; ++e) {
+        if (exact_all || fabsf(__fmul_rn(x[e], f[e])) >= thr)
+            m = fmaxf(m, fabsf(MODE == MODE_X ? __fdiv_rn(x[e], sv[e]) : __fmul_rn(x[e], sv[e])));
     }
     return m;
 }
@@ -102,29 +113,29 @@ __device__ __noinline__ float staged_candidates(uint32_t saddr, const uint32_t *
 //   (every element when !fast) get the exact code, one byte store each; the
 //   fast path has already stored the chunk's other codes.
 template <int MODE>
-__device__ __noinline__ void staged_ties(uint32_t saddr, const float *f, const float *__restrict__ sc, float scale,
-                                         float rsc, bool fast, int8_t *dst)
+__device__ __noinline__ void staged_ties(uint32_t raw_addr, uint32_t s_addr, float scale, float rsc, bool fast,
+                                         int8_t *dst)
 {
-    uint4 r;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(saddr));
-    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+    const uint4 r = lds_u4(raw_addr);
+    float sv[8], f[8], x[8];
+    chunk_factors<MODE>(s_addr, sv, f);
+    widen<__nv_bfloat16>(r, x);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-        const float x = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
-        const float a = __fmul_rn(x, f[e]);
+        const float a = __fmul_rn(x[e], f[e]);
         const float yy = __fmaf_rn(a, rsc, kRoundMagic);
         const float dd = __fmaf_rn(a, -rsc, __fadd_rn(yy, -kRoundMagic));
         if (!fast || !(fabsf(dd) < kTieLimit)) {
-            const float sv = __ldg(sc + e);
-            const float v = MODE == MODE_X ? __fdiv_rn(x, sv) : __fmul_rn(x, sv);
+            const float v = MODE == MODE_X ? __fdiv_rn(x[e], sv[e]) : __fmul_rn(x[e], sv[e]);
             const uint32_t cb = scale != 0.0f ? exact_code_bits(v, scale) : code_bits(0.0f);
             dst[e] = static_cast<int8_t>(cb & 0xFFu);
         }
     }
 }
 
-template <int MODE, int CH, bool BF>
-__global__ void __launch_bounds__(kQuantThreads, CH >= 14 ? 1 : 2)
+// THREADS = 256 (8 warps), or 512 (16 warps) where an SM holds one CTA.
+template <int MODE, int CH, int THREADS = kQuantThreads>
+__global__ void __launch_bounds__(THREADS, (CH >= 14 || THREADS > kQuantThreads) ? 1 : 2)
     row_quant_staged_kernel(const __nv_bfloat16 *__restrict__ in, int64_t rows, int64_t K,
                             const float *__restrict__ s, int log2g, int nslots, int8_t *__restrict__ q,
                             float *__restrict__ scale_out, int *__restrict__ zero, int nzero)
@@ -132,11 +143,12 @@ __global__ void __launch_bounds__(kQuantThreads, CH >= 14 ? 1 : 2)
     pdl_prologue();
     clear_ints(zero, nzero);
     constexpr int V = 8;
-    constexpr int WARPS = kQuantThreads / 32;
+    constexpr int WARPS = THREADS / 32;
     extern __shared__ __align__(128) uint8_t qs_smem[];
-    float *f_sm = reinterpret_cast<float *>(qs_smem);
-    uint32_t *fb_sm = reinterpret_cast<uint32_t *>(f_sm + K);
     __shared__ float red[2][WARPS];
+    __shared__ int okv[2][WARPS];
+    __shared__ int done_cnt[WARPS][kStagedMaxSlots];  // warps of a group done with a buffer
+    __shared__ uint32_t inflight[WARPS];               // buffers of a group with a copy in flight
     __shared__ int abort_sm;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -147,8 +159,11 @@ __global__ void __launch_bounds__(kQuantThreads, CH >= 14 ? 1 : 2)
     const int c0 = 32 * g + lane;
     const int cstep = 32 * G;
     const uint32_t row_bytes = static_cast<uint32_t>(K * 2);
-    const uint32_t slots = smem_u32(qs_smem) + static_cast<uint32_t>(staged_slots_offset(K, BF));
+    const uint32_t stab = smem_u32(qs_smem);
+    const float *s_sm = reinterpret_cast<const float *>(qs_smem);
+    const uint32_t slots = stab + static_cast<uint32_t>(staged_slots_offset(K));
     const uint32_t bars = slots + static_cast<uint32_t>(groups * nslots) * row_bytes;
+    const uint32_t tab_bar = bars + 8u * static_cast<uint32_t>(groups * nslots);
     auto slot_addr = [&](int j) { return slots + static_cast<uint32_t>(group * nslots + j) * row_bytes; };
     auto slot_bar = [&](int j) { return bars + 8u * static_cast<uint32_t>(group * nslots + j); };
     const bool leader = g == 0 && lane == 0;
@@ -156,106 +171,112 @@ __global__ void __launch_bounds__(kQuantThreads, CH >= 14 ? 1 : 2)
     const int64_t rstride = static_cast<int64_t>(gridDim.x) * groups;
 
     if (threadIdx.x == 0) {
-        for (int j = 0; j < groups * nslots; ++j)
+        for (int j = 0; j <= groups * nslots; ++j)
             mbar_init(bars + 8u * j, 1);
         abort_sm = 0;
         fence_barrier_init();
     }
+    for (int i = threadIdx.x; i < WARPS * kStagedMaxSlots; i += THREADS)
+        done_cnt[i / kStagedMaxSlots][i % kStagedMaxSlots] = 0;
+    if (threadIdx.x < WARPS)
+        inflight[threadIdx.x] = 0u;
     __syncthreads();
-    uint32_t pending = 0;  // leader: slots with a copy in flight
+    // s first, then the group's first rows
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(tab_bar, static_cast<uint32_t>(K * 4));
+        bulk_load(stab, s, static_cast<uint32_t>(K * 4), tab_bar);
+    }
     if (leader) {
+        uint32_t bits = 0;
         for (int j = 0; j < nslots; ++j) {
             const int64_t r = row0 + j * rstride;
             if (r < rows) {
                 mbar_arrive_expect_tx(slot_bar(j), row_bytes);
                 bulk_load(slot_addr(j), in + r * K, row_bytes, slot_bar(j));
-                pending |= 1u << j;
+                bits |= 1u << j;
             }
         }
+        atomicOr(&inflight[group], bits);
     }
-    // factor tables, staged while the first rows are in flight
-    const bool bad_divisor = __syncthreads_or(stage_factor_tables<MODE == MODE_X, BF>(
-                                 s, static_cast<int>(K), f_sm, fb_sm, threadIdx.x, blockDim.x)) != 0;
-    auto factor_pairs = [&](int c, float2 (&f2)[V / 2]) {
-#pragma unroll
-        for (int h = 0; h < V / 4; ++h) {
-            const float4 v4 = reinterpret_cast<const float4 *>(f_sm + static_cast<int64_t>(c) * V)[h];
-            f2[2 * h] = make_float2(v4.x, v4.y);
-            f2[2 * h + 1] = make_float2(v4.z, v4.w);
-        }
-    };
+    const bool tab_ok = bounded_wait(tab_bar, 0, kErrWaitRow, &abort_sm);
+    const bool tab_fail = __syncthreads_or(!tab_ok) != 0;
+    // divisors outside the range of the fast paths send every row to the exact path
+    int bad = 0;
+    if (MODE == MODE_X && !tab_fail)
+        for (int k = threadIdx.x; k < K; k += THREADS)
+            bad |= !div_operand_ok(s_sm[k]);
+    const bool bad_divisor = __syncthreads_or(bad) != 0;
+
+    // maximum over the G warps of this row: one value a warp, read back by
+    // the lanes in parallel; alternating buffers, so a buffer is rewritten
+    // only after every warp of the group has passed the barrier that follows
+    // its last read
+    // with it, whether every warp of the group had its row (the group then
+    // goes on or leaves together)
     int nred = 0;
-    auto group_max = [&](float v) -> float {
+    auto group_max = [&](float v, bool ok_w, bool &ok_g) -> float {
         v = warp_max(v);
-        if (G == 1)
+        if (G == 1) {
+            ok_g = ok_w;
             return v;
+        }
         float *r = red[nred & 1];
+        int *o = okv[nred & 1];
         ++nred;
-        if (lane == 0)
+        if (lane == 0) {
             r[warp] = v;
+            o[warp] = ok_w ? 1 : 0;
+        }
         named_barrier_sync(1 + group, 32 * G);
-        float m = r[group << log2g];
-        for (int j = 1; j < G; ++j)
-            m = fmaxf(m, r[(group << log2g) + j]);
-        return m;
-    };
-    auto group_sync = [&]() {
-        if (G == 1)
-            __syncwarp();
-        else
-            named_barrier_sync(1 + group, 32 * G);
+        ok_g = __all_sync(0xFFFFFFFFu, lane < G ? o[(group << log2g) + lane] != 0 : true);
+        return warp_max(lane < G ? r[(group << log2g) + lane] : 0.0f);
     };
 
     int j = 0;
-    for (int64_t row = row0; row < rows; row += rstride, ++j) {
+    for (int64_t row = row0; row < rows && !tab_fail; row += rstride, ++j) {
         const int slot = j % nslots;
         const uint32_t par = static_cast<uint32_t>(j / nslots) & 1u;
-        const bool ok = bounded_wait(slot_bar(slot), par, kErrWaitRow, &abort_sm);
-        if (!__all_sync(0xFFFFFFFFu, ok))
-            break;
-        if (leader)
-            pending &= ~(1u << slot);
+        const bool ok = __all_sync(0xFFFFFFFFu, bounded_wait(slot_bar(slot), par, kErrWaitRow, &abort_sm));
+        if (G == 1 && !ok)
+            break;  // (a group of several warps leaves together, after its exchange)
+        if (leader && ok)
+            atomicAnd(&inflight[group], ~(1u << slot));
         const uint32_t sbase = slot_addr(slot);
-        uint4 raw[CH];
-#pragma unroll
-        for (int i = 0; i < CH; ++i) {
-            const uint32_t a = sbase + static_cast<uint32_t>(c0 + cstep * i) * 16u;
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(raw[i].x), "=r"(raw[i].y), "=r"(raw[i].z), "=r"(raw[i].w)
-                         : "r"(a));
-        }
-        // 1. bounds of |v| per chunk, the row's largest bound A, the exact maximum E
+        // 1. the products a_k (kept for pass 2) and the bounds
+        float a[CH][V];
         float hm[CH];
         float am = 0.0f;
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
-            if constexpr (BF) {
-                const uint4 fb = *reinterpret_cast<const uint4 *>(fb_sm + static_cast<int64_t>(c0 + cstep * i) * 4);
-                uint32_t p = bf2_mul(raw[i].x & 0x7FFF7FFFu, fb.x);
-                p = bf2_max(p, bf2_mul(raw[i].y & 0x7FFF7FFFu, fb.y));
-                p = bf2_max(p, bf2_mul(raw[i].z & 0x7FFF7FFFu, fb.z));
-                p = bf2_max(p, bf2_mul(raw[i].w & 0x7FFF7FFFu, fb.w));
-                hm[i] = bf2_hmax_f32(p);
-            } else {
-                float x[V];
-                float2 f2[V / 2];
-                widen<__nv_bfloat16>(raw[i], x);
-                factor_pairs(c0 + cstep * i, f2);
-                float h = 0.0f;
-#pragma unroll
-                for (int e = 0; e < V; e += 2) {
-                    const float2 a = f2_mul(make_float2(x[e], x[e + 1]), f2[e / 2]);
-                    h = fmaxf(h, fmaxf(fabsf(a.x), fabsf(a.y)));
-                }
-                hm[i] = h;
-            }
+            const uint32_t c = static_cast<uint32_t>(c0 + cstep * i);
+            const uint4 r = lds_u4(sbase + c * 16u);
+            float sv[V], f[V], x[V];
+            chunk_factors<MODE>(stab + c * 32u, sv, f);
+            widen<__nv_bfloat16>(r, x);
+            const float2 p0 = f2_mul(make_float2(x[0], x[1]), make_float2(f[0], f[1]));
+            const float2 p1 = f2_mul(make_float2(x[2], x[3]), make_float2(f[2], f[3]));
+            const float2 p2 = f2_mul(make_float2(x[4], x[5]), make_float2(f[4], f[5]));
+            const float2 p3 = f2_mul(make_float2(x[6], x[7]), make_float2(f[6], f[7]));
+            a[i][0] = p0.x;
+            a[i][1] = p0.y;
+            a[i][2] = p1.x;
+            a[i][3] = p1.y;
+            a[i][4] = p2.x;
+            a[i][5] = p2.y;
+            a[i][6] = p3.x;
+            a[i][7] = p3.y;
+            const float h01 = fmaxf(fabsf(p0.x), fabsf(p0.y)), h23 = fmaxf(fabsf(p1.x), fabsf(p1.y));
+            const float h45 = fmaxf(fabsf(p2.x), fabsf(p2.y)), h67 = fmaxf(fabsf(p3.x), fabsf(p3.y));
+            hm[i] = fmaxf(fmaxf(h01, h23), fmaxf(h45, h67));
             am = fmaxf(am, hm[i]);
         }
-        const float A = group_max(am);
-        float E = A;  // fp32-bounded weights: the bounds are the values themselves
-        if (BF || MODE == MODE_X) {
-            const bool exact_all = bad_divisor || !(A >= kTinyQuotient) || !(A <= 0x1.fffffep127f);
-            const float thr = __fmul_rn(A, BF ? 0.96875f : kCandidateScale);
+        // 2. E, exact: this warp's candidates, then one exchange (weights:
+        // a_k is v_k itself)
+        float ew = warp_max(am);
+        if (MODE == MODE_X) {
+            const float Aw = ew;
+            const bool exact_all = bad_divisor || !(Aw >= kTinyQuotient) || !(Aw <= 0x1.fffffep127f);
+            const float thr = __fmul_rn(Aw, kCandidateScale);
             uint32_t cand = 0;
 #pragma unroll
             for (int i = 0; i < CH; ++i)
@@ -264,14 +285,17 @@ __global__ void __launch_bounds__(kQuantThreads, CH >= 14 ? 1 : 2)
             while (cand != 0u) {  // rare: the candidate elements exactly
                 const int i = __ffs(cand) - 1;
                 cand &= cand - 1u;
-                const int64_t c = c0 + cstep * i;
-                em = fmaxf(em, staged_candidates<MODE, BF>(sbase + static_cast<uint32_t>(c) * 16u, fb_sm + c * 4,
-                                                           f_sm + c * V, s + c * V, thr, exact_all));
+                const uint32_t c = static_cast<uint32_t>(c0 + cstep * i);
+                em = fmaxf(em, staged_candidates<MODE>(sbase + c * 16u, stab + c * 32u, thr, exact_all));
             }
-            E = group_max(em);
+            ew = em;
         }
+        bool go = true;
+        const float E = group_max(ew, ok, go);
+        if (!go)
+            break;  // some warp of the group timed out waiting for the row
 
-        // 2. scale and codes, from the registers
+        // 3. scale and codes, from the products in registers
         const float scale = scale_from_max(E);
         if (g == 0 && lane == 0)
             scale_out[row] = scale;
@@ -286,18 +310,14 @@ __global__ void __launch_bounds__(kQuantThreads, CH >= 14 ? 1 : 2)
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
             const int c = c0 + cstep * i;
-            float x[V];
             uint32_t y[V];
-            float2 f2[V / 2];
-            widen<__nv_bfloat16>(raw[i], x);
-            factor_pairs(c, f2);
             float dmax = 0.0f;
 #pragma unroll
             for (int e = 0; e < V; e += 2) {
-                const float2 a = f2_mul(make_float2(x[e], x[e + 1]), f2[e / 2]);
-                const float2 yy = f2_fma(a, rsc2, magic2);
+                const float2 av = make_float2(a[i][e], a[i][e + 1]);
+                const float2 yy = f2_fma(av, rsc2, magic2);
                 const float2 rr = f2_add(yy, nmagic2);
-                const float2 dd = f2_fma(a, nrsc2, rr);
+                const float2 dd = f2_fma(av, nrsc2, rr);
                 dmax = fmaxf(dmax, fmaxf(fabsf(dd.x), fabsf(dd.y)));
                 y[e] = __float_as_uint(yy.x);
                 y[e + 1] = __float_as_uint(yy.y);
@@ -308,25 +328,33 @@ __global__ void __launch_bounds__(kQuantThreads, CH >= 14 ? 1 : 2)
         while (ties != 0u) {  // rare: near ties; every element when the scale is outside the fast range
             const int i = __ffs(ties) - 1;
             ties &= ties - 1u;
-            const int64_t c = c0 + cstep * i;
-            staged_ties<MODE>(sbase + static_cast<uint32_t>(c) * 16u, f_sm + c * V, s + c * V, scale, rsc, fast,
-                              dst + c * V);
+            const uint32_t c = static_cast<uint32_t>(c0 + cstep * i);
+            staged_ties<MODE>(sbase + c * 16u, stab + c * 32u, scale, rsc, fast, dst + static_cast<int64_t>(c) * V);
         }
-        // every warp of the group is done with the slot: refill it
-        group_sync();
-        if (leader) {
-            const int64_t r = row + static_cast<int64_t>(nslots) * rstride;
-            if (r < rows) {
-                mbar_arrive_expect_tx(slot_bar(slot), row_bytes);
-                bulk_load(sbase, in + r * K, row_bytes, slot_bar(slot));
-                pending |= 1u << slot;
+        // 4. this warp is done with the buffer; the group's last refills it
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence_block();
+            if (atomicAdd(&done_cnt[group][slot], 1) == G - 1) {
+                done_cnt[group][slot] = 0;
+                const int64_t r = row + static_cast<int64_t>(nslots) * rstride;
+                if (r < rows) {
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    mbar_arrive_expect_tx(slot_bar(slot), row_bytes);
+                    bulk_load(sbase, in + r * K, row_bytes, slot_bar(slot));
+                    atomicOr(&inflight[group], 1u << slot);
+                }
             }
         }
     }
     // after a timeout the copies still in flight land before the CTA leaves
+    __syncthreads();
+    if (threadIdx.x == 0 && !tab_ok)
+        bounded_wait(tab_bar, 0, kErrWaitDrain, nullptr, kWaitTimeoutNs / 4);
     if (leader && abort_sm) {
+        const uint32_t pend = inflight[group];
         for (int k = 0; k < nslots; ++k)
-            if (pending & (1u << k)) {
+            if (pend & (1u << k)) {
                 // the phase a pending copy completes: parity of that slot's next use
                 int jj = j;
                 while (jj % nslots != k)
