@@ -26,6 +26,7 @@
 #include "sq_gptq.cuh"
 #include "sq_splitk.cuh"
 #include "sq_decode.cuh"
+#include "sq_slab.cuh"
 #include "sq_quant_staged.cuh"
 
 namespace {
@@ -785,9 +786,11 @@ sq_status launch_decode_cfg(const int8_t *xq, const float *sx, const int8_t *wq,
         std::fprintf(stderr, "sq decode M=%lld N=%lld K=%lld: BNX=%d units=%lld ctas=%d stages=%d smem=%d\n",
                      (long long)M, (long long)N, (long long)K, BNX, (long long)U, G, stages, smem);
     // tuning overrides (same arithmetic): SQ_DECODE_PREWAIT=0 waits for the
-    // quantiser before any weight load, SQ_DECODE_L2PF=0 drops the L2 prefetch
+    // quantiser before any weight load, SQ_DECODE_L2PF=1 adds the L2 prefetch
+    // (measured on B200: it delays the quantiser's completion, and with it the
+    // wait, by more than it saves for a 117 MB weight; neutral for 25 MB)
     static const int prewait = std::getenv("SQ_DECODE_PREWAIT") ? std::atoi(std::getenv("SQ_DECODE_PREWAIT")) : 1;
-    static const int l2pf = std::getenv("SQ_DECODE_L2PF") ? std::atoi(std::getenv("SQ_DECODE_L2PF")) : 1;
+    static const int l2pf = std::getenv("SQ_DECODE_L2PF") ? std::atoi(std::getenv("SQ_DECODE_L2PF")) : 0;
     const int flags = (prewait ? 1 : 0) | (prewait && l2pf ? 2 : 0);
     return launch_kernel(kernel, dim3(static_cast<unsigned>(G)), dim3(sq::kDecThreads), smem, st, 0, 0, tw, tx, sx, sw,
                          y, slots, cnt, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), U, G, stages,
@@ -806,6 +809,102 @@ sq_status launch_decode(const int8_t *xq, const float *sx, const int8_t *wq, con
     default:
         return launch_decode_cfg<128, OUT>(xq, sx, wq, sw, M, N, K, y, cnt, slots, in_dt, st);
     }
+}
+
+// ---- the slab GEMM: at most 32 tokens, whole output channels per CTA -------
+// Slabs are 16-channel groups, floor or ceil of R / G of them (R = N / 16);
+// G is the fewest CTAs (at most one an SM) that give the narrowest widest
+// slab, which is what sets the time.  Used where the narrower slab is at
+// least kSlabMinNt channels wide and the wider one fits one MMA (256).  The
+// MMA computes 128 token rows of which at most 32 are real, so the tensor
+// pipe does 4 to 16 times the useful work, and a narrow slab needs many MMAs
+// per weight byte: measured on B200, slabs of 32 or 48 channels are
+// MMA-bound (4096 x 14336 at M = 1: 57 us against 26 us for the
+// weight-streaming kernel), slabs of 192-208 are not far off the stream
+// (28672 x 4096: 30.7 against 31.8-33.9 us, the difference being the
+// stream's cross-CTA reduction).  SQ_DECODE_SLAB=0 turns it off.
+constexpr int64_t kSlabMinNt = 128;
+struct SlabPlan {
+    int G = 0, nt_lo = 0, nt_hi = 0;
+};
+
+inline SlabPlan plan_slab(int64_t M, int64_t N, int64_t sms)
+{
+    SlabPlan p;
+    static const bool on = !(std::getenv("SQ_DECODE_SLAB") && std::atoi(std::getenv("SQ_DECODE_SLAB")) == 0);
+    static const int64_t force = std::getenv("SQ_SLAB_CTAS") ? std::atoll(std::getenv("SQ_SLAB_CTAS")) : 0;
+    if (!on || M > 32 || N % 16 != 0)
+        return p;
+    const int64_t R = N / 16, gmax = std::min<int64_t>(R, sms);
+    const int64_t widest = (R + gmax - 1) / gmax;
+    if (16 * widest > sq::kSlabMaxNt || 16 * (R / gmax) < kSlabMinNt)
+        return p;
+    int64_t G = (R + widest - 1) / widest;  // fewest CTAs with that widest slab
+    if (force > 0)
+        G = std::min<int64_t>(force, gmax);
+    p.G = static_cast<int>(G);
+    p.nt_lo = static_cast<int>(16 * (R / G));
+    p.nt_hi = static_cast<int>(16 * ((R + G - 1) / G));
+    return p;
+}
+
+inline bool slab_applies(int64_t M, int64_t N)
+{
+    DeviceInfo di;
+    if (!device_info(di))
+        return false;
+    return plan_slab(M, N, di.sms).G > 0;
+}
+
+template <int BNX, int OUT>
+sq_status launch_slab_cfg(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw, int64_t M, int64_t N,
+                          int64_t K, void *y, sq_dtype in_dt, bool after_quant, cudaStream_t st)
+{
+    DeviceInfo di;
+    if (!device_info(di))
+        return SQ_ERR_CUDA;
+    const SlabPlan p = plan_slab(M, N, di.sms);
+    if (p.G == 0)
+        return SQ_ERR_UNSUPPORTED;
+    static const int force_kbs = std::getenv("SQ_SLAB_KBS") ? std::atoi(std::getenv("SQ_SLAB_KBS")) : 0;
+    const int kbs = force_kbs > 0 ? force_kbs : 2;
+    // the deepest ring that fits; after the library's quantiser, one that
+    // still leaves room for a quantiser CTA on the SM (the kernels overlap)
+    const int64_t budget = after_quant ? std::min<int64_t>(kMaxDynSmem, kSmSmemBytes - 1024 -
+                                                                            quant_smem_estimate(K, in_dt) - 1024)
+                                       : kMaxDynSmem;
+    int stages = 16;
+    while (stages > 2 && sq::slab_smem_bytes(BNX, p.nt_hi, stages, kbs) > budget)
+        --stages;
+    const int smem = sq::slab_smem_bytes(BNX, p.nt_hi, stages, kbs);
+    if (smem > kMaxDynSmem)
+        return SQ_ERR_UNSUPPORTED;
+    auto kernel = sq::gemm_slab_kernel<BNX, OUT>;
+    static std::atomic<uint64_t> attr_done{0};
+    if (!ensure_smem_attr(kernel, kMaxDynSmem, attr_done))
+        return SQ_ERR_CUDA;
+    CUtensorMap tlo, thi, tx;
+    if (!make_tmap_i8(&tlo, wq, N, K, p.nt_lo) || !make_tmap_i8(&thi, wq, N, K, p.nt_hi) ||
+        !make_tmap_i8(&tx, xq, M, K, BNX))
+        return SQ_ERR_CUDA;
+    if (debug_plan())
+        std::fprintf(stderr, "sq slab M=%lld N=%lld K=%lld: BNX=%d ctas=%d nt=%d/%d kbs=%d stages=%d smem=%d pre=%d\n",
+                     (long long)M, (long long)N, (long long)K, BNX, p.G, p.nt_lo, p.nt_hi, kbs, stages, smem,
+                     (int)after_quant);
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(p.G)), dim3(sq::kSlabThreads), smem, st, 0, 0, tlo, thi,
+                         tx, sx, sw, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), p.G, p.nt_hi,
+                         stages, kbs, after_quant ? 1 : 0);
+}
+
+template <int OUT>
+sq_status launch_slab(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw, int64_t M, int64_t N,
+                      int64_t K, void *y, sq_dtype in_dt, bool after_quant, cudaStream_t st)
+{
+    if (M <= 8)
+        return launch_slab_cfg<8, OUT>(xq, sx, wq, sw, M, N, K, y, in_dt, after_quant, st);
+    if (M <= 16)
+        return launch_slab_cfg<16, OUT>(xq, sx, wq, sw, M, N, K, y, in_dt, after_quant, st);
+    return launch_slab_cfg<32, OUT>(xq, sx, wq, sw, M, N, K, y, in_dt, after_quant, st);
 }
 
 // The stream-K tail of the pair GEMM is off unless SQ_GEMM_SK=1: measured on
@@ -891,20 +990,28 @@ inline int pick_pair_bn(int64_t M, int64_t N, int pairs)
     return best;
 }
 
-// The GEMM with or without a workspace (cnt, slots; null: none).  With one,
-// up to kDecodeMaxM tokens run the weight-streaming kernel and more run the
-// pair kernel with its stream-K tail; the caller has launched, right before,
-// a kernel of this library that clears the tile counters (the quantiser, or
-// the zeroing kernel of sq_w8a8_gemm_ws), which is also what lets the
-// few-token kernel request weights before its griddepcontrol.wait.
+// The GEMM with or without a workspace (cnt, slots; null: none).  Up to 32
+// tokens run the slab kernel (no workspace needed) where it applies.  With a
+// workspace, up to kDecodeMaxM tokens run the weight-streaming kernel and
+// more run the pair kernel with its stream-K tail; the caller has launched,
+// right before, a kernel of this library that clears the tile counters (the
+// quantiser, or the zeroing kernel of sq_w8a8_gemm_ws), which is also what
+// lets the few-token kernel request weights before its griddepcontrol.wait.
+// after_quant: the grid right before is the library's quantiser (so the slab
+// kernel may do the same).
 template <int OUT>
 sq_status launch_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
                       int64_t M, int64_t N, int64_t K, void *y, cudaStream_t st, int *cnt = nullptr,
-                      int32_t *slots = nullptr, sq_dtype in_dt = SQ_BF16)
+                      int32_t *slots = nullptr, sq_dtype in_dt = SQ_BF16, bool after_quant = false)
 {
     const float *nf = nullptr;
     const bool ws = cnt != nullptr && slots != nullptr;
-    if (ws && M <= kDecodeMaxM)
+    if (slab_applies(M, N))
+        return launch_slab<OUT>(xq, sx, wq, sw, M, N, K, y, in_dt, after_quant, st);
+    // SQ_DECODE_STREAM=0: the split-K kernel even with a workspace (tuning)
+    static const bool stream_on =
+        !(std::getenv("SQ_DECODE_STREAM") && std::atoi(std::getenv("SQ_DECODE_STREAM")) == 0);
+    if (ws && M <= kDecodeMaxM && stream_on)
         return launch_decode<OUT>(xq, sx, wq, sw, M, N, K, y, cnt, slots, in_dt, st);
     // weight tiles through the load/store unit (cp.async) or TMA
     static const bool lsu = std::getenv("SQ_SPLITK_LSU") && std::atoi(std::getenv("SQ_SPLITK_LSU")) == 1;
@@ -1369,8 +1476,8 @@ sq_status sq_linear(const void *x, sq_dtype in_dt, const float *s, const int8_t 
             : launch_quant_rows<float, sq::MODE_X>(static_cast<const float *>(x), M, K, s, xq, sx, st, cnt, ncnt);
     if (r != SQ_OK)
         return r;
-    return out_dt == SQ_BF16 ? launch_gemm<OUT_BF16>(xq, sx, wq, sw, M, N, K, y, st, cnt, slots, in_dt)
-                             : launch_gemm<OUT_F32>(xq, sx, wq, sw, M, N, K, y, st, cnt, slots, in_dt);
+    return out_dt == SQ_BF16 ? launch_gemm<OUT_BF16>(xq, sx, wq, sw, M, N, K, y, st, cnt, slots, in_dt, true)
+                             : launch_gemm<OUT_F32>(xq, sx, wq, sw, M, N, K, y, st, cnt, slots, in_dt, true);
 }
 
 size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K)
@@ -1398,6 +1505,11 @@ sq_status sq_w8a8_gemm_ws(const int8_t *xq, const float *sx, const int8_t *wq, c
     uint8_t *wsb = static_cast<uint8_t *>(workspace);
     int *cnt = reinterpret_cast<int *>(wsb + G.cnt);
     int32_t *slots = reinterpret_cast<int32_t *>(wsb + G.slots);
+    // the slab kernel needs no counters (and, after a grid of unknown origin,
+    // requests nothing before griddepcontrol.wait)
+    if (slab_applies(M, N))
+        return out_dt == SQ_BF16 ? launch_gemm<OUT_BF16>(xq, sx, wq, sw, M, N, K, y, st)
+                                 : launch_gemm<OUT_F32>(xq, sx, wq, sw, M, N, K, y, st);
     // clear the tile counters (a kernel of this library, so the GEMM after it
     // may start on its weight before griddepcontrol.wait)
     r = launch_kernel(sq::zero_f32_kernel, dim3(static_cast<unsigned>((G.ncnt + 255) / 256)), dim3(256), 0, st, 0, 0,
