@@ -248,10 +248,12 @@ inline int exact_fit_log2g(int64_t nch, int ch)
 template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false>
 sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
                                float *scale, int log2g, cudaStream_t st, const DeviceInfo &di, T *hout = nullptr,
-                               int *zero = nullptr, int nzero = 0)
+                               int *zero = nullptr, int nzero = 0, bool tab = true)
 {
     auto kernel = sq::row_quant_kernel<T, MODE, CH, FIT, BB, GLU>;
-    const int smem = static_cast<int>(sq::row_quant_smem(K, BB));
+    if (!tab && BB)
+        return SQ_ERR_UNSUPPORTED;  // the bf16 bound needs its table
+    const int smem = tab ? static_cast<int>(sq::row_quant_smem(K, BB)) : 0;
     static std::atomic<uint64_t> attr_done{0};
     // the kernel also has a little static shared memory (the group maxima)
     if (!ensure_smem_attr(kernel, kMaxDynSmem - 1024, attr_done))
@@ -286,7 +288,7 @@ sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float
         std::fprintf(stderr, "sq quant rows=%lld K=%lld: single pass CH=%d G=%d per_sm=%d blocks=%lld\n",
                      (long long)rows, (long long)K, CH, 1 << log2g, per_sm, (long long)blocks);
     return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(sq::kQuantThreads), smem, st, 0, 0, in, rows,
-                         K, s, log2g, q, scale, hout, zero, nzero);
+                         K, s, log2g, q, scale, hout, zero, nzero, tab ? 1 : 0);
 }
 
 // The quantiser with the gated feed-forward activation in front (rows of
@@ -413,6 +415,9 @@ bool launch_staged(const __nv_bfloat16 *in, int64_t rows, int64_t K, const float
     return false;
 }
 
+// Row counts below which the activation quantiser takes its few-row form.
+constexpr int64_t kFewRows = 256;
+
 // `zero` (may be null): nzero ints the quantiser kernel clears on the side.
 template <typename T, int MODE>
 sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
@@ -433,6 +438,30 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
     static const int force_kind = std::getenv("SQ_QUANT_KIND") ? std::atoi(std::getenv("SQ_QUANT_KIND")) : 0;
     constexpr int V = sq::Vec<T>::N;
     const int64_t nch = K / V;
+    // Few rows (decode): the latency of one row is the cost, and a factor
+    // table staged in every CTA for one row or two would be most of it.  So
+    // 8 warps a row, the fewest chunks a lane that cover it, and no table
+    // (each lane reads its own s_k).  SQ_QUANT_FEW=0 turns this off.
+    static const bool few_on = !(std::getenv("SQ_QUANT_FEW") && std::atoi(std::getenv("SQ_QUANT_FEW")) == 0);
+    if (few_on && force_kind != 2 && rows < kFewRows && nch <= (int64_t)32 * 16 * 8) {
+        int ch = 2;
+        while ((int64_t)32 * ch * 8 < nch)
+            ch *= 2;
+        const bool fit = (int64_t)32 * ch * 8 == nch;
+#define SQ_Q_FEW(CH_) (fit ? launch_row_quant_cfg<T, MODE, CH_, true, false>(in, rows, K, s, q, scale, 3, st, di, nullptr, zero, nzero, false) \
+                           : launch_row_quant_cfg<T, MODE, CH_, false, false>(in, rows, K, s, q, scale, 3, st, di, nullptr, zero, nzero, false))
+        switch (ch) {
+        case 2:
+            return SQ_Q_FEW(2);
+        case 4:
+            return SQ_Q_FEW(4);
+        case 8:
+            return SQ_Q_FEW(8);
+        default:
+            return SQ_Q_FEW(16);
+        }
+#undef SQ_Q_FEW
+    }
     // the bf16 bound while both factor tables stay small (about 3 CTAs per SM)
     const bool bb = V == 8 && sq::row_quant_smem(K, true) <= 64 * 1024;
     if (force_kind != 2 && sq::row_quant_smem(K, bb) <= kMaxDynSmem - 1024) {

@@ -520,8 +520,12 @@ template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false>
 __global__ void __launch_bounds__(kQuantThreads, (GLU ? (CH <= 8 ? 2 : 1) : (CH <= 8 ? 3 : 2)))
     row_quant_kernel(const T *__restrict__ in, int64_t rows, int64_t K, const float *__restrict__ s,
                      int log2g, int8_t *__restrict__ q, float *__restrict__ scale_out, T *__restrict__ hout,
-                     int *__restrict__ zero, int nzero)
+                     int *__restrict__ zero, int nzero, int tab)
 {
+    // tab = 0 (few rows, fp32 bound only): no factor table; each lane reads
+    // its chunks' s_k from global memory and takes the hardware reciprocal
+    // itself, and a chunk with an s_k outside the fast range bounds its
+    // elements by +inf, which sends the row to the exact path throughout
     pdl_prologue();
     clear_ints(zero, nzero);
     constexpr int V = Vec<T>::N;
@@ -565,15 +569,31 @@ __global__ void __launch_bounds__(kQuantThreads, (GLU ? (CH <= 8 ? 2 : 1) : (CH 
     if (row < rows)
         load_row(row);
     // factor tables staged while the first row's loads are in flight
-    const bool bad_divisor = __syncthreads_or(stage_factor_tables<MODE == MODE_X, BF>(
-                                 s, static_cast<int>(K), f_sm, fb_sm, threadIdx.x, blockDim.x)) != 0;
-    auto factor_pairs = [&](int c, float2 (&f2)[V / 2]) {
+    const bool bad_divisor =
+        tab ? __syncthreads_or(stage_factor_tables<MODE == MODE_X, BF>(s, static_cast<int>(K), f_sm, fb_sm,
+                                                                       threadIdx.x, blockDim.x)) != 0
+            : false;
+    // f_k of chunk c; without the table, whether some s_k of it is outside
+    // the range of the fast paths
+    auto factor_pairs = [&](int c, float2 (&f2)[V / 2]) -> bool {
+        bool bad = false;
 #pragma unroll
         for (int h = 0; h < V / 4; ++h) {
-            const float4 v4 = reinterpret_cast<const float4 *>(f_sm + static_cast<int64_t>(c) * V)[h];
+            float4 v4;
+            if (tab) {
+                v4 = reinterpret_cast<const float4 *>(f_sm + static_cast<int64_t>(c) * V)[h];
+            } else {
+                v4 = __ldg(reinterpret_cast<const float4 *>(s + static_cast<int64_t>(c) * V) + h);
+                if (MODE == MODE_X) {
+                    bad |= !div_operand_ok(v4.x) || !div_operand_ok(v4.y) || !div_operand_ok(v4.z) ||
+                           !div_operand_ok(v4.w);
+                    v4 = make_float4(rcp_approx(v4.x), rcp_approx(v4.y), rcp_approx(v4.z), rcp_approx(v4.w));
+                }
+            }
             f2[2 * h] = make_float2(v4.x, v4.y);
             f2[2 * h + 1] = make_float2(v4.z, v4.w);
         }
+        return bad;
     };
     // maximum over the G warps of this row; alternating buffers, so a buffer
     // is rewritten only after every warp of the group has passed the barrier
@@ -661,20 +681,23 @@ __global__ void __launch_bounds__(kQuantThreads, (GLU ? (CH <= 8 ? 2 : 1) : (CH 
                     float x[V];
                     float2 f2[V / 2];
                     widen<T>(raw[i], x);
-                    factor_pairs(c, f2);
+                    const bool bad = factor_pairs(c, f2);
                     float h = 0.0f;
 #pragma unroll
                     for (int e = 0; e < V; e += 2) {
                         const float2 a = f2_mul(make_float2(x[e], x[e + 1]), f2[e / 2]);
                         h = fmaxf(h, fmaxf(fabsf(a.x), fabsf(a.y)));
                     }
-                    hm[i] = h;
+                    hm[i] = bad ? __int_as_float(0x7f800000) : h;
                 }
                 am = fmaxf(am, hm[i]);
             }
         }
         const float A = group_max(am);
         float E = A;  // fp32-bounded weights: the bounds are the values themselves
+        // without the table an s_k outside the fast range shows as A = +inf,
+        // and the codes of such a row are all taken exactly too
+        const bool row_exact = !tab && MODE == MODE_X && !(A <= 0x1.fffffep127f);
         if (BF || MODE == MODE_X) {
             const bool exact_all = bad_divisor || !(A >= kTinyQuotient) || !(A <= 0x1.fffffep127f);
             const float thr = __fmul_rn(A, BF ? 0.96875f : kCandidateScale);
@@ -704,7 +727,7 @@ __global__ void __launch_bounds__(kQuantThreads, (GLU ? (CH <= 8 ? 2 : 1) : (CH 
         if (g == 0 && lane == 0)
             scale_out[row] = scale;
         const float rsc = rcp_approx(scale);
-        const bool fast = scale_in_fast_range(scale) && !bad_divisor;
+        const bool fast = scale_in_fast_range(scale) && !bad_divisor && !row_exact;
         const float2 rsc2 = make_float2(rsc, rsc);
         const float2 nrsc2 = make_float2(-rsc, -rsc);
         const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
