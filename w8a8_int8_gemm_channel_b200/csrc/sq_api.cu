@@ -952,6 +952,9 @@ bool gemm_sk_enabled()
 // rounds of the co-resident pairs, the last round and the partial one are
 // done stream-K: their k blocks are cut into one equal range per pair, and
 // tiles shared by several pairs are summed through int32 partials.
+// K from which the pair GEMM takes its tiles in groups of 8 m blocks.
+constexpr int64_t kPairGroupMinK = 16384;
+
 template <int BN, int STAGES, int OUT>
 sq_status launch_gemm_pair_cfg(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
                                int64_t M, int64_t N, int64_t K, void *y, cudaStream_t st, int32_t *slots = nullptr,
@@ -986,9 +989,14 @@ sq_status launch_gemm_pair_cfg(const int8_t *xq, const float *sx, const int8_t *
         std::fprintf(stderr, "sq gemm pair M=%lld N=%lld K=%lld: BN=%d stages=%d tiles=%lld pairs=%lld sk_first=%lld sk_units=%lld\n",
                      (long long)M, (long long)N, (long long)K, BN, STAGES, (long long)tiles, (long long)pairs,
                      (long long)sk_first, (long long)sk_units);
+    // tile order: groups of 8 m blocks for long K (less DRAM traffic, see
+    // pair_tile_mn), m fastest otherwise; SQ_PAIR_GROUP_M overrides
+    static const int force_gm = std::getenv("SQ_PAIR_GROUP_M") ? std::atoi(std::getenv("SQ_PAIR_GROUP_M")) : 0;
+    const int m_tiles = static_cast<int>((M + sq::kPairBM - 1) / sq::kPairBM);
+    const int group_m = force_gm > 0 ? force_gm : (K >= kPairGroupMinK ? 8 : m_tiles);
     return launch_kernel(kernel, dim3(static_cast<unsigned>(2 * pairs)), dim3(sq::kPairThreads), Cfg::SMEM_BYTES, st, 2,
                          1, ta, tb, sx, sw, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
-                         static_cast<int>(sk_first), sk_units, slots, cnt);
+                         static_cast<int>(sk_first), sk_units, slots, cnt, std::max(group_m, 1));
 }
 
 // Tile width of the pair GEMM: the fewest rounds of tiles over the

@@ -97,6 +97,25 @@ struct PairSched {
     __device__ __forceinline__ int first_sk_tile() const { return sk_first + static_cast<int>(u0 / KB); }
 };
 
+// Output tile t of the pair kernel -> (m block, n block).  Tiles go in
+// groups of up to group_m m blocks: within a group the m block varies
+// fastest, then the n block, and groups follow in m (group_m >= m_tiles: m
+// fastest throughout).  With groups of 8, the 74 pairs that work at the same
+// time touch about 8 + 10 tiles' k slices at M = 8192 instead of 32 + 3, so
+// more of each slice comes from L2: measured on B200, DRAM reads of 8192 x
+// 8192 x 28672 fell from 3.8 to 2.1 GB and its time by 5%, while 8192 x
+// 57344 x 8192 (DRAM reads 3.7 -> 2.8 GB) became 1.7% slower; the launcher
+// groups long-K shapes only.
+__device__ __forceinline__ void pair_tile_mn(int t, int m_tiles, int n_tiles, int group_m, int &m_blk, int &n_blk)
+{
+    const int per_group = group_m * n_tiles;
+    const int g = t / per_group;
+    const int r = t - g * per_group;
+    const int gm = min(group_m, m_tiles - g * group_m);  // m blocks in this group
+    m_blk = g * group_m + r % gm;
+    n_blk = r / gm;
+}
+
 // Partial-sum slot of CTA `cta` (blockIdx.x) of the pair kernel: ws holds
 // 2 slots per CTA of 128 rows x BN int32, column-chunk-major (32 columns of
 // 128 rows, the rows contiguous).
@@ -110,7 +129,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const float *__restrict__ sx, const float *__restrict__ sw, void *__restrict__ y,
                         int M, int N, int K, int sk_first, int64_t sk_units, int32_t *__restrict__ ws,
-                        int *__restrict__ cnt)
+                        int *__restrict__ cnt, int group_m)
 {
     pdl_prologue();
     using Cfg = PairCfg<BN, STAGES>;
@@ -166,6 +185,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     const int m_tiles = (M + kPairBM - 1) / kPairBM;
+    const int n_tiles = (N + BN - 1) / BN;
     const int k_blocks = (K + kBK - 1) / kBK;
 
     uint32_t issued_mask = 0, issued_parity = 0;  // producer: last phase issued per stage
@@ -178,7 +198,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             PairSched sch(pair, pairs, sk_first, k_blocks, sk_units);
             PairSeg sg;
             while (sch.next(sg)) {
-                const int m_blk = sg.tile % m_tiles, n_blk = sg.tile / m_tiles;
+                int m_blk, n_blk;
+                pair_tile_mn(sg.tile, m_tiles, n_tiles, group_m, m_blk, n_blk);
                 const int a_row = m_blk * kPairBM + static_cast<int>(rank) * 128;
                 const int b_row = n_blk * BN + static_cast<int>(rank) * (BN / 2);
                 for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
@@ -259,7 +280,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const int first_sk = sch.first_sk_tile();
         PairSeg sg;
         while (sch.next(sg)) {
-            const int m_blk = sg.tile % m_tiles, n_blk = sg.tile / m_tiles;
+            int m_blk, n_blk;
+            pair_tile_mn(sg.tile, m_tiles, n_tiles, group_m, m_blk, n_blk);
             const bool ok = bounded_wait(tfull_bar(acc), acc_phase, kErrWaitAccFull, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, ok))
                 break;
