@@ -72,8 +72,17 @@ L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
 # from one ncu capture each (--metrics dram__bytes_read.sum,dram__bytes_write.sum)
 # of `bench.py --case gemm:M,N,K`, taken on the kernel sources whose digest is
 # GEMM_TRAFFIC_DIGEST; reported only while the sources still have that digest.
-GEMM_TRAFFIC = {}
-GEMM_TRAFFIC_DIGEST = None
+GEMM_TRAFFIC = {
+    (2048, 10240, 8192): 122808320,
+    (2048, 8192, 8192): 97621760,
+    (2048, 57344, 8192): 731368704,
+    (2048, 8192, 28672): 514972672,
+    (8192, 10240, 8192): 837802496,
+    (8192, 8192, 8192): 684165888,
+    (8192, 57344, 8192): 5499106304,
+    (8192, 8192, 28672): 2997508352,
+}
+GEMM_TRAFFIC_DIGEST = "fa7fd8c3bf9a9833"
 
 
 # ---------------------------------------------------------------------------

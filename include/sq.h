@@ -269,17 +269,21 @@ SQ_API sq_status sq_w8a8_gemm(const int8_t *xq, const float *sx, const int8_t *w
  * shape ("quant_llm_int8", "The architecture: every piece explained": the
  * same int32 accumulation and outer-product dequantisation):
  *   - up to 128 tokens, the weight is streamed by one CTA per SM, each taking
- *     an equal share of the 128-channel x 128-byte weight blocks;
- *   - more tokens, the tiles that do not fill whole rounds of the CTA pairs
- *     (the last full round and the partial one) are split along K over all
- *     pairs.
+ *     an equal share of the 128-channel x 128-byte weight blocks (up to 32
+ *     tokens on layers whose output channels split into slabs of 128-256 per
+ *     SM, every CTA takes whole channels instead and the workspace is not
+ *     touched);
+ *   - more tokens: the same tiles as sq_w8a8_gemm; with SQ_GEMM_SK=1 in the
+ *     environment the tiles that do not fill whole rounds of the CTA pairs
+ *     are split along K over all pairs (off by default: slower on B200).
  *   A tile shared by several CTAs is summed through int32 partials in the
  *   workspace (exact: the result is the same bits as sq_w8a8_gemm's).
  *   workspace: device scratch of at least sq_w8a8_gemm_workspace_size(M, N,
  *   K) bytes, 16-byte aligned, owned by the caller, any contents; calls that
  *   run concurrently need separate workspaces.  A small kernel clears the
- *   workspace's tile counters before the GEMM.  Errors as sq_w8a8_gemm, plus
- *   SQ_ERR_INVALID_ARG for a missing or too small workspace.
+ *   workspace's tile counters before a GEMM that uses them.  Errors as
+ *   sq_w8a8_gemm, plus SQ_ERR_INVALID_ARG for a missing or too small
+ *   workspace.
  */
 SQ_API sq_status sq_w8a8_gemm_ws(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
                                  int64_t M, int64_t N, int64_t K, void *y, sq_dtype out_dt,

@@ -4,7 +4,10 @@ For up to 128 tokens sq_linear runs the activation quantiser and then a GEMM
 that streams the weight over every SM: the T x KB weight units (128 output
 channels x 128 bytes of K each) are cut into one contiguous range per CTA, a
 tile shared by several CTAs is summed through int32 partials in the
-workspace, and the quantiser clears the tiles' counters.  Every output is
+workspace, and the quantiser clears the tiles' counters.  (For at most 32
+tokens on layers of about 19K-38K output channels the slab kernel runs
+instead; tests/test_slab_gpu.py covers it, and the weight stream on those
+shapes in a child process.)  Every output is
 compared with the oracle's per-token quantisation, int32 GEMM and
 dequantisation ("quant_llm_int8", "The architecture: every piece
 explained"; "Understanding W8A8 INT8 LLM Quantization", "Why Activation
