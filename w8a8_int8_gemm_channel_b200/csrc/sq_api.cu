@@ -245,15 +245,13 @@ inline int exact_fit_log2g(int64_t nch, int ch)
     return -1;
 }
 
-template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false>
+template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false, bool TAB = true>
 sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
                                float *scale, int log2g, cudaStream_t st, const DeviceInfo &di, T *hout = nullptr,
-                               int *zero = nullptr, int nzero = 0, bool tab = true)
+                               int *zero = nullptr, int nzero = 0)
 {
-    auto kernel = sq::row_quant_kernel<T, MODE, CH, FIT, BB, GLU>;
-    if (!tab && BB)
-        return SQ_ERR_UNSUPPORTED;  // the bf16 bound needs its table
-    const int smem = tab ? static_cast<int>(sq::row_quant_smem(K, BB)) : 0;
+    auto kernel = sq::row_quant_kernel<T, MODE, CH, FIT, BB, GLU, TAB>;
+    const int smem = TAB ? static_cast<int>(sq::row_quant_smem(K, BB)) : 0;
     static std::atomic<uint64_t> attr_done{0};
     // the kernel also has a little static shared memory (the group maxima)
     if (!ensure_smem_attr(kernel, kMaxDynSmem - 1024, attr_done))
@@ -288,7 +286,7 @@ sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float
         std::fprintf(stderr, "sq quant rows=%lld K=%lld: single pass CH=%d G=%d per_sm=%d blocks=%lld\n",
                      (long long)rows, (long long)K, CH, 1 << log2g, per_sm, (long long)blocks);
     return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(sq::kQuantThreads), smem, st, 0, 0, in, rows,
-                         K, s, log2g, q, scale, hout, zero, nzero, tab ? 1 : 0);
+                         K, s, log2g, q, scale, hout, zero, nzero);
 }
 
 // The quantiser with the gated feed-forward activation in front (rows of
@@ -448,8 +446,8 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
         while ((int64_t)32 * ch * 8 < nch)
             ch *= 2;
         const bool fit = (int64_t)32 * ch * 8 == nch;
-#define SQ_Q_FEW(CH_) (fit ? launch_row_quant_cfg<T, MODE, CH_, true, false>(in, rows, K, s, q, scale, 3, st, di, nullptr, zero, nzero, false) \
-                           : launch_row_quant_cfg<T, MODE, CH_, false, false>(in, rows, K, s, q, scale, 3, st, di, nullptr, zero, nzero, false))
+#define SQ_Q_FEW(CH_) (fit ? launch_row_quant_cfg<T, MODE, CH_, true, false, false, false>(in, rows, K, s, q, scale, 3, st, di, nullptr, zero, nzero) \
+                           : launch_row_quant_cfg<T, MODE, CH_, false, false, false, false>(in, rows, K, s, q, scale, 3, st, di, nullptr, zero, nzero))
         switch (ch) {
         case 2:
             return SQ_Q_FEW(2);

@@ -516,13 +516,15 @@ __host__ __device__ constexpr int64_t row_quant_smem(int64_t K, bool bf) { retur
 // factor table in shared memory) instead of fp32.  GLU: each input row is
 // [gate | up] (2K values) and the row quantised is h = SiLU(gate) * up
 // (sq_glu.cuh), written to hout as well when hout is not null.
-template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false>
+template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false, bool TAB = true>
 __global__ void __launch_bounds__(kQuantThreads, (GLU ? (CH <= 8 ? 2 : 1) : (CH <= 8 ? 3 : 2)))
     row_quant_kernel(const T *__restrict__ in, int64_t rows, int64_t K, const float *__restrict__ s,
                      int log2g, int8_t *__restrict__ q, float *__restrict__ scale_out, T *__restrict__ hout,
-                     int *__restrict__ zero, int nzero, int tab)
+                     int *__restrict__ zero, int nzero)
 {
-    // tab = 0 (few rows, fp32 bound only): no factor table; each lane reads
+    static_assert(TAB || !BB, "the bf16 bound needs its table");
+    constexpr bool tab = TAB;
+    // TAB = false (few rows, fp32 bound only): no factor table; each lane reads
     // its chunks' s_k from global memory and takes the hardware reciprocal
     // itself, and a chunk with an s_k outside the fast range bounds its
     // elements by +inf, which sends the row to the exact path throughout
@@ -766,7 +768,7 @@ __global__ void __launch_bounds__(kQuantThreads, (GLU ? (CH <= 8 ? 2 : 1) : (CH 
             ties &= ties - 1u;
             const int64_t c = c0 + cstep * i;
             uint4 v;
-            if constexpr (GLU) {  // h exists only in the registers
+            if (GLU || !tab) {  // h exists only in the registers; few rows: latency counts, registers do not
                 v = raw[0];
 #pragma unroll
                 for (int j = 1; j < CH; ++j)
