@@ -321,9 +321,8 @@ SQ_API sq_status sq_w8a8_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M,
  * the workspace holds the int8 activations and their scales in between, and
  * the GEMM's tile counters and partial sums (the quantiser clears the
  * counters on every call, so the workspace may hold anything beforehand).
- * For M <= 128 the GEMM streams the weight over every SM and starts loading
- * weight tiles while the quantiser is still running (the quantiser waits
- * for all earlier work on the stream before it lets the GEMM start).
+ * For M <= 128 the GEMM streams the weight over every SM; its launch and
+ * set-up overlap the quantiser.
  * With the environment variable SQ_LINEAR_FUSED=1, up to 32 tokens are
  * instead quantised inside an older cluster split-K GEMM kernel (no
  * workspace; slower on B200).

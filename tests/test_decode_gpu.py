@@ -6,8 +6,10 @@ channels x 128 bytes of K each) are cut into one contiguous range per CTA, a
 tile shared by several CTAs is summed through int32 partials in the
 workspace, and the quantiser clears the tiles' counters.  (For at most 32
 tokens on layers of about 19K-38K output channels the slab kernel runs
-instead; tests/test_slab_gpu.py covers it, and the weight stream on those
-shapes in a child process.)  Every output is
+instead: tests/test_slab_gpu.py.)  With SQ_DECODE_STREAM=0 the split-K
+cluster kernel runs instead (K split across the CTAs of a cluster, partials
+summed through distributed shared memory); it is checked on the same shapes
+in a child process.  Every output is
 compared with the oracle's per-token quantisation, int32 GEMM and
 dequantisation ("quant_llm_int8", "The architecture: every piece
 explained"; "Understanding W8A8 INT8 LLM Quantization", "Why Activation
@@ -107,3 +109,44 @@ def test_linear_few_tokens_dirty_workspace_and_repeats(oracle):
     y2 = _run(xt, s, wq, sw, torch.bfloat16, ws)
     y_o, _, _, _ = oracle.linear(to_np(xt), s, wq, sw, "bf16")
     assert np.array_equal(y1, y_o) and np.array_equal(y2, y_o)
+
+
+CHILD_SPLITK = r'''
+import numpy as np
+import torch
+import w8a8_int8_gemm_channel_b200 as sq
+from oracle import oracle
+from w8a8_int8_gemm_channel_b200 import workloads as wls
+oracle.build()
+bits = lambda t: t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+for (M, N, K) in [(1, 6144, 4096), (8, 4096, 4096), (32, 4096, 14336), (33, 4112, 4112), (100, 6144, 4096), (7, 144, 208)]:
+    rng = np.random.default_rng(M * 3 + N + K)
+    x = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(torch.bfloat16)
+    s = rng.uniform(0.3, 8.0, K).astype(np.float32)
+    wq = wls.random_int8((N, K), seed=N + 1).numpy()
+    sw = (rng.uniform(0.5, 2.0, N) * 1e-3).astype(np.float32)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    ws = torch.full((max(sq.sq_linear_workspace_size(M, N, K), 16),), 0xFF, dtype=torch.uint8, device="cuda")
+    sq.sq_linear(x.cuda(), torch.from_numpy(s).cuda(), torch.from_numpy(wq).cuda(), torch.from_numpy(sw).cuda(), y, ws)
+    torch.cuda.synchronize()
+    y_o, _, _, _ = oracle.linear(bits(x), s, wq, sw, "bf16")
+    assert np.array_equal(bits(y), y_o), (M, N, K)
+st, code = sq.sq_device_status()
+assert st == sq.SQ_OK, hex(code)
+print("splitk-ok")
+'''
+
+
+def test_split_k_kernel_child_process():
+    """With SQ_DECODE_STREAM=0 (read once per process, so in a child) the
+    few-token shapes take the split-K cluster kernel; its outputs equal the
+    oracle's bit for bit."""
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SQ_DECODE_STREAM="0", PYTHONPATH=root)
+    r = subprocess.run([sys.executable, "-c", CHILD_SPLITK], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0 and "splitk-ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]

@@ -15,8 +15,8 @@ wider one fits one MMA (N of about 19K to 38K on 148 SMs).  Shapes cover
 every token-tile width and the token counts around them, one and two slab
 widths, the widest slab (256 channels), K that is not a multiple of the
 128-byte k block, and both output types.
-The weight-streaming kernel that the slab kernel replaces for M <= 32 is
-checked on the same shapes in a child process with SQ_DECODE_SLAB=0.
+The weight-streaming kernel is checked on the same shapes in a child process
+with SQ_DECODE_SLAB=0.
 """
 import numpy as np
 import pytest

@@ -760,6 +760,18 @@ inline int64_t quant_smem_estimate(int64_t K, sq_dtype dt)
 // units per CTA plus that cost per partial tile.
 constexpr int64_t kDecodeEpiUnits = 6;
 
+// Whether the few-token kernels request their first weight tiles before
+// griddepcontrol.wait when the grid before is the library's quantiser
+// (SQ_DECODE_PREWAIT=1).  Off by default: measured on B200 back to back,
+// those loads compete with the quantiser for HBM and delay its completion,
+// which every later step waits for (278 against 286 us for the 12-call decode
+// workload as one CUDA graph).
+inline bool decode_prewait()
+{
+    static const bool on = std::getenv("SQ_DECODE_PREWAIT") && std::atoi(std::getenv("SQ_DECODE_PREWAIT")) == 1;
+    return on;
+}
+
 inline int64_t decode_ctas(int64_t N, int64_t K, int64_t sms)
 {
     const int64_t T = (N + sq::kBM - 1) / sq::kBM, KB = (K + sq::kBK - 1) / sq::kBK, U = T * KB;
@@ -812,12 +824,12 @@ sq_status launch_decode_cfg(const int8_t *xq, const float *sx, const int8_t *wq,
     if (debug_plan())
         std::fprintf(stderr, "sq decode M=%lld N=%lld K=%lld: BNX=%d units=%lld ctas=%d stages=%d smem=%d\n",
                      (long long)M, (long long)N, (long long)K, BNX, (long long)U, G, stages, smem);
-    // tuning overrides (same arithmetic): SQ_DECODE_PREWAIT=0 waits for the
-    // quantiser before any weight load, SQ_DECODE_L2PF=1 adds the L2 prefetch
-    // (measured on B200: it delays the quantiser's completion, and with it the
-    // wait, by more than it saves for a 117 MB weight; neutral for 25 MB)
-    static const int prewait = std::getenv("SQ_DECODE_PREWAIT") ? std::atoi(std::getenv("SQ_DECODE_PREWAIT")) : 1;
+    // tuning override (same arithmetic): with the early weight loads on,
+    // SQ_DECODE_L2PF=1 adds an L2 prefetch of the CTA's whole range (measured
+    // on B200: it delays the quantiser's completion, and with it the wait, by
+    // more than it saves for a 117 MB weight; neutral for 25 MB)
     static const int l2pf = std::getenv("SQ_DECODE_L2PF") ? std::atoi(std::getenv("SQ_DECODE_L2PF")) : 0;
+    const bool prewait = decode_prewait();
     const int flags = (prewait ? 1 : 0) | (prewait && l2pf ? 2 : 0);
     return launch_kernel(kernel, dim3(static_cast<unsigned>(G)), dim3(sq::kDecThreads), smem, st, 0, 0, tw, tx, sx, sw,
                          y, slots, cnt, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), U, G, stages,
@@ -920,7 +932,7 @@ sq_status launch_slab_cfg(const int8_t *xq, const float *sx, const int8_t *wq, c
                      (int)after_quant);
     return launch_kernel(kernel, dim3(static_cast<unsigned>(p.G)), dim3(sq::kSlabThreads), smem, st, 0, 0, tlo, thi,
                          tx, sx, sw, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), p.G, p.nt_hi,
-                         stages, kbs, after_quant ? 1 : 0);
+                         stages, kbs, (after_quant && decode_prewait()) ? 1 : 0);
 }
 
 template <int OUT>
@@ -1025,15 +1037,27 @@ inline int pick_pair_bn(int64_t M, int64_t N, int pairs)
     return best;
 }
 
-// The GEMM with or without a workspace (cnt, slots; null: none).  Up to 32
-// tokens run the slab kernel (no workspace needed) where it applies.  With a
-// workspace, up to kDecodeMaxM tokens run the weight-streaming kernel and
-// more run the pair kernel with its stream-K tail; the caller has launched,
-// right before, a kernel of this library that clears the tile counters (the
-// quantiser, or the zeroing kernel of sq_w8a8_gemm_ws), which is also what
-// lets the few-token kernel request weights before its griddepcontrol.wait.
-// after_quant: the grid right before is the library's quantiser (so the slab
-// kernel may do the same).
+// The weight-streaming kernel runs for few tokens with a workspace unless
+// SQ_DECODE_STREAM=0 (the split-K cluster kernel then): measured on B200 back
+// to back, the two are within 1% of each other, the stream slightly ahead.
+inline bool decode_stream_on()
+{
+    static const bool on = !(std::getenv("SQ_DECODE_STREAM") && std::atoi(std::getenv("SQ_DECODE_STREAM")) == 0);
+    return on;
+}
+
+
+// The GEMM with or without a workspace (cnt, slots; null: none).
+//   - Up to 32 tokens on wide layers: the slab kernel (no workspace).
+//   - Up to kDecodeMaxM tokens otherwise: the split-K cluster kernel, or with
+//     SQ_DECODE_STREAM=1 and a workspace the weight-streaming kernel, whose
+//     tile counters the caller's kernel right before has cleared (the
+//     quantiser, or the zeroing kernel of sq_w8a8_gemm_ws).
+//   - More tokens: the pair kernel (with its stream-K tail under SQ_GEMM_SK=1
+//     and a workspace).
+// after_quant: the grid right before is the library's own quantiser, so the
+// few-token kernels may request their first weight tiles before
+// griddepcontrol.wait (that quantiser waited for every earlier grid).
 template <int OUT>
 sq_status launch_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
                       int64_t M, int64_t N, int64_t K, void *y, cudaStream_t st, int *cnt = nullptr,
@@ -1043,10 +1067,7 @@ sq_status launch_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const
     const bool ws = cnt != nullptr && slots != nullptr;
     if (slab_applies(M, N))
         return launch_slab<OUT>(xq, sx, wq, sw, M, N, K, y, in_dt, after_quant, st);
-    // SQ_DECODE_STREAM=0: the split-K kernel even with a workspace (tuning)
-    static const bool stream_on =
-        !(std::getenv("SQ_DECODE_STREAM") && std::atoi(std::getenv("SQ_DECODE_STREAM")) == 0);
-    if (ws && M <= kDecodeMaxM && stream_on)
+    if (ws && M <= kDecodeMaxM && decode_stream_on())
         return launch_decode<OUT>(xq, sx, wq, sw, M, N, K, y, cnt, slots, in_dt, st);
     // weight tiles through the load/store unit (cp.async) or TMA
     static const bool lsu = std::getenv("SQ_SPLITK_LSU") && std::atoi(std::getenv("SQ_SPLITK_LSU")) == 1;
@@ -1540,9 +1561,9 @@ sq_status sq_w8a8_gemm_ws(const int8_t *xq, const float *sx, const int8_t *wq, c
     uint8_t *wsb = static_cast<uint8_t *>(workspace);
     int *cnt = reinterpret_cast<int *>(wsb + G.cnt);
     int32_t *slots = reinterpret_cast<int32_t *>(wsb + G.slots);
-    // the slab kernel needs no counters (and, after a grid of unknown origin,
-    // requests nothing before griddepcontrol.wait)
-    if (slab_applies(M, N))
+    // the slab and split-K kernels need no counters (and, after a grid of
+    // unknown origin, request nothing before griddepcontrol.wait)
+    if (slab_applies(M, N) || (M <= kDecodeMaxM && !decode_stream_on()))
         return out_dt == SQ_BF16 ? launch_gemm<OUT_BF16>(xq, sx, wq, sw, M, N, K, y, st)
                                  : launch_gemm<OUT_F32>(xq, sx, wq, sw, M, N, K, y, st);
     // clear the tile counters (a kernel of this library, so the GEMM after it
