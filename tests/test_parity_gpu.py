@@ -153,7 +153,8 @@ QUANT_SHAPES = [(1, 16, torch.float32), (3, 48, torch.bfloat16), (37, 4096, torc
                 (130, 4112, torch.bfloat16), (5, 14336, torch.bfloat16), (2, 28672, torch.bfloat16),
                 (9, 8192, torch.float32), (4, 65536, torch.bfloat16), (2, 32768, torch.float32),
                 (2048, 4096, torch.bfloat16), (320, 14336, torch.bfloat16), (300, 8192, torch.bfloat16),
-                (513, 2048, torch.bfloat16), (257, 28672, torch.bfloat16), (260, 16384, torch.bfloat16)]
+                (513, 2048, torch.bfloat16), (257, 28672, torch.bfloat16), (260, 16384, torch.bfloat16),
+                (6, 8192, torch.bfloat16), (3, 32768, torch.bfloat16)]
 
 
 @pytest.mark.parametrize("R,K,dtype", QUANT_SHAPES)
@@ -185,6 +186,53 @@ def test_smooth_quant_weight(oracle, R, K, dtype):
     wq_o, sw_o = oracle.smooth_quant_weight(to_np(w), s_np)
     assert_bits_equal(to_np(sw), sw_o, "sw")
     assert_bits_equal(to_np(wq), wq_o, "wq")
+
+
+CHILD_FEW8 = r'''
+import numpy as np
+import torch
+import w8a8_int8_gemm_channel_b200 as sq
+from oracle import oracle
+from w8a8_int8_gemm_channel_b200 import workloads as wls
+oracle.build()
+bits = lambda t: t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+for (R, K) in [(5, 14336), (2, 28672), (4, 16384), (3, 32768), (7, 8208)]:
+    x = wls.random_tensor((R, K), R * 7 + K, dtype=torch.bfloat16)
+    x[1] = 0
+    if R > 2:
+        x[2] *= 1000
+    s = np.random.default_rng(K).uniform(0.25, 8.0, K).astype(np.float32)
+    xq = torch.empty(R, K, dtype=torch.int8, device="cuda")
+    sx = torch.empty(R, device="cuda")
+    sq.sq_quant_act(x.cuda(), torch.from_numpy(s).cuda(), xq, sx)
+    wq = torch.empty(R, K, dtype=torch.int8, device="cuda")
+    sw = torch.empty(R, device="cuda")
+    sq.sq_smooth_quant_weight(x.cuda(), torch.from_numpy(s).cuda(), wq, sw)
+    torch.cuda.synchronize()
+    xq_o, sx_o = oracle.quant_act(bits(x), s)
+    assert np.array_equal(xq.cpu().numpy(), xq_o) and np.array_equal(sx.cpu().numpy().view(np.uint32), sx_o.view(np.uint32)), (R, K)
+    wq_o, sw_o = oracle.smooth_quant_weight(bits(x), s)
+    assert np.array_equal(wq.cpu().numpy(), wq_o) and np.array_equal(sw.cpu().numpy().view(np.uint32), sw_o.view(np.uint32)), (R, K)
+st, code = sq.sq_device_status()
+assert st == sq.SQ_OK, hex(code)
+print("few8-ok")
+'''
+
+
+def test_few_row_quantiser_8_warps_child_process():
+    """Rows above 2 chunks a lane on 8 warps take the 16-warp few-row form by
+    default; with SQ_QUANT_FEW_THREADS=256 (read once per process, so in a
+    child) they take the 8-warp form (4, 8 and 16 chunks a lane, exact fits
+    and ragged rows).  Codes and scales equal the oracle's bit for bit."""
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SQ_QUANT_FEW_THREADS="256", PYTHONPATH=root)
+    r = subprocess.run([sys.executable, "-c", CHILD_FEW8], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0 and "few8-ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]
 
 
 # ---------------------------------------------------------------------------

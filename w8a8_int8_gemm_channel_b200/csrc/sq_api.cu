@@ -245,12 +245,13 @@ inline int exact_fit_log2g(int64_t nch, int ch)
     return -1;
 }
 
-template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false, bool TAB = true>
+template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false, bool TAB = true,
+          int THREADS = sq::kQuantThreads>
 sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q,
                                float *scale, int log2g, cudaStream_t st, const DeviceInfo &di, T *hout = nullptr,
                                int *zero = nullptr, int nzero = 0)
 {
-    auto kernel = sq::row_quant_kernel<T, MODE, CH, FIT, BB, GLU, TAB>;
+    auto kernel = sq::row_quant_kernel<T, MODE, CH, FIT, BB, GLU, TAB, THREADS>;
     const int smem = TAB ? static_cast<int>(sq::row_quant_smem(K, BB)) : 0;
     static std::atomic<uint64_t> attr_done{0};
     // the kernel also has a little static shared memory (the group maxima)
@@ -267,7 +268,7 @@ sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float
                 per_sm = e.second;
     }
     if (per_sm == 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, sq::kQuantThreads, smem) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, THREADS, smem) !=
                 cudaSuccess ||
             per_sm < 1) {
             cudaGetLastError();
@@ -278,14 +279,14 @@ sq_status launch_row_quant_cfg(const T *in, int64_t rows, int64_t K, const float
     }
     // few rows: spread each row over more warps so that every SM has work
     // (not for FIT, whose G is fixed by the row length)
-    while (!FIT && log2g < 3 && rows * (1 << log2g) < (int64_t)di.sms * per_sm * (sq::kQuantThreads / 32))
+    while (!FIT && log2g < 3 && rows * (1 << log2g) < (int64_t)di.sms * per_sm * (THREADS / 32))
         ++log2g;
-    const int slots = (sq::kQuantThreads / 32) >> log2g;
+    const int slots = (THREADS / 32) >> log2g;
     const int64_t blocks = std::min<int64_t>((rows + slots - 1) / slots, (int64_t)per_sm * di.sms);
     if (debug_plan())
         std::fprintf(stderr, "sq quant rows=%lld K=%lld: single pass CH=%d G=%d per_sm=%d blocks=%lld\n",
                      (long long)rows, (long long)K, CH, 1 << log2g, per_sm, (long long)blocks);
-    return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(sq::kQuantThreads), smem, st, 0, 0, in, rows,
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(THREADS), smem, st, 0, 0, in, rows,
                          K, s, log2g, q, scale, hout, zero, nzero);
 }
 
@@ -438,25 +439,47 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
     const int64_t nch = K / V;
     // Few rows (decode): the latency of one row is the cost, and a factor
     // table staged in every CTA for one row or two would be most of it.  So
-    // 8 warps a row, the fewest chunks a lane that cover it, and no table
-    // (each lane reads its own s_k).  SQ_QUANT_FEW=0 turns this off.
+    // one CTA a row, the fewest chunks a lane that cover it, and no table
+    // (each lane reads its own s_k): 8 warps while that is at most 2 chunks a
+    // lane, else 16 warps (measured at K = 14336 in the decode chain: 3.5
+    // chunks a lane on 16 warps took 4 us less a call than 7 on 8 warps; 32
+    // warps gained nothing more).  The 16-warp form is held to 64 registers
+    // a thread, half an SM's register file.
+    // SQ_QUANT_FEW=0 turns the few-row form off; SQ_QUANT_FEW_THREADS=256 or
+    // 512 fixes its CTA size (tuning).
     static const bool few_on = !(std::getenv("SQ_QUANT_FEW") && std::atoi(std::getenv("SQ_QUANT_FEW")) == 0);
+    static const int few_threads =
+        std::getenv("SQ_QUANT_FEW_THREADS") ? std::atoi(std::getenv("SQ_QUANT_FEW_THREADS")) : 0;
     if (few_on && force_kind != 2 && rows < kFewRows && nch <= (int64_t)32 * 16 * 8) {
-        int ch = 2;
-        while ((int64_t)32 * ch * 8 < nch)
+        const bool wide = few_threads == 512 || (few_threads != 256 && nch > (int64_t)32 * 8 * 2);
+        const int lg = wide ? 4 : 3;
+        int ch = wide ? 1 : 2;
+        while (((int64_t)32 * ch << lg) < nch)
             ch *= 2;
-        const bool fit = (int64_t)32 * ch * 8 == nch;
-#define SQ_Q_FEW(CH_) (fit ? launch_row_quant_cfg<T, MODE, CH_, true, false, false, false>(in, rows, K, s, q, scale, 3, st, di, nullptr, zero, nzero) \
-                           : launch_row_quant_cfg<T, MODE, CH_, false, false, false, false>(in, rows, K, s, q, scale, 3, st, di, nullptr, zero, nzero))
+        const bool fit = ((int64_t)32 * ch << lg) == nch;
+#define SQ_Q_FEW(CH_, TH_) (fit ? launch_row_quant_cfg<T, MODE, CH_, true, false, false, false, TH_>(in, rows, K, s, q, scale, lg, st, di, nullptr, zero, nzero) \
+                                : launch_row_quant_cfg<T, MODE, CH_, false, false, false, false, TH_>(in, rows, K, s, q, scale, lg, st, di, nullptr, zero, nzero))
+        if (wide) {
+            switch (ch) {
+            case 1:
+                return SQ_Q_FEW(1, 512);
+            case 2:
+                return SQ_Q_FEW(2, 512);
+            case 4:
+                return SQ_Q_FEW(4, 512);
+            default:
+                return SQ_Q_FEW(8, 512);
+            }
+        }
         switch (ch) {
         case 2:
-            return SQ_Q_FEW(2);
+            return SQ_Q_FEW(2, 256);
         case 4:
-            return SQ_Q_FEW(4);
+            return SQ_Q_FEW(4, 256);
         case 8:
-            return SQ_Q_FEW(8);
+            return SQ_Q_FEW(8, 256);
         default:
-            return SQ_Q_FEW(16);
+            return SQ_Q_FEW(16, 256);
         }
 #undef SQ_Q_FEW
     }

@@ -75,10 +75,34 @@ struct DecCfg {
 
 // shared memory: 1024 alignment slack, the ring, barriers (full, empty,
 // tfull[2], tempty[2], drain), the TMEM slot, the abort flag and the
-// last-contributor flag
+// last-contributor flag, then the token scales (at most 128 floats)
+constexpr int kDecSxBytes = 128 * 4;
 __host__ __device__ constexpr int dec_smem_bytes(int stage_bytes, int stages)
 {
-    return 1024 + stages * stage_bytes + (2 * stages + 5) * 8 + 16;
+    return 1024 + stages * stage_bytes + (2 * stages + 5) * 8 + 16 + kDecSxBytes;
+}
+
+// store_col_chunk with the token scales read from shared memory
+template <int OUT>
+__device__ __forceinline__ void dec_store_chunk(const uint32_t (&r)[32], float swn, const float *sx_s, int m0,
+                                                int M, void *__restrict__ y, int64_t n, int N)
+{
+    const int valid = min(32, M - m0);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        if (j < valid) {
+            const int64_t idx = static_cast<int64_t>(m0 + j) * N + n;
+            if constexpr (OUT == OUT_S32) {
+                reinterpret_cast<int32_t *>(y)[idx] = static_cast<int32_t>(r[j]);
+            } else {
+                const float o = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), sx_s[m0 + j]), swn);
+                if constexpr (OUT == OUT_F32)
+                    reinterpret_cast<float *>(y)[idx] = o;
+                else
+                    reinterpret_cast<__nv_bfloat16 *>(y)[idx] = __float2bfloat16_rn(o);
+            }
+        }
+    }
 }
 
 // barrier of the four epilogue warps (named barrier 2)
@@ -122,6 +146,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(gb + misc_off);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(gb + misc_off + 4);
     volatile int *last_flag = reinterpret_cast<volatile int *>(gb + misc_off + 8);
+    float *sx_s = reinterpret_cast<float *>(gb + misc_off + 16);
 
     const int64_t c = blockIdx.x;
     const int KB = (K + kBK - 1) / kBK;
@@ -248,6 +273,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;  // weight row within the tile
         const int et = threadIdx.x - 64;      // 0..127
+        // the token scales into shared memory while the weight streams, so
+        // that no store after the last MMA waits for a global load
+        if (OUT != OUT_S32 && et < M)
+            sx_s[et] = __ldg(sx + et);
+        dec_bar_sync();
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int64_t u = u0; u < u1;) {
@@ -256,12 +286,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             const int64_t seg_end = min(u1, (t + 1) * KB);
             u = seg_end;
             const bool whole = seg_begin == t * KB && seg_end == (t + 1) * KB;
+            const int64_t n = t * kBM + row;
+            const float swn = (OUT != OUT_S32 && n < N) ? __ldg(sw + n) : 0.0f;
             const bool ok = bounded_wait(tfull_bar(acc), acc_phase, kErrWaitAccFull, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, ok))
                 break;
             tc_fence_after_sync();
-            const int64_t n = t * kBM + row;
-            const float swn = (OUT != OUT_S32 && n < N) ? __ldg(sw + n) : 0.0f;
             const int slot = t == first_tile ? 0 : 1;
             int32_t *mine = dec_slot(ws, c, slot, BNX);
             const uint32_t lane_addr =
@@ -283,7 +313,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 }
                 if (whole) {
                     if (n < N)
-                        store_col_chunk<OUT>(r, swn, sx, cc * 32, M, y, n, N);
+                        dec_store_chunk<OUT>(r, swn, sx_s, cc * 32, M, y, n, N);
                 } else {
                     // this row's partial, the valid tokens only, 16 bytes at a time
                     int4 *dst = reinterpret_cast<int4 *>(mine + row * BNX + cc * 32);
@@ -326,31 +356,53 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         r[j] = 0u;
-                    // two contributors' loads in flight at a time
-                    for (int64_t c2 = cf; c2 <= cl; c2 += 2) {
-                        int4 a[8], b[8];
-                        const bool two = c2 + 1 <= cl;
-                        const int4 *pa = reinterpret_cast<const int4 *>(
+                    // this row's partial in contributor c2's slot
+                    auto part = [&](int64_t c2) {
+                        return reinterpret_cast<const int4 *>(
                             dec_slot(ws, c2, dec_start(c2, U, G) / KB == t ? 0 : 1, BNX) + row * BNX + cc * 32);
-                        const int4 *pb = two ? reinterpret_cast<const int4 *>(
-                                                   dec_slot(ws, c2 + 1, dec_start(c2 + 1, U, G) / KB == t ? 0 : 1,
-                                                            BNX) + row * BNX + cc * 32)
-                                             : pa;
+                    };
+                    auto add4 = [&](int v, int4 a) {
+                        r[4 * v] += static_cast<uint32_t>(a.x);
+                        r[4 * v + 1] += static_cast<uint32_t>(a.y);
+                        r[4 * v + 2] += static_cast<uint32_t>(a.z);
+                        r[4 * v + 3] += static_cast<uint32_t>(a.w);
+                    };
+                    if (nv <= 2) {
+                        // at most 8 tokens: four contributors' loads in flight at a time
+                        for (int64_t c2 = cf; c2 <= cl; c2 += 4) {
+                            int4 a[4][2];
 #pragma unroll
-                        for (int v = 0; v < 8; ++v) {
-                            a[v] = v < nv ? __ldcg(pa + v) : make_int4(0, 0, 0, 0);
-                            b[v] = (two && v < nv) ? __ldcg(pb + v) : make_int4(0, 0, 0, 0);
+                            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                                for (int v = 0; v < 2; ++v)
+                                    a[i][v] = (c2 + i <= cl && v < nv) ? __ldcg(part(c2 + i) + v) : make_int4(0, 0, 0, 0);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                                for (int v = 0; v < 2; ++v)
+                                    add4(v, a[i][v]);
                         }
+                    } else {
+                        // two contributors' loads in flight at a time
+                        for (int64_t c2 = cf; c2 <= cl; c2 += 2) {
+                            int4 a[8], b[8];
+                            const bool two = c2 + 1 <= cl;
+                            const int4 *pa = part(c2);
+                            const int4 *pb = two ? part(c2 + 1) : pa;
 #pragma unroll
-                        for (int v = 0; v < 8; ++v) {
-                            r[4 * v] += static_cast<uint32_t>(a[v].x) + static_cast<uint32_t>(b[v].x);
-                            r[4 * v + 1] += static_cast<uint32_t>(a[v].y) + static_cast<uint32_t>(b[v].y);
-                            r[4 * v + 2] += static_cast<uint32_t>(a[v].z) + static_cast<uint32_t>(b[v].z);
-                            r[4 * v + 3] += static_cast<uint32_t>(a[v].w) + static_cast<uint32_t>(b[v].w);
+                            for (int v = 0; v < 8; ++v) {
+                                a[v] = v < nv ? __ldcg(pa + v) : make_int4(0, 0, 0, 0);
+                                b[v] = (two && v < nv) ? __ldcg(pb + v) : make_int4(0, 0, 0, 0);
+                            }
+#pragma unroll
+                            for (int v = 0; v < 8; ++v) {
+                                add4(v, a[v]);
+                                add4(v, b[v]);
+                            }
                         }
                     }
                     if (n < N)
-                        store_col_chunk<OUT>(r, swn, sx, cc * 32, M, y, n, N);
+                        dec_store_chunk<OUT>(r, swn, sx_s, cc * 32, M, y, n, N);
                 }
             }
             dec_bar_sync();  // last_flag is rewritten by the next partial tile

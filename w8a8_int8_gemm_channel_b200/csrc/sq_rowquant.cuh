@@ -516,8 +516,12 @@ __host__ __device__ constexpr int64_t row_quant_smem(int64_t K, bool bf) { retur
 // factor table in shared memory) instead of fp32.  GLU: each input row is
 // [gate | up] (2K values) and the row quantised is h = SiLU(gate) * up
 // (sq_glu.cuh), written to hout as well when hout is not null.
-template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false, bool TAB = true>
-__global__ void __launch_bounds__(kQuantThreads, (GLU ? (CH <= 8 ? 2 : 1) : (CH <= 8 ? 3 : 2)))
+template <typename T, int MODE, int CH, bool FIT, bool BB, bool GLU = false, bool TAB = true,
+          int THREADS = kQuantThreads>
+__global__ void __launch_bounds__(THREADS, (THREADS >= 1024 ? 1
+                                            : THREADS > kQuantThreads ? 2
+                                            : GLU ? (CH <= 8 ? 2 : 1)
+                                                  : (CH <= 8 ? 3 : 2)))
     row_quant_kernel(const T *__restrict__ in, int64_t rows, int64_t K, const float *__restrict__ s,
                      int log2g, int8_t *__restrict__ q, float *__restrict__ scale_out, T *__restrict__ hout,
                      int *__restrict__ zero, int nzero)
@@ -532,7 +536,7 @@ __global__ void __launch_bounds__(kQuantThreads, (GLU ? (CH <= 8 ? 2 : 1) : (CH 
     clear_ints(zero, nzero);
     constexpr int V = Vec<T>::N;
     constexpr bool BF = BB && (V == 8);  // the bf16 bound
-    constexpr int WARPS = kQuantThreads / 32;
+    constexpr int WARPS = THREADS / 32;
     extern __shared__ float4 smem_f4[];
     float *f_sm = reinterpret_cast<float *>(smem_f4);
     uint32_t *fb_sm = reinterpret_cast<uint32_t *>(f_sm + K);

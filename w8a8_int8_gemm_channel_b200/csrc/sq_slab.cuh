@@ -57,11 +57,12 @@ __host__ __device__ constexpr int slab_col_stride(int nt) { return nt <= 128 ? 1
 
 // Shared-memory layout (offsets from the 1024-aligned base): the code tiles
 // of every stage and k block, then the weight tiles, then the barriers (full
-// and empty per stage, tfull, drain), the TMEM slot and the abort flag.  The
-// MMA reads 128 rows of a code tile; rows past BNX lie in the memory after
-// it, which the layout keeps inside the allocation.
+// and empty per stage, tfull, drain), the TMEM slot and the abort flag, then
+// the slab's weight scales (nt_max floats).  The MMA reads 128 rows of a code
+// tile; rows past BNX lie in the memory after it, which the layout keeps
+// inside the allocation.
 struct SlabLayout {
-    uint32_t w_off, bar_off, total;
+    uint32_t w_off, bar_off, sw_off, total;
 };
 
 __host__ __device__ constexpr SlabLayout slab_layout(int bnx, int nt_max, int stages, int kbs)
@@ -71,7 +72,8 @@ __host__ __device__ constexpr SlabLayout slab_layout(int bnx, int nt_max, int st
     const uint32_t footprint = xr - static_cast<uint32_t>(bnx * kBK) + static_cast<uint32_t>(kBM * kBK);
     const uint32_t end = (xr + wr > footprint ? xr + wr : footprint);
     const uint32_t bar = (end + 7u) & ~7u;
-    return SlabLayout{xr, bar, bar + static_cast<uint32_t>(2 * stages + 2) * 8u + 16u};
+    const uint32_t swo = (bar + static_cast<uint32_t>(2 * stages + 2) * 8u + 16u + 15u) & ~15u;
+    return SlabLayout{xr, bar, swo, swo + static_cast<uint32_t>(nt_max) * 4u};
 }
 
 // 1024 bytes of alignment slack on top of the layout
@@ -81,9 +83,10 @@ __host__ __device__ constexpr int slab_smem_bytes(int bnx, int nt_max, int stage
 }
 
 // Dequantise and store `valid` (<= 32, a multiple of 16) accumulator columns
-// of token m: channels n0 .. n0 + valid - 1, contiguous in y's row m.
+// of token m: channels n0 .. n0 + valid - 1, contiguous in y's row m.  sw_s
+// points at the shared-memory copy of sw[n0 .. n0 + valid - 1].
 template <int OUT>
-__device__ __forceinline__ void slab_store(const uint32_t (&r)[32], float sxm, const float *__restrict__ sw, int n0,
+__device__ __forceinline__ void slab_store(const uint32_t (&r)[32], float sxm, const float *sw_s, int n0,
                                            int valid, int N, void *__restrict__ y, int64_t m)
 {
     if constexpr (OUT == OUT_S32) {
@@ -94,10 +97,10 @@ __device__ __forceinline__ void slab_store(const uint32_t (&r)[32], float sxm, c
                 dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
     } else {
         float o[32];
-        const float4 *sw4 = reinterpret_cast<const float4 *>(sw + n0);
+        const float4 *sw4 = reinterpret_cast<const float4 *>(sw_s);
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
-            const float4 t = (v * 4 < valid) ? __ldg(sw4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 t = (v * 4 < valid) ? sw4[v] : make_float4(0.f, 0.f, 0.f, 0.f);
             o[4 * v] = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[4 * v])), sxm), t.x);
             o[4 * v + 1] = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[4 * v + 1])), sxm), t.y);
             o[4 * v + 2] = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[4 * v + 2])), sxm), t.z);
@@ -264,31 +267,50 @@ __global__ void __launch_bounds__(kSlabThreads, 1)
                 mma_commit(tfull_bar);
         }
     } else {
-        // epilogue warps 2..5: warp w reads TMEM lanes (tokens) 32 (w % 4) .. +31
+        // epilogue warps 2..5: warp w reads TMEM lanes (tokens) 32 (w % 4) .. +31.
+        // While the weight streams they bring the slab's weight scales into
+        // shared memory and each token's scale into a register, so that the
+        // stores after the last MMA wait for no global load.
         const int quarter = warp & 3;
+        const int64_t m = quarter * 32 + lane;
+        float *sw_s = reinterpret_cast<float *>(gb + L.sw_off);
+        if constexpr (OUT != OUT_S32)
+            for (int j = threadIdx.x - 64; j < nt; j += 128)
+                sw_s[j] = __ldg(sw + n0 + j);
+        const float sxm = (OUT != OUT_S32 && m < M) ? __ldg(sx + m) : 0.0f;
+        asm volatile("bar.sync 2, 128;" ::: "memory");  // the four epilogue warps
         const bool ok = bounded_wait(tfull_bar, 0, kErrWaitAccFull, abort_flag);
         if (__all_sync(0xFFFFFFFFu, ok) && quarter * 32 < M) {
             tc_fence_after_sync();
-            const int64_t m = quarter * 32 + lane;
-            const float sxm = (OUT != OUT_S32 && m < M) ? __ldg(sx + m) : 0.0f;
             const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
             // the accumulators written: every one when there are at least nacc MMAs
             const int nused = min(nacc, KB * (kBK / 32));
 #pragma unroll 1
             for (int cb = 0; cb * 32 < nt; ++cb) {
+                // two accumulators' loads in flight at a time, summed exactly
                 uint32_t r[32], q[32];
                 tmem_ld_32x32b_x32(lane_addr + static_cast<uint32_t>(cb * 32), r);
+                if (nused > 1)
+                    tmem_ld_32x32b_x32(lane_addr + static_cast<uint32_t>(cstride + cb * 32), q);
                 tmem_ld_wait();
+                if (nused > 1) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        r[j] += q[j];
+                }
 #pragma unroll 1
-                for (int a = 1; a < nused; ++a) {
+                for (int a = 2; a < nused; a += 2) {
+                    uint32_t q2[32];
                     tmem_ld_32x32b_x32(lane_addr + static_cast<uint32_t>(a * cstride + cb * 32), q);
+                    if (a + 1 < nused)
+                        tmem_ld_32x32b_x32(lane_addr + static_cast<uint32_t>((a + 1) * cstride + cb * 32), q2);
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        r[j] += q[j];  // exact int32 sums
+                        r[j] += q[j] + (a + 1 < nused ? q2[j] : 0u);
                 }
                 if (m < M)
-                    slab_store<OUT>(r, sxm, sw, n0 + cb * 32, min(32, nt - cb * 32), N, y, m);
+                    slab_store<OUT>(r, sxm, sw_s + cb * 32, n0 + cb * 32, min(32, nt - cb * 32), N, y, m);
             }
         }
     }
