@@ -154,7 +154,7 @@ QUANT_SHAPES = [(1, 16, torch.float32), (3, 48, torch.bfloat16), (37, 4096, torc
                 (9, 8192, torch.float32), (4, 65536, torch.bfloat16), (2, 32768, torch.float32),
                 (2048, 4096, torch.bfloat16), (320, 14336, torch.bfloat16), (300, 8192, torch.bfloat16),
                 (513, 2048, torch.bfloat16), (257, 28672, torch.bfloat16), (260, 16384, torch.bfloat16),
-                (6, 8192, torch.bfloat16), (3, 32768, torch.bfloat16)]
+                (6, 8192, torch.bfloat16), (3, 32768, torch.bfloat16), (100, 14336, torch.bfloat16)]
 
 
 @pytest.mark.parametrize("R,K,dtype", QUANT_SHAPES)
@@ -186,6 +186,71 @@ def test_smooth_quant_weight(oracle, R, K, dtype):
     wq_o, sw_o = oracle.smooth_quant_weight(to_np(w), s_np)
     assert_bits_equal(to_np(sw), sw_o, "sw")
     assert_bits_equal(to_np(wq), wq_o, "wq")
+
+
+# Few rows of more than 512 chunks: one thread-block cluster of C CTAs a row
+# (C = 8, 4, 2 as rows x C fits the SMs and every slice keeps >= 128 chunks),
+# slices of 1 to 8 chunks a thread, and slices cut raggedly (K / V not a
+# multiple of C).
+CLUSTER_SHAPES = [(1, 16384, torch.bfloat16), (2, 28672, torch.bfloat16), (20, 14336, torch.bfloat16),
+                  (30, 16384, torch.bfloat16), (40, 28672, torch.bfloat16), (70, 8192, torch.float32),
+                  (9, 8192, torch.float32), (5, 8208, torch.bfloat16), (18, 8192, torch.bfloat16),
+                  (17, 4112, torch.float32), (60, 16384, torch.bfloat16)]
+
+
+@pytest.mark.parametrize("R,K,dtype", CLUSTER_SHAPES)
+def test_quant_cluster_rows(oracle, R, K, dtype):
+    x = rand((R, K), seed=R * 13 + K, dtype=dtype)
+    x[0, K - 5] = 900.0  # the row maximum in the last slice
+    if R > 2:
+        x[1] = 0
+        x[2] *= 1000
+    s_np = np.random.default_rng(K + 3).uniform(0.25, 8.0, K).astype(np.float32)
+    xq = torch.empty(R, K, dtype=torch.int8, device="cuda")
+    sx = torch.empty(R, device="cuda")
+    sq.sq_quant_act(x.cuda(), to_dev(s_np), xq, sx)
+    xq_o, sx_o = oracle.quant_act(to_np(x), s_np)
+    assert_bits_equal(to_np(sx), sx_o, "sx")
+    assert_bits_equal(to_np(xq), xq_o, "xq")
+    wq = torch.empty(R, K, dtype=torch.int8, device="cuda")
+    sw = torch.empty(R, device="cuda")
+    sq.sq_smooth_quant_weight(x.cuda(), to_dev(s_np), wq, sw)
+    wq_o, sw_o = oracle.smooth_quant_weight(to_np(x), s_np)
+    assert_bits_equal(to_np(sw), sw_o, "sw")
+    assert_bits_equal(to_np(wq), wq_o, "wq")
+
+
+@pytest.mark.parametrize("K", [8192, 8208])
+@pytest.mark.parametrize("s_kind", ["ones", "random", "extreme"])
+def test_quant_cluster_fast_path_edges(oracle, s_kind, K):
+    """The edge rows (exact ties and their 1-ulp neighbours, tiny, subnormal
+    and huge rows, zero rows and zero chunks) repeated along a row of K = 8192
+    or 8208 fp32 values, so that every slice of the cluster holds them; for
+    "extreme", divisors outside the fast range in several slices."""
+    base = _edge_rows(256, 5)
+    x = np.tile(base, (1, (K + 255) // 256))[:, :K].copy()
+    rng = np.random.default_rng(16)
+    if s_kind == "ones":
+        s_np = np.ones(K, np.float32)
+    elif s_kind == "random":
+        s_np = rng.uniform(0.05, 20.0, K).astype(np.float32)
+    else:
+        s_np = rng.uniform(0.5, 2.0, K).astype(np.float32)
+        for col in (3, K // 2 + 1, K - 7):
+            s_np[col] = 1e-25
+            x[np.abs(x[:, col]) > 1e10, col] = 1.0  # keep x/s finite
+        s_np[9] = 1e25
+        s_np[K // 3] = 1e25
+    sc = np.float32(0.0123)
+    nt = (np.arange(K) % 200 - 100 + 0.5).astype(np.float32) * sc * s_np
+    nt[K // 2] = np.float32(127.0) * sc * s_np[K // 2]
+    x = np.vstack([x, nt.astype(np.float32)])
+    xq = torch.empty(x.shape, dtype=torch.int8, device="cuda")
+    sx = torch.empty(x.shape[0], device="cuda")
+    sq.sq_quant_act(to_dev(x), to_dev(s_np), xq, sx)
+    xq_o, sx_o = oracle.quant_act(x, s_np)
+    assert_bits_equal(to_np(sx), sx_o, "sx")
+    assert_bits_equal(to_np(xq), xq_o, "xq")
 
 
 CHILD_FEW8 = r'''
@@ -220,16 +285,17 @@ print("few8-ok")
 
 
 def test_few_row_quantiser_8_warps_child_process():
-    """Rows above 2 chunks a lane on 8 warps take the 16-warp few-row form by
-    default; with SQ_QUANT_FEW_THREADS=256 (read once per process, so in a
-    child) they take the 8-warp form (4, 8 and 16 chunks a lane, exact fits
-    and ragged rows).  Codes and scales equal the oracle's bit for bit."""
+    """Few long rows take the cluster form and, past the SM count, the 16-warp
+    form by default; with SQ_QUANT_CLUSTER=0 and SQ_QUANT_FEW_THREADS=256
+    (read once per process, so in a child) they take the 8-warp form (4, 8
+    and 16 chunks a lane, exact fits and ragged rows).  Codes and scales equal
+    the oracle's bit for bit."""
     import os
     import subprocess
     import sys
 
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    env = dict(os.environ, SQ_QUANT_FEW_THREADS="256", PYTHONPATH=root)
+    env = dict(os.environ, SQ_QUANT_FEW_THREADS="256", SQ_QUANT_CLUSTER="0", PYTHONPATH=root)
     r = subprocess.run([sys.executable, "-c", CHILD_FEW8], cwd=root, env=env, capture_output=True, text=True,
                        timeout=600)
     assert r.returncode == 0 and "few8-ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]

@@ -28,6 +28,7 @@
 #include "sq_decode.cuh"
 #include "sq_slab.cuh"
 #include "sq_quant_staged.cuh"
+#include "sq_quant_cluster.cuh"
 
 namespace {
 
@@ -414,6 +415,68 @@ bool launch_staged(const __nv_bfloat16 *in, int64_t rows, int64_t K, const float
     return false;
 }
 
+// The cluster form of the few-row quantiser: C CTAs a row (sq_quant_cluster.cuh).
+template <typename T, int MODE, int CH>
+sq_status launch_quant_cluster_cfg(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q, float *scale,
+                                   int C, cudaStream_t st, int *zero, int nzero)
+{
+    auto kernel = sq::row_quant_cluster_kernel<T, MODE, CH>;
+    if (debug_plan())
+        std::fprintf(stderr, "sq quant rows=%lld K=%lld: cluster of %d CTAs a row, CH=%d\n", (long long)rows,
+                     (long long)K, C, CH);
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(rows * C)), dim3(sq::kQuantClusterThreads), 0, st, C, 1,
+                         in, rows, K, s, q, scale, zero, nzero);
+}
+
+// Few rows of many chunks (more than 512: over 2 chunks a lane on 8 warps): a
+// cluster of C CTAs a row, the largest C in {8, 4, 2} that keeps one CTA an SM
+// (rows x C <= SMs) and leaves every CTA a slice of at least 128 chunks.
+// Measured in the decode chain of sq_linear calls (1 to 32 tokens) at
+// K = 14336: 4 to 8 SMs a row took about 2 us less a call than one.  At
+// K = 4096 (512 chunks) 2 to 4 SMs a row took 2 us more -- the two cluster
+// barriers outweigh the shorter slice -- so such rows keep the one-CTA forms.
+// Returns false (nothing launched) when no C qualifies.  SQ_QUANT_CLUSTER=0
+// turns the form off; SQ_QUANT_CLUSTER_MIN sets the smallest slice in chunks
+// (tuning).
+template <typename T, int MODE>
+bool launch_quant_cluster(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q, float *scale,
+                          cudaStream_t st, const DeviceInfo &di, int *zero, int nzero, sq_status &r)
+{
+    static const bool on = !(std::getenv("SQ_QUANT_CLUSTER") && std::atoi(std::getenv("SQ_QUANT_CLUSTER")) == 0);
+    static const int min_span =
+        std::getenv("SQ_QUANT_CLUSTER_MIN") ? std::max(32, std::atoi(std::getenv("SQ_QUANT_CLUSTER_MIN"))) : 128;
+    constexpr int V = sq::Vec<T>::N;
+    const int64_t nch = K / V;
+    // C >= 2 and CH <= 8 cover rows of up to 2 * 8 * 256 chunks
+    if (!on || nch <= (int64_t)32 * 8 * 2 || nch > (int64_t)2 * 8 * sq::kQuantClusterThreads)
+        return false;
+    int C = 0;
+    for (int c : {8, 4, 2})
+        if (C == 0 && rows * c <= di.sms && (nch + c - 1) / c >= min_span)
+            C = c;
+    if (C == 0)
+        return false;
+    const int64_t span = (nch + C - 1) / C;
+    int ch = 1;
+    while ((int64_t)sq::kQuantClusterThreads * ch < span)
+        ch *= 2;
+    switch (ch) {
+    case 1:
+        r = launch_quant_cluster_cfg<T, MODE, 1>(in, rows, K, s, q, scale, C, st, zero, nzero);
+        break;
+    case 2:
+        r = launch_quant_cluster_cfg<T, MODE, 2>(in, rows, K, s, q, scale, C, st, zero, nzero);
+        break;
+    case 4:
+        r = launch_quant_cluster_cfg<T, MODE, 4>(in, rows, K, s, q, scale, C, st, zero, nzero);
+        break;
+    default:
+        r = launch_quant_cluster_cfg<T, MODE, 8>(in, rows, K, s, q, scale, C, st, zero, nzero);
+        break;
+    }
+    return true;
+}
+
 // Row counts below which the activation quantiser takes its few-row form.
 constexpr int64_t kFewRows = 256;
 
@@ -450,6 +513,11 @@ sq_status launch_quant_rows(const T *in, int64_t rows, int64_t K, const float *s
     static const bool few_on = !(std::getenv("SQ_QUANT_FEW") && std::atoi(std::getenv("SQ_QUANT_FEW")) == 0);
     static const int few_threads =
         std::getenv("SQ_QUANT_FEW_THREADS") ? std::atoi(std::getenv("SQ_QUANT_FEW_THREADS")) : 0;
+    if (few_on && force_kind != 2 && rows < kFewRows) {
+        sq_status r = SQ_OK;
+        if (launch_quant_cluster<T, MODE>(in, rows, K, s, q, scale, st, di, zero, nzero, r))
+            return r;
+    }
     if (few_on && force_kind != 2 && rows < kFewRows && nch <= (int64_t)32 * 16 * 8) {
         const bool wide = few_threads == 512 || (few_threads != 256 && nch > (int64_t)32 * 8 * 2);
         const int lg = wide ? 4 : 3;

@@ -46,11 +46,6 @@ constexpr int kSplitWorkers = 192;  // warps 2..7
 constexpr int kMaxSplits = 8;
 constexpr int kFusedMaxSliceElems = 4096;  // K elements of one CTA's slice (128 KB / 32 tokens)
 
-__device__ __forceinline__ void st_shared_cluster_f32(uint32_t addr, float v)
-{
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-
 __device__ __forceinline__ void named_bar_sync(int id, int threads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
