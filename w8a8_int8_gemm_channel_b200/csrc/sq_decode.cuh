@@ -166,6 +166,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
+    if (producer) {
+        // the tensor maps are this launch's own parameters: fetched while
+        // the grid before still runs
+        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmX);
+    }
     if (warp == 1) {
         tmem_alloc(smem_u32(const_cast<uint32_t *>(tmem_slot)), Cfg::TMEM_COLS);
         tmem_relinquish();
@@ -174,9 +180,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
-    // Up to here nothing touched global memory.  Every thread but the
-    // producer waits for the grid before (the quantiser) now; the producer
-    // first requests weight tiles when that is allowed.
+    // Up to here nothing touched global memory but the tensor maps.  Every
+    // thread but the producer waits for the grid before (the quantiser) now;
+    // the producer first requests weight tiles when that is allowed.
     if (!(producer && (pre_wait & 1)))
         asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -186,8 +192,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            tma_prefetch_desc(&tmW);
-            tma_prefetch_desc(&tmX);
             const int64_t nu = u1 - u0;
             // units whose weight tile is requested before the wait
             const int pre = (pre_wait & 1) ? static_cast<int>(nu < stages ? nu : stages) : 0;

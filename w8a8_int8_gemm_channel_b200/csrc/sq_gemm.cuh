@@ -149,6 +149,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                    const float *__restrict__ sx, const float *__restrict__ sw,
                    void *__restrict__ y, int M, int N, int K)
 {
+    // the tensor maps are this launch's own parameters: fetched before the
+    // wait for the grid before
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
     pdl_prologue();
     using Cfg = GemmCfg<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
@@ -182,10 +188,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
-    }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(const_cast<uint32_t *>(tmem_slot)), Cfg::TMEM_COLS);

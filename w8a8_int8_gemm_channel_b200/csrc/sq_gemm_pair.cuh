@@ -131,6 +131,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                         int M, int N, int K, int sk_first, int64_t sk_units, int32_t *__restrict__ ws,
                         int *__restrict__ cnt, int group_m)
 {
+    // the tensor maps are this launch's own parameters: fetched before the
+    // wait for the grid before
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
     pdl_prologue();
     using Cfg = PairCfg<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
@@ -168,10 +174,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
-    }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(const_cast<uint32_t *>(tmem_slot)), Cfg::TMEM_COLS);

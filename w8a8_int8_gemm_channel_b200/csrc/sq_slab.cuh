@@ -181,6 +181,12 @@ __global__ void __launch_bounds__(kSlabThreads, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
+    if (producer) {
+        // the tensor maps are this launch's own parameters: fetched while
+        // the grid before still runs
+        tma_prefetch_desc(tmW);
+        tma_prefetch_desc(&tmX);
+    }
     if (warp == 1) {
         tmem_alloc(smem_u32(const_cast<uint32_t *>(tmem_slot)), kSlabTmemCols);
         tmem_relinquish();
@@ -189,7 +195,7 @@ __global__ void __launch_bounds__(kSlabThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
-    // Nothing has touched global memory yet.  Every thread but the producer
+    // Nothing but the tensor maps has touched global memory yet.  Every thread but the producer
     // waits for the grid before now; the producer first requests weight
     // tiles when that is allowed.
     if (!(producer && (pre_wait & 1)))
@@ -201,8 +207,6 @@ __global__ void __launch_bounds__(kSlabThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            tma_prefetch_desc(tmW);
-            tma_prefetch_desc(&tmX);
             const int pre = (pre_wait & 1) ? min(nsteps, stages) : 0;
             for (int s = 0; s < pre; ++s) {
                 const int n = step_kbs(s);

@@ -110,6 +110,13 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                        void *__restrict__ y, int M, int N, int K, int splits, int kb_per_split,
                        int stages, int kbs)
 {
+    // the tensor maps are this launch's own parameters: fetched before the
+    // wait for the grid before
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&tmW);
+        if (!FUSED)
+            tma_prefetch_desc(&tmX);
+    }
     pdl_prologue();
     static_assert(BNX % 32 == 0 && BNX <= 128, "token tile");
     static_assert(!FUSED || BNX == 32, "the fused prologue handles up to 32 tokens");
@@ -161,11 +168,6 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         *abort_flag = 0;
         *reinterpret_cast<volatile int *>(g + L.misc + 8) = 0;
         fence_barrier_init();
-    }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmW);
-        if (!FUSED)
-            tma_prefetch_desc(&tmX);
     }
     if (warp == 2 && lane == 0) {
         // request this CTA's whole weight slice into L2 at once: the ring's
