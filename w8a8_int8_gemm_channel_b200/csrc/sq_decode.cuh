@@ -351,6 +351,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             }
             dec_bar_sync();
             if (*last_flag) {
+                // On the range's last segment every stage of the ring has been
+                // consumed (the accumulator-full signal follows the last MMA),
+                // so with one token chunk (BNX = 32) the contributors' partials
+                // can land there: all of them in flight at once, whatever the
+                // register budget.  Thread `row` owns the 16-byte words
+                // (i, v, row), i the contributor and v the token quad, laid out
+                // so a warp's accesses are contiguous.
+                const int64_t S = cl - cf + 1;
+                const bool ring_free = seg_end == u1;
+                const int4 *land = reinterpret_cast<const int4 *>(gb + (sW - base));
 #pragma unroll 1
                 for (int cc = 0; cc < BNX / 32; ++cc) {
                     if (cc * 32 >= M)
@@ -371,7 +381,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                         r[4 * v + 2] += static_cast<uint32_t>(a.z);
                         r[4 * v + 3] += static_cast<uint32_t>(a.w);
                     };
-                    if (nv <= 2) {
+                    if (BNX == 32 && ring_free && S * nv * kBM * 16 <= static_cast<int64_t>(stages) * Cfg::STAGE_BYTES) {
+                        for (int64_t i = 0; i < S; ++i) {
+                            const int4 *p = part(cf + i);
+                            for (int v = 0; v < nv; ++v)
+                                cp_async_16(sW + static_cast<uint32_t>(((i * nv + v) * kBM + row) * 16), p + v, true);
+                        }
+                        cp_async_wait_all();
+                        for (int64_t i = 0; i < S; ++i) {
+#pragma unroll
+                            for (int v = 0; v < 8; ++v)
+                                if (v < nv)
+                                    add4(v, land[(i * nv + v) * kBM + row]);
+                        }
+                    } else if (nv <= 2) {
                         // at most 8 tokens: four contributors' loads in flight at a time
                         for (int64_t c2 = cf; c2 <= cl; c2 += 4) {
                             int4 a[4][2];
