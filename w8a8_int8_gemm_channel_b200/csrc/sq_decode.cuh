@@ -344,10 +344,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             dec_bar_sync();
             const int64_t cf = dec_owner(t * KB, U, G), cl = dec_owner((t + 1) * KB - 1, U, G);
             if (et == 0) {
-                __threadfence();
-                const int old = atomicAdd(cnt + t, 1);
+                // release: this CTA's partial (ordered before it by the
+                // barrier) precedes the count; acquire: the other
+                // contributors' partials precede the reads that follow
+                const int old = atom_add_acq_rel_gpu(cnt + t, 1);
                 *last_flag = old == static_cast<int>(cl - cf);
-                __threadfence();
             }
             dec_bar_sync();
             if (*last_flag) {

@@ -199,6 +199,14 @@ __device__ __forceinline__ bool bounded_wait_cluster(uint32_t bar, uint32_t pari
     }
 }
 
+// Atomic add with release and acquire semantics at GPU scope; returns the old value.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int *p, int v)
+{
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 // Split cluster barrier (not .aligned: the lanes of a warp may reach it apart).
 __device__ __forceinline__ void cluster_arrive()
 {
