@@ -843,13 +843,19 @@ inline int64_t quant_smem_estimate(int64_t K, sq_dtype dt)
 }
 
 // CTAs of the weight-streaming GEMM.  The units are cut into G equal
-// ranges; with G = S * T (T tiles, S <= KB) every range lies inside one tile,
+// ranges: with G = S * T (T tiles, S <= KB) every range lies inside one tile,
 // so a CTA has one partial tile to sum through the workspace instead of up
-// to two.  A partial tile's epilogue (stores, a release, a count, perhaps the
-// reduction) is a chain of global-memory round trips worth about
-// kDecodeEpiUnits units of streaming, so G is the choice with the fewest
-// units per CTA plus that cost per partial tile.
-constexpr int64_t kDecodeEpiUnits = 6;
+// to two; with G = T / D (D dividing T, for T above the SM count) every range
+// is D whole tiles and nothing is summed.  A shared tile's epilogue (stores,
+// a release, a count, the reduction) costs, in units of streaming, a fixed
+// kDecodeEpiUnits plus, per contributor, a part that grows with the tokens
+// (its partial's bytes); G is the choice with the fewest units per CTA plus
+// that cost.  Fitted to sq_linear calls on B200 (one call, L2 flushed): at
+// 1 to 16 tokens three or four CTAs a 4096-long tile were best, at 32 two,
+// from 64 one; with K = 14336 four at every token count; at 64 to 128
+// tokens and N = 28672, two whole tiles a CTA (42 -> 36 us, 52 -> 40 us).
+constexpr int64_t kDecodeEpiUnits = 4;
+inline int64_t decode_epi_units(int64_t M, int64_t S) { return kDecodeEpiUnits + (1 + std::min<int64_t>(M, 64) / 8) * S; }
 
 // Whether the few-token kernels request their first weight tiles before
 // griddepcontrol.wait when the grid before is the library's quantiser
@@ -863,21 +869,30 @@ inline bool decode_prewait()
     return on;
 }
 
-inline int64_t decode_ctas(int64_t N, int64_t K, int64_t sms)
+inline int64_t decode_ctas(int64_t M, int64_t N, int64_t K, int64_t sms)
 {
     const int64_t T = (N + sq::kBM - 1) / sq::kBM, KB = (K + sq::kBK - 1) / sq::kBK, U = T * KB;
     static const int64_t force = std::getenv("SQ_DECODE_CTAS") ? std::atoll(std::getenv("SQ_DECODE_CTAS")) : 0;
     if (force > 0)
         return std::min(force, std::min(U, sms));
     int64_t best = std::min(U, sms);
-    // the stream cut: ranges may span two tiles, so up to two partial tiles a CTA
-    int64_t best_cost = (U + best - 1) / best + (best < U ? 2 : 0) * kDecodeEpiUnits;
+    // the stream cut: ranges may span two tiles, so up to two partial tiles a
+    // CTA, each shared by about two CTAs
+    int64_t best_cost = (U + best - 1) / best + (best < U ? 2 * decode_epi_units(M, 2) : 0);
     for (int64_t S = 1; S <= KB && S * T <= sms; ++S) {
-        const int64_t G = S * T;
-        const int64_t cost = (KB + S - 1) / S + (S > 1 ? kDecodeEpiUnits : 0);
+        const int64_t cost = (KB + S - 1) / S + (S > 1 ? decode_epi_units(M, S) : 0);
         if (cost < best_cost) {
             best_cost = cost;
-            best = G;
+            best = S * T;
+        }
+    }
+    for (int64_t D = 2; D <= T && T > sms; ++D) {
+        if (T % D != 0 || T / D > sms)
+            continue;
+        const int64_t cost = D * KB;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = T / D;
         }
     }
     return best;
@@ -893,7 +908,7 @@ sq_status launch_decode_cfg(const int8_t *xq, const float *sx, const int8_t *wq,
     if (!device_info(di))
         return SQ_ERR_CUDA;
     const int64_t U = decode_units(N, K);
-    const int G = static_cast<int>(decode_ctas(N, K, std::min<int64_t>(di.sms, kDecodeMaxCtas)));
+    const int G = static_cast<int>(decode_ctas(M, N, K, std::min<int64_t>(di.sms, kDecodeMaxCtas)));
     // the deepest ring that still leaves room for a quantiser CTA on the SM
     // (the two kernels overlap), within the per-CTA limit
     static const int force_stages = std::getenv("SQ_DECODE_STAGES") ? std::atoi(std::getenv("SQ_DECODE_STAGES")) : 0;
