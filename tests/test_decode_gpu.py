@@ -4,7 +4,10 @@ For up to 128 tokens sq_linear runs the activation quantiser and then a GEMM
 that streams the weight over every SM: the T x KB weight units (128 output
 channels x 128 bytes of K each) are cut into one contiguous range per CTA, a
 tile shared by several CTAs is summed through int32 partials in the
-workspace, and the quantiser clears the tiles' counters.  (For at most 32
+workspace, and the quantiser clears the tiles' counters.  The plan weighs
+the streamed units per CTA against the reduction, whose cost grows with the
+tokens: from 64 tokens, or with more tiles than SMs, ranges of whole tiles
+(nothing summed) are chosen too.  (For at most 32
 tokens on layers of about 19K-38K output channels the slab kernel runs
 instead: tests/test_slab_gpu.py.)  With SQ_DECODE_STREAM=0 the split-K
 cluster kernel runs instead (K split across the CTAs of a cluster, partials
@@ -69,8 +72,14 @@ def _run(xt, s, wq, sw, out_dtype, ws=None):
 @pytest.mark.parametrize("M,N,K", [
     (1, 6144, 4096),      # 1536 units over 148 CTAs: tiles split over two CTAs
     (8, 4096, 4096),
-    (16, 28672, 4096),    # several whole tiles a CTA
+    (16, 28672, 4096),    # the slab kernel's shape (several whole tiles a CTA with SQ_DECODE_SLAB=0)
     (32, 4096, 14336),    # a tile spread over several CTAs
+    (32, 4096, 4096),     # two CTAs a tile
+    (40, 20480, 2048),    # more tiles than SMs: two whole tiles a CTA, nothing summed
+    (64, 28672, 1024),
+    (128, 6144, 1024),    # one CTA a tile, nothing summed
+    (100, 2048, 8192),    # 128-token tiles shared by three CTAs
+    (48, 1024, 8192),     # 64-token tiles shared by three CTAs
     (33, 4112, 4112),     # ragged N and K, 64-token tile
     (64, 1040, 3088),
     (100, 6144, 4096),    # 128-token tile
