@@ -20,12 +20,13 @@
 // Layout.  With a few rows, one CTA a row leaves most SMs idle, and a long
 // row's instructions on one SM are most of its latency.  Here the row's K / V
 // 16-byte chunks are cut into C contiguous slices (C = the cluster size: 2, 4
-// or 8), one per CTA, held in registers (CH chunks a thread).  The row maximum
-// is combined twice (the bound A, then the exact maximum E): across the warps
-// of a CTA through shared memory, then across the cluster -- every CTA stores
-// its maximum into each CTA's shared memory (distributed shared memory) and
-// waits at a cluster barrier, whose release / acquire orders those stores.
-// Every CTA of the cluster thus derives the same scale; CTA 0 stores it.
+// or 8), one per CTA, held in registers (CH chunks a thread).  Each warp
+// resolves its exact-maximum candidates against its own largest bound, so the
+// row's exact maximum E is combined once: across the warps of a CTA through
+// shared memory, then across the cluster -- every CTA stores its maximum into
+// each CTA's shared memory (distributed shared memory) and waits at a cluster
+// barrier, whose release / acquire orders those stores.  Every CTA of the
+// cluster thus derives the same scale; CTA 0 stores it.
 // The grid is rows x C CTAs: one cluster a row.
 #pragma once
 
@@ -52,8 +53,8 @@ __global__ void __launch_bounds__(kQuantClusterThreads, 2)
     constexpr int V = Vec<T>::N;
     constexpr int THREADS = kQuantClusterThreads;
     constexpr int WARPS = THREADS / 32;
-    __shared__ float red[2][WARPS];
-    __shared__ float cmax[2][kQuantClusterMax];
+    __shared__ float red[WARPS];
+    __shared__ float cmax[kQuantClusterMax];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int C = static_cast<int>(cluster_nctarank());
     const int rank = static_cast<int>(cluster_ctarank());
@@ -89,24 +90,24 @@ __global__ void __launch_bounds__(kQuantClusterThreads, 2)
         }
         return bad;
     };
-    // maximum over the row: the CTA's warps, then the cluster's CTAs (b: the
-    // exchange buffer, one per exchange, so none is rewritten)
-    auto row_max = [&](float v, int b) -> float {
+    // maximum over the row (called once): the CTA's warps, then the
+    // cluster's CTAs
+    auto row_max = [&](float v) -> float {
         v = warp_max(v);
         if (lane == 0)
-            red[b][warp] = v;
+            red[warp] = v;
         __syncthreads();
-        float m = red[b][0];
+        float m = red[0];
 #pragma unroll
         for (int j = 1; j < WARPS; ++j)
-            m = fmaxf(m, red[b][j]);
+            m = fmaxf(m, red[j]);
         if (static_cast<int>(threadIdx.x) < C)
-            st_shared_cluster_f32(map_shared_rank(smem_u32(&cmax[b][rank]), threadIdx.x), m);
+            st_shared_cluster_f32(map_shared_rank(smem_u32(&cmax[rank]), threadIdx.x), m);
         cluster_arrive();
         cluster_wait();
-        float r = cmax[b][0];
+        float r = cmax[0];
         for (int j = 1; j < C; ++j)
-            r = fmaxf(r, cmax[b][j]);
+            r = fmaxf(r, cmax[j]);
         return r;
     };
 
@@ -132,11 +133,18 @@ __global__ void __launch_bounds__(kQuantClusterThreads, 2)
             am = fmaxf(am, hm[i]);
         }
     }
-    const float A = row_max(am, 0);
+    // Each warp takes its own exact candidates, against its own largest
+    // bound A: the chunk holding the row's exact maximum has a bound within
+    // the candidate window of its warp's largest bound, so one exchange of
+    // the warps' exact maxima gives E.  A chunk whose bound is not finite (an
+    // s_k outside the fast range, or an overflowing product) is a candidate
+    // and has its codes taken exactly.
+    const float A = warp_max(am);
     float E = A;  // weights: the fp32 products are the values themselves
-    // an s_k outside the fast range shows as A = +inf; such a row's codes
-    // are all taken exactly too
-    const bool row_exact = MODE == MODE_X && !(A <= 0x1.fffffep127f);
+    uint32_t unbounded = 0;
+#pragma unroll
+    for (int i = 0; i < CH; ++i)
+        unbounded |= !(hm[i] <= 0x1.fffffep127f) ? (1u << i) : 0u;
     if (MODE == MODE_X) {
         const bool exact_all = !(A >= kTinyQuotient) || !(A <= 0x1.fffffep127f);
         const float thr = __fmul_rn(A, kCandidateScale);
@@ -158,7 +166,9 @@ __global__ void __launch_bounds__(kQuantClusterThreads, 2)
             const int64_t c = c0 + THREADS * i;
             em = fmaxf(em, chunk_exact_absmax<T, MODE>(v, s + c * V));
         }
-        E = row_max(em, 1);
+        E = row_max(em);
+    } else {
+        E = row_max(A);
     }
 
     // 2. scale and codes, from the registers
@@ -166,7 +176,7 @@ __global__ void __launch_bounds__(kQuantClusterThreads, 2)
     if (rank == 0 && threadIdx.x == 0)
         scale_out[row] = scale;
     const float rsc = rcp_approx(scale);
-    const bool fast = scale_in_fast_range(scale) && !row_exact;
+    const bool fast = scale_in_fast_range(scale);
     const float2 rsc2 = make_float2(rsc, rsc);
     const float2 nrsc2 = make_float2(-rsc, -rsc);
     const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
@@ -200,6 +210,7 @@ __global__ void __launch_bounds__(kQuantClusterThreads, 2)
             store_code_words(dst + static_cast<int64_t>(c) * V, y, V);
         }
     }
+    ties |= unbounded;
     while (ties != 0u) {  // rare: near ties; every chunk when the scale is outside the fast range
         const int i = __ffs(ties) - 1;
         ties &= ties - 1u;

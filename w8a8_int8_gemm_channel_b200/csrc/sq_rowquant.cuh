@@ -530,8 +530,9 @@ __global__ void __launch_bounds__(THREADS, (THREADS >= 1024 ? 1
     constexpr bool tab = TAB;
     // TAB = false (few rows, fp32 bound only): no factor table; each lane reads
     // its chunks' s_k from global memory and takes the hardware reciprocal
-    // itself, and a chunk with an s_k outside the fast range bounds its
-    // elements by +inf, which sends the row to the exact path throughout
+    // itself; a chunk with an s_k outside the fast range bounds its elements
+    // by +inf, which makes it an exact candidate and sends its codes to the
+    // exact path
     pdl_prologue();
     clear_ints(zero, nzero);
     constexpr int V = Vec<T>::N;
@@ -699,11 +700,19 @@ __global__ void __launch_bounds__(THREADS, (THREADS >= 1024 ? 1
                 am = fmaxf(am, hm[i]);
             }
         }
-        const float A = group_max(am);
+        // Each warp takes its own exact-maximum candidates against its own
+        // largest bound A, so one exchange of the warps' exact maxima gives E:
+        // the chunk holding the row's exact maximum has a bound within the
+        // candidate window of its warp's largest bound, as of the row's.  A
+        // chunk whose bound is not finite (without the table, an s_k outside
+        // the fast range; or an overflowing product) is a candidate and has
+        // its codes taken exactly.
+        const float A = warp_max(am);
         float E = A;  // fp32-bounded weights: the bounds are the values themselves
-        // without the table an s_k outside the fast range shows as A = +inf,
-        // and the codes of such a row are all taken exactly too
-        const bool row_exact = !tab && MODE == MODE_X && !(A <= 0x1.fffffep127f);
+        uint32_t unbounded = 0;
+#pragma unroll
+        for (int i = 0; i < CH; ++i)
+            unbounded |= !(hm[i] <= 0x1.fffffep127f) ? (1u << i) : 0u;
         if (BF || MODE == MODE_X) {
             const bool exact_all = bad_divisor || !(A >= kTinyQuotient) || !(A <= 0x1.fffffep127f);
             const float thr = __fmul_rn(A, BF ? 0.96875f : kCandidateScale);
@@ -726,6 +735,8 @@ __global__ void __launch_bounds__(THREADS, (THREADS >= 1024 ? 1
                 em = fmaxf(em, chunk_exact_absmax<T, MODE>(v, s + c * V));
             }
             E = group_max(em);
+        } else {
+            E = group_max(A);
         }
 
         // 2. scale and codes, from the registers
@@ -733,7 +744,7 @@ __global__ void __launch_bounds__(THREADS, (THREADS >= 1024 ? 1
         if (g == 0 && lane == 0)
             scale_out[row] = scale;
         const float rsc = rcp_approx(scale);
-        const bool fast = scale_in_fast_range(scale) && !bad_divisor && !row_exact;
+        const bool fast = scale_in_fast_range(scale) && !bad_divisor;
         const float2 rsc2 = make_float2(rsc, rsc);
         const float2 nrsc2 = make_float2(-rsc, -rsc);
         const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
@@ -767,6 +778,7 @@ __global__ void __launch_bounds__(THREADS, (THREADS >= 1024 ? 1
                 store_code_words(dst + static_cast<int64_t>(c) * V, y, V);
             }
         }
+        ties |= unbounded;
         while (ties != 0u) {  // rare: near ties; every chunk when the scale is outside the fast range
             const int i = __ffs(ties) - 1;
             ties &= ties - 1u;
