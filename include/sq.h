@@ -268,11 +268,13 @@ SQ_API sq_status sq_w8a8_gemm(const int8_t *xq, const float *sx, const int8_t *w
  * sq_w8a8_gemm with a workspace, which lets the GEMM use every SM whatever the
  * shape ("quant_llm_int8", "The architecture: every piece explained": the
  * same int32 accumulation and outer-product dequantisation):
- *   - up to 128 tokens, the weight is streamed by one CTA per SM, each taking
- *     an equal share of the 128-channel x 128-byte weight blocks (up to 32
- *     tokens on layers whose output channels split into slabs of 128-256 per
- *     SM, every CTA takes whole channels instead and the workspace is not
- *     touched);
+ *   - up to 128 tokens, the weight is streamed by at most one CTA per SM,
+ *     each taking an equal share of the 128-channel x 128-byte weight
+ *     blocks; where summing shared blocks would cost more than it saves
+ *     (typically from 64 tokens) the CTAs take whole 128-channel blocks
+ *     instead (up to 32 tokens on layers whose output channels split into
+ *     slabs of 128-256 per SM, every CTA takes whole channels and the
+ *     workspace is not touched);
  *   - more tokens: the same tiles as sq_w8a8_gemm; with SQ_GEMM_SK=1 in the
  *     environment the tiles that do not fill whole rounds of the CTA pairs
  *     are split along K over all pairs (off by default: slower on B200).
