@@ -1068,8 +1068,12 @@ bool gemm_sk_enabled()
 // rounds of the co-resident pairs, the last round and the partial one are
 // done stream-K: their k blocks are cut into one equal range per pair, and
 // tiles shared by several pairs are summed through int32 partials.
-// K from which the pair GEMM takes its tiles in groups of 8 m blocks.
-constexpr int64_t kPairGroupMinK = 16384;
+// The pair GEMM takes its tiles in groups of kPairGroupM m blocks (m fastest
+// within a group, then n; see pair_tile_mn): fewer operand re-reads from DRAM.  In the
+// Llama-3-70B step under the 1 kW power cap this mattered for K = 8192 as well
+// (2736 -> 2854 TOPS, three interleaved runs each on one B200), though a
+// single K = 8192 GEMM timed alone was no faster: the re-reads cost DRAM power.
+constexpr int kPairGroupM = 8;
 
 template <int BN, int STAGES, int OUT>
 sq_status launch_gemm_pair_cfg(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
@@ -1105,11 +1109,10 @@ sq_status launch_gemm_pair_cfg(const int8_t *xq, const float *sx, const int8_t *
         std::fprintf(stderr, "sq gemm pair M=%lld N=%lld K=%lld: BN=%d stages=%d tiles=%lld pairs=%lld sk_first=%lld sk_units=%lld\n",
                      (long long)M, (long long)N, (long long)K, BN, STAGES, (long long)tiles, (long long)pairs,
                      (long long)sk_first, (long long)sk_units);
-    // tile order: groups of 8 m blocks for long K (less DRAM traffic, see
-    // pair_tile_mn), m fastest otherwise; SQ_PAIR_GROUP_M overrides
+    // tile order: groups of kPairGroupM m blocks; SQ_PAIR_GROUP_M overrides
+    // (a value of at least the m block count gives the m-fastest order)
     static const int force_gm = std::getenv("SQ_PAIR_GROUP_M") ? std::atoi(std::getenv("SQ_PAIR_GROUP_M")) : 0;
-    const int m_tiles = static_cast<int>((M + sq::kPairBM - 1) / sq::kPairBM);
-    const int group_m = force_gm > 0 ? force_gm : (K >= kPairGroupMinK ? 8 : m_tiles);
+    const int group_m = force_gm > 0 ? force_gm : kPairGroupM;
     return launch_kernel(kernel, dim3(static_cast<unsigned>(2 * pairs)), dim3(sq::kPairThreads), Cfg::SMEM_BYTES, st, 2,
                          1, ta, tb, sx, sw, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
                          static_cast<int>(sk_first), sk_units, slots, cnt, std::max(group_m, 1));
