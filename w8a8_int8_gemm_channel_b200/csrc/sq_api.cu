@@ -854,6 +854,10 @@ inline int64_t quant_smem_estimate(int64_t K, sq_dtype dt)
 // 1 to 16 tokens three or four CTAs a 4096-long tile were best, at 32 two,
 // from 64 one; with K = 14336 four at every token count; at 64 to 128
 // tokens and N = 28672, two whole tiles a CTA (42 -> 36 us, 52 -> 40 us).
+// Small layers, whose units number at most the SMs, were once cut one unit
+// a CTA at no modelled reduction cost; costed like the rest they take fewer,
+// longer ranges (64 x 1024 x 2048: 44 -> 19 us; 1 x 1040 x 3088: 21.5 ->
+// 17.4 us; 128 x 2048 x 8192: 54 -> 40 us).
 constexpr int64_t kDecodeEpiUnits = 4;
 inline int64_t decode_epi_units(int64_t M, int64_t S) { return kDecodeEpiUnits + (1 + std::min<int64_t>(M, 64) / 8) * S; }
 
@@ -875,10 +879,17 @@ inline int64_t decode_ctas(int64_t M, int64_t N, int64_t K, int64_t sms)
     static const int64_t force = std::getenv("SQ_DECODE_CTAS") ? std::atoll(std::getenv("SQ_DECODE_CTAS")) : 0;
     if (force > 0)
         return std::min(force, std::min(U, sms));
-    int64_t best = std::min(U, sms);
-    // the stream cut: ranges may span two tiles, so up to two partial tiles a
-    // CTA, each shared by about two CTAs
-    int64_t best_cost = (U + best - 1) / best + (best < U ? 2 * decode_epi_units(M, 2) : 0);
+    int64_t best = 0, best_cost = INT64_MAX;
+    if (U > sms) {
+        // the stream cut over every SM: ranges of `per` units may span two
+        // tiles, each tile shared by about KB / per + 1 CTAs; the first
+        // partial tile's reduction overlaps the rest of the range, so the
+        // second's costs in full and the first's its fixed part
+        const int64_t per = (U + sms - 1) / sms;
+        const int64_t shared = std::max<int64_t>(2, (KB + per - 1) / per + 1);
+        best = sms;
+        best_cost = per + decode_epi_units(M, shared) + kDecodeEpiUnits;
+    }
     for (int64_t S = 1; S <= KB && S * T <= sms; ++S) {
         const int64_t cost = (KB + S - 1) / S + (S > 1 ? decode_epi_units(M, S) : 0);
         if (cost < best_cost) {
@@ -895,7 +906,7 @@ inline int64_t decode_ctas(int64_t M, int64_t N, int64_t K, int64_t sms)
             best = T / D;
         }
     }
-    return best;
+    return best > 0 ? best : std::min(U, sms);
 }
 
 template <int BNX, int OUT>
