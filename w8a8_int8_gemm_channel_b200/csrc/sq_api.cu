@@ -433,22 +433,23 @@ sq_status launch_quant_cluster_cfg(const T *in, int64_t rows, int64_t K, const f
 // (rows x C <= SMs) and leaves every CTA a slice of at least 128 chunks.
 // Measured in the decode chain of sq_linear calls (1 to 32 tokens) at
 // K = 14336: 4 to 8 SMs a row took about 2 us less a call than one.  At
-// K = 4096 (512 chunks) 2 to 4 SMs a row took 2 us more -- the two cluster
-// barriers outweigh the shorter slice -- so such rows keep the one-CTA forms.
+// K = 4096 (512 chunks) 2 to 4 SMs a row took 2 us more while the form
+// exchanged twice a row; with one exchange, 4 SMs a row came within 0.3 us a
+// pass of one (2 SMs: 5 us slower), so such rows keep the one-CTA forms.
 // Returns false (nothing launched) when no C qualifies.  SQ_QUANT_CLUSTER=0
-// turns the form off; SQ_QUANT_CLUSTER_MIN sets the smallest slice in chunks
-// (tuning).
+// turns the form off, =2 takes it for rows of 512 chunks or fewer too;
+// SQ_QUANT_CLUSTER_MIN sets the smallest slice in chunks (tuning).
 template <typename T, int MODE>
 bool launch_quant_cluster(const T *in, int64_t rows, int64_t K, const float *s, int8_t *q, float *scale,
                           cudaStream_t st, const DeviceInfo &di, int *zero, int nzero, sq_status &r)
 {
-    static const bool on = !(std::getenv("SQ_QUANT_CLUSTER") && std::atoi(std::getenv("SQ_QUANT_CLUSTER")) == 0);
+    static const int mode = std::getenv("SQ_QUANT_CLUSTER") ? std::atoi(std::getenv("SQ_QUANT_CLUSTER")) : 1;
     static const int min_span =
         std::getenv("SQ_QUANT_CLUSTER_MIN") ? std::max(32, std::atoi(std::getenv("SQ_QUANT_CLUSTER_MIN"))) : 128;
     constexpr int V = sq::Vec<T>::N;
     const int64_t nch = K / V;
     // C >= 2 and CH <= 8 cover rows of up to 2 * 8 * 256 chunks
-    if (!on || nch <= (int64_t)32 * 8 * 2 || nch > (int64_t)2 * 8 * sq::kQuantClusterThreads)
+    if (mode == 0 || (mode == 1 && nch <= (int64_t)32 * 8 * 2) || nch > (int64_t)2 * 8 * sq::kQuantClusterThreads)
         return false;
     int C = 0;
     for (int c : {8, 4, 2})
