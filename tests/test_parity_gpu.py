@@ -301,6 +301,51 @@ def test_few_row_quantiser_8_warps_child_process():
     assert r.returncode == 0 and "few8-ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]
 
 
+CHILD_CLUSTER_SHORT = r'''
+import numpy as np
+import torch
+import w8a8_int8_gemm_channel_b200 as sq
+from oracle import oracle
+from w8a8_int8_gemm_channel_b200 import workloads as wls
+oracle.build()
+bits = lambda t: t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+for (R, K, dt) in [(1, 4096, torch.bfloat16), (30, 4096, torch.bfloat16), (9, 4112, torch.bfloat16),
+                   (5, 4096, torch.float32), (37, 2048, torch.bfloat16)]:
+    x = wls.random_tensor((R, K), R * 11 + K, dtype=dt)
+    x[0, K - 3] = 700.0
+    if R > 2:
+        x[1] = 0
+        x[2] *= 1000
+    s = np.random.default_rng(K + 5).uniform(0.25, 8.0, K).astype(np.float32)
+    xq = torch.empty(R, K, dtype=torch.int8, device="cuda")
+    sx = torch.empty(R, device="cuda")
+    sq.sq_quant_act(x.cuda(), torch.from_numpy(s).cuda(), xq, sx)
+    torch.cuda.synchronize()
+    xin = bits(x) if dt == torch.bfloat16 else x.numpy()
+    xq_o, sx_o = oracle.quant_act(xin, s)
+    assert np.array_equal(xq.cpu().numpy(), xq_o) and np.array_equal(sx.cpu().numpy().view(np.uint32), sx_o.view(np.uint32)), (R, K)
+st, code = sq.sq_device_status()
+assert st == sq.SQ_OK, hex(code)
+print("cluster-short-ok")
+'''
+
+
+def test_cluster_form_on_short_rows_child_process():
+    """SQ_QUANT_CLUSTER=2 (read once per process, so in a child) gives rows of
+    512 chunks or fewer the cluster form too (clusters of 2, 4 and 8 CTAs with
+    slices of 128 to 129 chunks, ragged slices at K = 4112); codes and scales
+    equal the oracle's bit for bit."""
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SQ_QUANT_CLUSTER="2", PYTHONPATH=root)
+    r = subprocess.run([sys.executable, "-c", CHILD_CLUSTER_SHORT], cwd=root, env=env, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0 and "cluster-short-ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]
+
+
 # ---------------------------------------------------------------------------
 # GEMM: int32 accumulators and the dequantised output
 # ---------------------------------------------------------------------------
